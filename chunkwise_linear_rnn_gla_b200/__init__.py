@@ -1,0 +1,247 @@
+"""Chunkwise gated linear attention (GLA) for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/gla.h`` (``libgla.so``). Every
+step of the layer runs in the library's CUDA kernels; this module only checks
+tensors, allocates outputs and workspace with torch, and passes pointers and
+the current CUDA stream. There is no CPU fallback: without the built library
+every call raises.
+
+Layer (per batch b and head h; "Gated Linear Attention Transformers with
+Hardware-Efficient Training", atlas.scime.ai summary, section "Approach"):
+    S_t = diag(exp(log_a_t)) S_{t-1} + k_t^T v_t,    o_t = q_t S_t.
+Shapes: q, k, log_a [B,H,L,Dk]; v [B,H,L,Dv]; states [B,H,Dk,Dv] (fp32).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import GlaDesc, GlaError, load  # noqa: F401
+
+__all__ = ["gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum", "gla_fwd_workspace_size",
+           "gla_bwd_workspace_size", "gla_resolve", "gla_check_device_error", "gla_launch_count",
+           "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset",
+           "make_desc", "GlaError"]
+
+_TORCH_DTYPE = {torch.float32: "f32", torch.bfloat16: "bf16"}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check(status: int, what: str):
+    if status != _lib.GLA_OK:
+        raise GlaError(status, what)
+
+
+def _dt(t: torch.Tensor) -> str:
+    if t.dtype not in _TORCH_DTYPE:
+        raise TypeError("q/k/v/dO must be float32 or bfloat16, got %s" % t.dtype)
+    return _TORCH_DTYPE[t.dtype]
+
+
+def _need(t, name, shape, dtype, dev):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch.Tensor" % name)
+    if t.device != dev:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, dev))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if t.dtype != dtype:
+        raise TypeError("%s has dtype %s, expected %s" % (name, t.dtype, dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def make_desc(B, H, L, Dk, Dv, dtype="bf16", chunk=0, subchunk=0, state_mode="auto", impl="auto",
+              flags=0) -> GlaDesc:
+    return GlaDesc(B, H, L, Dk, Dv, _lib.DTYPE[dtype], chunk, subchunk, _lib.STATE_MODE[state_mode],
+                   _lib.IMPL[impl], flags)
+
+
+def gla_fwd_workspace_size(desc: GlaDesc) -> int:
+    return int(load().gla_fwd_workspace_size(ctypes.byref(desc)))
+
+
+def gla_bwd_workspace_size(desc: GlaDesc) -> int:
+    return int(load().gla_bwd_workspace_size(ctypes.byref(desc)))
+
+
+def gla_resolve(desc: GlaDesc):
+    """(chunk, subchunk, impl, state_mode) the library resolves `desc` to."""
+    c, sc, im, sm = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(load().gla_resolve(ctypes.byref(desc), ctypes.byref(c), ctypes.byref(sc), ctypes.byref(im),
+                              ctypes.byref(sm)), "gla_resolve")
+    inv_impl = {v: k for k, v in _lib.IMPL.items()}
+    inv_sm = {v: k for k, v in _lib.STATE_MODE.items()}
+    return c.value, sc.value, inv_impl[im.value], inv_sm[sm.value]
+
+
+def _workspace(nbytes: int, dev, workspace: Optional[torch.Tensor]):
+    if nbytes == 0:
+        return None, 0
+    if workspace is None:
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    if workspace.numel() * workspace.element_size() < nbytes:
+        raise ValueError("workspace too small: %d < %d bytes" % (workspace.numel() * workspace.element_size(), nbytes))
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def _desc_from(q, v, chunk, subchunk, state_mode, impl, flags=0):
+    B, H, L, Dk = q.shape
+    Dv = v.shape[-1]
+    return make_desc(B, H, L, Dk, Dv, _dt(q), chunk, subchunk, state_mode, impl, flags)
+
+
+def gla_fwd(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto", o=None, hT=None,
+            want_hT=True, workspace=None):
+    """Forward. Returns (o, hT); hT is None when want_hT is False and no hT
+    buffer is given. `workspace` (uint8 tensor) may be passed to reuse it."""
+    load()
+    dev = q.device
+    B, H, L, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", q.shape, dt, dev)
+    _need(v, "v", (B, H, L, Dv), dt, dev)
+    _need(log_a, "log_a", q.shape, torch.float32, dev)
+    if h0 is not None:
+        _need(h0, "h0", (B, H, Dk, Dv), torch.float32, dev)
+    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl)
+    if o is None:
+        o = torch.empty(B, H, L, Dv, dtype=dt, device=dev)
+    _need(o, "o", (B, H, L, Dv), dt, dev)
+    if hT is None and want_hT:
+        hT = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+    if hT is not None:
+        _need(hT, "hT", (B, H, Dk, Dv), torch.float32, dev)
+    ws, nbytes = _workspace(gla_fwd_workspace_size(desc), dev, workspace)
+    with torch.cuda.device(dev):
+        st = load().gla_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(h0), _ptr(o),
+                            _ptr(hT), _ptr(ws), nbytes, _stream(dev))
+    _check(st, "gla_fwd")
+    return o, hT
+
+
+def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto",
+            want_dh0=True, workspace=None, ws_from_fwd=False, out=None):
+    """Backward of <dO, o> + <dhT, hT>. Returns a dict with dq, dk, dv,
+    dlog_a and dh0. With ws_from_fwd=True the workspace must be the one the
+    matching gla_fwd call used (same inputs, same options)."""
+    load()
+    dev = q.device
+    B, H, L, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", q.shape, dt, dev)
+    _need(v, "v", (B, H, L, Dv), dt, dev)
+    _need(log_a, "log_a", q.shape, torch.float32, dev)
+    _need(dO, "dO", (B, H, L, Dv), dt, dev)
+    if h0 is not None:
+        _need(h0, "h0", (B, H, Dk, Dv), torch.float32, dev)
+    if dhT is not None:
+        _need(dhT, "dhT", (B, H, Dk, Dv), torch.float32, dev)
+    flags = _lib.FLAG_WS_FROM_FWD if ws_from_fwd else 0
+    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, flags)
+    if ws_from_fwd and workspace is None:
+        raise ValueError("ws_from_fwd needs the forward's workspace")
+    out = dict(out or {})
+    dq = out.get("dq")
+    if dq is None:
+        dq = torch.empty_like(q)
+    dk = out.get("dk")
+    if dk is None:
+        dk = torch.empty_like(k)
+    dv = out.get("dv")
+    if dv is None:
+        dv = torch.empty_like(v)
+    dla = out.get("dlog_a")
+    if dla is None:
+        dla = torch.empty_like(log_a)
+    dh0 = out.get("dh0")
+    if dh0 is None and want_dh0:
+        dh0 = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+    ws, nbytes = _workspace(gla_bwd_workspace_size(desc), dev, workspace)
+    with torch.cuda.device(dev):
+        st = load().gla_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(h0), _ptr(dO),
+                            _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dla), _ptr(dh0), _ptr(ws), nbytes,
+                            _stream(dev))
+    _check(st, "gla_bwd")
+    return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dh0": dh0}
+
+
+def gla_step(q, k, v, log_a, S, o=None):
+    """One decode step; S [B,H,Dk,Dv] fp32 is updated in place. Returns o [B,H,Dv]."""
+    load()
+    dev = q.device
+    B, H, Dk = q.shape
+    Dv = v.shape[-1]
+    dt = q.dtype
+    _need(k, "k", q.shape, dt, dev)
+    _need(v, "v", (B, H, Dv), dt, dev)
+    _need(log_a, "log_a", q.shape, torch.float32, dev)
+    _need(S, "S", (B, H, Dk, Dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, Dv, dtype=dt, device=dev)
+    _need(o, "o", (B, H, Dv), dt, dev)
+    desc = make_desc(B, H, 1, Dk, Dv, _dt(q))
+    with torch.cuda.device(dev):
+        st = load().gla_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(S), _ptr(o),
+                             _stream(dev))
+    _check(st, "gla_step")
+    return o
+
+
+def gla_chunk_cumsum(log_a, chunk=64, out=None):
+    """Per-chunk inclusive cumsum of log_a along L (restarting every `chunk`)."""
+    load()
+    dev = log_a.device
+    B, H, L, Dk = log_a.shape
+    _need(log_a, "log_a", log_a.shape, torch.float32, dev)
+    if out is None:
+        out = torch.empty_like(log_a)
+    desc = make_desc(B, H, L, Dk, 1, "f32", chunk)
+    with torch.cuda.device(dev):
+        st = load().gla_chunk_cumsum(ctypes.byref(desc), _ptr(log_a), _ptr(out), _stream(dev))
+    _check(st, "gla_chunk_cumsum")
+    return out
+
+
+def gla_check_device_error(stream=None) -> int:
+    s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
+    return int(load().gla_check_device_error(s))
+
+
+def gla_launch_count() -> int:
+    return int(load().gla_launch_count())
+
+
+def gla_launch_count_reset() -> None:
+    load().gla_launch_count_reset()
+
+
+def gla_profile_enable(on: bool = True) -> None:
+    load().gla_profile_enable(1 if on else 0)
+
+
+def gla_profile_read():
+    """{kernel name: (launches, total device ms)} of the recorded launches."""
+    lib = load()
+    cap = 64
+    names = (ctypes.c_char_p * cap)()
+    cnt = (ctypes.c_uint64 * cap)()
+    ms = (ctypes.c_double * cap)()
+    n = lib.gla_profile_read(names, cnt, ms, cap)
+    return {names[i].decode(): (int(cnt[i]), float(ms[i])) for i in range(min(n, cap))}
+
+
+def gla_profile_reset() -> None:
+    load().gla_profile_reset()

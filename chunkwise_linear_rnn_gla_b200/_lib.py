@@ -1,0 +1,98 @@
+"""ctypes declarations of the libgla C ABI (include/gla.h).
+
+Loading fails loudly: there is no Python or CPU fallback for any entry point.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libgla.so")
+
+GLA_OK = 0
+STATUS_NAMES = {0: "GLA_OK", 1: "GLA_ERR_INVALID_ARG", 2: "GLA_ERR_UNSUPPORTED", 3: "GLA_ERR_WORKSPACE",
+                4: "GLA_ERR_CUDA", 5: "GLA_ERR_TIMEOUT"}
+DTYPE = {"f32": 0, "bf16": 1}
+STATE_MODE = {"auto": 0, "materialized": 1, "nonmaterialized": 2}
+IMPL = {"auto": 0, "simt": 1, "tc": 2}
+FLAG_WS_FROM_FWD = 0x1
+
+# Every function the header declares, for the ABI-completeness test.
+EXPORTS = (
+    "gla_fwd_workspace_size", "gla_bwd_workspace_size", "gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum",
+    "gla_check_device_error", "gla_status_string", "gla_abi_version", "gla_resolve", "gla_launch_count",
+    "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset",
+)
+
+
+class GlaDesc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("L", ctypes.c_int64), ("Dk", ctypes.c_int64),
+                ("Dv", ctypes.c_int64), ("dtype", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("subchunk", ctypes.c_int32), ("state_mode", ctypes.c_int32), ("impl", ctypes.c_int32),
+                ("flags", ctypes.c_int32)]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+class GlaError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__("%s failed: %s (%s)" % (what, STATUS_NAMES.get(status, status), status_string(status)))
+
+
+def _declare(lib):
+    vp, sz, i32, u64 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_uint64
+    dp = ctypes.POINTER(GlaDesc)
+    lib.gla_fwd_workspace_size.argtypes = [dp]
+    lib.gla_fwd_workspace_size.restype = sz
+    lib.gla_bwd_workspace_size.argtypes = [dp]
+    lib.gla_bwd_workspace_size.restype = sz
+    lib.gla_fwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gla_fwd.restype = ctypes.c_int
+    lib.gla_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gla_bwd.restype = ctypes.c_int
+    lib.gla_step.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gla_step.restype = ctypes.c_int
+    lib.gla_chunk_cumsum.argtypes = [dp, vp, vp, vp]
+    lib.gla_chunk_cumsum.restype = ctypes.c_int
+    lib.gla_check_device_error.argtypes = [vp]
+    lib.gla_check_device_error.restype = ctypes.c_int
+    lib.gla_status_string.argtypes = [ctypes.c_int]
+    lib.gla_status_string.restype = ctypes.c_char_p
+    lib.gla_abi_version.restype = ctypes.c_int
+    lib.gla_resolve.argtypes = [dp, ctypes.POINTER(i32), ctypes.POINTER(i32), ctypes.POINTER(i32),
+                                ctypes.POINTER(i32)]
+    lib.gla_resolve.restype = ctypes.c_int
+    lib.gla_launch_count.restype = u64
+    lib.gla_launch_count_reset.restype = None
+    lib.gla_profile_enable.argtypes = [ctypes.c_int]
+    lib.gla_profile_enable.restype = None
+    lib.gla_profile_read.argtypes = [ctypes.POINTER(ctypes.c_char_p), ctypes.POINTER(u64),
+                                     ctypes.POINTER(ctypes.c_double), ctypes.c_int]
+    lib.gla_profile_read.restype = ctypes.c_int
+    lib.gla_profile_reset.restype = None
+
+
+def load(path: str = LIB_PATH):
+    """Load libgla.so (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise ImportError("libgla.so not found at %s: build it with "
+                                  "`python -m chunkwise_linear_rnn_gla_b200.build`" % path)
+            lib = ctypes.CDLL(path)
+            _declare(lib)
+            _lib = lib
+    return _lib
+
+
+def status_string(status: int) -> str:
+    try:
+        return load().gla_status_string(int(status)).decode()
+    except Exception:  # library not loadable: still produce a message
+        return STATUS_NAMES.get(status, "unknown")

@@ -1,0 +1,358 @@
+// C ABI of libgla: argument checks, defaults, workspace sizing, dispatch,
+// status strings and the measurement hooks (launch counter, per-kernel event
+// timing). The arithmetic lives in the kernel files.
+
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "gla_internal.h"
+
+namespace gla {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+// ---- per-kernel event timing ----------------------------------------------
+struct ProfRec {
+    int id;
+    cudaEvent_t a, b;
+};
+std::mutex g_mu;
+bool g_prof = false;
+std::vector<ProfRec> g_pending;
+std::vector<cudaEvent_t> g_pool;
+std::vector<const char*> g_names;
+std::vector<uint64_t> g_counts;
+std::vector<double> g_ms;
+thread_local cudaEvent_t t_begin = nullptr;
+
+int name_id(const char* name) {
+    for (size_t i = 0; i < g_names.size(); ++i)
+        if (g_names[i] == name || std::strcmp(g_names[i], name) == 0) return int(i);
+    g_names.push_back(name);
+    g_counts.push_back(0);
+    g_ms.push_back(0.0);
+    return int(g_names.size() - 1);
+}
+
+cudaEvent_t get_event() {
+    if (!g_pool.empty()) {
+        cudaEvent_t e = g_pool.back();
+        g_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    if (cudaEventCreate(&e) != cudaSuccess) return nullptr;
+    return e;
+}
+
+void drain_locked() {
+    for (auto& r : g_pending) {
+        float ms = 0.f;
+        if (cudaEventSynchronize(r.b) == cudaSuccess && cudaEventElapsedTime(&ms, r.a, r.b) == cudaSuccess) {
+            g_counts[r.id] += 1;
+            g_ms[r.id] += ms;
+        }
+        g_pool.push_back(r.a);
+        g_pool.push_back(r.b);
+    }
+    g_pending.clear();
+}
+
+// ---- device error word ------------------------------------------------------
+__device__ int g_device_error;
+
+}  // namespace
+
+void launch_begin(const char* name, cudaStream_t s) {
+    (void)name;
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    t_begin = nullptr;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_prof) return;
+    cudaEvent_t a = get_event();
+    if (a && cudaEventRecord(a, s) == cudaSuccess) t_begin = a;
+    else if (a) g_pool.push_back(a);
+}
+
+gla_status launch_end(const char* name, cudaStream_t s) {
+    const cudaError_t err = cudaGetLastError();
+    if (t_begin) {
+        std::lock_guard<std::mutex> lk(g_mu);
+        cudaEvent_t b = get_event();
+        if (b && cudaEventRecord(b, s) == cudaSuccess) {
+            g_pending.push_back(ProfRec{name_id(name), t_begin, b});
+        } else {
+            g_pool.push_back(t_begin);
+            if (b) g_pool.push_back(b);
+        }
+        t_begin = nullptr;
+        if (g_pending.size() > 4096) drain_locked();
+    }
+    return err == cudaSuccess ? GLA_OK : GLA_ERR_CUDA;
+}
+
+int* device_error_word() {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+    return static_cast<int*>(p);
+}
+
+}  // namespace gla
+
+using gla::Problem;
+
+namespace {
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// Fill `p` from `d` (defaults applied). Returns GLA_OK or an error status.
+gla_status resolve(const gla_desc* d, Problem& p) {
+    if (!d) return GLA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H < 1 || d->L < 1 || d->Dk < 1 || d->Dv < 1) return GLA_ERR_INVALID_ARG;
+    if (d->dtype != GLA_DTYPE_F32 && d->dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+    if (d->chunk != 0 && d->chunk != 16 && d->chunk != 32 && d->chunk != 64 && d->chunk != 128)
+        return GLA_ERR_INVALID_ARG;
+    if (d->subchunk < 0) return GLA_ERR_INVALID_ARG;
+    if (d->state_mode < GLA_STATE_AUTO || d->state_mode > GLA_STATE_NONMATERIALIZED) return GLA_ERR_INVALID_ARG;
+    if (d->impl < GLA_IMPL_AUTO || d->impl > GLA_IMPL_TC) return GLA_ERR_INVALID_ARG;
+    if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD)) return GLA_ERR_INVALID_ARG;
+    p.B = d->B;
+    p.H = d->H;
+    p.L = d->L;
+    p.K = d->Dk;
+    p.V = d->Dv;
+    p.BH = d->B * d->H;
+    p.bf16 = d->dtype == GLA_DTYPE_BF16;
+    p.flags = d->flags;
+    if (p.BH > 65535) return GLA_ERR_UNSUPPORTED;
+    int impl = d->impl;
+    if (impl == GLA_IMPL_AUTO) {
+        Problem probe = p;
+        probe.C = d->chunk ? d->chunk : 128;
+        probe.c = d->subchunk ? d->subchunk : 16;
+        probe.N = (p.L + probe.C - 1) / probe.C;
+        probe.impl = GLA_IMPL_TC;
+        probe.state_mode = d->state_mode;
+        impl = (p.bf16 && gla::tc_supported(probe)) ? GLA_IMPL_TC : GLA_IMPL_SIMT;
+    }
+    p.impl = impl;
+    if (impl == GLA_IMPL_SIMT) {
+        p.C = d->chunk ? d->chunk : 64;
+        p.c = d->subchunk ? d->subchunk : p.C;
+        if (d->state_mode == GLA_STATE_NONMATERIALIZED) return GLA_ERR_UNSUPPORTED;
+        p.state_mode = GLA_STATE_MATERIALIZED;
+    } else {
+        if (!p.bf16) return GLA_ERR_UNSUPPORTED;
+        p.C = d->chunk ? d->chunk : 128;
+        p.c = d->subchunk ? d->subchunk : 16;
+        p.state_mode = d->state_mode == GLA_STATE_AUTO ? GLA_STATE_NONMATERIALIZED : d->state_mode;
+    }
+    if (p.c > p.C || p.C % p.c != 0) return GLA_ERR_INVALID_ARG;
+    p.N = (p.L + p.C - 1) / p.C;
+    if (p.N > 65535) return GLA_ERR_UNSUPPORTED;
+    if (impl == GLA_IMPL_TC && !gla::tc_supported(p)) return GLA_ERR_UNSUPPORTED;
+    return GLA_OK;
+}
+
+size_t fwd_ws(const Problem& p) { return p.impl == GLA_IMPL_TC ? gla::tc_fwd_workspace(p) : gla::simt_fwd_workspace(p); }
+size_t bwd_ws(const Problem& p) { return p.impl == GLA_IMPL_TC ? gla::tc_bwd_workspace(p) : gla::simt_bwd_workspace(p); }
+
+gla_status check_ws(void* ws, size_t bytes, size_t need) {
+    if (need == 0) return GLA_OK;
+    if (!ws || !aligned(ws, 256) || bytes < need) return GLA_ERR_WORKSPACE;
+    return GLA_OK;
+}
+
+#define GLA_REQUIRE_PTR(ptr) \
+    do {                     \
+        if (!(ptr) || !aligned((ptr), 16)) return GLA_ERR_INVALID_ARG; \
+    } while (0)
+#define GLA_OPTIONAL_PTR(ptr) \
+    do {                      \
+        if ((ptr) && !aligned((ptr), 16)) return GLA_ERR_INVALID_ARG; \
+    } while (0)
+
+}  // namespace
+
+extern "C" {
+
+int gla_abi_version(void) { return GLA_ABI_VERSION; }
+
+const char* gla_status_string(gla_status s) {
+    switch (s) {
+        case GLA_OK: return "ok";
+        case GLA_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size or enum)";
+        case GLA_ERR_UNSUPPORTED: return "unsupported shape or option for the selected kernel path";
+        case GLA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case GLA_ERR_CUDA: return "CUDA runtime error or failed kernel launch";
+        case GLA_ERR_TIMEOUT: return "a device-side bounded wait ran out";
+    }
+    return "unknown status";
+}
+
+gla_status gla_resolve(const gla_desc* d, int32_t* chunk, int32_t* subchunk, int32_t* impl, int32_t* state_mode) {
+    Problem p{};
+    gla_status st = resolve(d, p);
+    if (st != GLA_OK) return st;
+    if (chunk) *chunk = p.C;
+    if (subchunk) *subchunk = p.c;
+    if (impl) *impl = p.impl;
+    if (state_mode) *state_mode = p.state_mode;
+    return GLA_OK;
+}
+
+size_t gla_fwd_workspace_size(const gla_desc* d) {
+    Problem p{};
+    if (resolve(d, p) != GLA_OK) return 0;
+    return fwd_ws(p);
+}
+
+size_t gla_bwd_workspace_size(const gla_desc* d) {
+    Problem p{};
+    if (resolve(d, p) != GLA_OK) return 0;
+    const size_t a = fwd_ws(p), b = bwd_ws(p);
+    return a > b ? a : b;
+}
+
+gla_status gla_fwd(const gla_desc* d, const void* q, const void* k, const void* v, const float* log_a,
+                   const float* h0, void* o, float* hT, void* workspace, size_t workspace_bytes, void* stream) {
+    Problem p{};
+    gla_status st = resolve(d, p);
+    if (st != GLA_OK) return st;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(v);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(o);
+    GLA_OPTIONAL_PTR(h0);
+    GLA_OPTIONAL_PTR(hT);
+    const size_t need = fwd_ws(p);
+    st = check_ws(workspace, workspace_bytes, need);
+    if (st != GLA_OK) return st;
+    gla::Arena a{static_cast<char*>(workspace), workspace_bytes, 0};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p.impl == GLA_IMPL_TC) return gla::tc_fwd(p, q, k, v, log_a, h0, o, hT, a, s);
+    return gla::simt_fwd(p, q, k, v, log_a, h0, o, hT, a, s);
+}
+
+gla_status gla_bwd(const gla_desc* d, const void* q, const void* k, const void* v, const float* log_a,
+                   const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dlog_a,
+                   float* dh0, void* workspace, size_t workspace_bytes, void* stream) {
+    Problem p{};
+    gla_status st = resolve(d, p);
+    if (st != GLA_OK) return st;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(v);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(dO);
+    GLA_REQUIRE_PTR(dq);
+    GLA_REQUIRE_PTR(dk);
+    GLA_REQUIRE_PTR(dv);
+    GLA_REQUIRE_PTR(dlog_a);
+    GLA_OPTIONAL_PTR(h0);
+    GLA_OPTIONAL_PTR(dhT);
+    GLA_OPTIONAL_PTR(dh0);
+    const size_t need = bwd_ws(p);
+    st = check_ws(workspace, workspace_bytes, need);
+    if (st != GLA_OK) return st;
+    gla::Arena a{static_cast<char*>(workspace), workspace_bytes, 0};
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (p.impl == GLA_IMPL_TC) return gla::tc_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s);
+    return gla::simt_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s);
+}
+
+gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void* v, const float* log_a, float* S,
+                    void* o, void* stream) {
+    if (!d) return GLA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H < 1 || d->Dk < 1 || d->Dv < 1) return GLA_ERR_INVALID_ARG;
+    if (d->dtype != GLA_DTYPE_F32 && d->dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(v);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(S);
+    GLA_REQUIRE_PTR(o);
+    if (d->B * d->H > 65535 || d->Dk > 8192) return GLA_ERR_UNSUPPORTED;
+    Problem p{};
+    p.B = d->B;
+    p.H = d->H;
+    p.L = 1;
+    p.K = d->Dk;
+    p.V = d->Dv;
+    p.BH = d->B * d->H;
+    p.bf16 = d->dtype == GLA_DTYPE_BF16;
+    return gla::step_launch(p, q, k, v, log_a, S, o, static_cast<cudaStream_t>(stream));
+}
+
+gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, void* stream) {
+    if (!d) return GLA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H < 1 || d->L < 1 || d->Dk < 1) return GLA_ERR_INVALID_ARG;
+    const int C = d->chunk ? d->chunk : 64;
+    if (C != 16 && C != 32 && C != 64 && C != 128) return GLA_ERR_INVALID_ARG;
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(Bcum);
+    Problem p{};
+    p.B = d->B;
+    p.H = d->H;
+    p.L = d->L;
+    p.K = d->Dk;
+    p.V = d->Dv;
+    p.BH = d->B * d->H;
+    p.C = C;
+    p.N = (p.L + C - 1) / C;
+    if (p.BH > 65535 || p.N > 65535) return GLA_ERR_UNSUPPORTED;
+    return gla::simt_chunk_cumsum(p, log_a, Bcum, static_cast<cudaStream_t>(stream));
+}
+
+gla_status gla_check_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GLA_ERR_CUDA;
+    int* w = gla::device_error_word();
+    if (!w) return GLA_ERR_CUDA;
+    int h = 0;
+    if (cudaMemcpy(&h, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return GLA_ERR_CUDA;
+    if (h != 0) {
+        const int zero = 0;
+        if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return GLA_ERR_CUDA;
+        return GLA_ERR_TIMEOUT;
+    }
+    return GLA_OK;
+}
+
+uint64_t gla_launch_count(void) { return gla::g_launches.load(); }
+void gla_launch_count_reset(void) { gla::g_launches.store(0); }
+
+void gla_profile_enable(int on) {
+    std::lock_guard<std::mutex> lk(gla::g_mu);
+    gla::g_prof = on != 0;
+}
+
+int gla_profile_read(const char** names, uint64_t* launches, double* total_ms, int cap) {
+    std::lock_guard<std::mutex> lk(gla::g_mu);
+    gla::drain_locked();
+    const int n = int(gla::g_names.size());
+    for (int i = 0; i < n && i < cap; ++i) {
+        if (names) names[i] = gla::g_names[i];
+        if (launches) launches[i] = gla::g_counts[i];
+        if (total_ms) total_ms[i] = gla::g_ms[i];
+    }
+    return n;
+}
+
+void gla_profile_reset(void) {
+    std::lock_guard<std::mutex> lk(gla::g_mu);
+    gla::drain_locked();
+    for (cudaEvent_t e : gla::g_pool) cudaEventDestroy(e);
+    gla::g_pool.clear();
+    gla::g_names.clear();
+    gla::g_counts.clear();
+    gla::g_ms.clear();
+}
+
+}  // extern "C"

@@ -1,0 +1,83 @@
+// Internal host-side interface between the C ABI (gla_api.cu) and the kernel
+// files. Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/gla.h"
+
+namespace gla {
+
+// Resolved problem: the descriptor after defaults and checks.
+struct Problem {
+    int64_t B, H, L, K, V;
+    int64_t BH;      // B*H
+    int C;           // chunk length
+    int c;           // sub-chunk length
+    int64_t N;       // number of chunks, ceil(L / C)
+    bool bf16;       // element type of q, k, v, o, dO, dq, dk, dv
+    int impl;        // GLA_IMPL_SIMT or GLA_IMPL_TC (never AUTO)
+    int state_mode;  // never AUTO
+    int flags;
+};
+
+// Bump allocator over the caller's workspace; every slice is 256-B aligned.
+struct Arena {
+    char* base;
+    size_t cap;
+    size_t used;
+    template <typename T>
+    T* take(size_t count) {
+        size_t off = (used + 255) & ~size_t(255);
+        size_t bytes = count * sizeof(T);
+        used = off + bytes;
+        return base ? reinterpret_cast<T*>(base + off) : nullptr;
+    }
+};
+
+// ---- launch bookkeeping (gla_api.cu) ------------------------------------
+// Every kernel launch goes through launch_begin/launch_end so that the
+// launch counter and the optional per-kernel event timing see it.
+void launch_begin(const char* name, cudaStream_t s);
+gla_status launch_end(const char* name, cudaStream_t s);
+
+// Device-side error word (set by kernels whose bounded waits run out).
+int* device_error_word();
+
+// ---- SIMT path (gla_simt.cu) ---------------------------------------------
+size_t simt_fwd_workspace(const Problem& p);
+size_t simt_bwd_workspace(const Problem& p);
+gla_status simt_chunk_cumsum(const Problem& p, const float* log_a, float* Bc, cudaStream_t s);
+gla_status simt_fwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
+                    const float* h0, void* o, float* hT, Arena& ws, cudaStream_t s);
+gla_status simt_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
+                    const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
+                    float* dlog_a, float* dh0, Arena& ws, cudaStream_t s);
+
+// ---- decode step (gla_step.cu) ---------------------------------------------
+gla_status step_launch(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
+                       float* S, void* o, cudaStream_t s);
+
+// ---- tensor-core path (gla_tc_*.cu) -----------------------------------------
+bool tc_supported(const Problem& p);
+size_t tc_fwd_workspace(const Problem& p);
+size_t tc_bwd_workspace(const Problem& p);
+gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
+                  const float* h0, void* o, float* hT, Arena& ws, cudaStream_t s);
+gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
+                  const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
+                  float* dlog_a, float* dh0, Arena& ws, cudaStream_t s);
+
+}  // namespace gla
+
+// Launch helper: bracket a <<<>>> launch with the bookkeeping hooks and return
+// GLA_ERR_CUDA from the enclosing function if the launch failed.
+#define GLA_LAUNCH(name, kernel, grid, block, smem, stream, ...)                   \
+    do {                                                                           \
+        ::gla::launch_begin(name, stream);                                         \
+        kernel<<<(grid), (block), (smem), (stream)>>>(__VA_ARGS__);                \
+        gla_status _st = ::gla::launch_end(name, stream);                          \
+        if (_st != GLA_OK) return _st;                                             \
+    } while (0)

@@ -1,0 +1,184 @@
+/*
+ * gla.h -- C ABI of libgla: chunkwise gated linear attention (GLA) on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The layer ("Gated Linear Attention Transformers with Hardware-Efficient
+ * Training", atlas.scime.ai summary, section "Approach"): per batch b and
+ * head h, with a data-dependent gate G_t = alpha_t^T 1 (rank one, constant
+ * along the value dimension), i.e. a per-key-channel decay,
+ *
+ *     S_t = diag(alpha_t) S_{t-1} + k_t^T v_t,      o_t = q_t S_t,
+ *
+ * alpha_t = exp(log_a_t) in [0,1]^{Dk}, S_{-1} = h0, hT = S_{L-1}. The output
+ * reads the state after the update. There is no 1/sqrt(Dk) scale and no
+ * normaliser inside the layer.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * Layout: all tensors are dense, row-major, contiguous, on the device:
+ *     q, k, log_a, dq, dk, dlog_a : [B, H, L, Dk]
+ *     v, o, dO, dv                : [B, H, L, Dv]
+ *     h0, hT, dhT, dh0, S         : [B, H, Dk, Dv]   (always fp32)
+ * q, k, v, o, dO, dq, dk, dv have the element type `desc->dtype` (fp32 or
+ * bf16); log_a, dlog_a and all states are fp32. Every arithmetic step
+ * accumulates in fp32.
+ * Ownership: the caller allocates and frees every buffer, including the
+ * workspace. The library never allocates device memory, never frees, and
+ * never synchronises (except gla_check_device_error).
+ * Execution: work is enqueued on `stream` (a cudaStream_t; NULL = the legacy
+ * default stream) on the current device; calls return before the GPU is
+ * done. Outputs must not alias inputs (except S in gla_step, updated in
+ * place).
+ * Errors: argument checks run on the host before any launch and return a
+ * status; nothing is thrown across the ABI. A failed launch returns
+ * GLA_ERR_CUDA. Device-side conditions (a bounded wait that ran out) are
+ * recorded in a device flag that gla_check_device_error reports.
+ * Alignment: device pointers must be 16-byte aligned; the workspace 256-byte
+ * aligned.
+ */
+#ifndef GLA_H_
+#define GLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define GLA_ABI_VERSION 1
+
+typedef enum gla_status {
+    GLA_OK = 0,
+    GLA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size, bad enum   */
+    GLA_ERR_UNSUPPORTED = 2, /* valid request this build has no kernel for    */
+    GLA_ERR_WORKSPACE = 3,   /* workspace missing, too small or misaligned    */
+    GLA_ERR_CUDA = 4,        /* a CUDA runtime call or kernel launch failed   */
+    GLA_ERR_TIMEOUT = 5      /* a device-side bounded wait ran out            */
+} gla_status;
+
+typedef enum gla_dtype {
+    GLA_DTYPE_F32 = 0,
+    GLA_DTYPE_BF16 = 1
+} gla_dtype;
+
+/* How the inter-chunk states are handled ("Approach" section: "materialized
+ * or non-materialized inter-chunk states"). */
+typedef enum gla_state_mode {
+    GLA_STATE_AUTO = 0,            /* library picks                            */
+    GLA_STATE_MATERIALIZED = 1,    /* write S_[i] of every chunk to workspace  */
+    GLA_STATE_NONMATERIALIZED = 2  /* keep S on chip while walking the chunks  */
+} gla_state_mode;
+
+/* Which kernel family runs. */
+typedef enum gla_impl {
+    GLA_IMPL_AUTO = 0,  /* tensor-core path for bf16, CUDA-core path for fp32 */
+    GLA_IMPL_SIMT = 1,  /* fp32 CUDA-core kernels for every dtype              */
+    GLA_IMPL_TC = 2     /* bf16 tensor-core kernels (tcgen05/TMEM/TMA)         */
+} gla_impl;
+
+/* Problem descriptor. B, H, L >= 1; Dk, Dv >= 1 (each path states its own
+ * supported set and returns GLA_ERR_UNSUPPORTED outside it). chunk = 0 and
+ * subchunk = 0 pick defaults; otherwise chunk must be one of 16, 32, 64, 128
+ * and subchunk must divide chunk. The result does not depend on chunk or
+ * subchunk beyond rounding. */
+typedef struct gla_desc {
+    int64_t B, H, L, Dk, Dv;
+    int32_t dtype;      /* gla_dtype                                   */
+    int32_t chunk;      /* C, the chunk length (0 = default)           */
+    int32_t subchunk;   /* c, the secondary chunk length (0 = default) */
+    int32_t state_mode; /* gla_state_mode                              */
+    int32_t impl;       /* gla_impl                                    */
+    int32_t flags;      /* GLA_FLAG_* bits                             */
+} gla_desc;
+
+/* gla_bwd: the workspace still holds what gla_fwd left in it for the same
+ * inputs and descriptor, so the backward may reuse those intermediates
+ * instead of recomputing them. The caller guarantees that nothing wrote the
+ * workspace or the inputs in between. */
+#define GLA_FLAG_WS_FROM_FWD 0x1
+
+/* Workspace bytes gla_fwd / gla_bwd need for `d` (0 when `d` is invalid).
+ * A buffer of gla_bwd_workspace_size bytes also serves gla_fwd, so one
+ * workspace can be shared by a forward and the following backward. */
+size_t gla_fwd_workspace_size(const gla_desc* d);
+size_t gla_bwd_workspace_size(const gla_desc* d);
+
+/* Forward: o[B,H,L,Dv] and, if hT != NULL, hT[B,H,Dk,Dv] = S_{L-1}.
+ * h0 may be NULL (zero initial state).
+ * Method: per-chunk log-space gate cumsum, inter-chunk state walk and
+ * intra-chunk secondary chunking, the chunkwise form of the recurrence
+ * ("Approach": I/O-aware chunkwise algorithm, two-level chunking). */
+gla_status gla_fwd(const gla_desc* d, const void* q, const void* k, const void* v,
+                   const float* log_a, const float* h0, void* o, float* hT,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* Backward of L = <dO, o> + <dhT, hT>: dq, dk [B,H,L,Dk], dv [B,H,L,Dv]
+ * (dtype), dlog_a [B,H,L,Dk] (fp32), dh0 [B,H,Dk,Dv] (fp32, may be NULL).
+ * h0 and dhT may be NULL (zero). The gate gradient is the closed form
+ *   dlog_a_t = sum_{s>=t} (q_s*dq_s - k_s*dk_s) + sum_v dhT[:,v]*hT[:,v]
+ * ("Approach": "a closed-form gradient for the gates that avoids
+ * materializing per-step states"). dq, dk, dv are the full gradients. */
+gla_status gla_bwd(const gla_desc* d, const void* q, const void* k, const void* v,
+                   const float* log_a, const float* h0, const void* dO, const float* dhT,
+                   void* dq, void* dk, void* dv, float* dlog_a, float* dh0,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/* One recurrent decode step for B*H independent states (d->L is ignored):
+ * S <- diag(exp(log_a)) S + k^T v (in place), then o = q S.
+ * q, k, log_a: [B,H,Dk]; v, o: [B,H,Dv]; S: [B,H,Dk,Dv] fp32. The recurrent
+ * form of the layer (podcast.app episode page, summary: "a gated,
+ * recurrent-style memory update"). */
+gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void* v,
+                    const float* log_a, float* S, void* o, void* stream);
+
+/* Per-chunk inclusive log-space gate cumsum: for chunk i and row j,
+ * Bcum[t = iC + j] = sum_{r=0..j} log_a[iC + r] per key channel, restarting
+ * at every chunk boundary (C = the descriptor's chunk). In/out [B,H,L,Dk]
+ * fp32. This is the first stage of every chunkwise pass; it is exported so
+ * that it can be checked and timed on its own. */
+gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, void* stream);
+
+/* Blocks until `stream` is idle, then reports (and clears) the device-side
+ * error flag: GLA_ERR_TIMEOUT if a bounded wait ran out in any kernel since
+ * the last check, GLA_ERR_CUDA on a sticky CUDA error, else GLA_OK. */
+gla_status gla_check_device_error(void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* gla_status_string(gla_status s);
+
+/* GLA_ABI_VERSION of the loaded library. */
+int gla_abi_version(void);
+
+/* Chunk and sub-chunk lengths gla_fwd/gla_bwd use for `d` after defaults
+ * are applied, and the kernel family (gla_impl) it resolves to; returns
+ * GLA_ERR_INVALID_ARG / GLA_ERR_UNSUPPORTED like the compute calls would. */
+gla_status gla_resolve(const gla_desc* d, int32_t* chunk, int32_t* subchunk,
+                       int32_t* impl, int32_t* state_mode);
+
+/* ---- measurement hooks (host-side counters; off the math path) ---------- */
+
+/* Number of kernels this library has launched since load (or the last
+ * reset). */
+uint64_t gla_launch_count(void);
+void gla_launch_count_reset(void);
+
+/* When enabled (on != 0), every kernel launch is bracketed by a pair of CUDA
+ * events recorded on the launching stream, so per-kernel device time can be
+ * read back with gla_profile_read. Events are created lazily on the first
+ * enabled launch (this is the only place the library creates CUDA objects)
+ * and destroyed by gla_profile_reset. */
+void gla_profile_enable(int on);
+
+/* Synchronises the recorded events and writes, for up to `cap` kernel
+ * names, the name (pointer to a static string), the number of launches and
+ * the summed device milliseconds. Returns the number of distinct kernels
+ * (which may exceed cap). */
+int gla_profile_read(const char** names, uint64_t* launches, double* total_ms, int cap);
+void gla_profile_reset(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLA_H_ */

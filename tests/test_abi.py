@@ -1,0 +1,106 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/gla.h declares, and rejects bad arguments on the host before any
+launch."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from chunkwise_linear_rnn_gla_b200 import build as gbuild
+from chunkwise_linear_rnn_gla_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    gbuild.build()
+    return _lib.load()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "gla.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gla_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_and_binding_agree():
+    assert sorted(_lib.EXPORTS) == declared_functions()
+
+
+def test_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_abi_version(lib):
+    assert lib.gla_abi_version() == 1
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert len(lib.gla_status_string(s)) > 0
+    assert lib.gla_status_string(99) == b"unknown status"
+
+
+def desc(**kw):
+    d = dict(B=1, H=1, L=64, Dk=64, Dv=64, dtype=0, chunk=0, subchunk=0, state_mode=0, impl=0, flags=0)
+    d.update(kw)
+    return _lib.GlaDesc(**d)
+
+
+def test_resolve_defaults(lib):
+    c, sc, im, sm = (ctypes.c_int32() for _ in range(4))
+    assert lib.gla_resolve(ctypes.byref(desc(dtype=0)), ctypes.byref(c), ctypes.byref(sc), ctypes.byref(im),
+                           ctypes.byref(sm)) == 0
+    assert (c.value, im.value) == (64, 1)  # fp32 -> CUDA-core path, chunk 64
+
+
+@pytest.mark.parametrize("bad", [dict(B=0), dict(L=0), dict(Dk=0), dict(dtype=7), dict(chunk=48), dict(chunk=-1),
+                                 dict(state_mode=9), dict(impl=5), dict(flags=0x100), dict(chunk=16, subchunk=32),
+                                 dict(chunk=64, subchunk=24, impl=1)])
+def test_bad_descriptor_rejected(lib, bad):
+    d = desc(**bad)
+    assert lib.gla_fwd_workspace_size(ctypes.byref(d)) == 0
+    st = lib.gla_fwd(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, None, 0, None)
+    assert st == 1  # GLA_ERR_INVALID_ARG
+
+
+def test_null_desc(lib):
+    assert lib.gla_fwd(None, 16, 16, 16, 16, None, 16, None, None, 0, None) == 1
+    assert lib.gla_step(None, 16, 16, 16, 16, 16, 16, None) == 1
+    assert lib.gla_fwd_workspace_size(None) == 0
+
+
+def test_null_and_misaligned_pointers(lib):
+    d = desc()
+    # null q
+    assert lib.gla_fwd(ctypes.byref(d), None, 16, 16, 16, None, 16, None, None, 0, None) == 1
+    # misaligned k
+    assert lib.gla_fwd(ctypes.byref(d), 16, 18, 16, 16, None, 16, None, None, 0, None) == 1
+    # misaligned optional h0
+    assert lib.gla_fwd(ctypes.byref(d), 16, 16, 16, 16, 24, 16, None, None, 0, None) == 1
+    # backward: null dlog_a
+    assert lib.gla_bwd(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, 16, 16, 16, None, None, None, 0, None) == 1
+
+
+def test_workspace_checks(lib):
+    d = desc()
+    need = lib.gla_fwd_workspace_size(ctypes.byref(d))
+    assert need > 0
+    assert lib.gla_bwd_workspace_size(ctypes.byref(d)) >= need
+    # missing workspace, too small, misaligned: all GLA_ERR_WORKSPACE before any launch
+    assert lib.gla_fwd(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, None, 0, None) == 3
+    assert lib.gla_fwd(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, 256, need - 1, None) == 3
+    assert lib.gla_fwd(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, 272, need, None) == 3
+
+
+def test_simt_rejects_nonmaterialized(lib):
+    d = desc(impl=1, state_mode=2)
+    assert lib.gla_fwd(ctypes.byref(d), 16, 16, 16, 16, None, 16, None, 256, 1 << 30, None) == 2
+
+
+def test_launch_counter_host_only(lib):
+    lib.gla_launch_count_reset()
+    assert lib.gla_launch_count() == 0

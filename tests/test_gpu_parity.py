@@ -1,0 +1,221 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 oracle, on the
+same seeded inputs, element by element.
+
+Small cases run every output of every head through the oracle; the full-size
+workloads (in the launch configuration the benchmark times) compare sampled
+heads -- all of L, Dk and Dv of each sampled head, which the oracle computes
+exactly since heads are independent.
+"""
+import numpy as np
+import pytest
+import torch
+
+import chunkwise_linear_rnn_gla_b200 as gla
+from chunkwise_linear_rnn_gla_b200 import build as gbuild
+from chunkwise_linear_rnn_gla_b200.inputs import WORKLOADS, make_inputs, make_step_inputs, to_f64_numpy
+from tests.parity import compare, heads, oracle_bwd, oracle_fwd, to_dev
+
+pytestmark = pytest.mark.gpu
+
+IMPLS = ["simt"]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    gbuild.build()
+    gla.load()
+
+
+def run_fwd(d, impl="auto", **kw):
+    o, hT = gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], d.get("h0"), impl=impl, **kw)
+    torch.cuda.synchronize()
+    return o, hT
+
+
+def run_bwd(d, impl="auto", **kw):
+    g = gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d.get("h0"), d.get("dhT"), impl=impl, **kw)
+    torch.cuda.synchronize()
+    return g
+
+
+def check_fwd(inp, dtype, impl, idx=None, **kw):
+    d = to_dev(inp)
+    o, hT = run_fwd(d, impl, **kw)
+    o_ref, hT_ref = oracle_fwd(inp, idx)
+    if idx is not None:
+        o, hT = heads(o, idx), heads(hT, idx)
+    compare("o", o, o_ref, dtype)
+    compare("hT", hT, hT_ref, dtype)
+
+
+def check_bwd(inp, dtype, impl, idx=None, **kw):
+    d = to_dev(inp)
+    g = run_bwd(d, impl, **kw)
+    ref = oracle_bwd(inp, idx)
+    for name in ("dq", "dk", "dv", "dlog_a", "dh0"):
+        val = g[name] if idx is None else heads(g[name], idx)
+        compare(name, val, ref[name], dtype)
+
+
+# ------------------------------------------------------------ small, all heads
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("L", [1, 63, 64, 65, 200])
+def test_small_shapes(impl, dtype, L):
+    inp = make_inputs(2, 2, L, 64, 64, dtype, seed=L, h0=True, dhT=True)
+    check_fwd(inp, dtype, impl)
+    check_bwd(inp, dtype, impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("chunk", [16, 32, 64, 128])
+def test_chunk_size_invariance(impl, chunk):
+    inp = make_inputs(1, 2, 300, 64, 128, "f32", seed=5, h0=True, dhT=True)
+    check_fwd(inp, "f32", impl, chunk=chunk)
+    check_bwd(inp, "f32", impl, chunk=chunk)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("KV", [(32, 48), (128, 256), (96, 64)])
+def test_head_dims(impl, KV):
+    K, V = KV
+    inp = make_inputs(1, 3, 130, K, V, "bf16", seed=K + V, h0=True, dhT=True)
+    check_fwd(inp, "bf16", impl)
+    check_bwd(inp, "bf16", impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_zero_and_unit_gates(impl):
+    inp = make_inputs(1, 2, 150, 64, 64, "f32", seed=11, h0=True, dhT=True)
+    la = inp["log_a"].clone()
+    la[:, 0] = -1e30  # head 0: alpha = 0 exactly
+    la[:, 1] = 0.0  # head 1: alpha = 1 (no decay)
+    inp["log_a"] = la
+    check_fwd(inp, "f32", impl)
+    check_bwd(inp, "f32", impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_strong_mixed_gates(impl):
+    # gates down to ~e^-5 per step: exercises the non-overflow guarantee
+    inp = make_inputs(1, 2, 256, 64, 64, "bf16", seed=12, h0=True, dhT=True, gate_scale=1.0)
+    check_fwd(inp, "bf16", impl)
+    check_bwd(inp, "bf16", impl)
+
+
+def test_ws_reuse_matches_recompute():
+    inp = make_inputs(2, 2, 200, 64, 64, "f32", seed=13, h0=True, dhT=True)
+    d = to_dev(inp)
+    desc = gla.make_desc(2, 2, 200, 64, 64, "f32")
+    ws = torch.empty(gla.gla_bwd_workspace_size(desc), dtype=torch.uint8, device="cuda")
+    gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], d["h0"], workspace=ws)
+    g1 = gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d["h0"], d["dhT"], workspace=ws, ws_from_fwd=True)
+    g2 = gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d["h0"], d["dhT"])
+    torch.cuda.synchronize()
+    for key in g1:
+        assert torch.equal(g1[key], g2[key]), key
+
+
+def test_chunk_cumsum_kernel():
+    inp = make_inputs(2, 3, 333, 80, 8, "f32", seed=14, with_grad=False)
+    la = inp["log_a"].cuda()
+    for C in (16, 64, 128):
+        out = gla.gla_chunk_cumsum(la, chunk=C)
+        torch.cuda.synchronize()
+        ref = np.zeros(la.shape)
+        x = to_f64_numpy(inp["log_a"])
+        for i0 in range(0, 333, C):
+            ref[:, :, i0:i0 + C] = np.cumsum(x[:, :, i0:i0 + C], axis=2)
+        np.testing.assert_allclose(to_f64_numpy(out), ref, rtol=0, atol=1e-5)
+
+
+# ------------------------------------------------------------- decode step
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_matches_oracle(dtype):
+    import oracle
+
+    B, H, K, V, T = 4, 2, 64, 96, 20
+    st = make_step_inputs(B, H, K, V, T, dtype, seed=15)
+    S = torch.randn(B, H, K, V, generator=torch.Generator().manual_seed(1)) * 0.1
+    S_ref = S.double().numpy()
+    Sd = S.cuda()
+    for t in range(T):
+        o = gla.gla_step(st["q"][t].cuda(), st["k"][t].cuda(), st["v"][t].cuda(), st["log_a"][t].cuda(), Sd)
+        o_ref, S_ref = oracle.step(to_f64_numpy(st["q"][t]), to_f64_numpy(st["k"][t]), to_f64_numpy(st["v"][t]),
+                                   to_f64_numpy(st["log_a"][t]), S_ref)
+        torch.cuda.synchronize()
+        compare("o_%d" % t, o, o_ref, dtype)
+    compare("S", Sd, S_ref, "f32" if dtype == "f32" else "bf16")
+
+
+def test_step_iterated_equals_fwd():
+    B, H, L, K, V = 2, 2, 70, 64, 64
+    inp = make_inputs(B, H, L, K, V, "f32", seed=16, h0=True)
+    d = to_dev(inp)
+    o, hT = run_fwd(d)
+    S = d["h0"].clone()
+    outs = []
+    for t in range(L):
+        outs.append(gla.gla_step(d["q"][:, :, t].contiguous(), d["k"][:, :, t].contiguous(),
+                                 d["v"][:, :, t].contiguous(), d["log_a"][:, :, t].contiguous(), S))
+    torch.cuda.synchronize()
+    torch.testing.assert_close(torch.stack(outs, 2), o, atol=1e-4, rtol=0)
+    torch.testing.assert_close(S, hT, atol=1e-4, rtol=0)
+
+
+def test_decode_workload_sampled():
+    """Decode workload shape (B=64, H=4, Dk=128, Dv=256, fp32 state): 16 steps,
+    every head against the oracle."""
+    import oracle
+
+    B, H, K, V, T = 64, 4, 128, 256, 16
+    st = make_step_inputs(B, H, K, V, T, "bf16", seed=17)
+    Sd = torch.zeros(B, H, K, V, device="cuda")
+    S_ref = np.zeros((B, H, K, V))
+    for t in range(T):
+        o = gla.gla_step(st["q"][t].cuda(), st["k"][t].cuda(), st["v"][t].cuda(), st["log_a"][t].cuda(), Sd)
+        o_ref, S_ref = oracle.step(to_f64_numpy(st["q"][t]), to_f64_numpy(st["k"][t]), to_f64_numpy(st["v"][t]),
+                                   to_f64_numpy(st["log_a"][t]), S_ref)
+    torch.cuda.synchronize()
+    compare("o_last", o, o_ref, "bf16")
+    compare("S", Sd, S_ref, "bf16")
+
+
+# ------------------------------------------------------- the named workloads
+def test_workload_tiny_f32():
+    w = WORKLOADS["tiny_f32"]
+    inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=0)
+    check_fwd(inp, "f32", "auto", chunk=w.chunk)
+    check_bwd(inp, "f32", "auto", chunk=w.chunk)
+
+
+def test_workload_340m_fwd():
+    w = WORKLOADS["gla340m_fwd"]
+    inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=0, with_grad=False)
+    check_fwd(inp, "bf16", "auto", idx=[0, 13, w.B * w.H - 1])
+
+
+def test_workload_1p3b_fwdbwd():
+    w = WORKLOADS["gla1p3b_fwdbwd"]
+    inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=0)
+    idx = [0, w.B * w.H - 1]
+    check_fwd(inp, "bf16", "auto", idx=idx)
+    check_bwd(inp, "bf16", "auto", idx=idx)
+
+
+@pytest.mark.parametrize("mode", ["materialized"])
+def test_workload_long16k(mode):
+    w = WORKLOADS["long16k"]
+    inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=0, z_mean=w.z_mean)
+    idx = [1]
+    check_fwd(inp, "bf16", "auto", idx=idx, state_mode=mode)
+    check_bwd(inp, "bf16", "auto", idx=idx, state_mode=mode)
+
+
+@pytest.mark.parametrize("L", [1024, 4096, 16384])
+def test_workload_sweep(L):
+    w = WORKLOADS["sweep_L%d" % L]
+    inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=0)
+    idx = [w.B * w.H - 1]
+    check_fwd(inp, "bf16", "auto", idx=idx)
+    check_bwd(inp, "bf16", "auto", idx=idx)
