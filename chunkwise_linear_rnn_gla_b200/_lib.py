@@ -23,7 +23,7 @@ FLAG_WS_FROM_FWD = 0x1
 EXPORTS = (
     "gla_fwd_workspace_size", "gla_bwd_workspace_size", "gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum",
     "gla_check_device_error", "gla_status_string", "gla_abi_version", "gla_resolve", "gla_launch_count",
-    "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset",
+    "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset", "gla_fwd_noalloc",
 )
 
 
@@ -75,6 +75,8 @@ def _declare(lib):
                                      ctypes.POINTER(ctypes.c_double), ctypes.c_int]
     lib.gla_profile_read.restype = ctypes.c_int
     lib.gla_profile_reset.restype = None
+    lib.gla_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
+    lib.gla_fwd_noalloc.restype = ctypes.c_int
 
 
 def load(path: str = LIB_PATH):

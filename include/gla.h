@@ -139,6 +139,34 @@ gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void*
  * that it can be checked and timed on its own. */
 gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, void* stream);
 
+/* ---- forward without any allocation ---------------------------------------
+ * The paper has no counterpart to this entry point; it exists for callers
+ * that cannot allocate device memory or provide a workspace: a plugin under
+ * a framework or server that owns every device allocation, a latency-critical
+ * loop that must not risk the implicit synchronisation of cudaMalloc/cudaFree,
+ * or a C caller with no device memory manager.
+ *
+ * gla_fwd_noalloc computes exactly what gla_fwd computes (same arguments,
+ * same layouts; the CUDA-core kernel path, chosen whatever d->impl says
+ * except that GLA_IMPL_TC or GLA_STATE_NONMATERIALIZED return
+ * GLA_ERR_UNSUPPORTED), but takes its scratch from a fixed array of
+ * GLA_NOALLOC_SCRATCH_BYTES bytes built into the library; it calls no
+ * cudaMalloc, cudaFree or other allocating routine.
+ *  - Every GPU that loads the library's kernels holds that array until the
+ *    process exits.
+ *  - A problem whose gla_fwd_workspace_size (with impl = GLA_IMPL_SIMT)
+ *    exceeds GLA_NOALLOC_SCRATCH_BYTES is rejected with GLA_ERR_WORKSPACE
+ *    before any launch.
+ *  - All calls on one device share the array and it keeps the last call's
+ *    contents; nothing in it needs clearing, but calls that overlap on the
+ *    GPU (other streams or host threads) race and must be serialised.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current): make that first call
+ *    before any stream capture begins. */
+#define GLA_NOALLOC_SCRATCH_BYTES (16u << 20)
+gla_status gla_fwd_noalloc(const gla_desc* d, const void* q, const void* k, const void* v,
+                           const float* log_a, const float* h0, void* o, float* hT, void* stream);
+
 /* Blocks until `stream` is idle, then reports (and clears) the device-side
  * error flag: GLA_ERR_TIMEOUT if a bounded wait ran out in any kernel since
  * the last check, GLA_ERR_CUDA on a sticky CUDA error, else GLA_OK. */
