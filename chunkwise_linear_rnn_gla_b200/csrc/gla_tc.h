@@ -1,0 +1,49 @@
+// Internal declarations of the tensor-core (tcgen05 / TMEM / TMA) path.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "gla_internal.h"
+#include "tc_prims.cuh"
+
+namespace gla {
+
+__device__ __forceinline__ uint32_t tc_smem_u32(const void* p) { return tc::smem_u32(p); }
+
+constexpr int kTcChunk = 128;  // C on the tensor-core path
+constexpr int kTcSub = 16;     // secondary chunk c
+constexpr int kTcBV = 64;      // value columns per walk CTA
+
+// Chunk-parallel gate preparation (gla_tc_prep.cu).
+size_t tc_prep_smem_bytes();
+gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const float* la, __nv_bfloat16* Qt,
+                          __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, float* Bout, cudaStream_t s);
+
+// Row-gated chunk walk (gla_tc_walk.cu). State X [K x 64-column tile] with the
+// gate on its rows. Per chunk i (in walk order):
+//   Y_i = A2_i X + Pm_i B1_i          (fused / output-only modes)
+//   X  <- diag(gam_i) X + A1_i^T B1_i  (fused / states-only modes)
+// Forward: A1 = K~, B1 = v, A2 = Q~, Pm = P, forward order, Y = o, X0 = h0.
+// dv:      A1 = Q~, B1 = dO, A2 = K~, Pm = P^T, reverse order, Y = dv, X0 = dhT.
+enum WalkMode : int { kWalkFused = 0, kWalkStatesOnly = 1, kWalkOutputOnly = 2 };
+
+struct WalkArgs {
+    const __nv_bfloat16* A1;  // [BH][L][K]
+    const __nv_bfloat16* B1;  // [BH][L][V]
+    const __nv_bfloat16* A2;  // [BH][L][K]
+    const __nv_bfloat16* Pm;  // [BH][N][128][128]
+    const float* gam;         // [BH][N][K]
+    const float* init;        // [BH][K][V] or null
+    float* fin;               // [BH][K][V] or null
+    __nv_bfloat16* Y;         // [BH][L][V]
+    __nv_bfloat16* states;    // [BH][N][K][V] (states-only: written; output-only: read)
+    int mode;
+    bool reverse;
+    bool p_transposed;
+};
+
+gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, const char* name);
+
+}  // namespace gla

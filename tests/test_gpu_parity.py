@@ -219,3 +219,38 @@ def test_workload_sweep(L):
     idx = [w.B * w.H - 1]
     check_fwd(inp, "bf16", "auto", idx=idx)
     check_bwd(inp, "bf16", "auto", idx=idx)
+
+
+# ------------------------------------------------ tensor-core forward path
+TC_SHAPES = [(1, 2, 1, 128, 64), (1, 2, 100, 128, 128), (2, 1, 128, 256, 64), (1, 2, 129, 128, 256),
+             (1, 1, 300, 256, 128), (2, 2, 512, 128, 64)]
+
+
+@pytest.mark.parametrize("mode", ["nonmaterialized", "materialized"])
+@pytest.mark.parametrize("shape", TC_SHAPES)
+def test_tc_forward(mode, shape):
+    B, H, L, K, V = shape
+    inp = make_inputs(B, H, L, K, V, "bf16", seed=L + K + V, h0=True, with_grad=False)
+    check_fwd(inp, "bf16", "tc", state_mode=mode)
+
+
+@pytest.mark.parametrize("mode", ["nonmaterialized", "materialized"])
+def test_tc_forward_extreme_gates(mode):
+    # head 0: alpha = 0 exactly; head 1: alpha = 1; head 2: strong decays (up to
+    # ~e^-6 per step, so sub-chunk spans exceed the factored fp32 range)
+    inp = make_inputs(1, 3, 260, 128, 64, "bf16", seed=21, h0=True, with_grad=False, gate_scale=1.0)
+    la = inp["log_a"].clone()
+    la[:, 0] = -1e30
+    la[:, 1] = 0.0
+    la[:, 2] = la[:, 2] * 3.0
+    inp["log_a"] = la
+    check_fwd(inp, "bf16", "tc", state_mode=mode)
+
+
+def test_tc_matches_simt_forward():
+    inp = make_inputs(2, 2, 700, 256, 128, "bf16", seed=22, h0=True, with_grad=False)
+    d = to_dev(inp)
+    o_tc, hT_tc = run_fwd(d, "tc")
+    o_s, hT_s = run_fwd(d, "simt")
+    compare("o tc-vs-simt", o_tc, to_f64_numpy(o_s), "bf16")
+    compare("hT tc-vs-simt", hT_tc, to_f64_numpy(hT_s), "bf16")
