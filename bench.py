@@ -82,6 +82,23 @@ def kernel_models(w, C):
                         bound="alu")
     m["simt_dlog_a"] = dict(bytes=th * K * 8, flops=th * K, bound="hbm")
     m["step"] = dict(bytes=2 * st, flops=4 * BH * K * V, bound="hbm")
+    # tensor-core path (bf16 operands, fp32 accumulate); C = 128
+    sb = BH * N * K * V * e  # one set of bf16 chunk states
+    pb = BH * N * C * C * e  # intra-chunk score matrices
+    m["tc_prep"] = dict(bytes=th * (2 * K * e + 4 * K + 2 * K * e) + pb + BH * N * K * 4,
+                        flops=th * C * K, bound="hbm")
+    m["tc_walk_states"] = dict(bytes=th * (K * e + V * e) + sb, flops=th * 2 * K * V, bound="hbm")
+    m["tc_walk_dstates"] = dict(bytes=th * (K * e + V * e) + sb, flops=th * 2 * K * V, bound="hbm")
+    m["tc_output"] = dict(bytes=th * (K * e + 2 * V * e) + pb + sb, flops=th * 2 * (K * V + C * V), bound="hbm")
+    m["tc_output_dv"] = dict(bytes=th * (K * e + 2 * V * e) + pb + sb, flops=th * 2 * (K * V + C * V), bound="hbm")
+    m["tc_walk_fwd"] = dict(bytes=th * (2 * K * e + 2 * V * e) + pb + 2 * st, flops=th * 2 * (2 * K * V + C * V),
+                            bound="hbm")
+    m["tc_walk_dv"] = dict(bytes=th * (2 * K * e + 2 * V * e) + pb + 2 * st, flops=th * 2 * (2 * K * V + C * V),
+                           bound="hbm")
+    m["tc_bwd_gemm"] = dict(bytes=th * (2 * V * e + 2 * K * e) + 2 * sb + pb, flops=th * 2 * (C * V + 2 * K * V),
+                            bound="hbm")
+    m["tc_bwd_intra"] = dict(bytes=th * (2 * K * e + 4 * K + 2 * K * e + 2 * K * e + 4 * K) + pb + 2 * sb,
+                             flops=th * 2 * C * K, bound="hbm")
     return m
 
 

@@ -37,13 +37,25 @@ struct WalkArgs {
     const float* gam;         // [BH][N][K]
     const float* init;        // [BH][K][V] or null
     float* fin;               // [BH][K][V] or null
+    float* fin2;              // second copy of the final state, or null
     __nv_bfloat16* Y;         // [BH][L][V]
-    __nv_bfloat16* states;    // [BH][N][K][V] (states-only: written; output-only: read)
+    __nv_bfloat16* states;    // [BH][N][K][V] bf16 state entering each chunk (written by
+                              // states-only mode and, when non-null, by fused mode; read by
+                              // output-only mode)
     int mode;
     bool reverse;
     bool p_transposed;
 };
 
 gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, const char* name);
+
+// Backward, chunk-parallel part (gla_tc_bwd.cu).
+gla_status tc_bwd_gemm_launch(const Problem& p, const void* dO, const void* v, const __nv_bfloat16* Sbuf,
+                              const __nv_bfloat16* Dbuf, __nv_bfloat16* dP, __nv_bfloat16* dQt, __nv_bfloat16* dKt,
+                              cudaStream_t s);
+gla_status tc_bwd_intra_launch(const Problem& p, const void* q, const void* k, const float* la,
+                               const __nv_bfloat16* dP, const __nv_bfloat16* dQt, const __nv_bfloat16* dKt,
+                               const __nv_bfloat16* Sbuf, const __nv_bfloat16* Dbuf, const float* hT,
+                               const float* dhT, void* dq, void* dk, float* dla, cudaStream_t s);
 
 }  // namespace gla

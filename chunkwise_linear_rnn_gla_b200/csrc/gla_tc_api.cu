@@ -1,13 +1,20 @@
-// Tensor-core path: support check, workspace layout and the kernel sequence
-// of the forward (and, for now, the backward).
+// Tensor-core path: support check, workspace layout and kernel sequences.
 //
 // Forward, non-materialised states (default):
-//   tc_prep  (chunk-parallel)  cumsum, Q~, K~, e^Gamma, intra-chunk P
-//   tc_walk  (fused)           per (head, 64-column tile): state walk on chip
-//                               and o = Q~ S + P v
+//   tc_prep      (chunk-parallel)  cumsum, Q~, K~, e^Gamma, intra-chunk P
+//   tc_walk_fwd  (per head and 64 value columns) state walk kept on chip,
+//                o = Q~ S + P v
 // Forward, materialised states:
-//   tc_prep, tc_walk (states only: writes S_[i] in bf16 to the workspace),
-//   tc_output (chunk-parallel: o = Q~ S_[i] + P v from the stored states)
+//   tc_prep, tc_walk_states (writes S_[i] in bf16), tc_output (chunk-parallel
+//   o = Q~ S_[i] + P v from the stored states)
+// Backward:
+//   [tc_prep]          unless the forward's workspace is reused
+//   [tc_walk_states]   unless the reused forward materialised its states
+//   tc_walk_dv         reverse walk: D_i chain, dv = K~ D_i + P^T dO, writes D_i
+//                      (materialised mode: tc_walk_dstates writes D_i, then the
+//                      chunk-parallel tc_output_dv computes dv)
+//   tc_bwd_gemm        dP = dO v^T, dQ~ = dO S_[i]^T, dK~ = v D_i^T (tcgen05)
+//   tc_bwd_intra       intra-chunk gradients, dq, dk, closed-form dlog a
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -21,17 +28,28 @@ namespace {
 
 struct TcBuffers {
     __nv_bfloat16 *Qt, *Kt, *P;
-    float* gam;
+    float *gam, *hT;
     __nv_bfloat16* states;
+    __nv_bfloat16 *Dbuf, *dP, *dQt, *dKt;
 };
 
-TcBuffers carve_fwd(const Problem& p, Arena& a) {
+// The backward layout extends the forward's, so a forward workspace can be
+// handed to the backward unchanged.
+TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
     TcBuffers b{};
     b.Qt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
     b.Kt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
     b.P = a.take<__nv_bfloat16>(size_t(p.BH * p.N * kTcChunk * kTcChunk));
     b.gam = a.take<float>(size_t(p.BH * p.N * p.K));
-    if (p.state_mode == GLA_STATE_MATERIALIZED) b.states = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
+    b.hT = a.take<float>(size_t(p.BH * p.K * p.V));
+    if (bwd || p.state_mode == GLA_STATE_MATERIALIZED)
+        b.states = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
+    if (bwd) {
+        b.Dbuf = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
+        b.dP = a.take<__nv_bfloat16>(size_t(p.BH * p.N * kTcChunk * kTcChunk));
+        b.dQt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
+        b.dKt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
+    }
     return b;
 }
 
@@ -49,24 +67,19 @@ bool tc_supported(const Problem& p) {
 
 size_t tc_fwd_workspace(const Problem& p) {
     Arena a{nullptr, 0, 0};
-    carve_fwd(p, a);
+    carve(p, a, false);
     return a.used;
 }
 
 size_t tc_bwd_workspace(const Problem& p) {
-    // interim: the backward runs the CUDA-core kernels after the forward's buffers
     Arena a{nullptr, 0, 0};
-    carve_fwd(p, a);
-    Problem ps = p;
-    ps.C = 64;
-    ps.c = 64;
-    ps.N = (p.L + 63) / 64;
-    return a.used + 256 + simt_bwd_workspace(ps);
+    carve(p, a, true);
+    return a.used;
 }
 
 gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v, const float* la, const float* h0,
                   void* o, float* hT, Arena& ws, cudaStream_t s) {
-    TcBuffers b = carve_fwd(p, ws);
+    TcBuffers b = carve(p, ws, false);
     if (ws.used > ws.cap) return GLA_ERR_WORKSPACE;
     gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, nullptr, s);
     if (st != GLA_OK) return st;
@@ -78,9 +91,8 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
     a.gam = b.gam;
     a.init = h0;
     a.fin = hT;
+    a.fin2 = b.hT;
     a.Y = static_cast<__nv_bfloat16*>(o);
-    a.reverse = false;
-    a.p_transposed = false;
     if (p.state_mode == GLA_STATE_NONMATERIALIZED) {
         a.mode = kWalkFused;
         return tc_walk_launch(p, a, s, "tc_walk_fwd");
@@ -90,26 +102,66 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
     st = tc_walk_launch(p, a, s, "tc_walk_states");
     if (st != GLA_OK) return st;
     a.mode = kWalkOutputOnly;
-    a.fin = nullptr;
+    a.fin = a.fin2 = nullptr;
     return tc_walk_launch(p, a, s, "tc_output");
 }
 
 gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* la, const float* h0,
                   const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dla, float* dh0, Arena& ws,
                   cudaStream_t s) {
-    // interim: CUDA-core backward (recomputes its own intermediates)
-    Arena a{nullptr, 0, 0};
-    carve_fwd(p, a);
-    Problem ps = p;
-    ps.impl = GLA_IMPL_SIMT;
-    ps.C = 64;
-    ps.c = 64;
-    ps.N = (p.L + 63) / 64;
-    ps.state_mode = GLA_STATE_MATERIALIZED;
-    ps.flags = 0;
-    const size_t off = (a.used + 255) & ~size_t(255);
-    Arena rest{ws.base + off, ws.cap > off ? ws.cap - off : 0, 0};
-    return simt_bwd(ps, q, k, v, la, h0, dO, dhT, dq, dk, dv, dla, dh0, rest, s);
+    TcBuffers b = carve(p, ws, true);
+    if (ws.used > ws.cap) return GLA_ERR_WORKSPACE;
+    const bool reuse = (p.flags & GLA_FLAG_WS_FROM_FWD) != 0;
+    gla_status st;
+    if (!reuse) {
+        st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, nullptr, s);
+        if (st != GLA_OK) return st;
+    }
+    if (!(reuse && p.state_mode == GLA_STATE_MATERIALIZED)) {
+        WalkArgs a{};
+        a.A1 = b.Kt;
+        a.B1 = static_cast<const __nv_bfloat16*>(v);
+        a.gam = b.gam;
+        a.init = h0;
+        a.fin = b.hT;
+        a.states = b.states;
+        a.mode = kWalkStatesOnly;
+        st = tc_walk_launch(p, a, s, "tc_walk_states");
+        if (st != GLA_OK) return st;
+    }
+    {
+        // D_i chain (reverse) and dv = K~ D_i + P^T dO
+        WalkArgs a{};
+        a.A1 = b.Qt;
+        a.B1 = static_cast<const __nv_bfloat16*>(dO);
+        a.A2 = b.Kt;
+        a.Pm = b.P;
+        a.gam = b.gam;
+        a.init = dhT;
+        a.fin = dh0;
+        a.Y = static_cast<__nv_bfloat16*>(dv);
+        a.states = b.Dbuf;
+        a.reverse = true;
+        if (p.state_mode == GLA_STATE_NONMATERIALIZED) {
+            a.mode = kWalkFused;
+            a.p_transposed = true;
+            st = tc_walk_launch(p, a, s, "tc_walk_dv");
+            if (st != GLA_OK) return st;
+        } else {
+            a.mode = kWalkStatesOnly;
+            st = tc_walk_launch(p, a, s, "tc_walk_dstates");
+            if (st != GLA_OK) return st;
+            a.mode = kWalkOutputOnly;
+            a.reverse = false;
+            a.p_transposed = true;
+            a.fin = nullptr;
+            st = tc_walk_launch(p, a, s, "tc_output_dv");
+            if (st != GLA_OK) return st;
+        }
+    }
+    st = tc_bwd_gemm_launch(p, dO, v, b.states, b.Dbuf, b.dP, b.dQt, b.dKt, s);
+    if (st != GLA_OK) return st;
+    return tc_bwd_intra_launch(p, q, k, la, b.dP, b.dQt, b.dKt, b.states, b.Dbuf, b.hT, dhT, dq, dk, dla, s);
 }
 
 }  // namespace gla

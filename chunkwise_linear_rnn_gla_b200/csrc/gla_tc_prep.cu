@@ -67,7 +67,25 @@ __device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float s0, float s1)
 // Pair index of (I, J), J < I, in [0, 28).
 __host__ __device__ constexpr int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }
 
+// cp.async 16-byte copy with zero fill when `valid` is false
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
+    const uint32_t n = valid ? 16u : 0u;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(tc_smem_u32(dst)), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+struct Stage {  // raw inputs of one channel tile, filled by cp.async
+    float la[C][KT];
+    __nv_bfloat16 q[C][KT];
+    __nv_bfloat16 k[C][KT];
+};
+
 struct PrepSmem {
+    Stage st[2];
+    __nv_bfloat16 qo[C][KT];  // Q~ / K~ tiles staged for coalesced stores
+    __nv_bfloat16 ko[C][KT];
     float B[C][KT];
     float qf[C][KT + 1];
     float kf[C][KT + 1];
@@ -107,8 +125,35 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
         for (int b = 0; b < 4; ++b) dg[a][b] = 0.f;
     const int I = warp;
     const int jr0 = 2 * (lane >> 2), s0 = 4 * (lane & 3);
+    // async copy of channel tile [c0, c0+KT) into stage buffer `sb`
+    auto issue = [&](int64_t c0, int sb) {
+        Stage& S = sm.st[sb];
+        for (int e = tid; e < C * (KT / 4); e += 256) {  // log a: 8 x 16 B per row
+            const int row = e / (KT / 4), cc = (e % (KT / 4)) * 4;
+            const bool ok = row < nvalid;
+            cp_async16(&S.la[row][cc], la + (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc, ok);
+        }
+        for (int e = tid; e < C * (KT / 8); e += 256) {  // q, k: 4 x 16 B per row
+            const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
+            const bool ok = row < nvalid;
+            const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc;
+            cp_async16(&S.q[row][cc], q + off, ok);
+            cp_async16(&S.k[row][cc], k + off, ok);
+        }
+        cp_async_commit();
+    };
+    issue(0, 0);
+    int sb = 0;
 
-    for (int64_t c0 = 0; c0 < K; c0 += KT) {
+    for (int64_t c0 = 0; c0 < K; c0 += KT, sb ^= 1) {
+        if (c0 + KT < K) {
+            issue(c0 + KT, sb ^ 1);
+            cp_async_wait_1();
+        } else {
+            cp_async_wait_0();
+        }
+        __syncthreads();
+        const Stage& S = sm.st[sb];
         // ---- phase 1: thread (channel cl, sub-chunk I) cumsum, factors, operands
         const int cl = lane;
         const int64_t ch = c0 + cl;
@@ -116,9 +161,7 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
         float run = 0.f;
 #pragma unroll
         for (int r = 0; r < SC; ++r) {
-            const int row = I * SC + r;
-            const float x = (row < nvalid) ? la[(bh * L + t0 + row) * K + ch] : 0.f;
-            run += x;
+            run += S.la[I * SC + r][cl];
             b[r] = run;
         }
         sm.tot[I][cl] = run;
@@ -154,12 +197,8 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
             const int row = I * SC + r;
             const float B = pre + b[r];
             sm.B[row][cl] = B;
-            float qv = 0.f, kv = 0.f;
-            if (row < nvalid) {
-                const int64_t off = (bh * L + t0 + row) * K + ch;
-                qv = __bfloat162float(q[off]);
-                kv = __bfloat162float(k[off]);
-            }
+            const float qv = __bfloat162float(S.q[row][cl]);
+            const float kv = __bfloat162float(S.k[row][cl]);
             const float a = __expf(B - rho);     // e^{B_j - rho_I} <= 1
             const float kfac = __expf(last - B); // e^{last_I - B_j} <= 1
             const float qhat = qv * a;
@@ -168,14 +207,20 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
             sm.kh[row][cl] = __float2bfloat16_rn(khat);
             sm.qf[row][cl] = qhat;
             sm.kf[row][cl] = unsafe ? 0.f : khat * eSpan;
-            if (row < nvalid) {
-                const int64_t off = (bh * L + t0 + row) * K + ch;
-                Qt[off] = __float2bfloat16_rn(qhat * eRho);
-                Kt[off] = __float2bfloat16_rn(khat * eGl);
-                if (Bout) Bout[off] = B;
-            }
+            sm.qo[row][cl] = __float2bfloat16_rn(qhat * eRho);
+            sm.ko[row][cl] = __float2bfloat16_rn(khat * eGl);
+            if (Bout && row < nvalid) Bout[(bh * L + t0 + row) * K + ch] = B;
         }
         __syncthreads();
+        // coalesced 16-byte stores of the Q~ and K~ tiles
+        for (int e = tid; e < C * (KT / 8); e += 256) {
+            const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
+            if (row < nvalid) {
+                const int64_t off = (bh * L + t0 + row) * K + c0 + cc;
+                *reinterpret_cast<uint4*>(Qt + off) = *reinterpret_cast<const uint4*>(&sm.qo[row][cc]);
+                *reinterpret_cast<uint4*>(Kt + off) = *reinterpret_cast<const uint4*>(&sm.ko[row][cc]);
+            }
+        }
 
         // ---- phase 2a: off-diagonal blocks on the tensor cores
 #pragma unroll

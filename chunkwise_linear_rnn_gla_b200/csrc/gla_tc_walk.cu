@@ -46,7 +46,8 @@ struct Bars {
     uint64_t empty[RING];
     uint64_t u_full[2], u_empty[2], o_full[2], o_empty[2];
     uint64_t v_full[2], v_empty[2];  // value tile, double-buffered outside the ring
-    uint64_t s_ready, s_free, s_load, drain;
+    uint64_t s_ready[2], s_free[2];  // bf16 state copy, double-buffered: written / read
+    uint64_t s_load, drain;
     uint32_t tmem_slot;
     int abort_flag;
 };
@@ -120,15 +121,15 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     k_walk(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
            const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmP,
            const __grid_constant__ CUtensorMap tmS, const float* __restrict__ gam, const float* __restrict__ init,
-           float* __restrict__ fin, __nv_bfloat16* __restrict__ Y, __nv_bfloat16* __restrict__ states, int64_t L,
-           int64_t N, int64_t V, int* err) {
-    constexpr int K = NH * 128;
+           float* __restrict__ fin, float* __restrict__ fin2, __nv_bfloat16* __restrict__ Y,
+           __nv_bfloat16* __restrict__ states, int64_t L, int64_t N, int64_t V, int64_t K, int* err) {
+    constexpr int KC = NH * 128;  // key channels owned by this CTA
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = base;
     uint8_t* vbuf = base + RING * PIECE;  // 2 x PIECE
-    uint8_t* sS = vbuf + 2 * PIECE;
-    Bars& bar = *reinterpret_cast<Bars*>(sS + K * 128);
+    uint8_t* sS = vbuf + 2 * PIECE;  // 2 x [KC x 64] bf16 copies of the state
+    Bars& bar = *reinterpret_cast<Bars*>(sS + 2 * KC * 128);
     volatile int* abort_flag = &bar.abort_flag;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -136,6 +137,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     const int v0 = blockIdx.x * BV;
     const int nsteps = MODE == kWalkOutputOnly ? 1 : int(N);
     const int first_chunk = MODE == kWalkOutputOnly ? int(blockIdx.y) : 0;
+    // states-only walks may split the key channels over blockIdx.y
+    const int kbase = MODE == kWalkStatesOnly ? int(blockIdx.y) * KC : 0;
     auto chunk_of = [&](int step) -> int {
         if (MODE == kWalkOutputOnly) return first_chunk;
         return REVERSE ? int(N) - 1 - step : step;
@@ -154,8 +157,10 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
             mbar_init(&bar.v_full[b], 1);
             mbar_init(&bar.v_empty[b], 1);
         }
-        mbar_init(&bar.s_ready, 128);
-        mbar_init(&bar.s_free, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar.s_ready[b], 128);
+            mbar_init(&bar.s_free[b], 1);
+        }
         mbar_init(&bar.s_load, 1);
         mbar_init(&bar.drain, 1);
         bar.abort_flag = 0;
@@ -205,7 +210,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
             };
             if (MODE == kWalkOutputOnly) {
                 const int i = first_chunk;
-                mbar_arrive_expect_tx(&bar.s_load, K * 128);
+                mbar_arrive_expect_tx(&bar.s_load, KC * 128);
                 tma_load_3d(sS, &tmS, v0, 0, int(bh * N + i), &bar.s_load);
             }
             bool ok = true;
@@ -218,7 +223,8 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                 if (!is_out) {
                     for (int h = 0; h < NH && ok; ++h) {
                         const int s = cur.take_pair();
-                        ok = load(s, &tmA1, 128 * h, row0, int(bh)) && load(s + 1, &tmA1, 128 * h + 64, row0, int(bh));
+                        ok = load(s, &tmA1, kbase + 128 * h, row0, int(bh)) &&
+                             load(s + 1, &tmA1, kbase + 128 * h + 64, row0, int(bh));
                     }
                     if (ok) ok = load_v(step, row0);
                 } else {
@@ -286,7 +292,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                     int sq[2 * NH];
                     for (int pc = 0; pc < 2 * NH; ++pc) sq[pc] = cur.take();
                     const int sp = cur.take_pair();
-                    if (MODE == kWalkFused) ok = mbar_wait(&bar.s_ready, uint32_t(step & 1), err, abort_flag);
+                    if (MODE == kWalkFused) ok = mbar_wait(&bar.s_ready[b], use_par, err, abort_flag);
                     if (ok) ok = mbar_wait(&bar.o_empty[b], use_par ^ 1u, err, abort_flag);
                     if (ok && MODE == kWalkOutputOnly) ok = mbar_wait(&bar.v_full[b], use_par, err, abort_flag);
                     for (int pc = 0; pc < 2 * NH && ok; ++pc) ok = wait_full(sq[pc]);
@@ -294,9 +300,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                     if (!ok) break;
                     tc_fence_after();
                     const uint32_t dO_ = tmem + col_O<NH>(b);
-                    const uint32_t s0 = smem_u32(sS);
+                    const uint32_t s0 = smem_u32(sS + b * KC * 128);
 #pragma unroll
-                    for (int kk = 0; kk < K / 16; ++kk)
+                    for (int kk = 0; kk < KC / 16; ++kk)
                         mma_bf16(dO_, sdesc_sw128(smem_u32(ring + sq[kk / 4] * PIECE) + (kk % 4) * 32, 16, 1024),
                                  sdesc_sw128(s0 + kk * 2048, 16, 1024), idQS, kk > 0 ? 1u : 0u);
                     const uint32_t p0 = smem_u32(ring + sp * PIECE);
@@ -308,7 +314,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                         mma_bf16(dO_, ad, sdesc_sw128(vb + kk * 2048, 16, 1024), idPV, 1u);
                     }
                     mma_commit(&bar.o_full[b]);
-                    if (MODE == kWalkFused) mma_commit(&bar.s_free);
+                    if (MODE == kWalkFused) mma_commit(&bar.s_free[b]);
                     for (int pc = 0; pc < 2 * NH; ++pc) mma_commit(&bar.empty[sq[pc]]);
                     mma_commit(&bar.empty[sp]);
                     mma_commit(&bar.empty[sp + 1]);
@@ -323,7 +329,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
         // ------------------------------------------------------ state epilogue
         if (MODE != kWalkOutputOnly) {
             const int q = warp & 3;
-            const int cq = 32 * q + lane;  // key channel within a 128-channel half
+            const int cq = kbase + 32 * q + lane;  // key channel (global index) in this CTA's first half
             const uint32_t lane_off = uint32_t(32 * q) << 16;
             // X0 = init tile (or zero) -> TMEM master and the bf16 copy in smem
             for (int h = 0; h < NH; ++h) {
@@ -334,7 +340,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                     for (int e = 0; e < 16; ++e)
                         x[e] = init ? init[(bh * K + c) * V + v0 + c16 * 16 + e] : 0.f;
                     tmem_st16(tmem + lane_off + col_S<NH>() + uint32_t(h * BV + c16 * 16), x);
-                    uint8_t* row = sS + c * 128;
+                    uint8_t* row = sS + (c - kbase) * 128;
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         const int chunk = c16 * 2 + half;
@@ -343,9 +349,9 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                         w.y = pack_bf16x2(x[half * 8 + 2], x[half * 8 + 3]);
                         w.z = pack_bf16x2(x[half * 8 + 4], x[half * 8 + 5]);
                         w.w = pack_bf16x2(x[half * 8 + 6], x[half * 8 + 7]);
-                        *reinterpret_cast<uint4*>(row + ((chunk ^ (c & 7)) * 16)) = w;
+                        *reinterpret_cast<uint4*>(row + ((chunk ^ ((c - kbase) & 7)) * 16)) = w;
                     }
-                    if (MODE == kWalkStatesOnly) {
+                    if (MODE == kWalkStatesOnly || states) {
                         __nv_bfloat16* dst = states + ((bh * N + chunk_of(0)) * K + c) * V + v0 + c16 * 16;
                         uint4 w0, w1;
                         w0.x = pack_bf16x2(x[0], x[1]);
@@ -364,7 +370,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bar.s_ready);
+            mbar_arrive(&bar.s_ready[0]);
             float g_next[NH];
             for (int h = 0; h < NH; ++h) g_next[h] = gam[(bh * N + chunk_of(0)) * K + 128 * h + cq];
             for (int step = 0; step < nsteps; ++step) {
@@ -376,67 +382,77 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                     for (int h = 0; h < NH; ++h) g_next[h] = gam[(bh * N + chunk_of(step + 1)) * K + 128 * h + cq];
                 if (!mbar_wait(&bar.u_full[b], use_par, err, abort_flag)) break;
                 tc_fence_after();
+                // X <- diag(g) X + U in TMEM, 32 columns per batch; keep the new
+                // state packed to bf16 in registers for the smem / global copy
+                uint32_t pk[NH][BV / 2];
+#pragma unroll
                 for (int h = 0; h < NH; ++h) {
 #pragma unroll
-                    for (int c16 = 0; c16 < BV / 16; ++c16) {
-                        float u[16], x[16];
-                        tmem_ld16(tmem + lane_off + col_U<NH>(b, h) + uint32_t(c16 * 16), u);
-                        tmem_ld16(tmem + lane_off + col_S<NH>() + uint32_t(h * BV + c16 * 16), x);
+                    for (int c32 = 0; c32 < BV / 32; ++c32) {
+                        float u[32], x[32];
+                        const uint32_t cu = col_U<NH>(b, h) + uint32_t(c32 * 32);
+                        const uint32_t cs = col_S<NH>() + uint32_t(h * BV + c32 * 32);
+                        tmem_ld16(tmem + lane_off + cu, u);
+                        tmem_ld16(tmem + lane_off + cu + 16, u + 16);
+                        tmem_ld16(tmem + lane_off + cs, x);
+                        tmem_ld16(tmem + lane_off + cs + 16, x + 16);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 16; ++e) x[e] = fmaf(g[h], x[e], u[e]);
-                        tmem_st16(tmem + lane_off + col_S<NH>() + uint32_t(h * BV + c16 * 16), x);
+                        for (int e = 0; e < 32; ++e) x[e] = fmaf(g[h], x[e], u[e]);
+                        tmem_st16(tmem + lane_off + cs, x);
+                        tmem_st16(tmem + lane_off + cs + 16, x + 16);
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) pk[h][c32 * 16 + e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
                     }
                 }
                 tmem_wait_st();
                 tc_fence_before();
                 mbar_arrive(&bar.u_empty[b]);
                 if (step + 1 == nsteps) break;  // the final state is written below
-                // S_[i+1] -> bf16 smem copy for the next output GEMM (after O_i read the old one)
-                if (MODE == kWalkFused && !mbar_wait(&bar.s_free, uint32_t(step & 1), err, abort_flag)) break;
-                for (int h = 0; h < NH; ++h) {
-                    const int c = 128 * h + cq;
-                    uint8_t* row = sS + c * 128;
+                if (MODE == kWalkFused) {
+                    // S_[i+1] -> bf16 copy in buffer (step+1)&1, last read by the output GEMM of step-1
+                    const int nb = (step + 1) & 1;
+                    if (step >= 1 &&
+                        !mbar_wait(&bar.s_free[nb], uint32_t(((step - 1) >> 1) & 1), err, abort_flag))
+                        break;
 #pragma unroll
-                    for (int c16 = 0; c16 < BV / 16; ++c16) {
-                        float x[16];
-                        tmem_ld16(tmem + lane_off + col_S<NH>() + uint32_t(h * BV + c16 * 16), x);
-                        tmem_wait_ld();
-                        uint4 w0, w1;
-                        w0.x = pack_bf16x2(x[0], x[1]);
-                        w0.y = pack_bf16x2(x[2], x[3]);
-                        w0.z = pack_bf16x2(x[4], x[5]);
-                        w0.w = pack_bf16x2(x[6], x[7]);
-                        w1.x = pack_bf16x2(x[8], x[9]);
-                        w1.y = pack_bf16x2(x[10], x[11]);
-                        w1.z = pack_bf16x2(x[12], x[13]);
-                        w1.w = pack_bf16x2(x[14], x[15]);
-                        if (MODE == kWalkFused) {
-                            *reinterpret_cast<uint4*>(row + (((2 * c16) ^ (c & 7)) * 16)) = w0;
-                            *reinterpret_cast<uint4*>(row + (((2 * c16 + 1) ^ (c & 7)) * 16)) = w1;
-                        } else {
-                            __nv_bfloat16* dst =
-                                states + ((bh * N + chunk_of(step + 1)) * K + c) * V + v0 + c16 * 16;
-                            reinterpret_cast<uint4*>(dst)[0] = w0;
-                            reinterpret_cast<uint4*>(dst)[1] = w1;
-                        }
+                    for (int h = 0; h < NH; ++h) {
+                        const int c = 128 * h + cq;
+                        uint8_t* row = sS + nb * KC * 128 + (c - kbase) * 128;
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch)
+                            *reinterpret_cast<uint4*>(row + ((ch ^ ((c - kbase) & 7)) * 16)) =
+                                make_uint4(pk[h][4 * ch], pk[h][4 * ch + 1], pk[h][4 * ch + 2], pk[h][4 * ch + 3]);
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&bar.s_ready[nb]);
+                }
+                if (MODE == kWalkStatesOnly || states) {
+#pragma unroll
+                    for (int h = 0; h < NH; ++h) {
+                        const int c = 128 * h + cq;
+                        uint4* dst = reinterpret_cast<uint4*>(states + ((bh * N + chunk_of(step + 1)) * K + c) * V + v0);
+#pragma unroll
+                        for (int ch = 0; ch < 8; ++ch)
+                            dst[ch] = make_uint4(pk[h][4 * ch], pk[h][4 * ch + 1], pk[h][4 * ch + 2], pk[h][4 * ch + 3]);
                     }
                 }
-                if (MODE == kWalkFused) {
-                    fence_proxy_async_smem();
-                    mbar_arrive(&bar.s_ready);
-                }
             }
-            if (fin && !*abort_flag) {
+            if ((fin || fin2) && !*abort_flag) {
                 for (int h = 0; h < NH; ++h) {
                     const int c = 128 * h + cq;
                     for (int c16 = 0; c16 < BV / 16; ++c16) {
                         float x[16];
                         tmem_ld16(tmem + lane_off + col_S<NH>() + uint32_t(h * BV + c16 * 16), x);
                         tmem_wait_ld();
-                        float4* dst = reinterpret_cast<float4*>(fin + (bh * K + c) * V + v0 + c16 * 16);
+                        for (int w = 0; w < 2; ++w) {
+                            float* f = w ? fin2 : fin;
+                            if (!f) continue;
+                            float4* dst = reinterpret_cast<float4*>(f + (bh * K + c) * V + v0 + c16 * 16);
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                            for (int e = 0; e < 4; ++e)
+                                dst[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                        }
                     }
                 }
             }
@@ -453,25 +469,18 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                 if (!mbar_wait(&bar.o_full[b], use_par, err, abort_flag)) break;
                 tc_fence_after();
                 const int64_t t = int64_t(chunk_of(step)) * C + r;
+                float y[BV];
 #pragma unroll
-                for (int c16 = 0; c16 < BV / 16; ++c16) {
-                    float y[16];
-                    tmem_ld16(tmem + lane_off + col_O<NH>(b) + uint32_t(c16 * 16), y);
-                    tmem_wait_ld();
-                    if (t < L) {
-                        uint4 w0, w1;
-                        w0.x = pack_bf16x2(y[0], y[1]);
-                        w0.y = pack_bf16x2(y[2], y[3]);
-                        w0.z = pack_bf16x2(y[4], y[5]);
-                        w0.w = pack_bf16x2(y[6], y[7]);
-                        w1.x = pack_bf16x2(y[8], y[9]);
-                        w1.y = pack_bf16x2(y[10], y[11]);
-                        w1.z = pack_bf16x2(y[12], y[13]);
-                        w1.w = pack_bf16x2(y[14], y[15]);
-                        uint4* dst = reinterpret_cast<uint4*>(Y + (bh * L + t) * V + v0 + c16 * 16);
-                        dst[0] = w0;
-                        dst[1] = w1;
-                    }
+                for (int c16 = 0; c16 < BV / 16; ++c16)
+                    tmem_ld16(tmem + lane_off + col_O<NH>(b) + uint32_t(c16 * 16), y + 16 * c16);
+                tmem_wait_ld();
+                if (t < L) {
+                    uint4* dst = reinterpret_cast<uint4*>(Y + (bh * L + t) * V + v0);
+#pragma unroll
+                    for (int ch = 0; ch < BV / 8; ++ch)
+                        dst[ch] = make_uint4(pack_bf16x2(y[8 * ch], y[8 * ch + 1]), pack_bf16x2(y[8 * ch + 2], y[8 * ch + 3]),
+                                             pack_bf16x2(y[8 * ch + 4], y[8 * ch + 5]),
+                                             pack_bf16x2(y[8 * ch + 6], y[8 * ch + 7]));
                 }
                 tc_fence_before();
                 mbar_arrive(&bar.o_empty[b]);
@@ -496,20 +505,22 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
 template <int NH, bool REVERSE, bool PT, int MODE>
 gla_status launch_walk(const Problem& p, const WalkArgs& a, const CUtensorMap* maps, cudaStream_t s,
                        const char* name) {
-    constexpr int K = NH * 128;
+    constexpr int KC = NH * 128;
     auto fn = k_walk<NH, REVERSE, PT, MODE>;
-    const size_t smem = 1024 + size_t(RING + 2) * PIECE + size_t(K) * 128 + sizeof(Bars);
+    const size_t smem = 1024 + size_t(RING + 2) * PIECE + 2 * size_t(KC) * 128 + sizeof(Bars);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    const dim3 grid(unsigned(p.V / BV), MODE == kWalkOutputOnly ? unsigned(p.N) : 1u, unsigned(p.BH));
+    const unsigned gy = MODE == kWalkOutputOnly ? unsigned(p.N)
+                        : MODE == kWalkStatesOnly ? unsigned(p.K / KC) : 1u;
+    const dim3 grid(unsigned(p.V / BV), gy, unsigned(p.BH));
     GLA_LAUNCH(name, fn, grid, kWalkThreads, smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], a.gam, a.init,
-               a.fin, a.Y, a.states, p.L, p.N, p.V, device_error_word());
+               a.fin, a.fin2, a.Y, a.states, p.L, p.N, p.V, p.K, device_error_word());
     return GLA_OK;
 }
 
 }  // namespace
 
-size_t tc_walk_smem_bytes(int K) { return 1024 + size_t(RING + 2) * PIECE + size_t(K) * 128 + sizeof(Bars); }
+
 
 gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, const char* name) {
     CUtensorMap maps[5];
@@ -528,7 +539,7 @@ gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, c
         if (!ok) break;
         else if (maps[m].opaque[0] == 0 && maps[m].opaque[1] == 0) maps[m] = maps[1];
     if (!ok) return GLA_ERR_CUDA;
-    const int NH = int(p.K / 128);
+    const int NH = a.mode == kWalkStatesOnly ? 1 : int(p.K / 128);  // states-only: one half per CTA
 #define GLA_WALK_CASE(nh_, rev_, pt_, mode_)                                                   \
     if (NH == nh_ && a.reverse == rev_ && a.p_transposed == pt_ && a.mode == mode_)            \
         return launch_walk<nh_, rev_, pt_, mode_>(p, a, maps, s, name);
@@ -537,9 +548,11 @@ gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, c
     GLA_WALK_CASE(1, true, true, kWalkFused)
     GLA_WALK_CASE(2, true, true, kWalkFused)
     GLA_WALK_CASE(1, false, false, kWalkStatesOnly)
-    GLA_WALK_CASE(2, false, false, kWalkStatesOnly)
+    GLA_WALK_CASE(1, true, false, kWalkStatesOnly)
     GLA_WALK_CASE(1, false, false, kWalkOutputOnly)
     GLA_WALK_CASE(2, false, false, kWalkOutputOnly)
+    GLA_WALK_CASE(1, false, true, kWalkOutputOnly)
+    GLA_WALK_CASE(2, false, true, kWalkOutputOnly)
 #undef GLA_WALK_CASE
     return GLA_ERR_UNSUPPORTED;
 }

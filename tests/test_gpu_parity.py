@@ -254,3 +254,48 @@ def test_tc_matches_simt_forward():
     o_s, hT_s = run_fwd(d, "simt")
     compare("o tc-vs-simt", o_tc, to_f64_numpy(o_s), "bf16")
     compare("hT tc-vs-simt", hT_tc, to_f64_numpy(hT_s), "bf16")
+
+
+# ----------------------------------------------- tensor-core backward path
+@pytest.mark.parametrize("mode", ["nonmaterialized", "materialized"])
+@pytest.mark.parametrize("shape", TC_SHAPES)
+def test_tc_backward(mode, shape):
+    B, H, L, K, V = shape
+    inp = make_inputs(B, H, L, K, V, "bf16", seed=L + K + V + 1, h0=True, dhT=True)
+    check_bwd(inp, "bf16", "tc", state_mode=mode)
+
+
+@pytest.mark.parametrize("mode", ["nonmaterialized", "materialized"])
+def test_tc_backward_extreme_gates(mode):
+    inp = make_inputs(1, 3, 260, 128, 64, "bf16", seed=23, h0=True, dhT=True, gate_scale=1.0)
+    la = inp["log_a"].clone()
+    la[:, 0] = -1e30
+    la[:, 1] = 0.0
+    la[:, 2] = la[:, 2] * 3.0
+    inp["log_a"] = la
+    check_bwd(inp, "bf16", "tc", state_mode=mode)
+
+
+@pytest.mark.parametrize("mode", ["nonmaterialized", "materialized"])
+def test_tc_ws_reuse_matches_recompute(mode):
+    inp = make_inputs(2, 2, 300, 256, 128, "bf16", seed=24, h0=True, dhT=True)
+    d = to_dev(inp)
+    desc = gla.make_desc(2, 2, 300, 256, 128, "bf16", impl="tc", state_mode=mode)
+    ws = torch.empty(gla.gla_bwd_workspace_size(desc), dtype=torch.uint8, device="cuda")
+    kw = dict(impl="tc", state_mode=mode)
+    gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], d["h0"], workspace=ws, **kw)
+    g1 = gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d["h0"], d["dhT"], workspace=ws, ws_from_fwd=True,
+                     **kw)
+    g2 = gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d["h0"], d["dhT"], **kw)
+    torch.cuda.synchronize()
+    for key in g1:
+        assert torch.equal(g1[key], g2[key]), key
+
+
+def test_tc_backward_matches_simt():
+    inp = make_inputs(1, 2, 400, 256, 128, "bf16", seed=25, h0=True, dhT=True)
+    d = to_dev(inp)
+    g_tc = run_bwd(d, "tc")
+    g_s = run_bwd(d, "simt")
+    for key in ("dq", "dk", "dv", "dlog_a", "dh0"):
+        compare(key + " tc-vs-simt", g_tc[key], to_f64_numpy(g_s[key]), "bf16")
