@@ -49,13 +49,18 @@ struct WalkArgs {
 
 gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, const char* name);
 
+// Chunk-parallel Y_i = A_i X_i + Pm_i B_i from stored bf16 chunk states X
+// (gla_tc_out.cu): forward o (A = Q~, Pm = P) and dv (A = K~, Pm = P^T).
+gla_status tc_chunk_out_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* X,
+                               const __nv_bfloat16* Pm, const __nv_bfloat16* Bv, bool p_transposed,
+                               __nv_bfloat16* Y, cudaStream_t s, const char* name);
+
 // Backward, chunk-parallel part (gla_tc_bwd.cu).
 gla_status tc_bwd_gemm_launch(const Problem& p, const void* dO, const void* v, const __nv_bfloat16* Sbuf,
                               const __nv_bfloat16* Dbuf, __nv_bfloat16* dP, __nv_bfloat16* dQt, __nv_bfloat16* dKt,
-                              cudaStream_t s);
+                              float* xdot, cudaStream_t s);
 gla_status tc_bwd_intra_launch(const Problem& p, const void* q, const void* k, const float* la,
                                const __nv_bfloat16* dP, const __nv_bfloat16* dQt, const __nv_bfloat16* dKt,
-                               const __nv_bfloat16* Sbuf, const __nv_bfloat16* Dbuf, const float* hT,
-                               const float* dhT, void* dq, void* dk, float* dla, cudaStream_t s);
+                               const float* xdot, void* dq, void* dk, float* dla, cudaStream_t s);
 
 }  // namespace gla

@@ -31,6 +31,7 @@ struct TcBuffers {
     float *gam, *hT;
     __nv_bfloat16* states;
     __nv_bfloat16 *Dbuf, *dP, *dQt, *dKt;
+    float* xdot;  // sum_v D_i * S_[i] per chunk and key channel
 };
 
 // The backward layout extends the forward's, so a forward workspace can be
@@ -49,6 +50,7 @@ TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
         b.dP = a.take<__nv_bfloat16>(size_t(p.BH * p.N * kTcChunk * kTcChunk));
         b.dQt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
         b.dKt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
+        b.xdot = a.take<float>(size_t(p.BH * p.N * p.K));
     }
     return b;
 }
@@ -101,9 +103,8 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
     a.mode = kWalkStatesOnly;
     st = tc_walk_launch(p, a, s, "tc_walk_states");
     if (st != GLA_OK) return st;
-    a.mode = kWalkOutputOnly;
-    a.fin = a.fin2 = nullptr;
-    return tc_walk_launch(p, a, s, "tc_output");
+    return tc_chunk_out_launch(p, b.Qt, b.states, b.P, static_cast<const __nv_bfloat16*>(v), false,
+                               static_cast<__nv_bfloat16*>(o), s, "tc_output");
 }
 
 gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* la, const float* h0,
@@ -151,17 +152,14 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
             a.mode = kWalkStatesOnly;
             st = tc_walk_launch(p, a, s, "tc_walk_dstates");
             if (st != GLA_OK) return st;
-            a.mode = kWalkOutputOnly;
-            a.reverse = false;
-            a.p_transposed = true;
-            a.fin = nullptr;
-            st = tc_walk_launch(p, a, s, "tc_output_dv");
+            st = tc_chunk_out_launch(p, b.Kt, b.Dbuf, b.P, static_cast<const __nv_bfloat16*>(dO), true,
+                                     static_cast<__nv_bfloat16*>(dv), s, "tc_output_dv");
             if (st != GLA_OK) return st;
         }
     }
-    st = tc_bwd_gemm_launch(p, dO, v, b.states, b.Dbuf, b.dP, b.dQt, b.dKt, s);
+    st = tc_bwd_gemm_launch(p, dO, v, b.states, b.Dbuf, b.dP, b.dQt, b.dKt, b.xdot, s);
     if (st != GLA_OK) return st;
-    return tc_bwd_intra_launch(p, q, k, la, b.dP, b.dQt, b.dKt, b.states, b.Dbuf, b.hT, dhT, dq, dk, dla, s);
+    return tc_bwd_intra_launch(p, q, k, la, b.dP, b.dQt, b.dKt, b.xdot, dq, dk, dla, s);
 }
 
 }  // namespace gla

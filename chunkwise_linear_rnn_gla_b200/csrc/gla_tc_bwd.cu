@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(192, 1)
     k_bwd_gemm(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmV,
                const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmD,
                __nv_bfloat16* __restrict__ dP, __nv_bfloat16* __restrict__ dQt, __nv_bfloat16* __restrict__ dKt,
-               int64_t L, int64_t N, int64_t K, int64_t V, int* err) {
+               float* __restrict__ xdot, int64_t L, int64_t N, int64_t K, int64_t V, int* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     GemmBars& bar = *reinterpret_cast<GemmBars*>(base + NSTAGE * 4 * PIECE);
@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGE; ++s) {
             mbar_init(&bar.full[s], 1);
-            mbar_init(&bar.empty[s], 1);
+            mbar_init(&bar.empty[s], 1 + 128);  // MMA commit + the 128 row-dot threads
         }
         mbar_init(&bar.done, 1);
         bar.abort_flag = 0;
@@ -129,7 +129,33 @@ __global__ void __launch_bounds__(192, 1)
         const int q = warp & 3;
         const int r = 32 * q + lane;
         const uint32_t lane_off = uint32_t(32 * q) << 16;
-        if (mbar_wait(&bar.done, 0, err, abort_flag)) {
+        // while the MMAs run: x[c] = sum_v D_i[c,v] S_[i][c,v] for this thread's key channel
+        float x = 0.f;
+        bool ok = true;
+        for (int vb = 0; vb < nvb; ++vb) {
+            const int s = vb % NSTAGE;
+            if (!mbar_wait(&bar.full[s], uint32_t((vb / NSTAGE) & 1), err, abort_flag)) {
+                ok = false;
+                break;
+            }
+            const uint8_t* st = base + s * 4 * PIECE;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch) {
+                const uint32_t off = uint32_t(r) * 128u + uint32_t((ch ^ (r & 7)) * 16);
+                const uint4 sv = *reinterpret_cast<const uint4*>(st + 2 * PIECE + off);
+                const uint4 dv = *reinterpret_cast<const uint4*>(st + 3 * PIECE + off);
+                const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv);
+                const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 a = __bfloat1622float2(s2[e]), b = __bfloat1622float2(d2[e]);
+                    x = fmaf(a.x, b.x, fmaf(a.y, b.y, x));
+                }
+            }
+            mbar_arrive(&bar.empty[s]);
+        }
+        if (ok) xdot[(bh * N + i) * K + 128 * kh + r] = x;
+        if (ok && mbar_wait(&bar.done, 0, err, abort_flag)) {
             tc_fence_after();
             const int64_t t = int64_t(i) * C + r;
             for (int part = 0; part < 3; ++part) {
@@ -198,29 +224,44 @@ __device__ __forceinline__ uint32_t scale2(uint32_t v, float s) {
 }
 __host__ __device__ constexpr int pidx(int I, int J) { return I * (I - 1) / 2 + J; }
 
+__device__ __forceinline__ void cpa16(void* dst, const void* src, bool valid) {
+    const uint32_t n = valid ? 16u : 0u;
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(tc_smem_u32(dst)), "l"(src), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cpa_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cpa_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+struct IntraStage {  // raw inputs of one 32-channel tile (cp.async)
+    float la[C][KT];
+    __nv_bfloat16 q[C][KT];
+    __nv_bfloat16 k[C][KT];
+};
+
 struct IntraSmem {
     __nv_bfloat16 dP[C][DPS];
-    float la[C][KT];
-    __nv_bfloat16 q[C][KT], k[C][KT], dQt[C][KT], dKt[C][KT];
-    float B[C][KT];
-    float a[C][KT + 1], kf[C][KT + 1];      // e^{B_j - rho_I}, e^{last_I - B_j}
-    float qf[C][KT + 1], kfD[C][KT + 1];    // fp32 operands of the diagonal blocks
-    __nv_bfloat16 qh[C][QS], kh[C][QS];     // bf16 operands of the off-diagonal blocks
-    float iq[C][KT + 1], ik[C][KT + 1];     // intra results
+    float dg[NS][SC][SC];   // diagonal blocks of dP in fp32: dg[I][j][s] = dP[16I+j][16I+s]
+    float dgT[NS][SC][SC];  // the same blocks transposed: dgT[I][s][j]
+    IntraStage st[2];
+    float a[C][KT + 1], kf[C][KT + 1];   // e^{B_j - rho_I}, e^{last_I - B_j}
+    __nv_bfloat16 qh[C][QS], kh[C][QS];  // bf16 operands of the off-diagonal blocks
+    float iq[C][KT + 1], ik[C][KT + 1];  // intra-chunk parts of dq, dk
     float d[28][KT];
-    float tot[NS][KT];
-    float EI[NS][KT], FI[NS][KT];
-    float carry[KT];
+    float tot[NS][KT], tot2[NS][KT];
+    float EI[NS][KT], FI[NS][KT], DI[NS][KT];
+    float eG[KT];
     unsigned unsafe_mask[NS];
 };
 
+// One CTA per (chunk, head); 8 warps, warp I <-> query/key sub-chunk I; key
+// channels in tiles of 32 (thread (channel = lane, sub-chunk = warp) in the
+// elementwise phases).
 __global__ void __launch_bounds__(256, 1)
     k_bwd_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                 const float* __restrict__ la, const __nv_bfloat16* __restrict__ dPg,
                 const __nv_bfloat16* __restrict__ dQt, const __nv_bfloat16* __restrict__ dKt,
-                const __nv_bfloat16* __restrict__ Sbuf, const __nv_bfloat16* __restrict__ Dbuf,
-                const float* __restrict__ hT, const float* __restrict__ dhT, __nv_bfloat16* __restrict__ dq,
-                __nv_bfloat16* __restrict__ dk, float* __restrict__ dla, int64_t L, int64_t N, int64_t K, int64_t V) {
+                const float* __restrict__ xdot, __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
+                float* __restrict__ dla, int64_t L, int64_t N, int64_t K) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     IntraSmem& sm = *reinterpret_cast<IntraSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -229,63 +270,65 @@ __global__ void __launch_bounds__(256, 1)
     const int nvalid = int(L - t0 < C ? L - t0 : C);
     const int g = lane >> 2, tq = lane & 3;
 
-    // dP of this chunk (bf16, zero above the diagonal) -> smem
     for (int e = tid; e < C * C / 8; e += 256) {
         const int row = e / (C / 8), cc = (e % (C / 8)) * 8;
-        *reinterpret_cast<uint4*>(&sm.dP[row][cc]) =
-            *reinterpret_cast<const uint4*>(dPg + ((bh * N + i) * C + row) * C + cc);
+        cpa16(&sm.dP[row][cc], dPg + ((bh * N + i) * C + row) * C + cc, true);
     }
-
-    for (int64_t c0 = 0; c0 < K; c0 += KT) {
-        __syncthreads();
-        // ---- stage the raw tile
-        for (int e = tid; e < C * KT; e += 256) {
-            const int row = e / KT, cc = e % KT;
+    auto issue = [&](int64_t c0, int sb) {
+        IntraStage& S = sm.st[sb];
+        for (int e = tid; e < C * (KT / 4); e += 256) {
+            const int row = e / (KT / 4), cc = (e % (KT / 4)) * 4;
             const bool ok = row < nvalid;
-            const int64_t off = (bh * L + t0 + row) * K + c0 + cc;
-            sm.la[row][cc] = ok ? la[off] : 0.f;
-            sm.q[row][cc] = ok ? q[off] : __float2bfloat16_rn(0.f);
-            sm.k[row][cc] = ok ? k[off] : __float2bfloat16_rn(0.f);
-            sm.dQt[row][cc] = ok ? dQt[off] : __float2bfloat16_rn(0.f);
-            sm.dKt[row][cc] = ok ? dKt[off] : __float2bfloat16_rn(0.f);
+            cpa16(&S.la[row][cc], la + (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc, ok);
         }
-        // ---- carry into this chunk from all later chunks: sum_v D_i * S_[i+1]
-        {
-            const int cl = tid >> 3, part = tid & 7;  // 32 channels x 8 threads
-            const int64_t ch = c0 + cl;
-            float acc = 0.f;
-            if (i + 1 < N) {
-                const __nv_bfloat16* Dr = Dbuf + ((bh * N + i) * K + ch) * V;
-                const __nv_bfloat16* Sr = Sbuf + ((bh * N + i + 1) * K + ch) * V;
-                for (int64_t v = part * 8; v < V; v += 64) {
-                    const uint4 dv4 = *reinterpret_cast<const uint4*>(Dr + v);
-                    const uint4 sv4 = *reinterpret_cast<const uint4*>(Sr + v);
-                    const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv4);
-                    const __nv_bfloat162* s2 = reinterpret_cast<const __nv_bfloat162*>(&sv4);
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float2 a = __bfloat1622float2(d2[e]), b = __bfloat1622float2(s2[e]);
-                        acc += a.x * b.x + a.y * b.y;
-                    }
-                }
-            } else if (dhT) {
-                const float* Dr = dhT + (bh * K + ch) * V;
-                const float* Sr = hT + (bh * K + ch) * V;
-                for (int64_t v = part; v < V; v += 8) acc += Dr[v] * Sr[v];
-            }
-            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-            acc += __shfl_xor_sync(0xffffffffu, acc, 4);
-            if (part == 0) sm.carry[cl] = acc;
+        for (int e = tid; e < C * (KT / 8); e += 256) {
+            const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
+            const bool ok = row < nvalid;
+            const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc;
+            cpa16(&S.q[row][cc], q + off, ok);
+            cpa16(&S.k[row][cc], k + off, ok);
+        }
+        cpa_commit();
+    };
+    issue(0, 0);
+    int sb = 0;
+    const int cl = lane, I = warp;
+
+    for (int64_t c0 = 0; c0 < K; c0 += KT, sb ^= 1) {
+        if (c0 + KT < K) {
+            issue(c0 + KT, sb ^ 1);
+            cpa_wait1();
+        } else {
+            cpa_wait0();
         }
         __syncthreads();
-        // ---- phase 1: thread (channel cl, sub-chunk I): cumsum, factors, operands
-        const int cl = lane, I = warp;
+        if (c0 == 0) {
+            for (int e = tid; e < NS * SC * SC; e += 256) {
+                const int I2 = e / (SC * SC), j = (e / SC) % SC, s_ = e % SC;
+                const float v = __bfloat162float(sm.dP[I2 * SC + j][I2 * SC + s_]);
+                sm.dg[I2][j][s_] = v;
+                sm.dgT[I2][s_][j] = v;
+            }
+        }
+        const IntraStage& S = sm.st[sb];
+        const int64_t ch = c0 + cl;
+        // inter-chunk parts of this thread's rows, used by the combine at the end
+        unsigned short hq[SC], hk[SC];
+#pragma unroll
+        for (int r = 0; r < SC; ++r) {
+            const int row = I * SC + r;
+            const bool ok = row < nvalid;
+            const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + ch;
+            hq[r] = ok ? reinterpret_cast<const unsigned short*>(dQt)[off] : 0;
+            hk[r] = ok ? reinterpret_cast<const unsigned short*>(dKt)[off] : 0;
+        }
+        const float xd = xdot[(bh * N + i) * K + ch];
+        // ---- phase 1: cumsum, factors, operands
         float b[SC];
         float run = 0.f;
 #pragma unroll
         for (int r = 0; r < SC; ++r) {
-            run += sm.la[I * SC + r][cl];
+            run += S.la[I * SC + r][cl];
             b[r] = run;
         }
         sm.tot[I][cl] = run;
@@ -305,6 +348,8 @@ __global__ void __launch_bounds__(256, 1)
         if (unsafe) atomicOr(&sm.unsafe_mask[I], 1u << cl);
         sm.EI[I][cl] = __expf(rho);
         sm.FI[I][cl] = __expf(gamma - last);
+        sm.DI[I][cl] = eSpan;
+        if (I == 0) sm.eG[cl] = __expf(gamma);
         {
             float lastJ = 0.f;
 #pragma unroll
@@ -317,32 +362,27 @@ __global__ void __launch_bounds__(256, 1)
         for (int r = 0; r < SC; ++r) {
             const int row = I * SC + r;
             const float Bv = pre + b[r];
-            sm.B[row][cl] = Bv;
             const float av = __expf(Bv - rho), kv = __expf(last - Bv);
-            const float qhat = __bfloat162float(sm.q[row][cl]) * av;
-            const float khat = __bfloat162float(sm.k[row][cl]) * kv;
             sm.a[row][cl] = av;
             sm.kf[row][cl] = kv;
-            sm.qf[row][cl] = qhat;
-            sm.kfD[row][cl] = unsafe ? 0.f : khat * eSpan;
-            sm.qh[row][cl] = __float2bfloat16_rn(qhat);
-            sm.kh[row][cl] = __float2bfloat16_rn(khat);
+            sm.qh[row][cl] = __float2bfloat16_rn(__bfloat162float(S.q[row][cl]) * av);
+            sm.kh[row][cl] = __float2bfloat16_rn(__bfloat162float(S.k[row][cl]) * kv);
         }
         __syncthreads();
-        // ---- phase 2a: off-diagonal blocks, warp I: dq rows of sub-chunk I, dk rows of sub-chunk I
+        // ---- phase 2a: off-diagonal blocks on the tensor cores
         {
             float aq[4][4], ak[4][4];
 #pragma unroll
             for (int n = 0; n < 4; ++n)
 #pragma unroll
                 for (int e = 0; e < 4; ++e) aq[n][e] = ak[n][e] = 0.f;
-            // dq_I += sum_{J<I} dP_IJ (K^_J * d_IJ)     (K^_J = k e^{last_J - B})
+            // dq_I += sum_{J<I} dP_IJ (K^_J * d_IJ)
             for (int J = 0; J < I; ++J) {
                 uint32_t A[4];
                 ldsm_x4(tc_smem_u32(&sm.dP[I * SC + (lane & 15)][J * SC + (lane >> 4) * 8]), A);
                 const float* dd = sm.d[pidx(I, J)];
 #pragma unroll
-                for (int nb2 = 0; nb2 < 2; ++nb2) {  // pairs of 8-channel blocks
+                for (int nb2 = 0; nb2 < 2; ++nb2) {
                     uint32_t Bf[4];
                     const int row = J * SC + (lane & 7) + ((lane >> 3) & 1) * 8;
                     const int col = nb2 * 16 + (lane >> 4) * 8;
@@ -352,7 +392,7 @@ __global__ void __launch_bounds__(256, 1)
                     mma16816(aq[2 * nb2 + 1], A, scale2(Bf[2], f1), scale2(Bf[3], f1));
                 }
             }
-            // dk_J += sum_{I>J} dP_IJ^T (Q^_I * d_IJ), here J = warp
+            // dk_J += sum_{I2>J} dP_{I2 J}^T (Q^_{I2} * d_{I2 J}), J = this warp
             const int J = warp;
             for (int I2 = J + 1; I2 < NS; ++I2) {
                 uint32_t A[4];
@@ -369,7 +409,6 @@ __global__ void __launch_bounds__(256, 1)
                     mma16816(ak[2 * nb2 + 1], A, scale2(Bf[2], f1), scale2(Bf[3], f1));
                 }
             }
-            // scale by the row factors and park in smem (fragment layout -> [row][channel])
 #pragma unroll
             for (int n = 0; n < 4; ++n) {
                 const int c = n * 8 + 2 * tq;
@@ -386,47 +425,62 @@ __global__ void __launch_bounds__(256, 1)
         __syncwarp();
         // ---- phase 2b: diagonal block of sub-chunk I in fp32 (lane = channel)
         {
-            const int c = lane, I2 = warp;
-            const unsigned um = sm.unsafe_mask[I2];
-            const bool exact = (um >> c) & 1u;
-            for (int jr = 0; jr < SC; ++jr) {
-                const int j = I2 * SC + jr;
-                float sq_ = 0.f, sk_ = 0.f;
-                for (int sr = 0; sr <= jr; ++sr) {  // dq_j += sum_{s<=j} dP_js k_s e^{B_j-B_s}
-                    const int s = I2 * SC + sr;
-                    const float w = __bfloat162float(sm.dP[j][s]);
-                    if (!exact) sq_ += w * sm.kfD[s][c];
-                    else sq_ += w * __bfloat162float(sm.k[s][c]) * expf(sm.B[j][c] - sm.B[s][c]);
+            const int c = lane;
+            const bool exact = (sm.unsafe_mask[I] >> c) & 1u;
+            if (!exact) {
+                float kv[SC], qv[SC];
+#pragma unroll
+                for (int r = 0; r < SC; ++r) {
+                    kv[r] = __bfloat162float(S.k[I * SC + r][c]) * sm.kf[I * SC + r][c] * eSpan;  // k_s e^{rho-B_s}
+                    qv[r] = __bfloat162float(S.q[I * SC + r][c]) * sm.a[I * SC + r][c];          // q_j e^{B_j-rho}
                 }
-                for (int sr = jr; sr < SC; ++sr) {  // dk_j += sum_{s'>=j} dP_{s'j} q_s' e^{B_s'-B_j}
-                    const int s = I2 * SC + sr;
-                    const float w = __bfloat162float(sm.dP[s][j]);
-                    if (!exact) sk_ += w * sm.qf[s][c];
-                    else sk_ += w * __bfloat162float(sm.q[s][c]) * expf(sm.B[s][c] - sm.B[j][c]);
+#pragma unroll
+                for (int j = 0; j < SC; ++j) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int s_ = 0; s_ <= j; ++s_) acc = fmaf(sm.dg[I][j][s_], kv[s_], acc);
+                    sm.iq[I * SC + j][c] += sm.a[I * SC + j][c] * acc;
                 }
-                if (!exact) {
-                    sq_ *= sm.a[j][c];
-                    // e^{B_s' - B_j} = a_s' * D_I * kf_j
-                    sk_ *= sm.kf[j][c] * eSpan;
+#pragma unroll
+                for (int s_ = 0; s_ < SC; ++s_) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int j = s_; j < SC; ++j) acc = fmaf(sm.dgT[I][s_][j], qv[j], acc);
+                    sm.ik[I * SC + s_][c] += sm.kf[I * SC + s_][c] * eSpan * acc;
                 }
-                sm.iq[j][c] += sq_;
-                sm.ik[j][c] += sk_;
+            } else {  // rare: the decay span leaves the fp32 range; exact log-space terms
+                for (int j = 0; j < SC; ++j) {
+                    float acc = 0.f;
+                    for (int s_ = 0; s_ <= j; ++s_)
+                        acc += sm.dg[I][j][s_] * __bfloat162float(S.k[I * SC + s_][c]) * expf(b[j] - b[s_]);
+                    sm.iq[I * SC + j][c] += acc;
+                }
+                for (int s_ = 0; s_ < SC; ++s_) {
+                    float acc = 0.f;
+                    for (int j = s_; j < SC; ++j)
+                        acc += sm.dgT[I][s_][j] * __bfloat162float(S.q[I * SC + j][c]) * expf(b[j] - b[s_]);
+                    sm.ik[I * SC + s_][c] += acc;
+                }
             }
         }
         __syncthreads();
-        // ---- combine, gate gradient (thread: channel cl, rows of sub-chunk I)
+        // ---- combine and closed-form gate gradient (thread: channel cl, rows of sub-chunk I)
         {
             const float E = sm.EI[I][cl], F = sm.FI[I][cl];
             float rr[SC];
-            float rs = 0.f;
-            const int64_t ch = c0 + cl;
+            float rs = 0.f, ks = 0.f;
 #pragma unroll
             for (int r = 0; r < SC; ++r) {
                 const int row = I * SC + r;
-                const float dqv = sm.a[row][cl] * E * __bfloat162float(sm.dQt[row][cl]) + sm.iq[row][cl];
-                const float dkv = sm.kf[row][cl] * F * __bfloat162float(sm.dKt[row][cl]) + sm.ik[row][cl];
-                rr[r] = __bfloat162float(sm.q[row][cl]) * dqv - __bfloat162float(sm.k[row][cl]) * dkv;
+                const float qv = __bfloat162float(S.q[row][cl]), kv = __bfloat162float(S.k[row][cl]);
+                const float dQi = __bfloat162float(__ushort_as_bfloat16(hq[r]));
+                const float dKi = __bfloat162float(__ushort_as_bfloat16(hk[r]));
+                const float kt = kv * sm.kf[row][cl] * F;  // K~_j = k_j e^{Gamma - B_j}
+                const float dqv = sm.a[row][cl] * E * dQi + sm.iq[row][cl];
+                const float dkv = sm.kf[row][cl] * F * dKi + sm.ik[row][cl];
+                rr[r] = qv * dqv - kv * dkv;
                 rs += rr[r];
+                ks += kt * dKi;
                 if (row < nvalid) {
                     const int64_t off = (bh * L + t0 + row) * K + ch;
                     dq[off] = __float2bfloat16_rn(dqv);
@@ -434,9 +488,15 @@ __global__ void __launch_bounds__(256, 1)
                 }
             }
             sm.tot[I][cl] = rs;
+            sm.tot2[I][cl] = ks;
             __syncthreads();
-            float suf = sm.carry[cl];
-            for (int J = I + 1; J < NS; ++J) suf += sm.tot[J][cl];
+            // carry from all later chunks: sum_v D_i S_[i+1] = e^Gamma sum_v D_i S_[i] + sum_j K~_j dK~_j
+            float suf = sm.eG[cl] * xd;
+#pragma unroll
+            for (int J = 0; J < NS; ++J) {
+                suf += sm.tot2[J][cl];
+                if (J > I) suf += sm.tot[J][cl];
+            }
 #pragma unroll
             for (int r = SC - 1; r >= 0; --r) {
                 suf += rr[r];
@@ -444,8 +504,11 @@ __global__ void __launch_bounds__(256, 1)
                 if (row < nvalid) dla[(bh * L + t0 + row) * K + ch] = suf;
             }
         }
+        __syncthreads();
     }
 }
+
+}  // namespace
 
 bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
     const uint64_t dims[3] = {inner, rows, outer};
@@ -454,11 +517,9 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
     return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-}  // namespace
-
 gla_status tc_bwd_gemm_launch(const Problem& p, const void* dO, const void* v, const __nv_bfloat16* Sbuf,
                               const __nv_bfloat16* Dbuf, __nv_bfloat16* dP, __nv_bfloat16* dQt, __nv_bfloat16* dKt,
-                              cudaStream_t s) {
+                              float* xdot, cudaStream_t s) {
     CUtensorMap m[4];
     memset(m, 0, sizeof(m));
     const uint64_t L = uint64_t(p.L), K = uint64_t(p.K), V = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
@@ -469,22 +530,20 @@ gla_status tc_bwd_gemm_launch(const Problem& p, const void* dO, const void* v, c
     if (cudaFuncSetAttribute(k_bwd_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.K / 128), unsigned(p.BH));
-    GLA_LAUNCH("tc_bwd_gemm", k_bwd_gemm, grid, 192, smem, s, m[0], m[1], m[2], m[3], dP, dQt, dKt, p.L, p.N, p.K,
-               p.V, device_error_word());
+    GLA_LAUNCH("tc_bwd_gemm", k_bwd_gemm, grid, 192, smem, s, m[0], m[1], m[2], m[3], dP, dQt, dKt, xdot, p.L, p.N,
+               p.K, p.V, device_error_word());
     return GLA_OK;
 }
 
 gla_status tc_bwd_intra_launch(const Problem& p, const void* q, const void* k, const float* la,
                                const __nv_bfloat16* dP, const __nv_bfloat16* dQt, const __nv_bfloat16* dKt,
-                               const __nv_bfloat16* Sbuf, const __nv_bfloat16* Dbuf, const float* hT,
-                               const float* dhT, void* dq, void* dk, float* dla, cudaStream_t s) {
+                               const float* xdot, void* dq, void* dk, float* dla, cudaStream_t s) {
     const size_t smem = sizeof(IntraSmem);
     if (cudaFuncSetAttribute(k_bwd_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     GLA_LAUNCH("tc_bwd_intra", k_bwd_intra, dim3(unsigned(p.N), unsigned(p.BH)), 256, smem, s,
-               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, dP, dQt, dKt, Sbuf,
-               Dbuf, hT, dhT, static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K,
-               p.V);
+               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, dP, dQt, dKt, xdot,
+               static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K);
     return GLA_OK;
 }
 

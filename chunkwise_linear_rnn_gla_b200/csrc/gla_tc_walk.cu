@@ -54,20 +54,32 @@ struct Bars {
 
 // Deterministic ring cursor shared (by construction) by producer and MMA
 // issuer: both walk the same schedule and therefore see the same slots.
+template <int R>
 struct Cursor {
     int pos = 0;
     __device__ int take() {
         const int s = pos;
-        pos = (pos + 1) % RING;
+        pos = (pos + 1) % R;
         return s;
     }
     __device__ int take_pair() {  // two adjacent slots (constant LBO)
-        if (pos == RING - 1) pos = 0;
-        if (pos & 1) pos = (pos + 1) % RING;
+        if (pos == R - 1) pos = 0;
+        if (pos & 1) pos = (pos + 1) % R;
         const int s = pos;
-        pos = (pos + 2) % RING;
+        pos = (pos + 2) % R;
         return s;
     }
+};
+
+// Per-mode resources: ring pieces, bf16 state copies in smem, TMEM columns.
+template <int NH, int MODE>
+struct WalkCfg {
+    static constexpr int ring = MODE == kWalkStatesOnly ? 4 : RING;
+    static constexpr int s_bufs = MODE == kWalkStatesOnly ? 0 : 2;
+    static constexpr uint32_t tmem_cols = MODE == kWalkStatesOnly ? (NH == 1 ? 256u : 512u) : 512u;
+    // the states-only walk has no output epilogue (warps 6-9)
+    static constexpr int threads = MODE == kWalkStatesOnly ? 192 : kWalkThreads;
+    static constexpr int min_blocks = MODE == kWalkStatesOnly ? 2 : 1;
 };
 
 struct Sched {
@@ -117,19 +129,20 @@ template <int NH>
 __device__ __forceinline__ uint32_t col_O(int b) { return uint32_t(3 * NH * BV + b * BV); }
 
 template <int NH, bool REVERSE, bool PT, int MODE>
-__global__ void __launch_bounds__(kWalkThreads, 1)
+__global__ void __launch_bounds__(WalkCfg<NH, MODE>::threads, WalkCfg<NH, MODE>::min_blocks)
     k_walk(const __grid_constant__ CUtensorMap tmA1, const __grid_constant__ CUtensorMap tmB1,
            const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmP,
            const __grid_constant__ CUtensorMap tmS, const float* __restrict__ gam, const float* __restrict__ init,
            float* __restrict__ fin, float* __restrict__ fin2, __nv_bfloat16* __restrict__ Y,
            __nv_bfloat16* __restrict__ states, int64_t L, int64_t N, int64_t V, int64_t K, int* err) {
     constexpr int KC = NH * 128;  // key channels owned by this CTA
+    using Cfg = WalkCfg<NH, MODE>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = base;
-    uint8_t* vbuf = base + RING * PIECE;  // 2 x PIECE
-    uint8_t* sS = vbuf + 2 * PIECE;  // 2 x [KC x 64] bf16 copies of the state
-    Bars& bar = *reinterpret_cast<Bars*>(sS + 2 * KC * 128);
+    uint8_t* vbuf = base + Cfg::ring * PIECE;  // 2 x PIECE
+    uint8_t* sS = vbuf + 2 * PIECE;             // s_bufs x [KC x 64] bf16 copies of the state
+    Bars& bar = *reinterpret_cast<Bars*>(sS + Cfg::s_bufs * KC * 128);
     volatile int* abort_flag = &bar.abort_flag;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -145,7 +158,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < RING; ++s) {
+        for (int s = 0; s < Cfg::ring; ++s) {
             mbar_init(&bar.full[s], 1);
             mbar_init(&bar.empty[s], 1);
         }
@@ -167,7 +180,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&bar.tmem_slot, 512);
+        tmem_alloc(&bar.tmem_slot, Cfg::tmem_cols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -183,7 +196,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
             tma_prefetch(&tmB1);
             tma_prefetch(&tmA2);
             tma_prefetch(&tmP);
-            Cursor cur;
+            Cursor<Cfg::ring> cur;
             uint32_t par = 0;            // parity of the next use, one bit per slot
             uint32_t pending = 0;        // slots with a load whose completion nobody waited for yet
             uint32_t pending_par = 0;
@@ -238,7 +251,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
             }
             // on abort, wait (bounded) for loads still in flight before the block exits
             if (!ok) {
-                for (int s = 0; s < RING; ++s)
+                for (int s = 0; s < Cfg::ring; ++s)
                     if ((pending >> s) & 1u) mbar_wait(&bar.full[s], (pending_par >> s) & 1u, nullptr, abort_flag);
                 for (int vb = 0; vb < 2; ++vb)
                     if ((vpend >> (2 * vb)) & 1u)
@@ -251,7 +264,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
             const uint32_t idU = idesc_bf16_f32(128, BV, true, true);
             const uint32_t idQS = idesc_bf16_f32(128, BV, false, true);
             const uint32_t idPV = idesc_bf16_f32(128, BV, PT, true);
-            Cursor cur;
+            Cursor<Cfg::ring> cur;
             uint32_t par = 0;
             bool ok = true;
             auto wait_full = [&](int slot) -> bool {
@@ -340,16 +353,18 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
                     for (int e = 0; e < 16; ++e)
                         x[e] = init ? init[(bh * K + c) * V + v0 + c16 * 16 + e] : 0.f;
                     tmem_st16(tmem + lane_off + col_S<NH>() + uint32_t(h * BV + c16 * 16), x);
-                    uint8_t* row = sS + (c - kbase) * 128;
+                    if (MODE == kWalkFused) {  // only the fused walk keeps a bf16 copy in smem
+                        uint8_t* row = sS + (c - kbase) * 128;
 #pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        const int chunk = c16 * 2 + half;
-                        uint4 w;
-                        w.x = pack_bf16x2(x[half * 8 + 0], x[half * 8 + 1]);
-                        w.y = pack_bf16x2(x[half * 8 + 2], x[half * 8 + 3]);
-                        w.z = pack_bf16x2(x[half * 8 + 4], x[half * 8 + 5]);
-                        w.w = pack_bf16x2(x[half * 8 + 6], x[half * 8 + 7]);
-                        *reinterpret_cast<uint4*>(row + ((chunk ^ ((c - kbase) & 7)) * 16)) = w;
+                        for (int half = 0; half < 2; ++half) {
+                            const int chunk = c16 * 2 + half;
+                            uint4 w;
+                            w.x = pack_bf16x2(x[half * 8 + 0], x[half * 8 + 1]);
+                            w.y = pack_bf16x2(x[half * 8 + 2], x[half * 8 + 3]);
+                            w.z = pack_bf16x2(x[half * 8 + 4], x[half * 8 + 5]);
+                            w.w = pack_bf16x2(x[half * 8 + 6], x[half * 8 + 7]);
+                            *reinterpret_cast<uint4*>(row + ((chunk ^ ((c - kbase) & 7)) * 16)) = w;
+                        }
                     }
                     if (MODE == kWalkStatesOnly || states) {
                         __nv_bfloat16* dst = states + ((bh * N + chunk_of(0)) * K + c) * V + v0 + c16 * 16;
@@ -491,7 +506,7 @@ __global__ void __launch_bounds__(kWalkThreads, 1)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc(tmem, Cfg::tmem_cols);
     }
 }
 
@@ -506,14 +521,15 @@ template <int NH, bool REVERSE, bool PT, int MODE>
 gla_status launch_walk(const Problem& p, const WalkArgs& a, const CUtensorMap* maps, cudaStream_t s,
                        const char* name) {
     constexpr int KC = NH * 128;
+    using Cfg = WalkCfg<NH, MODE>;
     auto fn = k_walk<NH, REVERSE, PT, MODE>;
-    const size_t smem = 1024 + size_t(RING + 2) * PIECE + 2 * size_t(KC) * 128 + sizeof(Bars);
+    const size_t smem = 1024 + size_t(Cfg::ring + 2) * PIECE + size_t(Cfg::s_bufs) * KC * 128 + sizeof(Bars);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const unsigned gy = MODE == kWalkOutputOnly ? unsigned(p.N)
                         : MODE == kWalkStatesOnly ? unsigned(p.K / KC) : 1u;
     const dim3 grid(unsigned(p.V / BV), gy, unsigned(p.BH));
-    GLA_LAUNCH(name, fn, grid, kWalkThreads, smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], a.gam, a.init,
+    GLA_LAUNCH(name, fn, grid, Cfg::threads, smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], a.gam, a.init,
                a.fin, a.fin2, a.Y, a.states, p.L, p.N, p.V, p.K, device_error_word());
     return GLA_OK;
 }
