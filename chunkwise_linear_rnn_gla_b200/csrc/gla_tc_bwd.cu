@@ -247,21 +247,27 @@ struct IntraSmem {
     __nv_bfloat16 qh[C][QS], kh[C][QS];  // bf16 operands of the off-diagonal blocks
     float iq[C][KT + 1], ik[C][KT + 1];  // intra-chunk parts of dq, dk
     float d[28][KT];
-    float tot[NS][KT], tot2[NS][KT];
+    float h8[NS][2][KT];   // per half sub-chunk: gate sums, then r sums
+    float k8[NS][2][KT];   // per half sub-chunk: sum_j K~_j dK~_j
+    float first[NS][KT];   // B offset of each sub-chunk's first row within its half 0
     float EI[NS][KT], FI[NS][KT], DI[NS][KT];
     float eG[KT];
     unsigned unsafe_mask[NS];
 };
 
-// One CTA per (chunk, head); 8 warps, warp I <-> query/key sub-chunk I; key
-// channels in tiles of 32 (thread (channel = lane, sub-chunk = warp) in the
-// elementwise phases).
-__global__ void __launch_bounds__(256, 1)
+// One CTA per (chunk, head), 16 warps. Elementwise phases: thread (channel =
+// lane, sub-chunk I = warp % 8, half = warp / 8) owns rows 8*half .. 8*half+7
+// of sub-chunk I. Off-diagonal and diagonal blocks: warps 0-7 form the dq
+// side (query sub-chunk I = warp), warps 8-15 the dk side (key sub-chunk
+// J = warp - 8). Key channels are processed in tiles of 32.
+__global__ void __launch_bounds__(512, 1)
     k_bwd_intra(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                 const float* __restrict__ la, const __nv_bfloat16* __restrict__ dPg,
                 const __nv_bfloat16* __restrict__ dQt, const __nv_bfloat16* __restrict__ dKt,
                 const float* __restrict__ xdot, __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk,
                 float* __restrict__ dla, int64_t L, int64_t N, int64_t K) {
+    constexpr int NT = 512;
+    constexpr int HR = SC / 2;  // rows per half sub-chunk
     extern __shared__ __align__(16) unsigned char smem_raw[];
     IntraSmem& sm = *reinterpret_cast<IntraSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -269,19 +275,21 @@ __global__ void __launch_bounds__(256, 1)
     const int64_t t0 = i * C;
     const int nvalid = int(L - t0 < C ? L - t0 : C);
     const int g = lane >> 2, tq = lane & 3;
+    const int cl = lane, I = warp & 7, half = warp >> 3;
+    const int r0 = I * SC + half * HR;  // first row owned in the elementwise phases
 
-    for (int e = tid; e < C * C / 8; e += 256) {
+    for (int e = tid; e < C * C / 8; e += NT) {
         const int row = e / (C / 8), cc = (e % (C / 8)) * 8;
         cpa16(&sm.dP[row][cc], dPg + ((bh * N + i) * C + row) * C + cc, true);
     }
     auto issue = [&](int64_t c0, int sb) {
         IntraStage& S = sm.st[sb];
-        for (int e = tid; e < C * (KT / 4); e += 256) {
+        for (int e = tid; e < C * (KT / 4); e += NT) {
             const int row = e / (KT / 4), cc = (e % (KT / 4)) * 4;
             const bool ok = row < nvalid;
             cpa16(&S.la[row][cc], la + (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc, ok);
         }
-        for (int e = tid; e < C * (KT / 8); e += 256) {
+        for (int e = tid; e < C * (KT / 8); e += NT) {
             const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
             const bool ok = row < nvalid;
             const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc;
@@ -292,7 +300,6 @@ __global__ void __launch_bounds__(256, 1)
     };
     issue(0, 0);
     int sb = 0;
-    const int cl = lane, I = warp;
 
     for (int64_t c0 = 0; c0 < K; c0 += KT, sb ^= 1) {
         if (c0 + KT < K) {
@@ -303,7 +310,7 @@ __global__ void __launch_bounds__(256, 1)
         }
         __syncthreads();
         if (c0 == 0) {
-            for (int e = tid; e < NS * SC * SC; e += 256) {
+            for (int e = tid; e < NS * SC * SC; e += NT) {
                 const int I2 = e / (SC * SC), j = (e / SC) % SC, s_ = e % SC;
                 const float v = __bfloat162float(sm.dP[I2 * SC + j][I2 * SC + s_]);
                 sm.dg[I2][j][s_] = v;
@@ -313,70 +320,73 @@ __global__ void __launch_bounds__(256, 1)
         const IntraStage& S = sm.st[sb];
         const int64_t ch = c0 + cl;
         // inter-chunk parts of this thread's rows, used by the combine at the end
-        unsigned short hq[SC], hk[SC];
+        unsigned short hq[HR], hk[HR];
 #pragma unroll
-        for (int r = 0; r < SC; ++r) {
-            const int row = I * SC + r;
+        for (int r = 0; r < HR; ++r) {
+            const int row = r0 + r;
             const bool ok = row < nvalid;
             const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + ch;
             hq[r] = ok ? reinterpret_cast<const unsigned short*>(dQt)[off] : 0;
             hk[r] = ok ? reinterpret_cast<const unsigned short*>(dKt)[off] : 0;
         }
         const float xd = xdot[(bh * N + i) * K + ch];
-        // ---- phase 1: cumsum, factors, operands
-        float b[SC];
+        // ---- phase 1: cumsum over the half sub-chunk, factors, operands
+        float b[HR];
         float run = 0.f;
 #pragma unroll
-        for (int r = 0; r < SC; ++r) {
-            run += S.la[I * SC + r][cl];
-            b[r] = run;
+        for (int r = 0; r < HR; ++r) {
+            run += S.la[r0 + r][cl];
+            b[r] = run;  // cumsum within this half
         }
-        sm.tot[I][cl] = run;
+        sm.h8[I][half][cl] = run;
+        if (half == 0) sm.first[I][cl] = b[0];
         if (tid < NS) sm.unsafe_mask[tid] = 0u;
         __syncthreads();
-        float pre = 0.f, gamma = 0.f;
+        float pre = 0.f, gamma = 0.f, lastJ[NS];
 #pragma unroll
         for (int J = 0; J < NS; ++J) {
-            const float t = sm.tot[J][cl];
+            const float t = sm.h8[J][0][cl] + sm.h8[J][1][cl];
             if (J < I) pre += t;
             gamma += t;
+            lastJ[J] = gamma;  // B at the last row of sub-chunk J
         }
-        const float rho = pre + b[0], last = pre + b[SC - 1];
-        const float span = rho - last;
+        const float rho = pre + sm.first[I][cl];        // B at the first row of sub-chunk I
+        const float last = lastJ[I];
+        const float hoff = pre + (half ? sm.h8[I][0][cl] : 0.f);  // B offset of this half
+        const float span = fmaxf(rho - last, 0.f);
         const bool unsafe = span > kUnsafeSpan;
         const float eSpan = unsafe ? 0.f : __expf(span);
-        if (unsafe) atomicOr(&sm.unsafe_mask[I], 1u << cl);
-        sm.EI[I][cl] = __expf(rho);
-        sm.FI[I][cl] = __expf(gamma - last);
-        sm.DI[I][cl] = eSpan;
-        if (I == 0) sm.eG[cl] = __expf(gamma);
-        {
-            float lastJ = 0.f;
+        if (half == 0) {
+            if (unsafe) atomicOr(&sm.unsafe_mask[I], 1u << cl);
+            // every exponent below is <= 0 in exact arithmetic; the clamps only absorb the
+            // rounding of cumsums summed in different orders (|B| can reach ~1e32 for alpha = 0)
+            sm.EI[I][cl] = __expf(fminf(rho, 0.f));
+            sm.FI[I][cl] = __expf(fminf(gamma - last, 0.f));
+            sm.DI[I][cl] = eSpan;
+            if (I == 0) sm.eG[cl] = __expf(fminf(gamma, 0.f));
 #pragma unroll
-            for (int J = 0; J < NS - 1; ++J) {
-                lastJ += sm.tot[J][cl];
-                if (J < I) sm.d[pidx(I, J)][cl] = __expf(rho - lastJ);
-            }
+            for (int J = 0; J < NS - 1; ++J)
+                if (J < I) sm.d[pidx(I, J)][cl] = __expf(fminf(rho - lastJ[J], 0.f));
         }
 #pragma unroll
-        for (int r = 0; r < SC; ++r) {
-            const int row = I * SC + r;
-            const float Bv = pre + b[r];
-            const float av = __expf(Bv - rho), kv = __expf(last - Bv);
+        for (int r = 0; r < HR; ++r) {
+            const int row = r0 + r;
+            const float Bv = hoff + b[r];
+            const float av = __expf(fminf(Bv - rho, 0.f)), kv = __expf(fminf(last - Bv, 0.f));
             sm.a[row][cl] = av;
             sm.kf[row][cl] = kv;
             sm.qh[row][cl] = __float2bfloat16_rn(__bfloat162float(S.q[row][cl]) * av);
             sm.kh[row][cl] = __float2bfloat16_rn(__bfloat162float(S.k[row][cl]) * kv);
         }
         __syncthreads();
-        // ---- phase 2a: off-diagonal blocks on the tensor cores
-        {
-            float aq[4][4], ak[4][4];
+        // ---- phase 2: warps 0-7 dq side of sub-chunk I, warps 8-15 dk side of sub-chunk J = I
+        if (half == 0) {
+            // off-diagonal: dq_I += sum_{J<I} dP_IJ (K^_J * d_IJ)
+            float aq[4][4];
 #pragma unroll
             for (int n = 0; n < 4; ++n)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) aq[n][e] = ak[n][e] = 0.f;
-            // dq_I += sum_{J<I} dP_IJ (K^_J * d_IJ)
+                for (int e = 0; e < 4; ++e) aq[n][e] = 0.f;
             for (int J = 0; J < I; ++J) {
                 uint32_t A[4];
                 ldsm_x4(tc_smem_u32(&sm.dP[I * SC + (lane & 15)][J * SC + (lane >> 4) * 8]), A);
@@ -392,8 +402,55 @@ __global__ void __launch_bounds__(256, 1)
                     mma16816(aq[2 * nb2 + 1], A, scale2(Bf[2], f1), scale2(Bf[3], f1));
                 }
             }
-            // dk_J += sum_{I2>J} dP_{I2 J}^T (Q^_{I2} * d_{I2 J}), J = this warp
-            const int J = warp;
+#pragma unroll
+            for (int n = 0; n < 4; ++n) {
+                const int c = n * 8 + 2 * tq;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int row = I * SC + g + 8 * hh;
+                    sm.iq[row][c] = aq[n][2 * hh] * sm.a[row][c];
+                    sm.iq[row][c + 1] = aq[n][2 * hh + 1] * sm.a[row][c + 1];
+                }
+            }
+            __syncwarp();
+            // diagonal block in fp32 (lane = channel)
+            const int c = lane;
+            const bool exact = (sm.unsafe_mask[I] >> c) & 1u;
+            if (!exact) {
+                float kv[SC];
+#pragma unroll
+                for (int r = 0; r < SC; ++r)
+                    kv[r] = __bfloat162float(S.k[I * SC + r][c]) * sm.kf[I * SC + r][c] * eSpan;  // k_s e^{rho-B_s}
+#pragma unroll
+                for (int j = 0; j < SC; ++j) {
+                    float acc = 0.f;
+#pragma unroll
+                    for (int s_ = 0; s_ <= j; ++s_) acc = fmaf(sm.dg[I][j][s_], kv[s_], acc);
+                    sm.iq[I * SC + j][c] += sm.a[I * SC + j][c] * acc;
+                }
+            } else {  // rare: the decay span leaves the fp32 range; exact log-space terms
+                float Bj[SC];
+                float run2 = 0.f;
+                for (int r = 0; r < I * SC; ++r) run2 += S.la[r][c];
+                for (int r = 0; r < SC; ++r) {
+                    run2 += S.la[I * SC + r][c];
+                    Bj[r] = run2;
+                }
+                for (int j = 0; j < SC; ++j) {
+                    float acc = 0.f;
+                    for (int s_ = 0; s_ <= j; ++s_)
+                        acc += sm.dg[I][j][s_] * __bfloat162float(S.k[I * SC + s_][c]) * expf(fminf(Bj[j] - Bj[s_], 0.f));
+                    sm.iq[I * SC + j][c] += acc;
+                }
+            }
+        } else {
+            // off-diagonal: dk_J += sum_{I2>J} dP_{I2 J}^T (Q^_{I2} * d_{I2 J}), J = I
+            const int J = I;
+            float ak[4][4];
+#pragma unroll
+            for (int n = 0; n < 4; ++n)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) ak[n][e] = 0.f;
             for (int I2 = J + 1; I2 < NS; ++I2) {
                 uint32_t A[4];
                 ldsm_x4_t(tc_smem_u32(&sm.dP[I2 * SC + (lane & 7) + (lane >> 4) * 8][J * SC + ((lane >> 3) & 1) * 8]), A);
@@ -414,93 +471,84 @@ __global__ void __launch_bounds__(256, 1)
                 const int c = n * 8 + 2 * tq;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    const int row = warp * SC + g + 8 * hh;
-                    sm.iq[row][c] = aq[n][2 * hh] * sm.a[row][c];
-                    sm.iq[row][c + 1] = aq[n][2 * hh + 1] * sm.a[row][c + 1];
+                    const int row = J * SC + g + 8 * hh;
                     sm.ik[row][c] = ak[n][2 * hh] * sm.kf[row][c];
                     sm.ik[row][c + 1] = ak[n][2 * hh + 1] * sm.kf[row][c + 1];
                 }
             }
-        }
-        __syncwarp();
-        // ---- phase 2b: diagonal block of sub-chunk I in fp32 (lane = channel)
-        {
+            __syncwarp();
             const int c = lane;
-            const bool exact = (sm.unsafe_mask[I] >> c) & 1u;
+            const bool exact = (sm.unsafe_mask[J] >> c) & 1u;
+            const float Dv = sm.DI[J][c];
             if (!exact) {
-                float kv[SC], qv[SC];
+                float qv[SC];
 #pragma unroll
-                for (int r = 0; r < SC; ++r) {
-                    kv[r] = __bfloat162float(S.k[I * SC + r][c]) * sm.kf[I * SC + r][c] * eSpan;  // k_s e^{rho-B_s}
-                    qv[r] = __bfloat162float(S.q[I * SC + r][c]) * sm.a[I * SC + r][c];          // q_j e^{B_j-rho}
-                }
-#pragma unroll
-                for (int j = 0; j < SC; ++j) {
-                    float acc = 0.f;
-#pragma unroll
-                    for (int s_ = 0; s_ <= j; ++s_) acc = fmaf(sm.dg[I][j][s_], kv[s_], acc);
-                    sm.iq[I * SC + j][c] += sm.a[I * SC + j][c] * acc;
-                }
+                for (int r = 0; r < SC; ++r)
+                    qv[r] = __bfloat162float(S.q[J * SC + r][c]) * sm.a[J * SC + r][c];  // q_j e^{B_j-rho}
 #pragma unroll
                 for (int s_ = 0; s_ < SC; ++s_) {
                     float acc = 0.f;
 #pragma unroll
-                    for (int j = s_; j < SC; ++j) acc = fmaf(sm.dgT[I][s_][j], qv[j], acc);
-                    sm.ik[I * SC + s_][c] += sm.kf[I * SC + s_][c] * eSpan * acc;
+                    for (int j = s_; j < SC; ++j) acc = fmaf(sm.dgT[J][s_][j], qv[j], acc);
+                    sm.ik[J * SC + s_][c] += sm.kf[J * SC + s_][c] * Dv * acc;
                 }
-            } else {  // rare: the decay span leaves the fp32 range; exact log-space terms
-                for (int j = 0; j < SC; ++j) {
-                    float acc = 0.f;
-                    for (int s_ = 0; s_ <= j; ++s_)
-                        acc += sm.dg[I][j][s_] * __bfloat162float(S.k[I * SC + s_][c]) * expf(b[j] - b[s_]);
-                    sm.iq[I * SC + j][c] += acc;
+            } else {
+                float Bj[SC];
+                float run2 = 0.f;
+                for (int r = 0; r < J * SC; ++r) run2 += S.la[r][c];
+                for (int r = 0; r < SC; ++r) {
+                    run2 += S.la[J * SC + r][c];
+                    Bj[r] = run2;
                 }
                 for (int s_ = 0; s_ < SC; ++s_) {
                     float acc = 0.f;
                     for (int j = s_; j < SC; ++j)
-                        acc += sm.dgT[I][s_][j] * __bfloat162float(S.q[I * SC + j][c]) * expf(b[j] - b[s_]);
-                    sm.ik[I * SC + s_][c] += acc;
+                        acc += sm.dgT[J][s_][j] * __bfloat162float(S.q[J * SC + j][c]) * expf(fminf(Bj[j] - Bj[s_], 0.f));
+                    sm.ik[J * SC + s_][c] += acc;
                 }
             }
         }
         __syncthreads();
-        // ---- combine and closed-form gate gradient (thread: channel cl, rows of sub-chunk I)
+        // ---- combine and closed-form gate gradient (thread: channel cl, rows r0 .. r0+7)
         {
             const float E = sm.EI[I][cl], F = sm.FI[I][cl];
-            float rr[SC];
+            float rr[HR];
             float rs = 0.f, ks = 0.f;
 #pragma unroll
-            for (int r = 0; r < SC; ++r) {
-                const int row = I * SC + r;
+            for (int r = 0; r < HR; ++r) {
+                const int row = r0 + r;
                 const float qv = __bfloat162float(S.q[row][cl]), kv = __bfloat162float(S.k[row][cl]);
                 const float dQi = __bfloat162float(__ushort_as_bfloat16(hq[r]));
                 const float dKi = __bfloat162float(__ushort_as_bfloat16(hk[r]));
-                const float kt = kv * sm.kf[row][cl] * F;  // K~_j = k_j e^{Gamma - B_j}
+                const float eGB = sm.kf[row][cl] * F;  // e^{Gamma - B_j}
                 const float dqv = sm.a[row][cl] * E * dQi + sm.iq[row][cl];
-                const float dkv = sm.kf[row][cl] * F * dKi + sm.ik[row][cl];
+                const float dkv = eGB * dKi + sm.ik[row][cl];
                 rr[r] = qv * dqv - kv * dkv;
                 rs += rr[r];
-                ks += kt * dKi;
+                ks += kv * eGB * dKi;  // K~_j dK~_j
                 if (row < nvalid) {
                     const int64_t off = (bh * L + t0 + row) * K + ch;
                     dq[off] = __float2bfloat16_rn(dqv);
                     dk[off] = __float2bfloat16_rn(dkv);
                 }
             }
-            sm.tot[I][cl] = rs;
-            sm.tot2[I][cl] = ks;
+            __syncthreads();  // everyone is done reading the gate sums in h8
+            sm.h8[I][half][cl] = rs;
+            sm.k8[I][half][cl] = ks;
             __syncthreads();
             // carry from all later chunks: sum_v D_i S_[i+1] = e^Gamma sum_v D_i S_[i] + sum_j K~_j dK~_j
             float suf = sm.eG[cl] * xd;
 #pragma unroll
-            for (int J = 0; J < NS; ++J) {
-                suf += sm.tot2[J][cl];
-                if (J > I) suf += sm.tot[J][cl];
-            }
+            for (int J = 0; J < NS; ++J)
 #pragma unroll
-            for (int r = SC - 1; r >= 0; --r) {
+                for (int hh = 0; hh < 2; ++hh) {
+                    suf += sm.k8[J][hh][cl];
+                    if (J > I || (J == I && hh > half)) suf += sm.h8[J][hh][cl];
+                }
+#pragma unroll
+            for (int r = HR - 1; r >= 0; --r) {
                 suf += rr[r];
-                const int row = I * SC + r;
+                const int row = r0 + r;
                 if (row < nvalid) dla[(bh * L + t0 + row) * K + ch] = suf;
             }
         }
@@ -541,7 +589,7 @@ gla_status tc_bwd_intra_launch(const Problem& p, const void* q, const void* k, c
     const size_t smem = sizeof(IntraSmem);
     if (cudaFuncSetAttribute(k_bwd_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    GLA_LAUNCH("tc_bwd_intra", k_bwd_intra, dim3(unsigned(p.N), unsigned(p.BH)), 256, smem, s,
+    GLA_LAUNCH("tc_bwd_intra", k_bwd_intra, dim3(unsigned(p.N), unsigned(p.BH)), 512, smem, s,
                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, dP, dQt, dKt, xdot,
                static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K);
     return GLA_OK;

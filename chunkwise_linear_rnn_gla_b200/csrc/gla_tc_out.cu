@@ -7,9 +7,11 @@
 // owns a 64-column tile of one head and loops over all chunks; every operand
 // of a chunk (A: 2K/128 pieces, X: K/128 pieces, Pm: 2 pieces, B: 1 piece, each
 // 128 rows x 128 bytes with the 128-byte swizzle) streams through one TMA ring
-// and is released by the MMAs of its own chunk, so the loads of the next
-// chunks overlap the current chunk's tcgen05 work. The fp32 accumulator is
-// double-buffered in TMEM and drained by four epilogue warps.
+// in the order the MMAs consume it; each group of four k-steps waits only for
+// its own pieces and releases them as soon as its MMAs complete, so the ring
+// stays full and the loads of later chunks overlap the current chunk's
+// tcgen05 work. The fp32 accumulator is double-buffered in TMEM and drained
+// by four epilogue warps.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -62,7 +64,6 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     k_chunk_out(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
                 const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmB,
                 __nv_bfloat16* __restrict__ Y, int64_t L, int64_t N, int64_t V, int* err) {
-    constexpr int K = NH * 128;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     OutBars& bar = *reinterpret_cast<OutBars*>(ring + RING * PIECE);
@@ -118,8 +119,10 @@ __global__ void __launch_bounds__(kOutThreads, 1)
             for (int it = 0; it < n_items && ok; ++it) {
                 const int i = chunk_of(it);
                 const int zs = int(bh * N + i);
-                for (int pc = 0; pc < 2 * NH && ok; ++pc) ok = load(cur.take(), &tmA, 64 * pc, i * C, int(bh));
-                for (int h = 0; h < NH && ok; ++h) ok = load(cur.take(), &tmX, v0, 128 * h, zs);
+                for (int h = 0; h < NH && ok; ++h) {  // X_h, then the two A pieces that pair with it
+                    ok = load(cur.take(), &tmX, v0, 128 * h, zs);
+                    for (int sub = 0; sub < 2 && ok; ++sub) ok = load(cur.take(), &tmA, 64 * (2 * h + sub), i * C, int(bh));
+                }
                 if (ok) {
                     const int sp = cur.take_pair();
                     ok = load(sp, &tmP, 0, 0, zs) && load(sp + 1, &tmP, 64, 0, zs);
@@ -144,25 +147,31 @@ __global__ void __launch_bounds__(kOutThreads, 1)
             bool ok = true;
             for (int it = 0; it < n_items && ok; ++it) {
                 const int b = it & 1;
-                int sa[2 * NH], sx[NH];
-                for (int pc = 0; pc < 2 * NH; ++pc) sa[pc] = cur.take();
-                for (int h = 0; h < NH; ++h) sx[h] = cur.take();
+                const uint32_t d = tmem + uint32_t(b * BV);
+                ok = mbar_wait(&bar.o_empty[b], uint32_t(((it >> 1) & 1) ^ 1), err, abort_flag);
+                for (int h = 0; h < NH && ok; ++h) {
+                    const int sx = cur.take();
+                    if (!(ok = wait_full(sx))) break;
+                    for (int sub = 0; sub < 2; ++sub) {
+                        const int sa = cur.take();
+                        if (!(ok = wait_full(sa))) break;
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(ring + sa * PIECE);
+                        const uint32_t x0 = smem_u32(ring + sx * PIECE) + sub * 64 * 128;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_bf16(d, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(x0 + kk * 2048, 16, 1024), idQS,
+                                     (h > 0 || sub > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&bar.empty[sa]);
+                    }
+                    if (ok) mma_commit(&bar.empty[sx]);
+                }
+                if (!ok) break;
                 const int sp = cur.take_pair();
                 const int sb = cur.take();
-                ok = mbar_wait(&bar.o_empty[b], uint32_t(((it >> 1) & 1) ^ 1), err, abort_flag);
-                for (int pc = 0; pc < 2 * NH && ok; ++pc) ok = wait_full(sa[pc]);
-                for (int h = 0; h < NH && ok; ++h) ok = wait_full(sx[h]);
-                if (ok) ok = wait_full(sp) && wait_full(sp + 1) && wait_full(sb);
+                ok = wait_full(sp) && wait_full(sp + 1) && wait_full(sb);
                 if (!ok) break;
                 tc_fence_after();
-                const uint32_t d = tmem + uint32_t(b * BV);
-#pragma unroll
-                for (int kk = 0; kk < K / 16; ++kk) {
-                    const int pc = kk / 4;  // 64-channel piece of A; its rows live in X piece pc/2
-                    const uint32_t a0 = smem_u32(ring + sa[pc] * PIECE) + (kk % 4) * 32;
-                    const uint32_t x0 = smem_u32(ring + sx[pc / 2] * PIECE) + (pc % 2) * 64 * 128 + (kk % 4) * 2048;
-                    mma_bf16(d, sdesc_sw128(a0, 16, 1024), sdesc_sw128(x0, 16, 1024), idQS, kk > 0 ? 1u : 0u);
-                }
                 const uint32_t p0 = smem_u32(ring + sp * PIECE);
                 const uint32_t b0 = smem_u32(ring + sb * PIECE);
 #pragma unroll
@@ -172,8 +181,6 @@ __global__ void __launch_bounds__(kOutThreads, 1)
                     mma_bf16(d, ad, sdesc_sw128(b0 + kk * 2048, 16, 1024), idPV, 1u);
                 }
                 mma_commit(&bar.o_full[b]);
-                for (int pc = 0; pc < 2 * NH; ++pc) mma_commit(&bar.empty[sa[pc]]);
-                for (int h = 0; h < NH; ++h) mma_commit(&bar.empty[sx[h]]);
                 mma_commit(&bar.empty[sp]);
                 mma_commit(&bar.empty[sp + 1]);
                 mma_commit(&bar.empty[sb]);

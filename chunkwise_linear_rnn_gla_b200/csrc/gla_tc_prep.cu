@@ -82,13 +82,12 @@ struct Stage {  // raw inputs of one channel tile, filled by cp.async
     __nv_bfloat16 k[C][KT];
 };
 
+constexpr int TS = C + 4;  // row stride of the transposed fp32 operands (16-byte aligned rows)
+
 struct PrepSmem {
-    Stage st[2];
-    __nv_bfloat16 qo[C][KT];  // Q~ / K~ tiles staged for coalesced stores
-    __nv_bfloat16 ko[C][KT];
-    float B[C][KT];
-    float qf[C][KT + 1];
-    float kf[C][KT + 1];
+    Stage st;
+    float qfT[KT][TS];  // q_jc e^{B_jc - rho_I}, channel-major for vector loads
+    float kfT[KT][TS];  // k_sc e^{rho_I - B_sc} (0 for channels that need the exact path)
     __nv_bfloat16 qh[C][QS];
     __nv_bfloat16 kh[C][QS];
     float tot[NS][KT];
@@ -96,12 +95,14 @@ struct PrepSmem {
     unsigned unsafe_mask[NS];
 };
 
-__global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict__ q,
-                                                 const __nv_bfloat16* __restrict__ k,
-                                                 const float* __restrict__ la, __nv_bfloat16* __restrict__ Qt,
-                                                 __nv_bfloat16* __restrict__ Kt, __nv_bfloat16* __restrict__ P,
-                                                 float* __restrict__ gam, float* __restrict__ Bout, int64_t L,
-                                                 int64_t K, int64_t N) {
+// One CTA per (chunk, head), 8 warps; warp I owns query sub-chunk I. Two CTAs
+// fit per SM so one CTA's loads overlap the other's arithmetic.
+__global__ void __launch_bounds__(256, 2) k_tc_prep(const __nv_bfloat16* __restrict__ q,
+                                                    const __nv_bfloat16* __restrict__ k,
+                                                    const float* __restrict__ la, __nv_bfloat16* __restrict__ Qt,
+                                                    __nv_bfloat16* __restrict__ Kt, __nv_bfloat16* __restrict__ P,
+                                                    float* __restrict__ gam, float* __restrict__ Bout, int64_t L,
+                                                    int64_t K, int64_t N) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     PrepSmem& sm = *reinterpret_cast<PrepSmem*>(smem_raw);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -125,35 +126,28 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
         for (int b = 0; b < 4; ++b) dg[a][b] = 0.f;
     const int I = warp;
     const int jr0 = 2 * (lane >> 2), s0 = 4 * (lane & 3);
-    // async copy of channel tile [c0, c0+KT) into stage buffer `sb`
-    auto issue = [&](int64_t c0, int sb) {
-        Stage& S = sm.st[sb];
-        for (int e = tid; e < C * (KT / 4); e += 256) {  // log a: 8 x 16 B per row
-            const int row = e / (KT / 4), cc = (e % (KT / 4)) * 4;
-            const bool ok = row < nvalid;
-            cp_async16(&S.la[row][cc], la + (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc, ok);
-        }
-        for (int e = tid; e < C * (KT / 8); e += 256) {  // q, k: 4 x 16 B per row
-            const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
-            const bool ok = row < nvalid;
-            const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc;
-            cp_async16(&S.q[row][cc], q + off, ok);
-            cp_async16(&S.k[row][cc], k + off, ok);
-        }
-        cp_async_commit();
-    };
-    issue(0, 0);
-    int sb = 0;
 
-    for (int64_t c0 = 0; c0 < K; c0 += KT, sb ^= 1) {
-        if (c0 + KT < K) {
-            issue(c0 + KT, sb ^ 1);
-            cp_async_wait_1();
-        } else {
+    for (int64_t c0 = 0; c0 < K; c0 += KT) {
+        // ---- stage the raw tile [128 rows x 32 channels]
+        {
+            Stage& S = sm.st;
+            for (int e = tid; e < C * (KT / 4); e += 256) {  // log a: 8 x 16 B per row
+                const int row = e / (KT / 4), cc = (e % (KT / 4)) * 4;
+                const bool ok = row < nvalid;
+                cp_async16(&S.la[row][cc], la + (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc, ok);
+            }
+            for (int e = tid; e < C * (KT / 8); e += 256) {  // q, k: 4 x 16 B per row
+                const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
+                const bool ok = row < nvalid;
+                const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc;
+                cp_async16(&S.q[row][cc], q + off, ok);
+                cp_async16(&S.k[row][cc], k + off, ok);
+            }
+            cp_async_commit();
             cp_async_wait_0();
         }
         __syncthreads();
-        const Stage& S = sm.st[sb];
+        const Stage& S = sm.st;
         // ---- phase 1: thread (channel cl, sub-chunk I) cumsum, factors, operands
         const int cl = lane;
         const int64_t ch = c0 + cl;
@@ -176,9 +170,10 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
         }
         const float rho = pre + b[0];
         const float last = pre + b[SC - 1];
-        const float eRho = __expf(rho);            // <= 1
-        const float eGl = __expf(gamma - last);     // <= 1
-        const float span = rho - last;              // >= 0
+        // exponents are <= 0 in exact arithmetic; the clamps absorb cumsum rounding
+        const float eRho = __expf(fminf(rho, 0.f));           // <= 1
+        const float eGl = __expf(fminf(gamma - last, 0.f));    // <= 1
+        const float span = fmaxf(rho - last, 0.f);             // >= 0
         const bool unsafe = span > kUnsafeSpan;
         const float eSpan = unsafe ? 0.f : __expf(span);
         if (unsafe) atomicOr(&sm.unsafe_mask[I], 1u << cl);
@@ -188,39 +183,32 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
 #pragma unroll
             for (int J = 0; J < NS - 1; ++J) {
                 lastJ += sm.tot[J][cl];
-                if (J < I) sm.d[pair_index(I, J)][cl] = __expf(rho - lastJ);
+                if (J < I) sm.d[pair_index(I, J)][cl] = __expf(fminf(rho - lastJ, 0.f));
             }
         }
-        if (I == 0 && gam) gam[(bh * N + i) * K + ch] = __expf(gamma);
+        if (I == 0 && gam) gam[(bh * N + i) * K + ch] = __expf(fminf(gamma, 0.f));
 #pragma unroll
         for (int r = 0; r < SC; ++r) {
             const int row = I * SC + r;
             const float B = pre + b[r];
-            sm.B[row][cl] = B;
             const float qv = __bfloat162float(S.q[row][cl]);
             const float kv = __bfloat162float(S.k[row][cl]);
-            const float a = __expf(B - rho);     // e^{B_j - rho_I} <= 1
-            const float kfac = __expf(last - B); // e^{last_I - B_j} <= 1
+            const float a = __expf(fminf(B - rho, 0.f));     // e^{B_j - rho_I} <= 1
+            const float kfac = __expf(fminf(last - B, 0.f)); // e^{last_I - B_j} <= 1
             const float qhat = qv * a;
             const float khat = kv * kfac;
             sm.qh[row][cl] = __float2bfloat16_rn(qhat);
             sm.kh[row][cl] = __float2bfloat16_rn(khat);
-            sm.qf[row][cl] = qhat;
-            sm.kf[row][cl] = unsafe ? 0.f : khat * eSpan;
-            sm.qo[row][cl] = __float2bfloat16_rn(qhat * eRho);
-            sm.ko[row][cl] = __float2bfloat16_rn(khat * eGl);
-            if (Bout && row < nvalid) Bout[(bh * L + t0 + row) * K + ch] = B;
-        }
-        __syncthreads();
-        // coalesced 16-byte stores of the Q~ and K~ tiles
-        for (int e = tid; e < C * (KT / 8); e += 256) {
-            const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
+            sm.qfT[cl][row] = qhat;
+            sm.kfT[cl][row] = unsafe ? 0.f : khat * eSpan;
             if (row < nvalid) {
-                const int64_t off = (bh * L + t0 + row) * K + c0 + cc;
-                *reinterpret_cast<uint4*>(Qt + off) = *reinterpret_cast<const uint4*>(&sm.qo[row][cc]);
-                *reinterpret_cast<uint4*>(Kt + off) = *reinterpret_cast<const uint4*>(&sm.ko[row][cc]);
+                const int64_t off = (bh * L + t0 + row) * K + ch;
+                Qt[off] = __float2bfloat16_rn(qhat * eRho);
+                Kt[off] = __float2bfloat16_rn(khat * eGl);
+                if (Bout) Bout[off] = B;
             }
         }
+        __syncthreads();
 
         // ---- phase 2a: off-diagonal blocks on the tensor cores
 #pragma unroll
@@ -254,36 +242,45 @@ __global__ void __launch_bounds__(256) k_tc_prep(const __nv_bfloat16* __restrict
         // ---- phase 2b: diagonal block (I,I) in fp32 on the CUDA cores
 #pragma unroll 8
         for (int c = 0; c < KT; ++c) {
-            const float qa = sm.qf[I * SC + jr0][c], qb = sm.qf[I * SC + jr0 + 1][c];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float kv = sm.kf[I * SC + s0 + e][c];
-                dg[0][e] += qa * kv;
-                dg[1][e] += qb * kv;
-            }
+            const float2 qa = *reinterpret_cast<const float2*>(&sm.qfT[c][I * SC + jr0]);
+            const float4 kb = *reinterpret_cast<const float4*>(&sm.kfT[c][I * SC + s0]);
+            dg[0][0] = fmaf(qa.x, kb.x, dg[0][0]);
+            dg[0][1] = fmaf(qa.x, kb.y, dg[0][1]);
+            dg[0][2] = fmaf(qa.x, kb.z, dg[0][2]);
+            dg[0][3] = fmaf(qa.x, kb.w, dg[0][3]);
+            dg[1][0] = fmaf(qa.y, kb.x, dg[1][0]);
+            dg[1][1] = fmaf(qa.y, kb.y, dg[1][1]);
+            dg[1][2] = fmaf(qa.y, kb.z, dg[1][2]);
+            dg[1][3] = fmaf(qa.y, kb.w, dg[1][3]);
         }
         const unsigned um = sm.unsafe_mask[I];
         if (um) {  // rare: channels whose decay span inside the sub-chunk leaves the fp32 range
             for (int c = 0; c < KT; ++c) {
                 if (!((um >> c) & 1u)) continue;
+                // per-chunk cumsum of this channel, recomputed from the staged gates
+                float Bj[SC];
+                float run2 = 0.f;
+                for (int r = 0; r < I * SC; ++r) run2 += S.la[r][c];
+                for (int r = 0; r < SC; ++r) {
+                    run2 += S.la[I * SC + r][c];
+                    Bj[r] = run2;
+                }
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
-                    const int j = I * SC + jr0 + a;
-                    if (j >= nvalid) continue;
-                    const float qv = __bfloat162float(q[(bh * L + t0 + j) * K + c0 + c]);
+                    const int jr = jr0 + a;
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int s = I * SC + s0 + e;
-                        if (s > j) continue;
-                        const float kv = __bfloat162float(k[(bh * L + t0 + s) * K + c0 + c]);
-                        dg[a][e] += qv * kv * expf(sm.B[j][c] - sm.B[s][c]);
+                        const int sr = s0 + e;
+                        if (sr > jr) continue;
+                        const float qv = __bfloat162float(S.q[I * SC + jr][c]);
+                        const float kv = __bfloat162float(S.k[I * SC + sr][c]);
+                        dg[a][e] += qv * kv * expf(fminf(Bj[jr] - Bj[sr], 0.f));
                     }
                 }
             }
         }
         __syncthreads();
     }
-
     // ---- write P (bf16, [128 x 128], zero above the diagonal)
     __nv_bfloat16* Pc = P + (bh * N + i) * C * C;
     const int g = lane >> 2, t = lane & 3;
