@@ -102,6 +102,28 @@ def kernel_models(w, C):
     return m
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
+# ncu capture of the default workload, with the SHA-1 of the kernel's source
+# file at capture time: a kernel whose source changed since reports null.
+NCU_TRAFFIC = {}
+
+
+def measured_traffic(name):
+    ent = NCU_TRAFFIC.get(name)
+    if not ent:
+        return None
+    nbytes, src, sha = ent
+    try:
+        import hashlib
+
+        with open(os.path.join(ROOT, "chunkwise_linear_rnn_gla_b200", "csrc", src), "rb") as f:
+            if hashlib.sha1(f.read()).hexdigest() != sha:
+                return None
+    except OSError:
+        return None
+    return nbytes
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock/throttle sampling during the timed region."""
@@ -200,7 +222,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="gla1p3b_fwdbwd")
     ap.add_argument("--kernel-impl", default="auto", choices=["auto", "simt", "tc"])
-    ap.add_argument("--state-mode", default="auto", choices=["auto", "materialized", "nonmaterialized"])
+    ap.add_argument("--state-mode", default="materialized", choices=["auto", "materialized", "nonmaterialized"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
@@ -364,6 +386,8 @@ def main():
                         "unit": "TFLOP/s", "frac": round(ach / pk, 4), "traffic": None}
             roof["peak_source"] = peaks_src
             roof["launch_ms"] = round(ms / n, 4)
+            roof["traffic"] = measured_traffic(name)
+            roof["alg_bytes"] = mdl["bytes"]
 
     alg = algorithmic_model(w, C)
     t_roof = max(alg["bytes"] / (peaks["hbm_gbs"] * 1e9), alg["flops"] / (peaks["bf16_tflops"] * 1e12))

@@ -49,6 +49,13 @@ struct WalkArgs {
 
 gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, const char* name);
 
+// Materialised state walk on [128 x 128] tiles with the state accumulated in
+// TMEM (gla_tc_states.cu); requires d_v % 128 == 0.
+bool tc_states_walk_supported(const Problem& p);
+gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
+                                 const float* init, float* fin, float* fin2, __nv_bfloat16* states, bool reverse,
+                                 cudaStream_t s, const char* name);
+
 // Chunk-parallel Y_i = A_i X_i + Pm_i B_i from stored bf16 chunk states X
 // (gla_tc_out.cu): forward o (A = Q~, Pm = P) and dv (A = K~, Pm = P^T).
 gla_status tc_chunk_out_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* X,

@@ -101,7 +101,9 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
     }
     a.states = b.states;
     a.mode = kWalkStatesOnly;
-    st = tc_walk_launch(p, a, s, "tc_walk_states");
+    st = tc_states_walk_supported(p)
+             ? tc_states_walk_launch(p, b.Kt, a.B1, b.gam, h0, hT, b.hT, b.states, false, s, "tc_walk_states")
+             : tc_walk_launch(p, a, s, "tc_walk_states");
     if (st != GLA_OK) return st;
     return tc_chunk_out_launch(p, b.Qt, b.states, b.P, static_cast<const __nv_bfloat16*>(v), false,
                                static_cast<__nv_bfloat16*>(o), s, "tc_output");
@@ -127,7 +129,9 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
         a.fin = b.hT;
         a.states = b.states;
         a.mode = kWalkStatesOnly;
-        st = tc_walk_launch(p, a, s, "tc_walk_states");
+        st = tc_states_walk_supported(p)
+                 ? tc_states_walk_launch(p, b.Kt, a.B1, b.gam, h0, b.hT, nullptr, b.states, false, s, "tc_walk_states")
+                 : tc_walk_launch(p, a, s, "tc_walk_states");
         if (st != GLA_OK) return st;
     }
     {
@@ -150,7 +154,9 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
             if (st != GLA_OK) return st;
         } else {
             a.mode = kWalkStatesOnly;
-            st = tc_walk_launch(p, a, s, "tc_walk_dstates");
+            st = tc_states_walk_supported(p) ? tc_states_walk_launch(p, b.Qt, a.B1, b.gam, dhT, dh0, nullptr, b.Dbuf,
+                                                                     true, s, "tc_walk_dstates")
+                                             : tc_walk_launch(p, a, s, "tc_walk_dstates");
             if (st != GLA_OK) return st;
             st = tc_chunk_out_launch(p, b.Kt, b.Dbuf, b.P, static_cast<const __nv_bfloat16*>(dO), true,
                                      static_cast<__nv_bfloat16*>(dv), s, "tc_output_dv");

@@ -424,8 +424,15 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
                 for (int j = 0; j < SC; ++j) {
                     float acc = 0.f;
+                    const float4* row4 = reinterpret_cast<const float4*>(sm.dg[I][j]);
 #pragma unroll
-                    for (int s_ = 0; s_ <= j; ++s_) acc = fmaf(sm.dg[I][j][s_], kv[s_], acc);
+                    for (int q4 = 0; q4 <= j / 4; ++q4) {  // broadcast 16-byte loads of the dP row
+                        const float4 w = row4[q4];
+                        if (4 * q4 + 0 <= j) acc = fmaf(w.x, kv[4 * q4 + 0], acc);
+                        if (4 * q4 + 1 <= j) acc = fmaf(w.y, kv[4 * q4 + 1], acc);
+                        if (4 * q4 + 2 <= j) acc = fmaf(w.z, kv[4 * q4 + 2], acc);
+                        if (4 * q4 + 3 <= j) acc = fmaf(w.w, kv[4 * q4 + 3], acc);
+                    }
                     sm.iq[I * SC + j][c] += sm.a[I * SC + j][c] * acc;
                 }
             } else {  // rare: the decay span leaves the fp32 range; exact log-space terms
@@ -488,8 +495,15 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
                 for (int s_ = 0; s_ < SC; ++s_) {
                     float acc = 0.f;
+                    const float4* row4 = reinterpret_cast<const float4*>(sm.dgT[J][s_]);
 #pragma unroll
-                    for (int j = s_; j < SC; ++j) acc = fmaf(sm.dgT[J][s_][j], qv[j], acc);
+                    for (int q4 = s_ / 4; q4 < SC / 4; ++q4) {
+                        const float4 w = row4[q4];
+                        if (4 * q4 + 0 >= s_) acc = fmaf(w.x, qv[4 * q4 + 0], acc);
+                        if (4 * q4 + 1 >= s_) acc = fmaf(w.y, qv[4 * q4 + 1], acc);
+                        if (4 * q4 + 2 >= s_) acc = fmaf(w.z, qv[4 * q4 + 2], acc);
+                        if (4 * q4 + 3 >= s_) acc = fmaf(w.w, qv[4 * q4 + 3], acc);
+                    }
                     sm.ik[J * SC + s_][c] += sm.kf[J * SC + s_][c] * Dv * acc;
                 }
             } else {

@@ -32,7 +32,7 @@ using namespace tc;
 constexpr int C = kTcChunk;
 constexpr int BV = kTcBV;
 constexpr uint32_t PIECE = 16384;
-constexpr int RING = 12;
+constexpr int RING = 6;  // >= the 3 pieces one MMA group holds; two CTAs fit per SM
 constexpr int kOutThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
 
 struct OutBars {
@@ -60,7 +60,7 @@ struct OutCursor {
 };
 
 template <int NH, bool PT>
-__global__ void __launch_bounds__(kOutThreads, 1)
+__global__ void __launch_bounds__(kOutThreads, 2)
     k_chunk_out(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
                 const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmB,
                 __nv_bfloat16* __restrict__ Y, int64_t L, int64_t N, int64_t V, int* err) {
@@ -234,9 +234,9 @@ gla_status launch_out(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, 
     const size_t smem = 1024 + size_t(RING) * PIECE + sizeof(OutBars);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    // one wave of CTAs (one per SM at this shared-memory size); each walks every gy-th chunk
+    // one wave of CTAs (two per SM at this shared-memory size); each walks every gy-th chunk
     const int64_t tiles = (p.V / BV) * p.BH;
-    int64_t gy = 148 / tiles;
+    int64_t gy = 296 / tiles;
     if (gy > p.N) gy = p.N;
     if (gy < 1) gy = 1;
     const dim3 grid(unsigned(p.V / BV), unsigned(gy), unsigned(p.BH));
