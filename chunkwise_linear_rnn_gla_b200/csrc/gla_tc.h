@@ -16,10 +16,10 @@ constexpr int kTcChunk = 128;  // C on the tensor-core path
 constexpr int kTcSub = 16;     // secondary chunk c
 constexpr int kTcBV = 64;      // value columns per walk CTA
 
-// Chunk-parallel gate preparation (gla_tc_prep.cu).
-size_t tc_prep_smem_bytes();
+// Chunk-parallel gate preparation (gla_tc_prep.cu): Q~, K~, e^Gamma and the
+// masked intra-chunk scores P.
 gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const float* la, __nv_bfloat16* Qt,
-                          __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, float* Bout, cudaStream_t s);
+                          __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, cudaStream_t s);
 
 // Row-gated chunk walk (gla_tc_walk.cu). State X [K x 64-column tile] with the
 // gate on its rows. Per chunk i (in walk order):
@@ -62,12 +62,10 @@ gla_status tc_chunk_out_launch(const Problem& p, const __nv_bfloat16* A, const _
                                const __nv_bfloat16* Pm, const __nv_bfloat16* Bv, bool p_transposed,
                                __nv_bfloat16* Y, cudaStream_t s, const char* name);
 
-// Backward, chunk-parallel part (gla_tc_bwd.cu).
-gla_status tc_bwd_gemm_launch(const Problem& p, const void* dO, const void* v, const __nv_bfloat16* Sbuf,
-                              const __nv_bfloat16* Dbuf, __nv_bfloat16* dP, __nv_bfloat16* dQt, __nv_bfloat16* dKt,
-                              float* xdot, cudaStream_t s);
-gla_status tc_bwd_intra_launch(const Problem& p, const void* q, const void* k, const float* la,
-                               const __nv_bfloat16* dP, const __nv_bfloat16* dQt, const __nv_bfloat16* dKt,
-                               const float* xdot, void* dq, void* dk, float* dla, cudaStream_t s);
+// Backward, chunk-parallel part (gla_tc_bwd.cu): dq, dk and dlog a from dO, v,
+// the stored states S_[i] and D_i, Q~ and e^Gamma.
+gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
+                               const void* v, const __nv_bfloat16* Qt, const float* gam, const __nv_bfloat16* Sbuf,
+                               const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, cudaStream_t s);
 
 }  // namespace gla

@@ -13,8 +13,8 @@
 //   tc_walk_dv         reverse walk: D_i chain, dv = K~ D_i + P^T dO, writes D_i
 //                      (materialised mode: tc_walk_dstates writes D_i, then the
 //                      chunk-parallel tc_output_dv computes dv)
-//   tc_bwd_gemm        dP = dO v^T, dQ~ = dO S_[i]^T, dK~ = v D_i^T (tcgen05)
-//   tc_bwd_intra       intra-chunk gradients, dq, dk, closed-form dlog a
+//   tc_bwd_chunk       dP = dO v^T, dQ~ = dO S_[i]^T, dK~ = v D_i^T and the
+//                      intra-chunk terms on tcgen05, dq, dk, closed-form dlog a
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -30,8 +30,7 @@ struct TcBuffers {
     __nv_bfloat16 *Qt, *Kt, *P;
     float *gam, *hT;
     __nv_bfloat16* states;
-    __nv_bfloat16 *Dbuf, *dP, *dQt, *dKt;
-    float* xdot;  // sum_v D_i * S_[i] per chunk and key channel
+    __nv_bfloat16* Dbuf;
 };
 
 // The backward layout extends the forward's, so a forward workspace can be
@@ -45,13 +44,7 @@ TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
     b.hT = a.take<float>(size_t(p.BH * p.K * p.V));
     if (bwd || p.state_mode == GLA_STATE_MATERIALIZED)
         b.states = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
-    if (bwd) {
-        b.Dbuf = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
-        b.dP = a.take<__nv_bfloat16>(size_t(p.BH * p.N * kTcChunk * kTcChunk));
-        b.dQt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
-        b.dKt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
-        b.xdot = a.take<float>(size_t(p.BH * p.N * p.K));
-    }
+    if (bwd) b.Dbuf = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
     return b;
 }
 
@@ -83,7 +76,7 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
                   void* o, float* hT, Arena& ws, cudaStream_t s) {
     TcBuffers b = carve(p, ws, false);
     if (ws.used > ws.cap) return GLA_ERR_WORKSPACE;
-    gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, nullptr, s);
+    gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, s);
     if (st != GLA_OK) return st;
     WalkArgs a{};
     a.A1 = b.Kt;
@@ -117,7 +110,7 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
     const bool reuse = (p.flags & GLA_FLAG_WS_FROM_FWD) != 0;
     gla_status st;
     if (!reuse) {
-        st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, nullptr, s);
+        st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, s);
         if (st != GLA_OK) return st;
     }
     if (!(reuse && p.state_mode == GLA_STATE_MATERIALIZED)) {
@@ -163,9 +156,7 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
             if (st != GLA_OK) return st;
         }
     }
-    st = tc_bwd_gemm_launch(p, dO, v, b.states, b.Dbuf, b.dP, b.dQt, b.dKt, b.xdot, s);
-    if (st != GLA_OK) return st;
-    return tc_bwd_intra_launch(p, q, k, la, b.dP, b.dQt, b.dKt, b.xdot, dq, dk, dla, s);
+    return tc_bwd_chunk_launch(p, q, k, la, dO, v, b.Qt, b.gam, b.states, b.Dbuf, dq, dk, dla, s);
 }
 
 }  // namespace gla

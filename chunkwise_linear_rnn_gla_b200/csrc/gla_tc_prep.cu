@@ -1,30 +1,36 @@
-// Chunk-parallel preparation for the tensor-core path (bf16 inputs, C = 128,
-// secondary chunk c = 16, so 8 sub-chunks per chunk).
+// Chunk-parallel preparation for the tensor-core path (bf16 inputs, C = 128).
 //
 // For every chunk i of every head this kernel computes, once:
 //   B_j   = sum_{r<=j} log a_r          per-chunk inclusive gate cumsum (fp32)
 //   Q~_j  = q_j * e^{B_j}               (bf16, operand of the inter-chunk output GEMM)
 //   K~_j  = k_j * e^{Gamma - B_j}       (bf16, operand of the state-update GEMM)
-//   e^Gamma                             (fp32 per key channel)
-//   P_js  = sum_c q_jc k_sc e^{B_jc - B_sc} for s <= j (bf16 [128 x 128])
-// P is built with two-level (secondary) chunking ("Gated Linear Attention
-// Transformers with Hardware-Efficient Training", atlas.scime.ai summary,
-// section "Approach": "two-level (secondary) chunking so most intra-chunk
-// matmuls use half-precision tensor cores"):
-//  * off-diagonal sub-chunk blocks (query sub-chunk I > key sub-chunk J) are
-//    bf16 tensor-core GEMMs of gate-rescaled operands
-//        P_IJ = (q_I * e^{B_I - rho_I}) (k_J * e^{last_J - B_J} * e^{rho_I - last_J})^T
-//    with rho_I = B at the first row of I and last_J = B at the last row of
-//    J; every factor is <= 1, so nothing overflows whatever the gates;
-//  * diagonal blocks are fp32 sums on the CUDA cores,
-//        P_js = sum_c (q_jc e^{B_jc - rho_I}) (k_sc e^{last_I - B_sc} e^{rho_I - last_I}),
-//    and for a channel whose within-sub-chunk decay span rho_I - last_I
-//    exceeds 80 (where e^{span} would leave the fp32 range) the terms are
-//    computed one by one as q_jc k_sc exp(B_jc - B_sc) (log space).
-// The exponentials are shared: every per-row factor is one exp of a
-// non-positive log-space difference, and Q~, K~ reuse them through
-// per-sub-chunk factors (e^{rho_I}, e^{Gamma - last_I}).
+//   e^Gamma                             (fp32 per key channel, Gamma = B at the chunk's last row)
+//   P_js  = sum_c q_jc k_sc e^{B_jc - B_sc} for s <= j, 0 above (bf16 [128 x 128])
+//
+// The intra-chunk scores follow the chunk form of the gated recurrence
+// ("Gated Linear Attention Transformers with Hardware-Efficient Training",
+// atlas.scime.ai summary, "Approach"): P = (q * e^B)(k * e^{-B})^T, masked.
+// The pages split this into 16-row secondary chunks so that the factors never
+// leave the half-precision range. Here the range is bounded per key channel
+// instead: when Gamma_c >= -64, every e^{+-B_jc} lies in [e^-64, e^64], so the
+// whole 128 x 128 block is ONE tcgen05 GEMM over the key channels,
+//     P = Q~ K^0^T,   K^0_s = k_s * e^{-B_s} = K~_s * e^{-Gamma},
+// with bf16 operands (the same relative rounding as the secondary-chunk
+// products: each term of the sum is q k e^{B_j - B_s} up to two bf16
+// roundings). A channel whose chunk decay exceeds the bound (Gamma_c < -64,
+// e.g. a gate of exactly 0) gets a zero K^0 column, and its terms are added on
+// the CUDA cores one by one as q_jc k_sc exp(B_jc - B_sc) (log space).
+//
+// Roles (one CTA per chunk, 288 threads, two CTAs per SM): warps 0-7 (warp
+// I = rows 16I .. 16I+15, lane = a pair of adjacent key channels) load log a,
+// q and k of one 64-channel piece straight into registers (8-, 4- and 4-byte
+// coalesced loads), do the cumsum and the elementwise work, write Q~/K~ to HBM
+// and the swizzled operand piece to shared memory; warp 8 owns TMEM and issues
+// the four MMAs of each piece as soon as it is complete (operand pieces are
+// double-buffered); at the end warps 0-7 read P back from TMEM (warp w: lanes
+// 32(w%4).., columns 64(w/4) ..) and store it.
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -35,298 +41,273 @@
 namespace gla {
 namespace {
 
-constexpr int C = 128;   // chunk
-constexpr int SC = 16;   // sub-chunk
-constexpr int NS = 8;    // sub-chunks per chunk
-constexpr int KT = 32;   // key channels per tile
-constexpr int QS = KT + 8;  // bf16 row stride of the mma operands (conflict-free ldmatrix)
-constexpr float kUnsafeSpan = 80.f;
+using namespace tc;
 
-__device__ __forceinline__ void ldmatrix_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
-                 : "r"(addr));
-}
+constexpr int C = kTcChunk;
+constexpr int KP = 64;                      // key channels per piece
+constexpr uint32_t PIECE = 16384;           // one [128 x 64] bf16 operand piece
+constexpr int kThreads = 288;
+constexpr float kSafeDecay = 64.f;          // |B| bound for the tensor-core form
 
-__device__ __forceinline__ void mma_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
-                                          uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t scale_bf16x2(uint32_t v, float s0, float s1) {
-    __nv_bfloat162 h = *reinterpret_cast<__nv_bfloat162*>(&v);
-    float2 f = __bfloat1622float2(h);
-    __nv_bfloat162 r = __floats2bfloat162_rn(f.x * s0, f.y * s1);
-    return *reinterpret_cast<uint32_t*>(&r);
-}
-
-// Pair index of (I, J), J < I, in [0, 28).
-__host__ __device__ constexpr int pair_index(int I, int J) { return I * (I - 1) / 2 + J; }
-
-// cp.async 16-byte copy with zero fill when `valid` is false
-__device__ __forceinline__ void cp_async16(void* dst, const void* src, bool valid) {
-    const uint32_t n = valid ? 16u : 0u;
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(tc_smem_u32(dst)), "l"(src), "r"(n) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
-
-struct Stage {  // raw inputs of one channel tile, filled by cp.async
-    float la[C][KT];
-    __nv_bfloat16 q[C][KT];
-    __nv_bfloat16 k[C][KT];
+struct PrepBars {
+    float tot[2][8][KP];  // per-piece, per 16-row segment gate sums (first: 8-byte aligned)
+    uint64_t ops_ready[2], mma_done[2], p_done, drain;
+    uint32_t tmem_slot;
+    int abort_flag;
+    int nuns;
+    unsigned short uns[256];  // key channels that take the exact path
 };
 
-constexpr int TS = C + 4;  // row stride of the transposed fp32 operands (16-byte aligned rows)
+constexpr uint32_t kTabOff = 4 * PIECE + (uint32_t(sizeof(PrepBars)) + 15u) / 16u * 16u;  // exact-path tables
 
-struct PrepSmem {
-    Stage st;
-    float qfT[KT][TS];  // q_jc e^{B_jc - rho_I}, channel-major for vector loads
-    float kfT[KT][TS];  // k_sc e^{rho_I - B_sc} (0 for channels that need the exact path)
-    __nv_bfloat16 qh[C][QS];
-    __nv_bfloat16 kh[C][QS];
-    float tot[NS][KT];
-    float d[28][KT];
-    unsigned unsafe_mask[NS];
-};
+// byte offset of (row, channel c64 of a piece) in a K-major SW128 piece
+__device__ __forceinline__ uint32_t piece_off(int row, int c64) {
+    return uint32_t(row) * 128u + uint32_t(((c64 >> 3) ^ (row & 7)) << 4) + uint32_t(c64 & 7) * 2u;
+}
 
-// One CTA per (chunk, head), 8 warps; warp I owns query sub-chunk I. Two CTAs
-// fit per SM so one CTA's loads overlap the other's arithmetic.
-__global__ void __launch_bounds__(256, 2) k_tc_prep(const __nv_bfloat16* __restrict__ q,
-                                                    const __nv_bfloat16* __restrict__ k,
-                                                    const float* __restrict__ la, __nv_bfloat16* __restrict__ Qt,
-                                                    __nv_bfloat16* __restrict__ Kt, __nv_bfloat16* __restrict__ P,
-                                                    float* __restrict__ gam, float* __restrict__ Bout, int64_t L,
-                                                    int64_t K, int64_t N) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    PrepSmem& sm = *reinterpret_cast<PrepSmem*>(smem_raw);
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t i = blockIdx.x, bh = blockIdx.y;
-    const int64_t t0 = i * C;
+__global__ void __launch_bounds__(kThreads, 2)
+    k_tc_prep(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const float* __restrict__ la,
+              __nv_bfloat16* __restrict__ Qt, __nv_bfloat16* __restrict__ Kt, __nv_bfloat16* __restrict__ P,
+              float* __restrict__ gam, int64_t L, int64_t K, int64_t N, int* err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // operand buffers: [b][Q~ piece, K^0 piece], b = piece parity
+    PrepBars& bar = *reinterpret_cast<PrepBars*>(base + 4 * PIECE);
+    volatile int* abort_flag = &bar.abort_flag;
+    const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+    const int i = blockIdx.x;
+    const int64_t bh = blockIdx.y;
+    const int64_t t0 = int64_t(i) * C;
     const int nvalid = int(L - t0 < C ? L - t0 : C);
+    const int npiece = int(K / KP);
 
-    // off-diagonal accumulators: warp I owns query sub-chunk I, key blocks J < I
-    float acc[NS - 1][2][4];
-#pragma unroll
-    for (int J = 0; J < NS - 1; ++J)
-#pragma unroll
-        for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[J][nb][e] = 0.f;
-    // diagonal accumulators: rows jr0, jr0+1; cols s0..s0+3 of block (I,I)
-    float dg[2][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-        for (int b = 0; b < 4; ++b) dg[a][b] = 0.f;
-    const int I = warp;
-    const int jr0 = 2 * (lane >> 2), s0 = 4 * (lane & 3);
+    if (tid == 0) {
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar.ops_ready[b], 256);
+            mbar_init(&bar.mma_done[b], 1);
+        }
+        mbar_init(&bar.p_done, 1);
+        mbar_init(&bar.drain, 1);
+        bar.abort_flag = 0;
+        bar.nuns = 0;
+        fence_barrier_init();
+    }
+    if (warp == 8) {
+        tmem_alloc(&bar.tmem_slot, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar.tmem_slot;
 
-    for (int64_t c0 = 0; c0 < K; c0 += KT) {
-        // ---- stage the raw tile [128 rows x 32 channels]
-        {
-            Stage& S = sm.st;
-            for (int e = tid; e < C * (KT / 4); e += 256) {  // log a: 8 x 16 B per row
-                const int row = e / (KT / 4), cc = (e % (KT / 4)) * 4;
-                const bool ok = row < nvalid;
-                cp_async16(&S.la[row][cc], la + (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc, ok);
+    if (warp == 8) {
+        if (lane == 0) {
+            const uint32_t id = idesc_bf16_f32(128, 128, false, false);
+            bool ok = true;
+            for (int t = 0; t < npiece && ok; ++t) {
+                const int b = t & 1;
+                ok = mbar_wait(&bar.ops_ready[b], uint32_t((t >> 1) & 1), err, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t a0 = smem_u32(base + b * 2 * PIECE), b0 = a0 + PIECE;
+#pragma unroll
+                for (int kk = 0; kk < KP / 16; ++kk)
+                    mma_bf16(tmem, sdesc_sw128(a0 + kk * 32, 16, 1024), sdesc_sw128(b0 + kk * 32, 16, 1024), id,
+                             (t > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bar.mma_done[b]);
             }
-            for (int e = tid; e < C * (KT / 8); e += 256) {  // q, k: 4 x 16 B per row
-                const int row = e / (KT / 8), cc = (e % (KT / 8)) * 8;
-                const bool ok = row < nvalid;
-                const int64_t off = (bh * L + t0 + (ok ? row : 0)) * K + c0 + cc;
-                cp_async16(&S.q[row][cc], q + off, ok);
-                cp_async16(&S.k[row][cc], k + off, ok);
+            if (ok) mma_commit(&bar.p_done);
+            mma_commit(&bar.drain);
+            mbar_drain(&bar.drain, 0);
+        }
+    } else {
+        const int I = warp;
+        const int cp = 2 * lane;  // channel pair within the piece
+        // Every compute thread passes every named barrier, also after a wait gave up (bar.sync
+        // has no time limit); a failed wait only skips the work.
+        bool ok = true;
+        for (int t = 0; t < npiece; ++t) {
+            const int b = t & 1;
+            const int64_t ch = int64_t(KP) * t + cp;
+            // rows past the end of the sequence (last chunk) read the last valid row and are zeroed
+            const int64_t rb = (bh * L + t0) * K + ch;
+            const float* lap = la + rb;
+            const __nv_bfloat16* qp = q + rb;
+            const __nv_bfloat16* kp = k + rb;
+            float2 bb[16];
+            uint32_t qv[16], kv[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int row = 16 * I + r;
+                const bool v = row < nvalid;
+                const uint32_t o = uint32_t(v ? row : nvalid - 1) * uint32_t(K);
+                const float2 l2 = *reinterpret_cast<const float2*>(lap + o);
+                const uint32_t qq = *reinterpret_cast<const uint32_t*>(qp + o);
+                const uint32_t kk = *reinterpret_cast<const uint32_t*>(kp + o);
+                // gate cumsums in base-2 units: e^x = 2^(x log2 e)
+                bb[r] = v ? make_float2(l2.x * kLog2e, l2.y * kLog2e) : make_float2(0.f, 0.f);
+                qv[r] = v ? qq : 0u;
+                kv[r] = v ? kk : 0u;
             }
-            cp_async_commit();
-            cp_async_wait_0();
-        }
-        __syncthreads();
-        const Stage& S = sm.st;
-        // ---- phase 1: thread (channel cl, sub-chunk I) cumsum, factors, operands
-        const int cl = lane;
-        const int64_t ch = c0 + cl;
-        float b[SC];
-        float run = 0.f;
+            float2 run = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int r = 0; r < SC; ++r) {
-            run += S.la[I * SC + r][cl];
-            b[r] = run;
-        }
-        sm.tot[I][cl] = run;
-        if (tid < NS) sm.unsafe_mask[tid] = 0u;
-        __syncthreads();
-        float pre = 0.f, gamma = 0.f;
-#pragma unroll
-        for (int J = 0; J < NS; ++J) {
-            const float t = sm.tot[J][cl];
-            if (J < I) pre += t;
-            gamma += t;
-        }
-        const float rho = pre + b[0];
-        const float last = pre + b[SC - 1];
-        // exponents are <= 0 in exact arithmetic; the clamps absorb cumsum rounding
-        const float eRho = __expf(fminf(rho, 0.f));           // <= 1
-        const float eGl = __expf(fminf(gamma - last, 0.f));    // <= 1
-        const float span = fmaxf(rho - last, 0.f);             // >= 0
-        const bool unsafe = span > kUnsafeSpan;
-        const float eSpan = unsafe ? 0.f : __expf(span);
-        if (unsafe) atomicOr(&sm.unsafe_mask[I], 1u << cl);
-        // pair factors e^{rho_I - last_J} for J < I (last_J = cumsum through sub-chunk J)
-        {
-            float lastJ = 0.f;
-#pragma unroll
-            for (int J = 0; J < NS - 1; ++J) {
-                lastJ += sm.tot[J][cl];
-                if (J < I) sm.d[pair_index(I, J)][cl] = __expf(fminf(rho - lastJ, 0.f));
+            for (int r = 0; r < 16; ++r) {
+                run.x += bb[r].x;
+                run.y += bb[r].y;
+                bb[r] = run;
             }
-        }
-        if (I == 0 && gam) gam[(bh * N + i) * K + ch] = __expf(fminf(gamma, 0.f));
+            *reinterpret_cast<float2*>(&bar.tot[b][I][cp]) = run;
+            named_sync(1, 256);
+            float2 pre = make_float2(0.f, 0.f), gamma = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int r = 0; r < SC; ++r) {
-            const int row = I * SC + r;
-            const float B = pre + b[r];
-            const float qv = __bfloat162float(S.q[row][cl]);
-            const float kv = __bfloat162float(S.k[row][cl]);
-            const float a = __expf(fminf(B - rho, 0.f));     // e^{B_j - rho_I} <= 1
-            const float kfac = __expf(fminf(last - B, 0.f)); // e^{last_I - B_j} <= 1
-            const float qhat = qv * a;
-            const float khat = kv * kfac;
-            sm.qh[row][cl] = __float2bfloat16_rn(qhat);
-            sm.kh[row][cl] = __float2bfloat16_rn(khat);
-            sm.qfT[cl][row] = qhat;
-            sm.kfT[cl][row] = unsafe ? 0.f : khat * eSpan;
-            if (row < nvalid) {
-                const int64_t off = (bh * L + t0 + row) * K + ch;
-                Qt[off] = __float2bfloat16_rn(qhat * eRho);
-                Kt[off] = __float2bfloat16_rn(khat * eGl);
-                if (Bout) Bout[off] = B;
-            }
-        }
-        __syncthreads();
-
-        // ---- phase 2a: off-diagonal blocks on the tensor cores
-#pragma unroll
-        for (int ks = 0; ks < KT / 16; ++ks) {
-            uint32_t a0, a1, a2, a3;
-            {
-                const int row = I * SC + (lane & 15);
-                const int col = ks * 16 + (lane >> 4) * 8;
-                ldmatrix_x4(tc_smem_u32(&sm.qh[row][col]), a0, a1, a2, a3);
-            }
-            const int t = lane & 3;
-            const int ca = ks * 16 + 2 * t, cb = ks * 16 + 8 + 2 * t;
-#pragma unroll
-            for (int J = 0; J < NS - 1; ++J) {
+            for (int J = 0; J < 8; ++J) {
+                const float2 v = *reinterpret_cast<const float2*>(&bar.tot[b][J][cp]);
                 if (J < I) {
-                    uint32_t b0, b1, b2, b3;
-                    const int row = J * SC + (lane & 7) + ((lane >> 4) << 3);
-                    const int col = ks * 16 + ((lane >> 3) & 1) * 8;
-                    ldmatrix_x4(tc_smem_u32(&sm.kh[row][col]), b0, b1, b2, b3);
-                    const float* dd = sm.d[pair_index(I, J)];
-                    const float dA = dd[ca], dB = dd[ca + 1], dC = dd[cb], dD = dd[cb + 1];
-                    b0 = scale_bf16x2(b0, dA, dB);
-                    b1 = scale_bf16x2(b1, dC, dD);
-                    b2 = scale_bf16x2(b2, dA, dB);
-                    b3 = scale_bf16x2(b3, dC, dD);
-                    mma_16816(acc[J][0], a0, a1, a2, a3, b0, b1);
-                    mma_16816(acc[J][1], a0, a1, a2, a3, b2, b3);
+                    pre.x += v.x;
+                    pre.y += v.y;
+                }
+                gamma.x += v.x;
+                gamma.y += v.y;
+            }
+            const bool unsafe0 = gamma.x < -kSafeDecay * kLog2e, unsafe1 = gamma.y < -kSafeDecay * kLog2e;
+            const float eNG0 = unsafe0 ? 0.f : exp2_ftz(fmaxf(-gamma.x, 0.f));  // e^{-Gamma} <= e^64
+            const float eNG1 = unsafe1 ? 0.f : exp2_ftz(fmaxf(-gamma.y, 0.f));
+            if (I == 0) {
+                *reinterpret_cast<float2*>(gam + (bh * N + i) * K + ch) =
+                    make_float2(exp2_ftz(fminf(gamma.x, 0.f)), exp2_ftz(fminf(gamma.y, 0.f)));
+                if (unsafe0) bar.uns[atomicAdd(&bar.nuns, 1)] = (unsigned short)ch;
+                if (unsafe1) bar.uns[atomicAdd(&bar.nuns, 1)] = (unsigned short)(ch + 1);
+            }
+            // the operand buffer of this parity is free once the MMAs of piece t-2 are done
+            if (t >= 2) ok = ok && mbar_wait(&bar.mma_done[b], uint32_t(((t >> 1) - 1) & 1), err, abort_flag);
+            uint8_t* opQ = base + b * 2 * PIECE;
+            uint8_t* opK = opQ + PIECE;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const int row = 16 * I + r;
+                const float Bx = pre.x + bb[r].x, By = pre.y + bb[r].y;
+                const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qv[r]));
+                const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kv[r]));
+                // exponents are <= 0 in exact arithmetic; the clamps absorb cumsum rounding
+                const float qt0 = qf.x * exp2_ftz(fminf(Bx, 0.f)), qt1 = qf.y * exp2_ftz(fminf(By, 0.f));
+                const float kt0 = kf.x * exp2_ftz(fminf(gamma.x - Bx, 0.f));
+                const float kt1 = kf.y * exp2_ftz(fminf(gamma.y - By, 0.f));
+                const uint32_t qh = pack_bf16x2(qt0, qt1);
+                const uint32_t o = piece_off(row, cp);
+                if (ok) {
+                    *reinterpret_cast<uint32_t*>(opQ + o) = qh;
+                    *reinterpret_cast<uint32_t*>(opK + o) = pack_bf16x2(kt0 * eNG0, kt1 * eNG1);
+                }
+                if (row < nvalid) {
+                    const int64_t off = (bh * L + t0 + row) * K + ch;
+                    *reinterpret_cast<uint32_t*>(Qt + off) = qh;
+                    *reinterpret_cast<uint32_t*>(Kt + off) = pack_bf16x2(kt0, kt1);
                 }
             }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar.ops_ready[b]);
         }
-        // ---- phase 2b: diagonal block (I,I) in fp32 on the CUDA cores
-#pragma unroll 8
-        for (int c = 0; c < KT; ++c) {
-            const float2 qa = *reinterpret_cast<const float2*>(&sm.qfT[c][I * SC + jr0]);
-            const float4 kb = *reinterpret_cast<const float4*>(&sm.kfT[c][I * SC + s0]);
-            dg[0][0] = fmaf(qa.x, kb.x, dg[0][0]);
-            dg[0][1] = fmaf(qa.x, kb.y, dg[0][1]);
-            dg[0][2] = fmaf(qa.x, kb.z, dg[0][2]);
-            dg[0][3] = fmaf(qa.x, kb.w, dg[0][3]);
-            dg[1][0] = fmaf(qa.y, kb.x, dg[1][0]);
-            dg[1][1] = fmaf(qa.y, kb.y, dg[1][1]);
-            dg[1][2] = fmaf(qa.y, kb.z, dg[1][2]);
-            dg[1][3] = fmaf(qa.y, kb.w, dg[1][3]);
-        }
-        const unsigned um = sm.unsafe_mask[I];
-        if (um) {  // rare: channels whose decay span inside the sub-chunk leaves the fp32 range
-            for (int c = 0; c < KT; ++c) {
-                if (!((um >> c) & 1u)) continue;
-                // per-chunk cumsum of this channel, recomputed from the staged gates
-                float Bj[SC];
-                float run2 = 0.f;
-                for (int r = 0; r < I * SC; ++r) run2 += S.la[r][c];
-                for (int r = 0; r < SC; ++r) {
-                    run2 += S.la[I * SC + r][c];
-                    Bj[r] = run2;
-                }
-#pragma unroll
-                for (int a = 0; a < 2; ++a) {
-                    const int jr = jr0 + a;
+        named_sync(1, 256);  // the list of exact-path channels is complete
+        // ---- P from TMEM: thread = row, 64 columns
+        const int q4 = warp & 3, h = warp >> 2;
+        const int row = 32 * q4 + lane;
+        // tcgen05.ld is warp-collective: the condition must be the same for the whole warp
+        const bool have = __all_sync(0xffffffffu, ok && mbar_wait(&bar.p_done, 0, err, abort_flag));
+        const int nuns = bar.nuns;  // the same for every compute thread
+        // exact terms of the channels beyond the bound, accumulated column-major in
+        // X[col][row] (fp32, the operand memory, free once P is complete); 8 channels per
+        // round, warp w building the cumsum / q / k columns of one of them
+        float* X = reinterpret_cast<float*>(base);
+        float* tabB = reinterpret_cast<float*>(base + kTabOff);
+        float* tabQ = tabB + 8 * C;
+        float* tabK = tabQ + 8 * C;
+        if (nuns > 0) {
+            if (have)
+                for (int jj = 0; jj < 64; ++jj) X[(64 * h + jj) * C + row] = 0.f;
+            for (int b0 = 0; b0 < nuns; b0 += 8) {
+                named_sync(1, 256);
+                const int u = b0 + warp;
+                if (have && u < nuns) {
+                    const int ch = bar.uns[u];
+                    float a[4], qa[4], ka[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int sr = s0 + e;
-                        if (sr > jr) continue;
-                        const float qv = __bfloat162float(S.q[I * SC + jr][c]);
-                        const float kv = __bfloat162float(S.k[I * SC + sr][c]);
-                        dg[a][e] += qv * kv * expf(fminf(Bj[jr] - Bj[sr], 0.f));
+                        const int tk = 4 * lane + e;
+                        const bool v = tk < nvalid;
+                        const int64_t off = (bh * L + t0 + (v ? tk : 0)) * K + ch;
+                        a[e] = v ? la[off] : 0.f;
+                        qa[e] = v ? __bfloat162float(q[off]) : 0.f;
+                        ka[e] = v ? __bfloat162float(k[off]) : 0.f;
                     }
+                    a[1] += a[0];
+                    a[2] += a[1];
+                    a[3] += a[2];
+                    float incl = a[3];
+#pragma unroll
+                    for (int d = 1; d < 32; d <<= 1) {
+                        const float o = __shfl_up_sync(0xffffffffu, incl, d);
+                        if (lane >= d) incl += o;
+                    }
+                    const float excl = incl - a[3];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        tabB[warp * C + 4 * lane + e] = excl + a[e];
+                        tabQ[warp * C + 4 * lane + e] = qa[e];
+                        tabK[warp * C + 4 * lane + e] = ka[e];
+                    }
+                }
+                named_sync(1, 256);
+                const int nb = !have ? 0 : nuns - b0 < 8 ? nuns - b0 : 8;
+                for (int w2 = 0; w2 < nb; ++w2) {
+                    const float Bi = tabB[w2 * C + row], qi = tabQ[w2 * C + row];
+                    const int jend = row < 64 * h + 63 ? row : 64 * h + 63;
+                    for (int j = 64 * h; j <= jend; ++j)
+                        X[j * C + row] += qi * tabK[w2 * C + j] * __expf(fminf(Bi - tabB[w2 * C + j], 0.f));
                 }
             }
         }
-        __syncthreads();
-    }
-    // ---- write P (bf16, [128 x 128], zero above the diagonal)
-    __nv_bfloat16* Pc = P + (bh * N + i) * C * C;
-    const int g = lane >> 2, t = lane & 3;
+        if (have) {
+            tc_fence_after();
+            uint4* dst = reinterpret_cast<uint4*>(P + ((bh * N + i) * C + row) * C + 64 * h);
 #pragma unroll
-    for (int J = 0; J < NS - 1; ++J) {
-        if (J < I) {
+            for (int c16 = 0; c16 < 4; ++c16) {
+                float y[16];
+                tmem_ld16(tmem + (uint32_t(32 * q4) << 16) + uint32_t(64 * h + 16 * c16), y);
+                tmem_wait_ld();
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                const int col = J * SC + nb * 8 + 2 * t;
-                const int r0 = I * SC + g;
-                *reinterpret_cast<uint32_t*>(&Pc[r0 * C + col]) = tc::pack_bf16x2(acc[J][nb][0], acc[J][nb][1]);
-                *reinterpret_cast<uint32_t*>(&Pc[(r0 + 8) * C + col]) =
-                    tc::pack_bf16x2(acc[J][nb][2], acc[J][nb][3]);
+                for (int e = 0; e < 16; ++e) {
+                    const int col = 64 * h + 16 * c16 + e;
+                    float v = y[e];
+                    if (nuns > 0) v += X[col * C + row];
+                    y[e] = col <= row ? v : 0.f;
+                }
+                dst[2 * c16] = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]), pack_bf16x2(y[4], y[5]),
+                                          pack_bf16x2(y[6], y[7]));
+                dst[2 * c16 + 1] = make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]),
+                                              pack_bf16x2(y[12], y[13]), pack_bf16x2(y[14], y[15]));
             }
         }
     }
-#pragma unroll
-    for (int a = 0; a < 2; ++a) {
-        const int jrel = jr0 + a;
-        float v[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) v[e] = (s0 + e <= jrel) ? dg[a][e] : 0.f;
-        const int row = I * SC + jrel;
-        *reinterpret_cast<uint32_t*>(&Pc[row * C + I * SC + s0]) = tc::pack_bf16x2(v[0], v[1]);
-        *reinterpret_cast<uint32_t*>(&Pc[row * C + I * SC + s0 + 2]) = tc::pack_bf16x2(v[2], v[3]);
-    }
-    // zero blocks right of the diagonal: row block I, columns (I+1)*16 .. 127
-    const int zc0 = (I + 1) * SC;
-    for (int e = lane; e < SC * (C - zc0) / 2; e += 32) {
-        const int r = e / ((C - zc0) / 2), cc = zc0 + 2 * (e % ((C - zc0) / 2));
-        *reinterpret_cast<uint32_t*>(&Pc[(I * SC + r) * C + cc]) = 0u;
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
     }
 }
+
+constexpr size_t kSmem = 1024 + kTabOff + 3 * 8 * C * sizeof(float);
 
 }  // namespace
 
-size_t tc_prep_smem_bytes() { return sizeof(PrepSmem); }
-
 gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const float* la, __nv_bfloat16* Qt,
-                          __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, float* Bout, cudaStream_t s) {
-    const size_t sm = sizeof(PrepSmem);
-    if (cudaFuncSetAttribute(k_tc_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, int(sm)) != cudaSuccess)
+                          __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, cudaStream_t s) {
+    if (cudaFuncSetAttribute(k_tc_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    GLA_LAUNCH("tc_prep", k_tc_prep, dim3(unsigned(p.N), unsigned(p.BH)), 256, sm, s,
-               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, Qt, Kt, P, gam, Bout,
-               p.L, p.K, p.N);
+    GLA_LAUNCH("tc_prep", k_tc_prep, dim3(unsigned(p.N), unsigned(p.BH)), kThreads, kSmem, s,
+               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, Qt, Kt, P, gam, p.L,
+               p.K, p.N, device_error_word());
     return GLA_OK;
 }
 

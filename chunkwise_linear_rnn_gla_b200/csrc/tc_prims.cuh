@@ -65,6 +65,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// The same test, but the thread may be suspended until the phase completes
+// or about `sleep_ns` nanoseconds have passed, so a waiting warp does not
+// take issue slots from the warps doing the work.
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t parity, uint32_t sleep_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(sleep_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity to complete. Gives up
 // after ~`limit_cycles` SM cycles, records kErrWaitTimeout in *err (device
 // memory) and in *abort (shared memory), and returns false. A set *abort
@@ -76,14 +91,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
     const long long t0 = clock64();
     while (true) {
         if (*abort) return false;
-        for (int i = 0; i < 64; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (clock64() - t0 > limit_cycles) {
             if (err) atomicExch(err, kErrWaitTimeout);
             *abort = 1;
             return false;
         }
     }
+}
+
+// Bounded wait that ignores the abort flag: lets copies and MMAs that were
+// already issued land before a block that gave up exits.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, long long limit_cycles = 2000000000LL) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait_sleep(bar, parity, 20000u))
+        if (clock64() - t0 > limit_cycles) return;
+}
+
+// Named barrier over the first `nthreads` threads of the block (id 1..15).
+__device__ __forceinline__ void named_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // ---------------------------------------------------------------- fences
@@ -136,6 +163,16 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
         : "r"(taddr));
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 8 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float* v) {
+    uint32_t r[8];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float* v) {
@@ -193,6 +230,16 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
     const uint32_t chunk = (col >> 3) ^ (row & 7u);
     return row * 128u + chunk * 16u + (col & 7u) * 2u;
+}
+
+// 2^x with the PTX ex2.approx instruction (results below the normal range
+// flush to zero). Gate factors are evaluated as e^x = 2^(x log2 e) with the
+// gate cumsums kept in base-2 units.
+constexpr float kLog2e = 1.4426950408889634f;  // log2(e)
+__device__ __forceinline__ float exp2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
