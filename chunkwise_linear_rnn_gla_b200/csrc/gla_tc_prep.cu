@@ -145,8 +145,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float2 l2 = *reinterpret_cast<const float2*>(lap + o);
                 const uint32_t qq = *reinterpret_cast<const uint32_t*>(qp + o);
                 const uint32_t kk = *reinterpret_cast<const uint32_t*>(kp + o);
-                // gate cumsums in base-2 units: e^x = 2^(x log2 e)
-                bb[r] = v ? make_float2(l2.x * kLog2e, l2.y * kLog2e) : make_float2(0.f, 0.f);
+                bb[r] = v ? make_float2(l2.x, l2.y) : make_float2(0.f, 0.f);
                 qv[r] = v ? qq : 0u;
                 kv[r] = v ? kk : 0u;
             }
@@ -170,12 +169,12 @@ __global__ void __launch_bounds__(kThreads, 2)
                 gamma.x += v.x;
                 gamma.y += v.y;
             }
-            const bool unsafe0 = gamma.x < -kSafeDecay * kLog2e, unsafe1 = gamma.y < -kSafeDecay * kLog2e;
-            const float eNG0 = unsafe0 ? 0.f : exp2_ftz(fmaxf(-gamma.x, 0.f));  // e^{-Gamma} <= e^64
-            const float eNG1 = unsafe1 ? 0.f : exp2_ftz(fmaxf(-gamma.y, 0.f));
+            const bool unsafe0 = gamma.x < -kSafeDecay, unsafe1 = gamma.y < -kSafeDecay;
+            const float eNG0 = unsafe0 ? 0.f : __expf(fmaxf(-gamma.x, 0.f));  // e^{-Gamma} <= e^64
+            const float eNG1 = unsafe1 ? 0.f : __expf(fmaxf(-gamma.y, 0.f));
             if (I == 0) {
                 *reinterpret_cast<float2*>(gam + (bh * N + i) * K + ch) =
-                    make_float2(exp2_ftz(fminf(gamma.x, 0.f)), exp2_ftz(fminf(gamma.y, 0.f)));
+                    make_float2(__expf(fminf(gamma.x, 0.f)), __expf(fminf(gamma.y, 0.f)));
                 if (unsafe0) bar.uns[atomicAdd(&bar.nuns, 1)] = (unsigned short)ch;
                 if (unsafe1) bar.uns[atomicAdd(&bar.nuns, 1)] = (unsigned short)(ch + 1);
             }
@@ -190,9 +189,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float2 qf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&qv[r]));
                 const float2 kf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&kv[r]));
                 // exponents are <= 0 in exact arithmetic; the clamps absorb cumsum rounding
-                const float qt0 = qf.x * exp2_ftz(fminf(Bx, 0.f)), qt1 = qf.y * exp2_ftz(fminf(By, 0.f));
-                const float kt0 = kf.x * exp2_ftz(fminf(gamma.x - Bx, 0.f));
-                const float kt1 = kf.y * exp2_ftz(fminf(gamma.y - By, 0.f));
+                const float qt0 = qf.x * __expf(fminf(Bx, 0.f)), qt1 = qf.y * __expf(fminf(By, 0.f));
+                const float kt0 = kf.x * __expf(fminf(gamma.x - Bx, 0.f));
+                const float kt1 = kf.y * __expf(fminf(gamma.y - By, 0.f));
                 const uint32_t qh = pack_bf16x2(qt0, qt1);
                 const uint32_t o = piece_off(row, cp);
                 if (ok) {

@@ -34,27 +34,36 @@ namespace {
 using namespace tc;
 
 constexpr int C = kTcChunk;
-constexpr int BVS = 64;   // value columns per CTA
 constexpr uint32_t PIECE = 16384;
-constexpr int NSLOT = 2;  // chunks in flight: (A pair, B piece) each
-constexpr uint32_t SLOT_BYTES = 3 * PIECE;
 constexpr int kThreads = 192;
 
+// Tile of BVS value columns (64 or 128): chunks in flight, bytes per chunk
+// (the key-channel pair of A pieces and BVS / 64 value pieces), CTAs per SM.
+template <int BVS>
+struct StCfg {
+    static constexpr int nslot = BVS == 128 ? 3 : 2;
+    static constexpr uint32_t slot_bytes = uint32_t(2 + BVS / 64) * PIECE;
+    static constexpr int min_blocks = BVS == 128 ? 1 : 2;
+    static constexpr size_t smem = 1024 + size_t(nslot) * slot_bytes;
+};
+
 struct StBars {
-    uint64_t full[NSLOT], empty[NSLOT];
+    uint64_t full[3], empty[3];
     uint64_t u_full[2], u_empty[2], drain;
     uint32_t tmem_slot;
     int abort_flag;
 };
 
-template <bool REVERSE>
-__global__ void __launch_bounds__(kThreads, 2)
+template <int BVS, bool REVERSE>
+__global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
     k_states_walk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const float* __restrict__ gam, const float* __restrict__ init, float* __restrict__ fin,
                   float* __restrict__ fin2, __nv_bfloat16* __restrict__ states, int64_t L, int64_t N, int64_t V,
                   int64_t K, int* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    constexpr int NSLOT = StCfg<BVS>::nslot;
+    constexpr uint32_t SLOT_BYTES = StCfg<BVS>::slot_bytes;
     StBars& bar = *reinterpret_cast<StBars*>(ring + NSLOT * SLOT_BYTES);
     volatile int* abort_flag = &bar.abort_flag;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -103,7 +112,9 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mbar_arrive_expect_tx(&bar.full[s], SLOT_BYTES);
                 tma_load_3d(st, &tmA, kbase, row0, int(bh), &bar.full[s]);
                 tma_load_3d(st + PIECE, &tmA, kbase + 64, row0, int(bh), &bar.full[s]);
-                tma_load_3d(st + 2 * PIECE, &tmB, v0, row0, int(bh), &bar.full[s]);
+#pragma unroll
+                for (int q = 0; q < BVS / 64; ++q)
+                    tma_load_3d(st + (2 + q) * PIECE, &tmB, v0 + 64 * q, row0, int(bh), &bar.full[s]);
             }
             if (!ok)
                 for (int w = step - NSLOT; w < step; ++w)
@@ -139,7 +150,14 @@ __global__ void __launch_bounds__(kThreads, 2)
         const uint32_t lane_off = uint32_t(32 * q4) << 16;
         float x[BVS];
 #pragma unroll
-        for (int e = 0; e < BVS; ++e) x[e] = init ? init[(bh * K + c) * V + v0 + e] : 0.f;
+        for (int e = 0; e < BVS / 4; ++e) {
+            const float4 v4 = init ? reinterpret_cast<const float4*>(init + (bh * K + c) * V + v0)[e]
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            x[4 * e] = v4.x;
+            x[4 * e + 1] = v4.y;
+            x[4 * e + 2] = v4.z;
+            x[4 * e + 3] = v4.w;
+        }
         bool ok = true;
         float g_next = gam[(bh * N + chunk_of(0)) * K + c];
         for (int step = 0; step < nsteps; ++step) {
@@ -147,26 +165,30 @@ __global__ void __launch_bounds__(kThreads, 2)
             const int ci = chunk_of(step);
             const float g = g_next;  // loaded one step ahead, off the critical path
             if (step + 1 < nsteps) g_next = gam[(bh * N + chunk_of(step + 1)) * K + c];
-            // the state entering chunk ci, in bf16
-            uint4* dst = reinterpret_cast<uint4*>(states + ((bh * N + ci) * K + c) * V + v0);
+            // the state entering chunk ci, in bf16 (32-byte stores: one full sector each)
+            __nv_bfloat16* dst = states + ((bh * N + ci) * K + c) * V + v0;
 #pragma unroll
-            for (int ch = 0; ch < BVS / 8; ++ch)
-                dst[ch] = make_uint4(pack_bf16x2(x[8 * ch], x[8 * ch + 1]), pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]),
-                                     pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]),
-                                     pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]));
+            for (int ch = 0; ch < BVS / 16; ++ch) {
+                uint32_t w[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(x[16 * ch + 2 * e], x[16 * ch + 2 * e + 1]);
+                st_global_v8(dst + 16 * ch, w);
+            }
             // tcgen05.ld is warp-collective: the condition must be the same for the whole warp
             ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar.u_full[b], uint32_t((step >> 1) & 1), err, abort_flag));
             if (!ok) break;
             tc_fence_after();
-            float u[BVS];
 #pragma unroll
-            for (int c16 = 0; c16 < BVS / 16; ++c16)
-                tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 16 * c16), u + 16 * c16);
-            tmem_wait_ld();
+            for (int c32 = 0; c32 < BVS / 32; ++c32) {
+                float u[32];
+                tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32), u);
+                tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32 + 16), u + 16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[32 * c32 + e] = fmaf(g, x[32 * c32 + e], u[e]);
+            }
             tc_fence_before();
             mbar_arrive(&bar.u_empty[b]);
-#pragma unroll
-            for (int e = 0; e < BVS; ++e) x[e] = fmaf(g, x[e], u[e]);
         }
         if (ok) {
             for (int w = 0; w < 2; ++w) {
@@ -195,7 +217,7 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
 
 }  // namespace
 
-bool tc_states_walk_supported(const Problem& p) { return p.V % BVS == 0; }
+bool tc_states_walk_supported(const Problem& p) { return p.V % 64 == 0; }
 
 gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
                                  const float* init, float* fin, float* fin2, __nv_bfloat16* states, bool reverse,
@@ -205,11 +227,15 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
     if (!(map3(&m[0], A, uint64_t(p.K), uint64_t(p.L), uint64_t(p.BH)) &&
           map3(&m[1], B, uint64_t(p.V), uint64_t(p.L), uint64_t(p.BH))))
         return GLA_ERR_CUDA;
-    const size_t smem = 1024 + size_t(NSLOT) * SLOT_BYTES + sizeof(StBars);
-    auto fn = reverse ? k_states_walk<true> : k_states_walk<false>;
+    // 128-column tiles halve the re-reads of the key operand through L2 when d_v allows
+    const bool wide = p.V % 128 == 0;
+    const int bvs = wide ? 128 : 64;
+    const size_t smem = (wide ? StCfg<128>::smem : StCfg<64>::smem) + sizeof(StBars);
+    auto fn = wide ? (reverse ? k_states_walk<128, true> : k_states_walk<128, false>)
+                   : (reverse ? k_states_walk<64, true> : k_states_walk<64, false>);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    const dim3 grid(unsigned(p.V / BVS), unsigned(p.K / 128), unsigned(p.BH));
+    const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH));
     GLA_LAUNCH(name, fn, grid, kThreads, smem, s, m[0], m[1], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
                device_error_word());
     return GLA_OK;

@@ -232,6 +232,13 @@ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
     return row * 128u + chunk * 16u + (col & 7u) * 2u;
 }
 
+// 32-byte global store (sm_100): a full sector per thread. p must be 32-byte aligned.
+__device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]),
+                 "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+
 // 2^x with the PTX ex2.approx instruction (results below the normal range
 // flush to zero). Gate factors are evaluated as e^x = 2^(x log2 e) with the
 // gate cumsums kept in base-2 units.

@@ -11,7 +11,8 @@
  *
  * alpha_t = exp(log_a_t) in [0,1]^{Dk}, S_{-1} = h0, hT = S_{L-1}. The output
  * reads the state after the update. There is no 1/sqrt(Dk) scale and no
- * normaliser inside the layer.
+ * normaliser inside the layer. log_a must be finite and <= 0: a gate of
+ * exactly zero is passed as a large negative value (e.g. -1e30), not -inf.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
