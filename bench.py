@@ -86,7 +86,7 @@ def kernel_models(w, C):
     sb = BH * N * K * V * e  # one set of bf16 chunk states
     pb = BH * N * C * C * e  # intra-chunk score matrices
     m["tc_prep"] = dict(bytes=th * (2 * K * e + 4 * K + 2 * K * e) + pb + BH * N * K * 4,
-                        flops=th * C * K, bound="hbm")
+                        flops=th * 2 * C * K, bound="hbm")
     m["tc_walk_states"] = dict(bytes=th * (K * e + V * e) + sb, flops=th * 2 * K * V, bound="hbm")
     m["tc_walk_dstates"] = dict(bytes=th * (K * e + V * e) + sb, flops=th * 2 * K * V, bound="hbm")
     m["tc_output"] = dict(bytes=th * (K * e + 2 * V * e) + pb + sb, flops=th * 2 * (K * V + C * V), bound="hbm")
@@ -95,10 +95,11 @@ def kernel_models(w, C):
                             bound="hbm")
     m["tc_walk_dv"] = dict(bytes=th * (2 * K * e + 2 * V * e) + pb + 2 * st, flops=th * 2 * (2 * K * V + C * V),
                            bound="hbm")
-    m["tc_bwd_gemm"] = dict(bytes=th * (2 * V * e + 2 * K * e) + 2 * sb + pb, flops=th * 2 * (C * V + 2 * K * V),
-                            bound="hbm")
-    m["tc_bwd_intra"] = dict(bytes=th * (2 * K * e + 4 * K + 2 * K * e + 2 * K * e + 4 * K) + pb + 2 * sb,
-                             flops=th * 2 * C * K, bound="hbm")
+    # fused chunk backward: reads dO, v, S_[i], D_i, Q~, q, k, log a, e^Gamma; writes dq, dk, dlog a.
+    # flops: dP, dO S^T, v D^T and the two intra-chunk GEMMs
+    m["tc_bwd_chunk"] = dict(bytes=th * (2 * V * e + K * e + 2 * K * e + 4 * K + 2 * K * e + 4 * K) + 2 * sb
+                             + BH * N * K * 4,
+                             flops=th * (2 * C * V + 4 * K * V + 4 * C * K), bound="hbm")
     return m
 
 
@@ -229,9 +230,10 @@ def main():
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    from chunkwise_linear_rnn_gla_b200 import dp
+
+    env = dp.rank_env()
+    world, rank, local_rank = env.world, env.rank, env.local_rank
 
     from chunkwise_linear_rnn_gla_b200.inputs import WORKLOADS
 
@@ -267,7 +269,7 @@ def main():
 
     from chunkwise_linear_rnn_gla_b200.inputs import make_inputs
 
-    inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=rank)
+    inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=dp.shard_seed(0, rank))
     d = {k: v.to(dev) for k, v in inp.items()}
     desc = gla.make_desc(w.B, w.H, w.L, w.K, w.V, w.dtype, 0, 0, args.state_mode, args.kernel_impl)
     C, sc, impl_name, mode = gla.gla_resolve(desc)
@@ -314,13 +316,10 @@ def main():
     step_ms = [a.elapsed_time(b) for a, b in ev]
     total_ms = sum(step_ms)
     prof = gla.gla_profile_read()
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = dp.max_over_ranks(total_ms)
     ms_per_step = total_ms / args.steps
     tokens_per_step = w.B * w.L * world
-    value = tokens_per_step / (ms_per_step / 1e3)
+    value = dp.job_throughput(w.B * w.L, world, ms_per_step)
 
     # ---------------- end to end through the public API, host buffers
     e2e = None
@@ -349,12 +348,9 @@ def main():
             e2e_step()
         b_.record(stream)
         torch.cuda.synchronize(dev)
-        e2e_ms = a_.elapsed_time(b_) / args.e2e_steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-        e2e = {"value": tokens_per_step / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+        e2e_ms = dp.max_over_ranks(a_.elapsed_time(b_) / args.e2e_steps)
+        e2e = {"value": dp.job_throughput(w.B * w.L, world, e2e_ms), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
 
     # ---------------- roofline of the dominant kernel
@@ -407,7 +403,7 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
                 "data": "synthetic (seeded N(0,1)/sqrt(d_k) q,k,v; log_a = logsigmoid(N(0,1))/16; dO ~ N(0,1))",
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V,
-                           "global_batch": w.B * world, "seq_len": w.L, "chunk": C, "subchunk": sc,
+                           "global_batch": dp.global_batch(w.B, world), "seq_len": w.L, "chunk": C, "subchunk": sc,
                            "kernel_impl": impl_name, "state_mode": mode, "parallelism": "dp%d" % world,
                            "l2": "flushed between timed steps (512 MB write)"},
                 "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cb, "e2e": e2e,

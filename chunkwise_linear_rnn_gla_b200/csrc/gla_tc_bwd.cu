@@ -81,6 +81,7 @@ struct BwdBars {
     uint64_t accA, qt_full, qk_full, dpm_ready, khat_ready, xd_ready, accB, drain;
     uint32_t tmem_slot;
     int abort_flag;
+    int any_exact;  // some key channel of this CTA is beyond the bound
     float xd[128];  // sum_v D_i[c,v] S_[i][c,v]
 };
 
@@ -96,7 +97,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_chunk(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmD,
                 const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmQ,
-                const __grid_constant__ CUtensorMap tmK, const __nv_bfloat16* __restrict__ q,
+                const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmDQ,
+                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDLA,
+                const __nv_bfloat16* __restrict__ q,
                 const __nv_bfloat16* __restrict__ k, const float* __restrict__ la, const float* __restrict__ gam,
                 __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, float* __restrict__ dla, int64_t L,
                 int64_t N, int64_t K, int64_t V, int* err) {
@@ -124,6 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&bar.accB, 1);
         mbar_init(&bar.drain, 1);
         bar.abort_flag = 0;
+        bar.any_exact = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -287,31 +291,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
             // per-chunk cumsum along the tokens (base-2 units: e^x = 2^(x log2 e)), gate table
             // into TMEM, K^0 operand into shared memory
+            // four quarters of 32 tokens; all loads of a quarter are issued before the (sequential) scan
             float B = 0.f;
 #pragma unroll 1
-            for (int g = 0; g < C / 16; ++g) {
-                float lav[16], kv[16];
+            for (int hf = 0; hf < 4; ++hf) {
+                float lav[32];
+                unsigned short kraw[32];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int t = 16 * g + r;
-                    const uint32_t o = roff(t);
-                    const float l = lap[o];
-                    const float kk = __bfloat162float(kp[o]);
-                    lav[r] = t < nvalid ? l * kLog2e : 0.f;
-                    kv[r] = t < nvalid ? kk : 0.f;
+                for (int r = 0; r < 32; ++r) {
+                    const uint32_t o = roff(32 * hf + r);
+                    lav[r] = lap[o];
+                    kraw[r] = reinterpret_cast<const unsigned short*>(kp)[o];
                 }
-                float tb[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int t = 16 * g + r;
-                    B += lav[r];
-                    const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; only used when safe
-                    tb[r] = safe ? e : B;
-                    *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c)) =
-                        __float2bfloat16_rn(safe ? kv[r] * e : 0.f);
+                for (int g = 0; g < 2; ++g) {
+                    float tb[16];
+#pragma unroll
+                    for (int r = 0; r < 16; ++r) {
+                        const int t = 32 * hf + 16 * g + r;
+                        const bool v = t < nvalid;
+                        B += v ? lav[16 * g + r] * kLog2e : 0.f;
+                        const float kv = v ? __bfloat162float(__ushort_as_bfloat16(kraw[16 * g + r])) : 0.f;
+                        const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; used when safe
+                        tb[r] = safe ? e : B;
+                        *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c)) =
+                            __float2bfloat16_rn(safe ? kv * e : 0.f);
+                    }
+                    tmem_st16(tmem + lane_off + 384u + uint32_t(32 * hf + 16 * g), tb);
                 }
-                tmem_st16(tmem + lane_off + 384u + uint32_t(16 * g), tb);
             }
+            if (__any_sync(0xffffffffu, !safe) && lane == 0) atomicOr(&bar.any_exact, 1);
             tmem_wait_st();
             fence_proxy_async_smem();
             tc_fence_before();
@@ -360,6 +369,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_sync(3, 256);
         float* xch = reinterpret_cast<float*>(base + DPM_OFF);  // free once the exact pass is done
+        // dq and dk are staged (bf16, 128-byte swizzle) over the Q~ and K^0 tiles and written by TMA
+        // stores, unless those areas hold exact-path terms
+        const bool stage = bar.any_exact == 0;
+        const bool issuer = gate_warp && c == 0;
         const int tlo = gate_warp ? 0 : C / 2;
         float kin = 0.f, rsum = 0.f;  // sum_s K~_s (v_s D_i^T) and sum_s r_s over this half
         float eGam = 0.f, Gam = 0.f;  // Gamma in base-2 units
@@ -374,16 +387,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 eGam = safe ? __fdividef(1.f, v8[7]) : exp2_ftz(fminf(v8[7], 0.f));
             }
 #pragma unroll 1
-            for (int g = tlo / 8; g < tlo / 8 + C / 16; ++g) {
-                float vQ[8], vJ[8], vI[8], vT[8];
-                tmem_ld8(tmem + lane_off + 128u + uint32_t(8 * g), vQ);
-                tmem_ld8(tmem + lane_off + 256u + uint32_t(8 * g), vJ);
-                tmem_ld8(tmem + lane_off + 0u + uint32_t(8 * g), vI);
-                tmem_ld8(tmem + lane_off + 384u + uint32_t(8 * g), vT);
+            for (int g = tlo / 16; g < tlo / 16 + C / 32; ++g) {
+                float vQ[16], vJ[16], vI[16], vT[16];
+                tmem_ld16(tmem + lane_off + 128u + uint32_t(16 * g), vQ);
+                tmem_ld16(tmem + lane_off + 256u + uint32_t(16 * g), vJ);
+                tmem_ld16(tmem + lane_off + 0u + uint32_t(16 * g), vI);
+                tmem_ld16(tmem + lane_off + 384u + uint32_t(16 * g), vT);
                 tmem_wait_ld();
 #pragma unroll
-                for (int r = 0; r < 8; ++r) {
-                    const int t = 8 * g + r;
+                for (int r = 0; r < 16; ++r) {
+                    const int t = 16 * g + r;
                     const float qv = qs(t), kv = ks(t);
                     float eGB, dqv, dkv;
                     if (safe) {
@@ -401,7 +414,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float rr = qv * dqv - kv * dkv;
                     rsum += rr;
                     rbuf[t * C + c] = rr;
-                    if (t < nvalid) {
+                    if (stage) {
+                        *reinterpret_cast<__nv_bfloat16*>(base + QT_OFF + tile_off(t, c)) = __float2bfloat16_rn(dqv);
+                        *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c)) = __float2bfloat16_rn(dkv);
+                    } else if (t < nvalid) {
                         dq[rb + int64_t(t) * K] = __float2bfloat16_rn(dqv);
                         dk[rb + int64_t(t) * K] = __float2bfloat16_rn(dkv);
                     }
@@ -410,16 +426,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             xch[(gate_warp ? 0 : 128) + c] = kin;
             if (!gate_warp) xch[256 + c] = rsum;
         }
+        fence_proxy_async_smem();
         named_sync(3, 256);
+        if (issuer && ok && stage) {  // rows past the end of the sequence are clipped by the TMA unit
+            for (int h = 0; h < 2; ++h) {
+                tma_store_3d(&tmDQ, 128 * kh + 64 * h, i * C, int(bh), base + QT_OFF + h * PIECE);
+                tma_store_3d(&tmDK, 128 * kh + 64 * h, i * C, int(bh), base + KH_OFF + h * PIECE);
+            }
+            bulk_commit();
+        }
         if (ok) {
-            // reverse cumsum; the carry from all later chunks is e^Gamma x_c + sum_s K~_s (v_s D_i^T)
+            // reverse cumsum in place; the carry from all later chunks is e^Gamma x_c + sum_s K~_s (v_s D_i^T)
             float suf = eGam * bar.xd[c] + xch[c] + xch[128 + c] + (gate_warp ? xch[256 + c] : 0.f);
 #pragma unroll 4
             for (int t = tlo + C / 2 - 1; t >= tlo; --t) {
                 suf += rbuf[t * C + c];
-                if (t < nvalid) dla[rb + int64_t(t) * K] = suf;
+                rbuf[t * C + c] = suf;
             }
         }
+        fence_proxy_async_smem();
+        named_sync(3, 256);
+        if (issuer && ok) {
+            tma_store_3d(&tmDLA, 128 * kh, i * C, int(bh), rbuf);  // dense [128 tokens x 128 channels] fp32
+            bulk_commit();
+        }
+        if (issuer) bulk_wait_all();
     }
     tc_fence_before();
     __syncthreads();
@@ -437,6 +468,14 @@ bool map_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, 
     return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// [outer][rows][inner] fp32 tensor, box [128 rows x 128 inner], no swizzle
+bool map_f32_tile(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
+    const uint64_t dims[3] = {inner, rows, outer};
+    const uint64_t strides[2] = {inner * 4, inner * rows * 4};
+    const uint32_t box[3] = {128, 128, 1};
+    return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 constexpr size_t kSmem = 1024 + KH_OFF + 2 * PIECE + sizeof(BwdBars);
 static_assert(kSmem <= 232448, "shared memory");
 
@@ -445,17 +484,19 @@ static_assert(kSmem <= 232448, "shared memory");
 gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
                                const void* v, const __nv_bfloat16* Qt, const float* gam, const __nv_bfloat16* Sbuf,
                                const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, cudaStream_t s) {
-    CUtensorMap m[7];
+    CUtensorMap m[10];
     memset(m, 0, sizeof(m));
     const uint64_t L = uint64_t(p.L), K = uint64_t(p.K), V = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
     if (!(map_sw128(&m[0], dO, V, L, BH) && map_sw128(&m[1], v, V, L, BH) && map_sw128(&m[2], Sbuf, V, K, BH * N) &&
           map_sw128(&m[3], Dbuf, V, K, BH * N) && map_sw128(&m[4], Qt, K, L, BH) && map_sw128(&m[5], q, K, L, BH) &&
-          map_sw128(&m[6], k, K, L, BH)))
+          map_sw128(&m[6], k, K, L, BH) && map_sw128(&m[7], dq, K, L, BH) && map_sw128(&m[8], dk, K, L, BH) &&
+          map_f32_tile(&m[9], dla, K, L, BH)))
         return GLA_ERR_CUDA;
     if (cudaFuncSetAttribute(k_bwd_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.K / 128), unsigned(p.BH));
-    GLA_LAUNCH("tc_bwd_chunk", k_bwd_chunk, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6],
+    GLA_LAUNCH("tc_bwd_chunk", k_bwd_chunk, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
+               m[8], m[9],
                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, gam,
                static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K, p.V,
                device_error_word());

@@ -43,8 +43,8 @@ template <int BVS>
 struct StCfg {
     static constexpr int nslot = BVS == 128 ? 3 : 2;
     static constexpr uint32_t slot_bytes = uint32_t(2 + BVS / 64) * PIECE;
-    static constexpr int min_blocks = BVS == 128 ? 1 : 2;
-    static constexpr size_t smem = 1024 + size_t(nslot) * slot_bytes;
+    static constexpr int min_blocks = 1;
+    static constexpr size_t smem = 1024 + size_t(nslot) * slot_bytes + size_t(BVS / 64) * PIECE;  // + staging
 };
 
 struct StBars {
@@ -57,6 +57,7 @@ struct StBars {
 template <int BVS, bool REVERSE>
 __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
     k_states_walk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmS,
                   const float* __restrict__ gam, const float* __restrict__ init, float* __restrict__ fin,
                   float* __restrict__ fin2, __nv_bfloat16* __restrict__ states, int64_t L, int64_t N, int64_t V,
                   int64_t K, int* err) {
@@ -64,7 +65,7 @@ __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NSLOT = StCfg<BVS>::nslot;
     constexpr uint32_t SLOT_BYTES = StCfg<BVS>::slot_bytes;
-    StBars& bar = *reinterpret_cast<StBars*>(ring + NSLOT * SLOT_BYTES);
+    StBars& bar = *reinterpret_cast<StBars*>(ring + NSLOT * SLOT_BYTES + (BVS / 64) * PIECE);
     volatile int* abort_flag = &bar.abort_flag;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int v0 = blockIdx.x * BVS;
@@ -158,38 +159,53 @@ __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
             x[4 * e + 2] = v4.z;
             x[4 * e + 3] = v4.w;
         }
+        // the bf16 copy of each entering state is staged in shared memory (128-byte swizzle) and
+        // written by TMA stores issued by one thread, so the register file never waits on the stores
+        uint8_t* stg = ring + NSLOT * SLOT_BYTES;
+        const bool issuer = row == 0;
         bool ok = true;
         float g_next = gam[(bh * N + chunk_of(0)) * K + c];
+        // every epilogue thread passes every named barrier, also after a wait gave up (bar.sync has
+        // no time limit); a failed wait only skips the work
         for (int step = 0; step < nsteps; ++step) {
             const int b = step & 1;
             const int ci = chunk_of(step);
             const float g = g_next;  // loaded one step ahead, off the critical path
             if (step + 1 < nsteps) g_next = gam[(bh * N + chunk_of(step + 1)) * K + c];
-            // the state entering chunk ci, in bf16 (32-byte stores: one full sector each)
-            __nv_bfloat16* dst = states + ((bh * N + ci) * K + c) * V + v0;
+            if (issuer) bulk_wait_read_all();  // the previous step's stores have read the staging tile
+            named_sync(1, 128);
 #pragma unroll
-            for (int ch = 0; ch < BVS / 16; ++ch) {
-                uint32_t w[8];
+            for (int ch = 0; ch < BVS / 8; ++ch)
+                *reinterpret_cast<uint4*>(stg + (ch >> 3) * PIECE + uint32_t(row) * 128u +
+                                          uint32_t(((ch & 7) ^ (row & 7)) << 4)) =
+                    make_uint4(pack_bf16x2(x[8 * ch], x[8 * ch + 1]), pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]),
+                               pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]), pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]));
+            fence_proxy_async_smem();
+            named_sync(1, 128);
+            if (issuer && ok) {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) w[e] = pack_bf16x2(x[16 * ch + 2 * e], x[16 * ch + 2 * e + 1]);
-                st_global_v8(dst + 16 * ch, w);
+                for (int q = 0; q < BVS / 64; ++q)
+                    tma_store_3d(&tmS, v0 + 64 * q, kbase, int(bh * N + ci), stg + q * PIECE);
+                bulk_commit();
             }
             // tcgen05.ld is warp-collective: the condition must be the same for the whole warp
             ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar.u_full[b], uint32_t((step >> 1) & 1), err, abort_flag));
-            if (!ok) break;
-            tc_fence_after();
+            if (ok) {
+                tc_fence_after();
 #pragma unroll
-            for (int c32 = 0; c32 < BVS / 32; ++c32) {
-                float u[32];
-                tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32), u);
-                tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32 + 16), u + 16);
-                tmem_wait_ld();
+                for (int c32 = 0; c32 < BVS / 32; ++c32) {
+                    float u[32];
+                    tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32), u);
+                    tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32 + 16), u + 16);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) x[32 * c32 + e] = fmaf(g, x[32 * c32 + e], u[e]);
+                    for (int e = 0; e < 32; ++e) x[32 * c32 + e] = fmaf(g, x[32 * c32 + e], u[e]);
+                }
+                tc_fence_before();
+                mbar_arrive(&bar.u_empty[b]);
             }
-            tc_fence_before();
-            mbar_arrive(&bar.u_empty[b]);
         }
+        if (issuer) bulk_wait_all();
         if (ok) {
             for (int w = 0; w < 2; ++w) {
                 float* f = w ? fin2 : fin;
@@ -222,10 +238,11 @@ bool tc_states_walk_supported(const Problem& p) { return p.V % 64 == 0; }
 gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
                                  const float* init, float* fin, float* fin2, __nv_bfloat16* states, bool reverse,
                                  cudaStream_t s, const char* name) {
-    CUtensorMap m[2];
+    CUtensorMap m[3];
     memset(m, 0, sizeof(m));
     if (!(map3(&m[0], A, uint64_t(p.K), uint64_t(p.L), uint64_t(p.BH)) &&
-          map3(&m[1], B, uint64_t(p.V), uint64_t(p.L), uint64_t(p.BH))))
+          map3(&m[1], B, uint64_t(p.V), uint64_t(p.L), uint64_t(p.BH)) &&
+          map3(&m[2], states, uint64_t(p.V), uint64_t(p.K), uint64_t(p.BH * p.N))))
         return GLA_ERR_CUDA;
     // 128-column tiles halve the re-reads of the key operand through L2 when d_v allows
     const bool wide = p.V % 128 == 0;
@@ -236,7 +253,7 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH));
-    GLA_LAUNCH(name, fn, grid, kThreads, smem, s, m[0], m[1], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
+    GLA_LAUNCH(name, fn, grid, kThreads, smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
                device_error_word());
     return GLA_OK;
 }
