@@ -106,7 +106,14 @@ def kernel_models(w, C):
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
 # ncu capture of the default workload, with the SHA-1 of the kernel's source
 # file at capture time: a kernel whose source changed since reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    "tc_prep": (76091392, "gla_tc_prep.cu", "c13be6f89c9b31d2bd2b53818730823b54d1811c"),
+    "tc_walk_states": (81700608, "gla_tc_states.cu", "58f1386a9107887b164f169c977a3b54ba03f471"),
+    "tc_output": (135941632, "gla_tc_out.cu", "073a31fe6a7d0be948a8a8d5796fb1e1e26cc317"),
+    "tc_walk_dstates": (74450688, "gla_tc_states.cu", "58f1386a9107887b164f169c977a3b54ba03f471"),
+    "tc_output_dv": (135902208, "gla_tc_out.cu", "073a31fe6a7d0be948a8a8d5796fb1e1e26cc317"),
+    "tc_bwd_chunk": (333266432, "gla_tc_bwd.cu", "058567593b0333a4e9b7914c6cf6905947952374"),
+}
 
 
 def measured_traffic(name):

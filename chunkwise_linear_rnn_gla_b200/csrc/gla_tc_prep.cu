@@ -65,10 +65,30 @@ __device__ __forceinline__ uint32_t piece_off(int row, int c64) {
     return uint32_t(row) * 128u + uint32_t(((c64 >> 3) ^ (row & 7)) << 4) + uint32_t(c64 & 7) * 2u;
 }
 
+// Rows of one 64-channel piece: log a (channel pair, fp32) and q, k (bf16 pairs) of rows 16I .. 16I+15.
+// Rows past the end of the sequence (last chunk only) read the last valid row and are zeroed.
+template <int K, bool FULL>
+__device__ __forceinline__ void load_rows(const float* lap, const __nv_bfloat16* qp, const __nv_bfloat16* kp, int I,
+                                          int nvalid, float2* bb, uint32_t* qv, uint32_t* kv) {
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+        const int row = 16 * I + r;
+        const bool v = FULL || row < nvalid;
+        const uint32_t o = uint32_t(FULL ? row : (v ? row : nvalid - 1)) * uint32_t(K);
+        const float2 l2 = *reinterpret_cast<const float2*>(lap + o);
+        const uint32_t qq = *reinterpret_cast<const uint32_t*>(qp + o);
+        const uint32_t kk = *reinterpret_cast<const uint32_t*>(kp + o);
+        bb[r] = v ? l2 : make_float2(0.f, 0.f);
+        qv[r] = v ? qq : 0u;
+        kv[r] = v ? kk : 0u;
+    }
+}
+
+template <int K>
 __global__ void __launch_bounds__(kThreads, 2)
     k_tc_prep(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k, const float* __restrict__ la,
               __nv_bfloat16* __restrict__ Qt, __nv_bfloat16* __restrict__ Kt, __nv_bfloat16* __restrict__ P,
-              float* __restrict__ gam, int64_t L, int64_t K, int64_t N, int* err) {
+              float* __restrict__ gam, int64_t L, int64_t N, int* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     // operand buffers: [b][Q~ piece, K^0 piece], b = piece parity
@@ -130,25 +150,13 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int t = 0; t < npiece; ++t) {
             const int b = t & 1;
             const int64_t ch = int64_t(KP) * t + cp;
-            // rows past the end of the sequence (last chunk) read the last valid row and are zeroed
             const int64_t rb = (bh * L + t0) * K + ch;
-            const float* lap = la + rb;
-            const __nv_bfloat16* qp = q + rb;
-            const __nv_bfloat16* kp = k + rb;
             float2 bb[16];
             uint32_t qv[16], kv[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const int row = 16 * I + r;
-                const bool v = row < nvalid;
-                const uint32_t o = uint32_t(v ? row : nvalid - 1) * uint32_t(K);
-                const float2 l2 = *reinterpret_cast<const float2*>(lap + o);
-                const uint32_t qq = *reinterpret_cast<const uint32_t*>(qp + o);
-                const uint32_t kk = *reinterpret_cast<const uint32_t*>(kp + o);
-                bb[r] = v ? make_float2(l2.x, l2.y) : make_float2(0.f, 0.f);
-                qv[r] = v ? qq : 0u;
-                kv[r] = v ? kk : 0u;
-            }
+            if (nvalid == C)
+                load_rows<K, true>(la + rb, q + rb, k + rb, I, nvalid, bb, qv, kv);
+            else
+                load_rows<K, false>(la + rb, q + rb, k + rb, I, nvalid, bb, qv, kv);
             float2 run = make_float2(0.f, 0.f);
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
@@ -302,11 +310,12 @@ constexpr size_t kSmem = 1024 + kTabOff + 3 * 8 * C * sizeof(float);
 
 gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const float* la, __nv_bfloat16* Qt,
                           __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, cudaStream_t s) {
-    if (cudaFuncSetAttribute(k_tc_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
+    auto fn = p.K == 256 ? k_tc_prep<256> : k_tc_prep<128>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    GLA_LAUNCH("tc_prep", k_tc_prep, dim3(unsigned(p.N), unsigned(p.BH)), kThreads, kSmem, s,
+    GLA_LAUNCH("tc_prep", fn, dim3(unsigned(p.N), unsigned(p.BH)), kThreads, kSmem, s,
                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, Qt, Kt, P, gam, p.L,
-               p.K, p.N, device_error_word());
+               p.N, device_error_word());
     return GLA_OK;
 }
 
