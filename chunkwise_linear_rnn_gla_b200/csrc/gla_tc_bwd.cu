@@ -61,9 +61,10 @@ using namespace tc;
 
 constexpr int C = kTcChunk;
 constexpr uint32_t PIECE = 16384;
-constexpr int NSTAGE = 3;  // each stage: dO, v, S, D pieces for 64 value columns
+constexpr int NSTAGE = 2;  // each stage: dO, v, S, D pieces for 64 value columns
 constexpr uint32_t STAGE_BYTES = 4 * PIECE;
-constexpr uint32_t KH_OFF = NSTAGE * STAGE_BYTES;  // K^0 operand, 2 pieces
+constexpr uint32_t LA_OFF = 8 * PIECE;             // log a tile, fp32 [128 tokens][128 channels], read by the prologue
+constexpr uint32_t KH_OFF = 12 * PIECE;            // k tile, rescaled in place into the K^0 operand, 2 pieces
 constexpr uint32_t DPM_OFF = 0;                    // after the value loop: masked dP (bf16), 2 pieces
 constexpr uint32_t QT_OFF = 2 * PIECE;             //                       Q~ tile, 2 pieces
 constexpr uint32_t RB_OFF = 4 * PIECE;             //                       r = q dq - k dk, fp32 [128][128]
@@ -78,7 +79,7 @@ constexpr float kSafeGam = 1.6038109e-28f;  // e^-64
 
 struct BwdBars {
     uint64_t full[NSTAGE], empty[NSTAGE];
-    uint64_t accA, qt_full, qk_full, dpm_ready, khat_ready, xd_ready, accB, drain;
+    uint64_t pro_full, accA, qt_full, qk_full, dpm_ready, khat_ready, xd_ready, accB, drain;
     uint32_t tmem_slot;
     int abort_flag;
     int any_exact;  // some key channel of this CTA is beyond the bound
@@ -99,6 +100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmDQ,
                 const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDLA,
+                const __grid_constant__ CUtensorMap tmLA,
                 const __nv_bfloat16* __restrict__ q,
                 const __nv_bfloat16* __restrict__ k, const float* __restrict__ la, const float* __restrict__ gam,
                 __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, float* __restrict__ dla, int64_t L,
@@ -118,6 +120,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar.full[s], 1);
             mbar_init(&bar.empty[s], 1 + 128);  // MMA commit + the 128 row threads
         }
+        mbar_init(&bar.pro_full, 1);
         mbar_init(&bar.accA, 1);
         mbar_init(&bar.qt_full, 1);
         mbar_init(&bar.qk_full, 1);
@@ -141,6 +144,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            // the gate prologue's inputs first: log a (dense fp32) and k (into the K^0 operand area)
+            mbar_arrive_expect_tx(&bar.pro_full, 4 * PIECE + 2 * PIECE);
+            tma_load_3d(base + LA_OFF, &tmLA, 128 * kh, i * C, int(bh), &bar.pro_full);
+            tma_load_3d(base + KH_OFF, &tmK, 128 * kh, i * C, int(bh), &bar.pro_full);
+            tma_load_3d(base + KH_OFF + PIECE, &tmK, 128 * kh + 64, i * C, int(bh), &bar.pro_full);
             bool ok = true;
             int vb = 0;
             for (; vb < nvb && ok; ++vb) {
@@ -156,8 +164,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(st + 2 * PIECE, &tmS, 64 * vb, 128 * kh, int(bh * N + i), &bar.full[s]);
                 tma_load_3d(st + 3 * PIECE, &tmD, 64 * vb, 128 * kh, int(bh * N + i), &bar.full[s]);
             }
-            // the Q~ tile goes where stage 0 was, once every stage has been consumed
-            if (ok && mbar_wait(&bar.accA, 0, err, abort_flag) && mbar_wait(&bar.xd_ready, 0, err, abort_flag)) {
+            // the Q~ tile goes where stage 0 was once every stage has been consumed; q and k go where
+            // the prologue's log a tile was
+            if (ok && mbar_wait(&bar.accA, 0, err, abort_flag) && mbar_wait(&bar.xd_ready, 0, err, abort_flag) &&
+                mbar_wait(&bar.khat_ready, 0, err, abort_flag)) {
                 mbar_arrive_expect_tx(&bar.qt_full, 2 * PIECE);
                 tma_load_3d(base + QT_OFF, &tmQt, 128 * kh, i * C, int(bh), &bar.qt_full);
                 tma_load_3d(base + QT_OFF + PIECE, &tmQt, 128 * kh + 64, i * C, int(bh), &bar.qt_full);
@@ -173,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int w = vb - NSTAGE; w < vb; ++w)
                     if (w >= 0) mbar_drain(&bar.full[w % NSTAGE], uint32_t((w / NSTAGE) & 1));
             }
+            mbar_drain(&bar.pro_full, 0);
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -232,7 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         // rows past the end of the sequence (last chunk) read the last valid row and are zeroed
         const int64_t rb = (bh * L + t0) * K + chg;
         const float* lap = la + rb;
-        const __nv_bfloat16* kp = k + rb;
         auto roff = [&](int t) -> uint32_t { return uint32_t(t < nvalid ? t : nvalid - 1) * uint32_t(K); };
         if (!gate_warp) {
             // x_c = sum_v D_i[c,v] S_[i][c,v] from the staged tiles
@@ -291,34 +301,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
             // per-chunk cumsum along the tokens (base-2 units: e^x = 2^(x log2 e)), gate table
             // into TMEM, K^0 operand into shared memory
-            // four quarters of 32 tokens; all loads of a quarter are issued before the (sequential) scan
+            // per-chunk cumsum along the tokens from the staged tiles (rows past the end of the
+            // sequence are zero-filled by TMA), in base-2 units: e^x = 2^(x log2 e)
+            const bool pro = __all_sync(0xffffffffu, mbar_wait(&bar.pro_full, 0, err, abort_flag));
+            const float* sLA = reinterpret_cast<const float*>(base + LA_OFF);
             float B = 0.f;
 #pragma unroll 1
-            for (int hf = 0; hf < 4; ++hf) {
-                float lav[32];
-                unsigned short kraw[32];
+            for (int g = 0; g < C / 16 && pro; ++g) {
+                float tb[16];
 #pragma unroll
-                for (int r = 0; r < 32; ++r) {
-                    const uint32_t o = roff(32 * hf + r);
-                    lav[r] = lap[o];
-                    kraw[r] = reinterpret_cast<const unsigned short*>(kp)[o];
+                for (int r = 0; r < 16; ++r) {
+                    const int t = 16 * g + r;
+                    B += sLA[t * C + c] * kLog2e;
+                    __nv_bfloat16* kslot = reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c));
+                    const float kv = __bfloat162float(*kslot);
+                    const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; used when safe
+                    tb[r] = safe ? e : B;
+                    *kslot = __float2bfloat16_rn(safe ? kv * e : 0.f);  // K^0 in place of k
                 }
-#pragma unroll
-                for (int g = 0; g < 2; ++g) {
-                    float tb[16];
-#pragma unroll
-                    for (int r = 0; r < 16; ++r) {
-                        const int t = 32 * hf + 16 * g + r;
-                        const bool v = t < nvalid;
-                        B += v ? lav[16 * g + r] * kLog2e : 0.f;
-                        const float kv = v ? __bfloat162float(__ushort_as_bfloat16(kraw[16 * g + r])) : 0.f;
-                        const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; used when safe
-                        tb[r] = safe ? e : B;
-                        *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c)) =
-                            __float2bfloat16_rn(safe ? kv * e : 0.f);
-                    }
-                    tmem_st16(tmem + lane_off + 384u + uint32_t(32 * hf + 16 * g), tb);
-                }
+                tmem_st16(tmem + lane_off + 384u + uint32_t(16 * g), tb);
             }
             if (__any_sync(0xffffffffu, !safe) && lane == 0) atomicOr(&bar.any_exact, 1);
             tmem_wait_st();
@@ -484,19 +485,19 @@ static_assert(kSmem <= 232448, "shared memory");
 gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
                                const void* v, const __nv_bfloat16* Qt, const float* gam, const __nv_bfloat16* Sbuf,
                                const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, cudaStream_t s) {
-    CUtensorMap m[10];
+    CUtensorMap m[11];
     memset(m, 0, sizeof(m));
     const uint64_t L = uint64_t(p.L), K = uint64_t(p.K), V = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
     if (!(map_sw128(&m[0], dO, V, L, BH) && map_sw128(&m[1], v, V, L, BH) && map_sw128(&m[2], Sbuf, V, K, BH * N) &&
           map_sw128(&m[3], Dbuf, V, K, BH * N) && map_sw128(&m[4], Qt, K, L, BH) && map_sw128(&m[5], q, K, L, BH) &&
           map_sw128(&m[6], k, K, L, BH) && map_sw128(&m[7], dq, K, L, BH) && map_sw128(&m[8], dk, K, L, BH) &&
-          map_f32_tile(&m[9], dla, K, L, BH)))
+          map_f32_tile(&m[9], dla, K, L, BH) && map_f32_tile(&m[10], la, K, L, BH)))
         return GLA_ERR_CUDA;
     if (cudaFuncSetAttribute(k_bwd_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.K / 128), unsigned(p.BH));
     GLA_LAUNCH("tc_bwd_chunk", k_bwd_chunk, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
-               m[8], m[9],
+               m[8], m[9], m[10],
                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, gam,
                static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K, p.V,
                device_error_word());

@@ -35,7 +35,9 @@ using namespace tc;
 
 constexpr int C = kTcChunk;
 constexpr uint32_t PIECE = 16384;
-constexpr int kThreads = 192;
+// warp 0 TMA, warp 1 MMA, then one group of four epilogue warps per 64 value columns
+template <int BVS>
+constexpr int st_threads() { return 64 + 128 * (BVS / 64); }
 
 // Tile of BVS value columns (64 or 128): chunks in flight, bytes per chunk
 // (the key-channel pair of A pieces and BVS / 64 value pieces), CTAs per SM.
@@ -55,7 +57,7 @@ struct StBars {
 };
 
 template <int BVS, bool REVERSE>
-__global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
+__global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     k_states_walk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmS,
                   const float* __restrict__ gam, const float* __restrict__ init, float* __restrict__ fin,
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&bar.u_full[b], 1);
-            mbar_init(&bar.u_empty[b], 128);
+            mbar_init(&bar.u_empty[b], 128 * (BVS / 64));
         }
         mbar_init(&bar.drain, 1);
         bar.abort_flag = 0;
@@ -144,24 +146,28 @@ __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
             mbar_drain(&bar.drain, 0);
         }
     } else {
-        // state epilogue: thread = key channel (TMEM lane), 64 value columns in registers
+        // state epilogue: BVS / 64 groups of four warps; thread = key channel (TMEM lane), the 64 value
+        // columns of its group in registers
         const int q4 = warp & 3;
+        const int grp = (warp - 2) >> 2;
         const int row = 32 * q4 + lane;
         const int64_t c = kbase + row;
+        const int col0 = 64 * grp;  // first value column of the group within the tile
         const uint32_t lane_off = uint32_t(32 * q4) << 16;
-        float x[BVS];
+        float x[64];
 #pragma unroll
-        for (int e = 0; e < BVS / 4; ++e) {
-            const float4 v4 = init ? reinterpret_cast<const float4*>(init + (bh * K + c) * V + v0)[e]
+        for (int e = 0; e < 16; ++e) {
+            const float4 v4 = init ? reinterpret_cast<const float4*>(init + (bh * K + c) * V + v0 + col0)[e]
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
             x[4 * e] = v4.x;
             x[4 * e + 1] = v4.y;
             x[4 * e + 2] = v4.z;
             x[4 * e + 3] = v4.w;
         }
-        // the bf16 copy of each entering state is staged in shared memory (128-byte swizzle) and
-        // written by TMA stores issued by one thread, so the register file never waits on the stores
-        uint8_t* stg = ring + NSLOT * SLOT_BYTES;
+        // the bf16 copy of each entering state is staged in shared memory (128-byte swizzle, one
+        // piece per group) and written by a TMA store issued by one thread of the group, so the
+        // register file never waits on the stores
+        uint8_t* stg = ring + NSLOT * SLOT_BYTES + grp * PIECE;
         const bool issuer = row == 0;
         bool ok = true;
         float g_next = gam[(bh * N + chunk_of(0)) * K + c];
@@ -172,20 +178,17 @@ __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
             const int ci = chunk_of(step);
             const float g = g_next;  // loaded one step ahead, off the critical path
             if (step + 1 < nsteps) g_next = gam[(bh * N + chunk_of(step + 1)) * K + c];
-            if (issuer) bulk_wait_read_all();  // the previous step's stores have read the staging tile
-            named_sync(1, 128);
+            if (issuer) bulk_wait_read_all();  // the previous step's store has read the staging piece
+            named_sync(1 + grp, 128);
 #pragma unroll
-            for (int ch = 0; ch < BVS / 8; ++ch)
-                *reinterpret_cast<uint4*>(stg + (ch >> 3) * PIECE + uint32_t(row) * 128u +
-                                          uint32_t(((ch & 7) ^ (row & 7)) << 4)) =
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(stg + uint32_t(row) * 128u + uint32_t((ch ^ (row & 7)) << 4)) =
                     make_uint4(pack_bf16x2(x[8 * ch], x[8 * ch + 1]), pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]),
                                pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]), pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]));
             fence_proxy_async_smem();
-            named_sync(1, 128);
+            named_sync(1 + grp, 128);
             if (issuer && ok) {
-#pragma unroll
-                for (int q = 0; q < BVS / 64; ++q)
-                    tma_store_3d(&tmS, v0 + 64 * q, kbase, int(bh * N + ci), stg + q * PIECE);
+                tma_store_3d(&tmS, v0 + col0, kbase, int(bh * N + ci), stg);
                 bulk_commit();
             }
             // tcgen05.ld is warp-collective: the condition must be the same for the whole warp
@@ -193,10 +196,10 @@ __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
             if (ok) {
                 tc_fence_after();
 #pragma unroll
-                for (int c32 = 0; c32 < BVS / 32; ++c32) {
+                for (int c32 = 0; c32 < 2; ++c32) {
                     float u[32];
-                    tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32), u);
-                    tmem_ld16(tmem + lane_off + uint32_t(b * BVS + 32 * c32 + 16), u + 16);
+                    tmem_ld16(tmem + lane_off + uint32_t(b * BVS + col0 + 32 * c32), u);
+                    tmem_ld16(tmem + lane_off + uint32_t(b * BVS + col0 + 32 * c32 + 16), u + 16);
                     tmem_wait_ld();
 #pragma unroll
                     for (int e = 0; e < 32; ++e) x[32 * c32 + e] = fmaf(g, x[32 * c32 + e], u[e]);
@@ -210,9 +213,9 @@ __global__ void __launch_bounds__(kThreads, StCfg<BVS>::min_blocks)
             for (int w = 0; w < 2; ++w) {
                 float* f = w ? fin2 : fin;
                 if (!f) continue;
-                float4* d4 = reinterpret_cast<float4*>(f + (bh * K + c) * V + v0);
+                float4* d4 = reinterpret_cast<float4*>(f + (bh * K + c) * V + v0 + col0);
 #pragma unroll
-                for (int e = 0; e < BVS / 4; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
+                for (int e = 0; e < 16; ++e) d4[e] = make_float4(x[4 * e], x[4 * e + 1], x[4 * e + 2], x[4 * e + 3]);
             }
         }
     }
@@ -253,7 +256,7 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH));
-    GLA_LAUNCH(name, fn, grid, kThreads, smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
+    GLA_LAUNCH(name, fn, grid, wide ? st_threads<128>() : st_threads<64>(), smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
                device_error_word());
     return GLA_OK;
 }
