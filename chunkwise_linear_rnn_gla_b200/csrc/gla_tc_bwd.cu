@@ -37,11 +37,12 @@
 // [128,256) dQ^T; [256,384) dK~^T inter part (v D^T); [384,512) per-token gate
 // table (e^{-B}, or B itself for a channel beyond the bound).
 //
-// Roles (320 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
+// Roles (576 threads): warp 0 TMA producer; warp 1 TMEM owner and MMA issuer;
 // warps 2-5 "row" warps (x_c = sum_v D S from the staged tiles, then the dP
 // epilogue: mask, bf16, swizzled shared tile); warps 6-9 "gate" warps
-// (thread = key channel: cumsum, gate table, K^0 operand; at the end dq, dk
-// and the gate gradient).
+// (thread = key channel: cumsum from the staged log-gate tile, gate table, K^0
+// operand); at the end warps 2-17 in four groups of 32 tokens form dq, dk and
+// the gate gradient, staged in shared memory and written by TMA stores.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -73,7 +74,8 @@ constexpr uint32_t KS_OFF = 10 * PIECE;            //                       k ti
 // after the intra MMAs: exact-path dk terms for tokens 0-63 over the Q~ tile and for tokens
 // 64-127 over K^0; after the exact pass: per-channel sums exchanged between the warp groups
 // over the masked dP tile
-constexpr int kThreads = 320;
+constexpr int kThreads = 576;
+constexpr int kFinal = 512;  // threads of the final phase: warps 2-17
 constexpr float kSafeDecay = 64.f;
 constexpr float kSafeGam = 1.6038109e-28f;  // e^-64
 
@@ -232,11 +234,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_drain(&bar.drain, 0);
         }
     } else {
-        // ---- warps 2-9: thread = key channel c of this CTA's 128 (TMEM lane c); warps 2-5 are
-        // the row warps, warps 6-9 the gate warps; both groups cover the four lane quadrants
+        // ---- warps 2-17: thread = key channel c of this CTA's 128 (TMEM lane c); warps 2-5 are
+        // the row warps, warps 6-9 the gate warps, warps 10-17 join for the final phase only; each
+        // group of four warps covers the four lane quadrants
         const int q4 = warp & 3;
         const int c = 32 * q4 + lane;
-        const bool gate_warp = warp >= 6;
+        const bool row_warp = warp < 6;
+        const bool gate_warp = warp >= 6 && warp < 10;
+        const int fgrp = (warp - 2) >> 2;  // final-phase group: tokens 32 fgrp .. 32 fgrp + 31
         const uint32_t lane_off = uint32_t(32 * q4) << 16;
         const int64_t chg = int64_t(128) * kh + c;
         const bool safe = gam[(bh * N + i) * K + chg] >= kSafeGam;
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int64_t rb = (bh * L + t0) * K + chg;
         const float* lap = la + rb;
         auto roff = [&](int t) -> uint32_t { return uint32_t(t < nvalid ? t : nvalid - 1) * uint32_t(K); };
-        if (!gate_warp) {
+        if (row_warp) {
             // x_c = sum_v D_i[c,v] S_[i][c,v] from the staged tiles
             float x = 0.f;
             bool ok = true;
@@ -298,11 +303,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
                 mbar_arrive(&bar.dpm_ready);
             }
-        } else {
-            // per-chunk cumsum along the tokens (base-2 units: e^x = 2^(x log2 e)), gate table
-            // into TMEM, K^0 operand into shared memory
+        } else if (gate_warp) {
             // per-chunk cumsum along the tokens from the staged tiles (rows past the end of the
-            // sequence are zero-filled by TMA), in base-2 units: e^x = 2^(x log2 e)
+            // sequence are zero-filled by TMA) in base-2 units, e^x = 2^(x log2 e); gate table into
+            // TMEM; the k tile becomes the K^0 operand in place
             const bool pro = __all_sync(0xffffffffu, mbar_wait(&bar.pro_full, 0, err, abort_flag));
             const float* sLA = reinterpret_cast<const float*>(base + LA_OFF);
             float B = 0.f;
@@ -327,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             mbar_arrive(&bar.khat_ready);
         }
-        // ---- final phase, warps 2-9: tokens [0,64) on the gate warps, [64,128) on the row warps.
+        // ---- final phase, warps 2-17: four groups of 32 tokens.
         float* rbuf = reinterpret_cast<float*>(base + RB_OFF);  // [t][c]: exact dq terms, then r
         auto xk = [&](int t) -> float* {                        // [t][c]: exact dk terms
             return reinterpret_cast<float*>(base + (t < C / 2 ? QT_OFF : KH_OFF)) + (t & (C / 2 - 1)) * C + c;
@@ -368,13 +372,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *xk(t) = ek;
             }
         }
-        named_sync(3, 256);
+        named_sync(3, kFinal);
         float* xch = reinterpret_cast<float*>(base + DPM_OFF);  // free once the exact pass is done
         // dq and dk are staged (bf16, 128-byte swizzle) over the Q~ and K^0 tiles and written by TMA
         // stores, unless those areas hold exact-path terms
         const bool stage = bar.any_exact == 0;
         const bool issuer = gate_warp && c == 0;
-        const int tlo = gate_warp ? 0 : C / 2;
+        const int tlo = 32 * fgrp;
         float kin = 0.f, rsum = 0.f;  // sum_s K~_s (v_s D_i^T) and sum_s r_s over this half
         float eGam = 0.f, Gam = 0.f;  // Gamma in base-2 units
         if (ok) {
@@ -388,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 eGam = safe ? __fdividef(1.f, v8[7]) : exp2_ftz(fminf(v8[7], 0.f));
             }
 #pragma unroll 1
-            for (int g = tlo / 16; g < tlo / 16 + C / 32; ++g) {
+            for (int g = tlo / 16; g < tlo / 16 + 2; ++g) {
                 float vQ[16], vJ[16], vI[16], vT[16];
                 tmem_ld16(tmem + lane_off + 128u + uint32_t(16 * g), vQ);
                 tmem_ld16(tmem + lane_off + 256u + uint32_t(16 * g), vJ);
@@ -424,11 +428,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
             }
-            xch[(gate_warp ? 0 : 128) + c] = kin;
-            if (!gate_warp) xch[256 + c] = rsum;
+            xch[128 * fgrp + c] = kin;
+            xch[512 + 128 * fgrp + c] = rsum;
         }
         fence_proxy_async_smem();
-        named_sync(3, 256);
+        named_sync(3, kFinal);
         if (issuer && ok && stage) {  // rows past the end of the sequence are clipped by the TMA unit
             for (int h = 0; h < 2; ++h) {
                 tma_store_3d(&tmDQ, 128 * kh + 64 * h, i * C, int(bh), base + QT_OFF + h * PIECE);
@@ -438,15 +442,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (ok) {
             // reverse cumsum in place; the carry from all later chunks is e^Gamma x_c + sum_s K~_s (v_s D_i^T)
-            float suf = eGam * bar.xd[c] + xch[c] + xch[128 + c] + (gate_warp ? xch[256 + c] : 0.f);
+            float suf = eGam * bar.xd[c];
+#pragma unroll
+            for (int f = 0; f < 4; ++f) suf += xch[128 * f + c] + (f > fgrp ? xch[512 + 128 * f + c] : 0.f);
 #pragma unroll 4
-            for (int t = tlo + C / 2 - 1; t >= tlo; --t) {
+            for (int t = tlo + 31; t >= tlo; --t) {
                 suf += rbuf[t * C + c];
                 rbuf[t * C + c] = suf;
             }
         }
         fence_proxy_async_smem();
-        named_sync(3, 256);
+        named_sync(3, kFinal);
         if (issuer && ok) {
             tma_store_3d(&tmDLA, 128 * kh, i * C, int(bh), rbuf);  // dense [128 tokens x 128 channels] fp32
             bulk_commit();
