@@ -81,3 +81,25 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
         gla_status _st = ::gla::launch_end(name, stream);                          \
         if (_st != GLA_OK) return _st;                                             \
     } while (0)
+
+// Launch with programmatic dependent launch: the kernel's CTAs may start (and run
+// their prologue: barrier init, TMEM allocation, tensor-map prefetch) while the
+// previous kernel on the stream drains. Every kernel launched this way executes
+// tc::pdl_wait() before it touches global memory that earlier work writes or reads.
+#define GLA_LAUNCH_PDL(name, kernel, grid, block, smem, strm_, ...)                              \
+    do {                                                                                          \
+        ::gla::launch_begin(name, strm_);                                                        \
+        cudaLaunchConfig_t _cfg = {};                                                             \
+        _cfg.gridDim = dim3(grid);                                                                \
+        _cfg.blockDim = dim3(block);                                                              \
+        _cfg.dynamicSmemBytes = (smem);                                                           \
+        _cfg.stream = (strm_);                                                                   \
+        cudaLaunchAttribute _attr[1];                                                             \
+        _attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;                         \
+        _attr[0].val.programmaticStreamSerializationAllowed = 1;                                  \
+        _cfg.attrs = _attr;                                                                       \
+        _cfg.numAttrs = 1;                                                                        \
+        (void)cudaLaunchKernelEx(&_cfg, kernel, __VA_ARGS__);                                     \
+        gla_status _st = ::gla::launch_end(name, strm_);                                         \
+        if (_st != GLA_OK) return _st;                                                            \
+    } while (0)

@@ -143,6 +143,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_slot;
+    // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
+    // nothing below touches global memory before that kernel has completed
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -502,7 +506,7 @@ gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, c
     if (cudaFuncSetAttribute(k_bwd_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.K / 128), unsigned(p.BH));
-    GLA_LAUNCH("tc_bwd_chunk", k_bwd_chunk, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
+    GLA_LAUNCH_PDL("tc_bwd_chunk", k_bwd_chunk, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
                m[8], m[9], m[10],
                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, gam,
                static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K, p.V,

@@ -95,6 +95,10 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_slot;
+    // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
+    // nothing below touches global memory before that kernel has completed
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -239,7 +243,7 @@ gla_status launch_out(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, 
     const int64_t items = p.BH * p.N * (p.V / OutCfg<NQ>::bvo);
     const int64_t sms = sm_count();
     const unsigned grid = unsigned(items < sms ? items : sms);
-    GLA_LAUNCH(name, fn, dim3(grid), kOutThreads, smem, s, m[0], m[1], m[2], m[3], Y, p.L, p.N, p.V, p.BH,
+    GLA_LAUNCH_PDL(name, fn, dim3(grid), kOutThreads, smem, s, m[0], m[1], m[2], m[3], Y, p.L, p.N, p.V, p.BH,
                device_error_word());
     return GLA_OK;
 }

@@ -120,6 +120,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_slot;
+    // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
+    // nothing below touches global memory before that kernel has completed
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 8) {
         if (lane == 0) {
@@ -313,7 +317,7 @@ gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const 
     auto fn = p.K == 256 ? k_tc_prep<256> : k_tc_prep<128>;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    GLA_LAUNCH("tc_prep", fn, dim3(unsigned(p.N), unsigned(p.BH)), kThreads, kSmem, s,
+    GLA_LAUNCH_PDL("tc_prep", fn, dim3(unsigned(p.N), unsigned(p.BH)), kThreads, kSmem, s,
                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, Qt, Kt, P, gam, p.L,
                p.N, device_error_word());
     return GLA_OK;

@@ -97,6 +97,10 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_slot;
+    // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
+    // nothing below touches global memory before that kernel has completed
+    pdl_launch_dependents();
+    pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -256,7 +260,7 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH));
-    GLA_LAUNCH(name, fn, grid, wide ? st_threads<128>() : st_threads<64>(), smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
+    GLA_LAUNCH_PDL(name, fn, grid, wide ? st_threads<128>() : st_threads<64>(), smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
                device_error_word());
     return GLA_OK;
 }

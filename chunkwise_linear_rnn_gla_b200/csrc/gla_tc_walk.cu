@@ -187,6 +187,10 @@ __global__ void __launch_bounds__(WalkCfg<NH, MODE>::threads, WalkCfg<NH, MODE>:
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = bar.tmem_slot;
+    // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
+    // nothing below touches global memory before that kernel has completed
+    pdl_launch_dependents();
+    pdl_wait();
     const Sched sched{nsteps, MODE};
 
     if (warp == 0) {
@@ -529,7 +533,7 @@ gla_status launch_walk(const Problem& p, const WalkArgs& a, const CUtensorMap* m
     const unsigned gy = MODE == kWalkOutputOnly ? unsigned(p.N)
                         : MODE == kWalkStatesOnly ? unsigned(p.K / KC) : 1u;
     const dim3 grid(unsigned(p.V / BV), gy, unsigned(p.BH));
-    GLA_LAUNCH(name, fn, grid, Cfg::threads, smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], a.gam, a.init,
+    GLA_LAUNCH_PDL(name, fn, grid, Cfg::threads, smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], a.gam, a.init,
                a.fin, a.fin2, a.Y, a.states, p.L, p.N, p.V, p.K, device_error_word());
     return GLA_OK;
 }
