@@ -107,12 +107,12 @@ def kernel_models(w, C):
 # ncu capture of the default workload, with the SHA-1 of the kernel's source
 # file at capture time: a kernel whose source changed since reports null.
 NCU_TRAFFIC = {
-    "tc_prep": (76091392, "gla_tc_prep.cu", "c13be6f89c9b31d2bd2b53818730823b54d1811c"),
-    "tc_walk_states": (81700608, "gla_tc_states.cu", "58f1386a9107887b164f169c977a3b54ba03f471"),
-    "tc_output": (135941632, "gla_tc_out.cu", "073a31fe6a7d0be948a8a8d5796fb1e1e26cc317"),
-    "tc_walk_dstates": (74450688, "gla_tc_states.cu", "58f1386a9107887b164f169c977a3b54ba03f471"),
-    "tc_output_dv": (135902208, "gla_tc_out.cu", "073a31fe6a7d0be948a8a8d5796fb1e1e26cc317"),
-    "tc_bwd_chunk": (333266432, "gla_tc_bwd.cu", "058567593b0333a4e9b7914c6cf6905947952374"),
+    "tc_prep": (74569728, "gla_tc_prep.cu", "33a8a99db46d13e3db1856e62934183d4c9ac1d7"),
+    "tc_walk_states": (82017792, "gla_tc_states.cu", "e49ec5c3d4704810b8c99f795fb0035014e1a95e"),
+    "tc_output": (136148992, "gla_tc_out.cu", "646393dd6c7c3f3ca6530ee79c6aa6cff1ffd9c8"),
+    "tc_walk_dstates": (73954816, "gla_tc_states.cu", "e49ec5c3d4704810b8c99f795fb0035014e1a95e"),
+    "tc_output_dv": (136209920, "gla_tc_out.cu", "646393dd6c7c3f3ca6530ee79c6aa6cff1ffd9c8"),
+    "tc_bwd_chunk": (335615744, "gla_tc_bwd.cu", "ffb14ef24fd5c05266f070ee0ac32252c2b63af9"),
 }
 
 
