@@ -145,6 +145,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bar.tmem_slot;
     // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
     // nothing below touches global memory before that kernel has completed
+    if (threadIdx.x == 0) {  // tensor maps are kernel parameters: fetch them while the previous kernel drains
+        tma_prefetch(&tmDO);
+        tma_prefetch(&tmV);
+        tma_prefetch(&tmS);
+        tma_prefetch(&tmD);
+        tma_prefetch(&tmQt);
+        tma_prefetch(&tmQ);
+        tma_prefetch(&tmK);
+        tma_prefetch(&tmLA);
+    }
     pdl_launch_dependents();
     pdl_wait();
 

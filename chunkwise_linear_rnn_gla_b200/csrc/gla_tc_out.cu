@@ -97,15 +97,17 @@ __global__ void __launch_bounds__(kOutThreads, 1)
     const uint32_t tmem = bar.tmem_slot;
     // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
     // nothing below touches global memory before that kernel has completed
+    if (threadIdx.x == 0) {  // tensor maps are kernel parameters: fetch them while the previous kernel drains
+        tma_prefetch(&tmA);
+        tma_prefetch(&tmX);
+        tma_prefetch(&tmP);
+        tma_prefetch(&tmB);
+    }
     pdl_launch_dependents();
     pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch(&tmA);
-            tma_prefetch(&tmX);
-            tma_prefetch(&tmP);
-            tma_prefetch(&tmB);
             bool ok = true;
             int gc = 0;  // groups issued
             for (int it = 0; it < n_items && ok; ++it) {

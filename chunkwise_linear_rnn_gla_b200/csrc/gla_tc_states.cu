@@ -43,15 +43,18 @@ constexpr int st_threads() { return 64 + 128 * (BVS / 64); }
 // (the key-channel pair of A pieces and BVS / 64 value pieces), CTAs per SM.
 template <int BVS>
 struct StCfg {
-    static constexpr int nslot = BVS == 128 ? 3 : 2;
+    static constexpr int nslot = 2;
+    static constexpr int nu = 3;  // TMEM accumulators for the chunk products: the MMAs run up to three chunks ahead
     static constexpr uint32_t slot_bytes = uint32_t(2 + BVS / 64) * PIECE;
     static constexpr int min_blocks = 1;
-    static constexpr size_t smem = 1024 + size_t(nslot) * slot_bytes + size_t(BVS / 64) * PIECE;  // + staging
+    // + two staging pieces per epilogue group (double-buffered bf16 state for the TMA stores)
+    static constexpr size_t smem = 1024 + size_t(nslot) * slot_bytes + size_t(2 * (BVS / 64)) * PIECE;
+    static constexpr uint32_t tmem_cols = 3 * BVS <= 256 ? 256u : 512u;
 };
 
 struct StBars {
     uint64_t full[3], empty[3];
-    uint64_t u_full[2], u_empty[2], drain;
+    uint64_t u_full[3], u_empty[3], drain;
     uint32_t tmem_slot;
     int abort_flag;
 };
@@ -67,7 +70,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NSLOT = StCfg<BVS>::nslot;
     constexpr uint32_t SLOT_BYTES = StCfg<BVS>::slot_bytes;
-    StBars& bar = *reinterpret_cast<StBars*>(ring + NSLOT * SLOT_BYTES + (BVS / 64) * PIECE);
+    StBars& bar = *reinterpret_cast<StBars*>(ring + NSLOT * SLOT_BYTES + 2 * (BVS / 64) * PIECE);
     volatile int* abort_flag = &bar.abort_flag;
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int v0 = blockIdx.x * BVS;
@@ -81,7 +84,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
             mbar_init(&bar.full[s], 1);
             mbar_init(&bar.empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
+        for (int b = 0; b < 3; ++b) {
             mbar_init(&bar.u_full[b], 1);
             mbar_init(&bar.u_empty[b], 128 * (BVS / 64));
         }
@@ -90,7 +93,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
         fence_barrier_init();
     }
     if (warp == 1) {
-        tmem_alloc(&bar.tmem_slot, 2 * BVS);
+        tmem_alloc(&bar.tmem_slot, StCfg<BVS>::tmem_cols);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -99,13 +102,16 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     const uint32_t tmem = bar.tmem_slot;
     // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
     // nothing below touches global memory before that kernel has completed
+    if (threadIdx.x == 0) {  // tensor maps are kernel parameters: fetch them while the previous kernel drains
+        tma_prefetch(&tmA);
+        tma_prefetch(&tmB);
+        tma_prefetch(&tmS);
+    }
     pdl_launch_dependents();
     pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
-            tma_prefetch(&tmA);
-            tma_prefetch(&tmB);
             bool ok = true;
             int step = 0;
             for (; step < nsteps && ok; ++step) {
@@ -133,8 +139,8 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
             const uint32_t id = idesc_bf16_f32(128, BVS, true, true);
             bool ok = true;
             for (int step = 0; step < nsteps && ok; ++step) {
-                const int s = step % NSLOT, b = step & 1;
-                ok = mbar_wait(&bar.u_empty[b], uint32_t(((step >> 1) & 1) ^ 1), err, abort_flag) &&
+                const int s = step % NSLOT, b = step % 3;
+                ok = mbar_wait(&bar.u_empty[b], uint32_t(((step / 3) & 1) ^ 1), err, abort_flag) &&
                      mbar_wait(&bar.full[s], uint32_t((step / NSLOT) & 1), err, abort_flag);
                 if (!ok) break;
                 tc_fence_after();
@@ -171,18 +177,19 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
         // the bf16 copy of each entering state is staged in shared memory (128-byte swizzle, one
         // piece per group) and written by a TMA store issued by one thread of the group, so the
         // register file never waits on the stores
-        uint8_t* stg = ring + NSLOT * SLOT_BYTES + grp * PIECE;
+        uint8_t* stg0 = ring + NSLOT * SLOT_BYTES + 2 * grp * PIECE;
         const bool issuer = row == 0;
         bool ok = true;
         float g_next = gam[(bh * N + chunk_of(0)) * K + c];
         // every epilogue thread passes every named barrier, also after a wait gave up (bar.sync has
         // no time limit); a failed wait only skips the work
         for (int step = 0; step < nsteps; ++step) {
-            const int b = step & 1;
+            const int b = step % 3;
             const int ci = chunk_of(step);
+            uint8_t* stg = stg0 + (step & 1) * PIECE;
             const float g = g_next;  // loaded one step ahead, off the critical path
             if (step + 1 < nsteps) g_next = gam[(bh * N + chunk_of(step + 1)) * K + c];
-            if (issuer) bulk_wait_read_all();  // the previous step's store has read the staging piece
+            if (issuer) bulk_wait_read_but1();  // the store of two steps ago has read this staging piece
             named_sync(1 + grp, 128);
 #pragma unroll
             for (int ch = 0; ch < 8; ++ch)
@@ -196,7 +203,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
                 bulk_commit();
             }
             // tcgen05.ld is warp-collective: the condition must be the same for the whole warp
-            ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar.u_full[b], uint32_t((step >> 1) & 1), err, abort_flag));
+            ok = __all_sync(0xffffffffu, ok && mbar_wait(&bar.u_full[b], uint32_t((step / 3) & 1), err, abort_flag));
             if (ok) {
                 tc_fence_after();
 #pragma unroll
@@ -227,7 +234,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 2 * BVS);
+        tmem_dealloc(tmem, StCfg<BVS>::tmem_cols);
     }
 }
 

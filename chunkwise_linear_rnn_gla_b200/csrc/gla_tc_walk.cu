@@ -189,6 +189,12 @@ __global__ void __launch_bounds__(WalkCfg<NH, MODE>::threads, WalkCfg<NH, MODE>:
     const uint32_t tmem = bar.tmem_slot;
     // programmatic dependent launch: the prologue above overlapped the previous kernel's tail;
     // nothing below touches global memory before that kernel has completed
+    if (threadIdx.x == 0) {  // tensor maps are kernel parameters: fetch them while the previous kernel drains
+        tma_prefetch(&tmA1);
+        tma_prefetch(&tmB1);
+        tma_prefetch(&tmA2);
+        tma_prefetch(&tmP);
+    }
     pdl_launch_dependents();
     pdl_wait();
     const Sched sched{nsteps, MODE};
@@ -196,10 +202,6 @@ __global__ void __launch_bounds__(WalkCfg<NH, MODE>::threads, WalkCfg<NH, MODE>:
     if (warp == 0) {
         // ------------------------------------------------------ TMA producer
         if (lane == 0) {
-            tma_prefetch(&tmA1);
-            tma_prefetch(&tmB1);
-            tma_prefetch(&tmA2);
-            tma_prefetch(&tmP);
             Cursor<Cfg::ring> cur;
             uint32_t par = 0;            // parity of the next use, one bit per slot
             uint32_t pending = 0;        // slots with a load whose completion nobody waited for yet
