@@ -67,10 +67,10 @@ constexpr uint32_t STAGE_BYTES = 4 * PIECE;
 constexpr uint32_t LA_OFF = 8 * PIECE;             // log a tile, fp32 [128 tokens][128 channels], read by the prologue
 constexpr uint32_t KH_OFF = 12 * PIECE;            // k tile, rescaled in place into the K^0 operand, 2 pieces
 constexpr uint32_t DPM_OFF = 0;                    // after the value loop: masked dP (bf16), 2 pieces
-constexpr uint32_t QT_OFF = 2 * PIECE;             //                       Q~ tile, 2 pieces
+constexpr uint32_t QT_OFF = LA_OFF;                // once the prologue is done: Q~ tile, 2 pieces
 constexpr uint32_t RB_OFF = 4 * PIECE;             //                       r = q dq - k dk, fp32 [128][128]
-constexpr uint32_t QS_OFF = 8 * PIECE;             //                       q tile, 2 pieces
-constexpr uint32_t KS_OFF = 10 * PIECE;            //                       k tile, 2 pieces
+constexpr uint32_t QS_OFF = LA_OFF + 2 * PIECE;    // once the prologue is done: q tile, 2 pieces
+constexpr uint32_t KS_OFF = 2 * PIECE;             // after the value loop: k tile, 2 pieces
 // after the intra MMAs: exact-path dk terms for tokens 0-63 over the Q~ tile and for tokens
 // 64-127 over K^0; after the exact pass: per-channel sums exchanged between the warp groups
 // over the masked dP tile
@@ -180,19 +180,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tma_load_3d(st + 2 * PIECE, &tmS, 64 * vb, 128 * kh, int(bh * N + i), &bar.full[s]);
                 tma_load_3d(st + 3 * PIECE, &tmD, 64 * vb, 128 * kh, int(bh * N + i), &bar.full[s]);
             }
-            // the Q~ tile goes where stage 0 was once every stage has been consumed; q and k go where
-            // the prologue's log a tile was
-            if (ok && mbar_wait(&bar.accA, 0, err, abort_flag) && mbar_wait(&bar.xd_ready, 0, err, abort_flag) &&
-                mbar_wait(&bar.khat_ready, 0, err, abort_flag)) {
+            // Q~ and q go where the prologue's log a tile was as soon as the prologue is done (usually
+            // before the last value stage is consumed); k goes where stage 0 was once the value loop
+            // (MMAs and the row warps' reads) is over
+            if (ok && mbar_wait(&bar.khat_ready, 0, err, abort_flag)) {
                 mbar_arrive_expect_tx(&bar.qt_full, 2 * PIECE);
                 tma_load_3d(base + QT_OFF, &tmQt, 128 * kh, i * C, int(bh), &bar.qt_full);
                 tma_load_3d(base + QT_OFF + PIECE, &tmQt, 128 * kh + 64, i * C, int(bh), &bar.qt_full);
-                // raw q and k tiles for the elementwise epilogue
+                // raw q and k tiles for the elementwise epilogue (one barrier for both)
                 mbar_arrive_expect_tx(&bar.qk_full, 4 * PIECE);
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < 2; ++h)
                     tma_load_3d(base + QS_OFF + h * PIECE, &tmQ, 128 * kh + 64 * h, i * C, int(bh), &bar.qk_full);
-                    tma_load_3d(base + KS_OFF + h * PIECE, &tmK, 128 * kh + 64 * h, i * C, int(bh), &bar.qk_full);
-                }
+                if (mbar_wait(&bar.accA, 0, err, abort_flag) && mbar_wait(&bar.xd_ready, 0, err, abort_flag))
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_3d(base + KS_OFF + h * PIECE, &tmK, 128 * kh + 64 * h, i * C, int(bh), &bar.qk_full);
                 mbar_drain(&bar.qt_full, 0);
                 mbar_drain(&bar.qk_full, 0);
             } else if (!ok) {
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tma_store_3d(&tmDLA, 128 * kh, i * C, int(bh), rbuf);  // dense [128 tokens x 128 channels] fp32
             bulk_commit();
         }
-        if (issuer) bulk_wait_all();
+        if (issuer) bulk_wait_read_all();  // the stores finish on their own; the CTA may exit once they have read smem
     }
     tc_fence_before();
     __syncthreads();

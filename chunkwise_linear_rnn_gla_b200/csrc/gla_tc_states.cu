@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
                 mbar_arrive(&bar.u_empty[b]);
             }
         }
-        if (issuer) bulk_wait_all();
+        if (issuer) bulk_wait_read_all();  // the stores finish on their own; the CTA may exit once they have read smem
         if (ok) {
             for (int w = 0; w < 2; ++w) {
                 float* f = w ? fin2 : fin;
