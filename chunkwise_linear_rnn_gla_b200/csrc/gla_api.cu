@@ -151,7 +151,9 @@ gla_status resolve(const gla_desc* d, Problem& p) {
         if (!p.bf16) return GLA_ERR_UNSUPPORTED;
         p.C = d->chunk ? d->chunk : 128;
         p.c = d->subchunk ? d->subchunk : 16;
-        p.state_mode = d->state_mode == GLA_STATE_AUTO ? GLA_STATE_NONMATERIALIZED : d->state_mode;
+        // materialised states are the faster mode on this path (the backward needs the stored states in
+        // either mode); non-materialised keeps the forward's footprint free of them
+        p.state_mode = d->state_mode == GLA_STATE_AUTO ? GLA_STATE_MATERIALIZED : d->state_mode;
     }
     if (p.c > p.C || p.C % p.c != 0) return GLA_ERR_INVALID_ARG;
     p.N = (p.L + p.C - 1) / p.C;

@@ -66,7 +66,7 @@ typedef enum gla_dtype {
 /* How the inter-chunk states are handled ("Approach" section: "materialized
  * or non-materialized inter-chunk states"). */
 typedef enum gla_state_mode {
-    GLA_STATE_AUTO = 0,            /* library picks                            */
+    GLA_STATE_AUTO = 0,            /* library picks: materialised              */
     GLA_STATE_MATERIALIZED = 1,    /* write S_[i] of every chunk to workspace  */
     GLA_STATE_NONMATERIALIZED = 2  /* keep S on chip while walking the chunks  */
 } gla_state_mode;
