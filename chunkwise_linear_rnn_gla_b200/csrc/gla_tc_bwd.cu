@@ -42,13 +42,15 @@
 // epilogue: mask, bf16, swizzled shared tile); warps 6-9 "gate" warps
 // (thread = key channel: cumsum from the staged log-gate tile, gate table, K^0
 // operand); at the end warps 2-17 in four groups of 32 tokens form dq, dk and
-// the gate gradient, staged in shared memory and written by TMA stores.
+// the gate gradient: dq and dk staged in shared memory and written by one TMA
+// store per group, dlog a written directly (128-byte rows per warp store).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
 #include <cstring>
+#include <type_traits>
 
 #include "gla_common.cuh"
 #include "gla_internal.h"
@@ -78,6 +80,7 @@ constexpr int kThreads = 576;
 constexpr int kFinal = 512;  // threads of the final phase: warps 2-17
 constexpr float kSafeDecay = 64.f;
 constexpr float kSafeGam = 1.6038109e-28f;  // e^-64
+constexpr uint32_t kStaggerNs = 8000;       // start offset of every other first-wave CTA
 
 struct BwdBars {
     uint64_t full[NSTAGE], empty[NSTAGE];
@@ -101,12 +104,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmD,
                 const __grid_constant__ CUtensorMap tmQt, const __grid_constant__ CUtensorMap tmQ,
                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmDQ,
-                const __grid_constant__ CUtensorMap tmDK, const __grid_constant__ CUtensorMap tmDLA,
+                const __grid_constant__ CUtensorMap tmDK,
                 const __grid_constant__ CUtensorMap tmLA,
                 const __nv_bfloat16* __restrict__ q,
                 const __nv_bfloat16* __restrict__ k, const float* __restrict__ la, const float* __restrict__ gam,
                 __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, float* __restrict__ dla, int64_t L,
-                int64_t N, int64_t K, int64_t V, int* err) {
+                int64_t N, int64_t K, int64_t V, uint32_t stagger_ns, uint32_t n_first, int* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     BwdBars& bar = *reinterpret_cast<BwdBars*>(base + KH_OFF + 2 * PIECE);
@@ -160,6 +163,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            // The CTAs of the first wave are released together (by the dependency wait) and would stay
+            // in lockstep: all streaming at once, then all in their epilogues with HBM idle. Every
+            // other first-wave CTA starts a fraction of a CTA's lifetime later, so that the loads of
+            // one half overlap the epilogues of the other, in this wave and in the ones that follow.
+            const uint32_t lin = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+            if (stagger_ns > 0 && lin < n_first && (lin & 1u)) {
+                const uint64_t until = global_ns() + stagger_ns;  // bounded: the host caps stagger_ns
+                while (global_ns() < until) __nanosleep(256);
+            }
             // the gate prologue's inputs first: log a (dense fp32) and k (into the K^0 operand area)
             mbar_arrive_expect_tx(&bar.pro_full, 4 * PIECE + 2 * PIECE);
             tma_load_3d(base + LA_OFF, &tmLA, 128 * kh, i * C, int(bh), &bar.pro_full);
@@ -329,14 +341,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int g = 0; g < C / 16 && pro; ++g) {
                 float tb[16];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int t = 16 * g + r;
-                    B += sLA[t * C + c] * kLog2e;
-                    __nv_bfloat16* kslot = reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c));
-                    const float kv = __bfloat162float(*kslot);
-                    const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; used when safe
-                    tb[r] = safe ? e : B;
-                    *kslot = __float2bfloat16_rn(safe ? kv * e : 0.f);  // K^0 in place of k
+                for (int h = 0; h < 2; ++h) {
+                    // the loads of 8 tokens first, so that none waits behind a store of the group
+                    float lv[8], kv[8];
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const int t = 16 * g + 8 * h + r;
+                        lv[r] = sLA[t * C + c];
+                        kv[r] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + KH_OFF + tile_off(t, c)));
+                    }
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        B += lv[r] * kLog2e;
+                        const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; used when safe
+                        tb[8 * h + r] = safe ? e : B;
+                        kv[r] = safe ? kv[r] * e : 0.f;
+                    }
+#pragma unroll
+                    for (int r = 0; r < 8; ++r)  // K^0 in place of k
+                        *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(16 * g + 8 * h + r, c)) =
+                            __float2bfloat16_rn(kv[r]);
                 }
                 tmem_st16(tmem + lane_off + 384u + uint32_t(16 * g), tb);
             }
@@ -392,9 +416,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // dq and dk are staged (bf16, 128-byte swizzle) over the Q~ and K^0 tiles and written by TMA
         // stores, unless those areas hold exact-path terms
         const bool stage = bar.any_exact == 0;
-        const bool issuer = gate_warp && c == 0;
+        // one thread per group of 32 tokens issues that group's TMA stores (rows past the end of the
+        // sequence are clipped by the TMA unit; a group entirely past it stores nothing)
+        const bool issuer = ((warp - 2) & 3) == 0 && lane == 0;
+        const bool grp_rows = 32 * fgrp < nvalid;
         const int tlo = 32 * fgrp;
-        float kin = 0.f, rsum = 0.f;  // sum_s K~_s (v_s D_i^T) and sum_s r_s over this half
+        float kin = 0.f, rsum = 0.f;  // sum_s K~_s (v_s D_i^T) and sum_s r_s over this group
         float eGam = 0.f, Gam = 0.f;  // Gamma in base-2 units
         if (ok) {
             tc_fence_after();
@@ -406,71 +433,82 @@ __global__ void __launch_bounds__(kThreads, 1)
                 Gam = safe ? 0.f : v8[7];
                 eGam = safe ? __fdividef(1.f, v8[7]) : exp2_ftz(fminf(v8[7], 0.f));
             }
+            // tokens of the group in reverse order: rbuf keeps the suffix sum of r within the group,
+            // the carry from later groups and chunks is added once every group's sum is known
+            auto run = [&](auto all_safe) {
 #pragma unroll 1
-            for (int g = tlo / 16; g < tlo / 16 + 2; ++g) {
-                float vQ[16], vJ[16], vI[16], vT[16];
-                tmem_ld16(tmem + lane_off + 128u + uint32_t(16 * g), vQ);
-                tmem_ld16(tmem + lane_off + 256u + uint32_t(16 * g), vJ);
-                tmem_ld16(tmem + lane_off + 0u + uint32_t(16 * g), vI);
-                tmem_ld16(tmem + lane_off + 384u + uint32_t(16 * g), vT);
-                tmem_wait_ld();
+                for (int g = tlo / 8 + 3; g >= tlo / 8; --g) {
+                    float vQ[8], vJ[8], vI[8], vT[8];
+                    tmem_ld8(tmem + lane_off + 128u + uint32_t(8 * g), vQ);
+                    tmem_ld8(tmem + lane_off + 256u + uint32_t(8 * g), vJ);
+                    tmem_ld8(tmem + lane_off + 0u + uint32_t(8 * g), vI);
+                    tmem_ld8(tmem + lane_off + 384u + uint32_t(8 * g), vT);
+                    tmem_wait_ld();
+                    // loads of the 8 tokens first, so that none waits behind a store of the group
+                    float qv[8], kv[8];
 #pragma unroll
-                for (int r = 0; r < 16; ++r) {
-                    const int t = 16 * g + r;
-                    const float qv = qs(t), kv = ks(t);
-                    float eGB, dqv, dkv;
-                    if (safe) {
-                        const float e = vT[r];  // e^{-B_t}
-                        eGB = eGam * e;
-                        dqv = __fdividef(vQ[r], e);
-                        dkv = eGB * vJ[r] + e * vI[r];
-                    } else {
-                        const float Bt = vT[r];
-                        eGB = exp2_ftz(fminf(Gam - Bt, 0.f));
-                        dqv = exp2_ftz(fminf(Bt, 0.f)) * vQ[r] + rbuf[t * C + c];
-                        dkv = eGB * vJ[r] + *xk(t);
+                    for (int r = 0; r < 8; ++r) {
+                        qv[r] = qs(8 * g + r);
+                        kv[r] = ks(8 * g + r);
                     }
-                    kin = fmaf(kv * eGB, vJ[r], kin);
-                    const float rr = qv * dqv - kv * dkv;
-                    rsum += rr;
-                    rbuf[t * C + c] = rr;
-                    if (stage) {
-                        *reinterpret_cast<__nv_bfloat16*>(base + QT_OFF + tile_off(t, c)) = __float2bfloat16_rn(dqv);
-                        *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c)) = __float2bfloat16_rn(dkv);
-                    } else if (t < nvalid) {
-                        dq[rb + int64_t(t) * K] = __float2bfloat16_rn(dqv);
-                        dk[rb + int64_t(t) * K] = __float2bfloat16_rn(dkv);
+#pragma unroll
+                    for (int r = 7; r >= 0; --r) {
+                        const int t = 8 * g + r;
+                        float eGB, dqv, dkv;
+                        if (decltype(all_safe)::value || safe) {
+                            const float e = vT[r];  // e^{-B_t}
+                            eGB = eGam * e;
+                            dqv = __fdividef(vQ[r], e);
+                            dkv = fmaf(eGB, vJ[r], e * vI[r]);
+                        } else {
+                            const float Bt = vT[r];
+                            eGB = exp2_ftz(fminf(Gam - Bt, 0.f));
+                            dqv = exp2_ftz(fminf(Bt, 0.f)) * vQ[r] + rbuf[t * C + c];
+                            dkv = eGB * vJ[r] + *xk(t);
+                        }
+                        kin = fmaf(kv[r] * eGB, vJ[r], kin);
+                        rsum += fmaf(qv[r], dqv, -kv[r] * dkv);
+                        rbuf[t * C + c] = rsum;
+                        if (stage) {
+                            *reinterpret_cast<__nv_bfloat16*>(base + QT_OFF + tile_off(t, c)) = __float2bfloat16_rn(dqv);
+                            *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(t, c)) = __float2bfloat16_rn(dkv);
+                        } else if (t < nvalid) {
+                            dq[rb + int64_t(t) * K] = __float2bfloat16_rn(dqv);
+                            dk[rb + int64_t(t) * K] = __float2bfloat16_rn(dkv);
+                        }
                     }
                 }
-            }
+            };
+            if (__all_sync(0xffffffffu, safe))
+                run(std::true_type{});
+            else
+                run(std::false_type{});
             xch[128 * fgrp + c] = kin;
             xch[512 + 128 * fgrp + c] = rsum;
         }
         fence_proxy_async_smem();
-        named_sync(3, kFinal);
-        if (issuer && ok && stage) {  // rows past the end of the sequence are clipped by the TMA unit
+        named_sync(4 + fgrp, 128);
+        if (issuer && ok && stage && grp_rows) {
             for (int h = 0; h < 2; ++h) {
-                tma_store_3d(&tmDQ, 128 * kh + 64 * h, i * C, int(bh), base + QT_OFF + h * PIECE);
-                tma_store_3d(&tmDK, 128 * kh + 64 * h, i * C, int(bh), base + KH_OFF + h * PIECE);
+                tma_store_3d(&tmDQ, 128 * kh + 64 * h, i * C + tlo, int(bh), base + QT_OFF + h * PIECE + tlo * 128);
+                tma_store_3d(&tmDK, 128 * kh + 64 * h, i * C + tlo, int(bh), base + KH_OFF + h * PIECE + tlo * 128);
             }
             bulk_commit();
         }
+        named_sync(3, kFinal);  // every group's sums are in xch
         if (ok) {
-            // reverse cumsum in place; the carry from all later chunks is e^Gamma x_c + sum_s K~_s (v_s D_i^T)
-            float suf = eGam * bar.xd[c];
+            // the carry from all later chunks is e^Gamma x_c + sum_s K~_s (v_s D_i^T); the later
+            // groups of this chunk add their sums of r. dlog a goes straight to global memory: a
+            // warp writes 32 consecutive channels (128 bytes) of one token per store
+            float carry = eGam * bar.xd[c];
 #pragma unroll
-            for (int f = 0; f < 4; ++f) suf += xch[128 * f + c] + (f > fgrp ? xch[512 + 128 * f + c] : 0.f);
-#pragma unroll 4
-            for (int t = tlo + 31; t >= tlo; --t) {
-                suf += rbuf[t * C + c];
-                rbuf[t * C + c] = suf;
-            }
-        }
-        fence_proxy_async_smem();
-        named_sync(3, kFinal);
-        if (issuer && ok) {
-            tma_store_3d(&tmDLA, 128 * kh, i * C, int(bh), rbuf);  // dense [128 tokens x 128 channels] fp32
-            bulk_commit();
+            for (int f = 0; f < 4; ++f) carry += xch[128 * f + c] + (f > fgrp ? xch[512 + 128 * f + c] : 0.f);
+            float dv[32];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) dv[u] = rbuf[(tlo + u) * C + c] + carry;
+#pragma unroll
+            for (int u = 0; u < 32; ++u)
+                if (tlo + u < nvalid) dla[rb + int64_t(tlo + u) * K] = dv[u];
         }
         if (issuer) bulk_wait_read_all();  // the stores finish on their own; the CTA may exit once they have read smem
     }
@@ -483,10 +521,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // [outer][rows][inner] bf16 tensor, box [128 rows x 64 inner], 128-byte swizzle
-bool map_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
+bool map_sw128(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer,
+               uint32_t box_rows = 128) {
     const uint64_t dims[3] = {inner, rows, outer};
     const uint64_t strides[2] = {inner * 2, inner * rows * 2};
-    const uint32_t box[3] = {64, 128, 1};
+    const uint32_t box[3] = {64, box_rows, 1};
     return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
@@ -506,22 +545,25 @@ static_assert(kSmem <= 232448, "shared memory");
 gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
                                const void* v, const __nv_bfloat16* Qt, const float* gam, const __nv_bfloat16* Sbuf,
                                const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, cudaStream_t s) {
-    CUtensorMap m[11];
+    CUtensorMap m[10];
     memset(m, 0, sizeof(m));
     const uint64_t L = uint64_t(p.L), K = uint64_t(p.K), V = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
     if (!(map_sw128(&m[0], dO, V, L, BH) && map_sw128(&m[1], v, V, L, BH) && map_sw128(&m[2], Sbuf, V, K, BH * N) &&
           map_sw128(&m[3], Dbuf, V, K, BH * N) && map_sw128(&m[4], Qt, K, L, BH) && map_sw128(&m[5], q, K, L, BH) &&
-          map_sw128(&m[6], k, K, L, BH) && map_sw128(&m[7], dq, K, L, BH) && map_sw128(&m[8], dk, K, L, BH) &&
-          map_f32_tile(&m[9], dla, K, L, BH) && map_f32_tile(&m[10], la, K, L, BH)))
+          map_sw128(&m[6], k, K, L, BH) && map_sw128(&m[7], dq, K, L, BH, 32) && map_sw128(&m[8], dk, K, L, BH, 32) &&
+          map_f32_tile(&m[9], la, K, L, BH)))
         return GLA_ERR_CUDA;
     if (cudaFuncSetAttribute(k_bwd_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.K / 128), unsigned(p.BH));
+    // one CTA per SM: stagger the first wave only when there are later waves for it to shape
+    const int64_t sms = sm_count();
+    const uint32_t stagger = int64_t(grid.x) * grid.y * grid.z > sms ? kStaggerNs : 0u;
     GLA_LAUNCH_PDL("tc_bwd_chunk", k_bwd_chunk, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
-               m[8], m[9], m[10],
+               m[8], m[9],
                static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, gam,
-               static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K, p.V,
-               device_error_word());
+               static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K, p.V, stagger,
+               unsigned(sms), device_error_word());
     return GLA_OK;
 }
 

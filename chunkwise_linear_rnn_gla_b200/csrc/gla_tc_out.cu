@@ -229,13 +229,6 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
     return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
-int sm_count() {
-    int dev = 0, n = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-        return 148;
-    return n > 0 ? n : 148;
-}
-
 template <int NH, int NQ, bool PT>
 gla_status launch_out(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, cudaStream_t s, const char* name) {
     auto fn = k_chunk_out<NH, NQ, PT>;

@@ -36,5 +36,12 @@ bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const 
     return r == CUDA_SUCCESS;
 }
 
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 148;
+    return n > 0 ? n : 148;
+}
+
 }  // namespace tc
 }  // namespace gla

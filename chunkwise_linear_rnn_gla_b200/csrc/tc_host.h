@@ -15,5 +15,8 @@ namespace tc {
 bool encode_tmap(CUtensorMap* map, CUtensorMapDataType dt, uint32_t rank, const void* base, const uint64_t* dims,
                  const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swizzle);
 
+// Number of SMs of the current device (148 if the query fails).
+int sm_count();
+
 }  // namespace tc
 }  // namespace gla
