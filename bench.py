@@ -234,6 +234,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed step eagerly instead of replaying it from a CUDA graph")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
 
@@ -300,7 +302,32 @@ def main():
 
     stream = torch.cuda.current_stream(dev)
 
-    def timed_pass(kernel_events):
+    # The step is captured once into a CUDA graph (the library's launches are capture-safe: host-side
+    # tensor maps, no allocation or synchronisation) and replayed, as a training loop would; the
+    # per-kernel timing pass stays eager because it needs an event pair around every launch.
+    graph, graph_launches, graph_note = None, 0, "eager"
+    if not args.no_graph:
+        try:
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(stream)
+            with torch.cuda.stream(side):
+                step()
+            stream.wait_stream(side)
+            torch.cuda.synchronize(dev)
+            graph = torch.cuda.CUDAGraph()
+            gla.gla_launch_count_reset()
+            with torch.cuda.graph(graph):
+                step()
+            graph_launches = gla.gla_launch_count()
+            for _ in range(max(3, args.warmup)):
+                graph.replay()
+            torch.cuda.synchronize(dev)
+            graph_note = "cuda_graph"
+        except Exception as ex:  # capture is an optimisation: report and time the eager step
+            graph, graph_note = None, "eager (graph capture failed: %s)" % type(ex).__name__
+            torch.cuda.synchronize(dev)
+
+    def timed_pass(kernel_events, use_graph=False):
         """K steps between barriers and synchronisations; L2 flushed before each step. Returns the
         summed step time (CUDA events on the launching stream) and our kernel launches."""
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
@@ -313,11 +340,14 @@ def main():
         for i in range(args.steps):
             flush.fill_(float(i))  # evict L2 (126 MB) between timed steps
             ev[i][0].record(stream)
-            step()
+            if use_graph:
+                graph.replay()
+            else:
+                step()
             ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
         gla.gla_profile_enable(False)
-        n_launch = gla.gla_launch_count()
+        n_launch = graph_launches * args.steps if use_graph else gla.gla_launch_count()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize(dev)
@@ -326,13 +356,15 @@ def main():
     # pass A: the step as a user runs it (headline time, clocks, launch count)
     clocks = ClockSampler(dev.index if world == 1 else local_rank)
     clocks.start()
-    total_ms, launches = timed_pass(False)
+    total_ms, launches = timed_pass(False, use_graph=graph is not None)
     clk = clocks.stop()
+    eager_ms = timed_pass(False)[0] if graph is not None else total_ms
     # pass B: the same K steps with a CUDA event pair around every kernel launch, for the per-kernel
     # durations of the roofline (the events between kernels lengthen the step, so pass A is the headline)
     prof_total_ms, _ = timed_pass(True)
     prof = gla.gla_profile_read()
     total_ms = dp.max_over_ranks(total_ms)
+    eager_ms = dp.max_over_ranks(eager_ms)
     ms_per_step = total_ms / args.steps
     tokens_per_step = w.B * w.L * world
     value = dp.job_throughput(w.B * w.L, world, ms_per_step)
@@ -424,7 +456,8 @@ def main():
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V,
                            "global_batch": dp.global_batch(w.B, world), "seq_len": w.L, "chunk": C, "subchunk": sc,
                            "kernel_impl": impl_name, "state_mode": mode, "parallelism": "dp%d" % world,
-                           "l2": "flushed between timed steps (512 MB write)"},
+                           "l2": "flushed between timed steps (512 MB write)", "step_launch": graph_note,
+                           "eager_ms_per_step": round(eager_ms / args.steps, 5)},
                 "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cb, "e2e": e2e,
                 "gpu_launches": int(launches), "clocks": clk, "kernels": kernels}
         print(json.dumps(line), flush=True)
