@@ -299,3 +299,45 @@ def test_tc_backward_matches_simt():
     g_s = run_bwd(d, "simt")
     for key in ("dq", "dk", "dv", "dlog_a", "dh0"):
         compare(key + " tc-vs-simt", g_tc[key], to_f64_numpy(g_s[key]), "bf16")
+
+
+@pytest.mark.parametrize("mode", ["materialized", "nonmaterialized"])
+def test_tc_step_replays_from_cuda_graph(mode):
+    """The fwd+bwd step captured into a CUDA graph and replayed gives the eager results bit for bit
+    (the kernels read and write fixed buffers; nothing in the path allocates or synchronises)."""
+    B, H, L, K, V = 2, 2, 300, 256, 128
+    inp = make_inputs(B, H, L, K, V, "bf16", seed=26, h0=True, dhT=True)
+    d = to_dev(inp)
+    desc = gla.make_desc(B, H, L, K, V, "bf16", impl="tc", state_mode=mode)
+    ws = torch.empty(gla.gla_bwd_workspace_size(desc), dtype=torch.uint8, device="cuda")
+    kw = dict(impl="tc", state_mode=mode)
+    o = torch.empty_like(d["v"])
+    hT = torch.empty(B, H, K, V, device="cuda")
+    outs = {"dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]), "dv": torch.empty_like(d["v"]),
+            "dlog_a": torch.empty_like(d["log_a"]), "dh0": torch.empty(B, H, K, V, device="cuda")}
+
+    def step():
+        gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], d["h0"], o=o, hT=hT, workspace=ws, **kw)
+        gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d["h0"], d["dhT"], workspace=ws, ws_from_fwd=True,
+                    out=outs, **kw)
+
+    step()
+    torch.cuda.synchronize()
+    eager = {"o": o.clone(), "hT": hT.clone(), **{k: v.clone() for k, v in outs.items()}}
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for t in [o, hT, *outs.values()]:
+        t.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    got = {"o": o, "hT": hT, **outs}
+    for key in eager:
+        assert torch.equal(got[key], eager[key]), key
+
