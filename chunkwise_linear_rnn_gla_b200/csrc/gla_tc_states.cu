@@ -6,16 +6,16 @@
 //   backward: D_{N-1} = dhT, D_{i-1} = diag(e^{Gamma_i}) D_i + Q~_i^T dO_i,   dh0 = D_{-1}
 // writing the state that enters every chunk to HBM in bf16.
 //
-// One CTA owns a [128 key channels x 64 value columns] tile of one head's
-// state. The chunk products U_i = A_i^T B_i (M = 128 channels, N = 64 values,
+// One CTA owns a [128 key channels x BVS value columns] tile of one head's
+// state (BVS = 128, or 64 when there are few heads). The chunk products U_i = A_i^T B_i (M = 128 channels, N = 64 values,
 // K = 128 tokens, operands by TMA with the 128-byte swizzle) do not depend on
-// the state, so the tcgen05 MMAs run ahead of the recurrence into a
-// double-buffered TMEM accumulator; the fp32 state itself lives in the
-// registers of four epilogue warps (thread = key channel, 64 values), which
-// per chunk store the bf16 copy of the entering state and apply
-// S <- e^{Gamma} S + U. Nothing on the tensor-core side waits for the
+// the state, so the tcgen05 MMAs run up to three chunks ahead of the
+// recurrence (three TMEM accumulators); the fp32 state itself lives in the
+// registers of BVS / 64 groups of four epilogue warps (thread = key channel,
+// 64 values), which per chunk store the bf16 copy of the entering state and
+// apply S <- e^{Gamma} S + U. Nothing on the tensor-core side waits for the
 // epilogue except the reuse of a TMEM buffer, so the walk runs at the speed
-// of its loads. Two CTAs fit per SM.
+// of its loads. One CTA per SM.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -41,10 +41,12 @@ constexpr int st_threads() { return 64 + 128 * (BVS / 64); }
 
 // Tile of BVS value columns (64 or 128): chunks in flight, bytes per chunk
 // (the key-channel pair of A pieces and BVS / 64 value pieces), CTAs per SM.
+// The narrow tile is used when the wide grid would leave most SMs idle (few
+// heads, long sequences): each walk is then bound by the chunks it has in
+// flight, so it keeps four of them.
 template <int BVS>
 struct StCfg {
-    static constexpr int nslot = 2;
-    static constexpr int nu = 3;  // TMEM accumulators for the chunk products: the MMAs run up to three chunks ahead
+    static constexpr int nslot = BVS == 64 ? 4 : 2;
     static constexpr uint32_t slot_bytes = uint32_t(2 + BVS / 64) * PIECE;
     static constexpr int min_blocks = 1;
     // + two staging pieces per epilogue group (double-buffered bf16 state for the TMA stores)
@@ -53,7 +55,7 @@ struct StCfg {
 };
 
 struct StBars {
-    uint64_t full[3], empty[3];
+    uint64_t full[4], empty[4];
     uint64_t u_full[3], u_empty[3], drain;
     uint32_t tmem_slot;
     int abort_flag;
@@ -258,8 +260,10 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
           map3(&m[1], B, uint64_t(p.V), uint64_t(p.L), uint64_t(p.BH)) &&
           map3(&m[2], states, uint64_t(p.V), uint64_t(p.K), uint64_t(p.BH * p.N))))
         return GLA_ERR_CUDA;
-    // 128-column tiles halve the re-reads of the key operand through L2 when d_v allows
-    const bool wide = p.V % 128 == 0;
+    // 128-column tiles halve the re-reads of the key operand through L2 when d_v allows and the grid
+    // still covers half of the SMs; otherwise 64-column tiles with more chunks in flight
+    const int64_t wide_ctas = p.BH * (p.K / 128) * (p.V / 128);
+    const bool wide = p.V % 128 == 0 && 2 * wide_ctas >= sm_count();
     const int bvs = wide ? 128 : 64;
     const size_t smem = (wide ? StCfg<128>::smem : StCfg<64>::smem) + sizeof(StBars);
     auto fn = wide ? (reverse ? k_states_walk<128, true> : k_states_walk<128, false>)
