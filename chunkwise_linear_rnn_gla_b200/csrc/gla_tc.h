@@ -51,10 +51,14 @@ gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, c
 
 // Materialised state walk on [128 x 128] tiles with the state accumulated in
 // TMEM (gla_tc_states.cu); requires d_v % 128 == 0.
+// A walk over few heads and many chunks is split into segments that run in
+// parallel (two passes and a scan over the segment end states); `segbuf`
+// holds tc_walk_seg_floats(p) floats of workspace (null: never split).
 bool tc_states_walk_supported(const Problem& p);
+size_t tc_walk_seg_floats(const Problem& p);
 gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
-                                 const float* init, float* fin, float* fin2, __nv_bfloat16* states, bool reverse,
-                                 cudaStream_t s, const char* name);
+                                 const float* init, float* fin, float* fin2, __nv_bfloat16* states, float* segbuf,
+                                 bool reverse, cudaStream_t s, const char* name);
 
 // Chunk-parallel Y_i = A_i X_i + Pm_i B_i from stored bf16 chunk states X
 // (gla_tc_out.cu): forward o (A = Q~, Pm = P) and dv (A = K~, Pm = P^T).

@@ -30,6 +30,7 @@ struct TcBuffers {
     __nv_bfloat16 *Qt, *Kt, *P;
     float *gam, *hT;
     __nv_bfloat16* states;
+    float* segbuf;  // segmented state walks: end states and entering states per segment
     __nv_bfloat16* Dbuf;
 };
 
@@ -42,8 +43,11 @@ TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
     b.P = a.take<__nv_bfloat16>(size_t(p.BH * p.N * kTcChunk * kTcChunk));
     b.gam = a.take<float>(size_t(p.BH * p.N * p.K));
     b.hT = a.take<float>(size_t(p.BH * p.K * p.V));
-    if (bwd || p.state_mode == GLA_STATE_MATERIALIZED)
+    if (bwd || p.state_mode == GLA_STATE_MATERIALIZED) {
         b.states = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
+        const size_t nseg = tc_walk_seg_floats(p);
+        if (nseg) b.segbuf = a.take<float>(nseg);
+    }
     if (bwd) b.Dbuf = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
     return b;
 }
@@ -95,7 +99,7 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
     a.states = b.states;
     a.mode = kWalkStatesOnly;
     st = tc_states_walk_supported(p)
-             ? tc_states_walk_launch(p, b.Kt, a.B1, b.gam, h0, hT, b.hT, b.states, false, s, "tc_walk_states")
+             ? tc_states_walk_launch(p, b.Kt, a.B1, b.gam, h0, hT, b.hT, b.states, b.segbuf, false, s, "tc_walk_states")
              : tc_walk_launch(p, a, s, "tc_walk_states");
     if (st != GLA_OK) return st;
     return tc_chunk_out_launch(p, b.Qt, b.states, b.P, static_cast<const __nv_bfloat16*>(v), false,
@@ -123,7 +127,7 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
         a.states = b.states;
         a.mode = kWalkStatesOnly;
         st = tc_states_walk_supported(p)
-                 ? tc_states_walk_launch(p, b.Kt, a.B1, b.gam, h0, b.hT, nullptr, b.states, false, s, "tc_walk_states")
+                 ? tc_states_walk_launch(p, b.Kt, a.B1, b.gam, h0, b.hT, nullptr, b.states, b.segbuf, false, s, "tc_walk_states")
                  : tc_walk_launch(p, a, s, "tc_walk_states");
         if (st != GLA_OK) return st;
     }
@@ -148,7 +152,7 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
         } else {
             a.mode = kWalkStatesOnly;
             st = tc_states_walk_supported(p) ? tc_states_walk_launch(p, b.Qt, a.B1, b.gam, dhT, dh0, nullptr, b.Dbuf,
-                                                                     true, s, "tc_walk_dstates")
+                                                                     b.segbuf, true, s, "tc_walk_dstates")
                                              : tc_walk_launch(p, a, s, "tc_walk_dstates");
             if (st != GLA_OK) return st;
             st = tc_chunk_out_launch(p, b.Kt, b.Dbuf, b.P, static_cast<const __nv_bfloat16*>(dO), true,

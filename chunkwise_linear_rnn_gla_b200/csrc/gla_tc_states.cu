@@ -61,13 +61,65 @@ struct StBars {
     int abort_flag;
 };
 
+// A long walk over few heads is split into segments of sg.len chunks that run
+// in parallel: pass 1 walks every segment from a zero state (segment 0 from
+// the true initial state, storing its states) and keeps the end states;
+// a scan over the segments turns them into the true state entering each
+// segment (S_in[g+1] = diag(prod of e^{Gamma} over segment g) S_in[g] +
+// E[g], all fp32); pass 2 walks segments 1.. again from those states and
+// stores theirs. A plain walk is one segment.
+constexpr int kMaxSegs = 16;
+
+struct WalkSegs {
+    int first;              // first segment of this launch
+    int len;                // chunks (walk steps) per segment
+    int store_all;          // every segment stores its states (else segment 0 only)
+    int64_t stride;         // elements between the per-segment [BH][K][V] fp32 blocks of init_seg / fin
+    const float* init_seg;  // start states of segments >= 1, indexed by segment (null: zero)
+};
+
+// S_in[g] for g = 1 .. G-1 from the pass-1 end states E[g] (E[0] is exact), and the final state.
+// One block per state row (head, key channel), one thread per four value columns; the first G
+// threads form the decay of every segment (the product of e^{Gamma} over its chunks) first.
+template <bool REVERSE>
+__global__ void __launch_bounds__(128) k_walk_seg_scan(const float* __restrict__ E, const float* __restrict__ gam,
+                                                       float* __restrict__ S_in, float* __restrict__ fin,
+                                                       float* __restrict__ fin2, int64_t N, int64_t K, int64_t V,
+                                                       int64_t BH, int G, int len) {
+    __shared__ float dec[kMaxSegs];
+    pdl_wait();  // the end states of pass 1
+    const int64_t row = blockIdx.x;  // bh * K + c
+    const int64_t bh = row / K, c = row % K;
+    const int t = threadIdx.x;
+    if (t < G) {
+        float d = 1.f;
+        const int s_end = (t + 1) * len < N ? (t + 1) * len : int(N);
+        for (int st = t * len; st < s_end; ++st) d *= gam[(bh * N + (REVERSE ? N - 1 - st : st)) * K + c];
+        dec[t] = d;
+    }
+    __syncthreads();
+    const int64_t stride = BH * K * V;
+    for (int64_t v4 = t; v4 < V / 4; v4 += blockDim.x) {
+        const int64_t e4 = row * (V / 4) + v4;
+        float4 x = reinterpret_cast<const float4*>(E)[e4];
+        for (int g = 1; g < G; ++g) {
+            reinterpret_cast<float4*>(S_in + g * stride)[e4] = x;
+            const float d = dec[g];
+            const float4 u = reinterpret_cast<const float4*>(E + g * stride)[e4];
+            x = make_float4(fmaf(d, x.x, u.x), fmaf(d, x.y, u.y), fmaf(d, x.z, u.z), fmaf(d, x.w, u.w));
+        }
+        if (fin) reinterpret_cast<float4*>(fin)[e4] = x;
+        if (fin2) reinterpret_cast<float4*>(fin2)[e4] = x;
+    }
+}
+
 template <int BVS, bool REVERSE>
 __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     k_states_walk(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmS,
                   const float* __restrict__ gam, const float* __restrict__ init, float* __restrict__ fin,
                   float* __restrict__ fin2, __nv_bfloat16* __restrict__ states, int64_t L, int64_t N, int64_t V,
-                  int64_t K, int* err) {
+                  int64_t K, int64_t BH, WalkSegs sg, int* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NSLOT = StCfg<BVS>::nslot;
@@ -77,9 +129,15 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int v0 = blockIdx.x * BVS;
     const int kbase = blockIdx.y * 128;
-    const int64_t bh = blockIdx.z;
-    const int nsteps = int(N);
-    auto chunk_of = [&](int step) -> int { return REVERSE ? int(N) - 1 - step : step; };
+    // blockIdx.z = head + BH * (segment - sg.first); a segment is sg.len consecutive steps of the walk
+    const int64_t bh = blockIdx.z % BH;
+    const int seg = sg.first + int(blockIdx.z / BH);
+    const int s0 = seg * sg.len;
+    const int nsteps = int(N) - s0 < sg.len ? int(N) - s0 : sg.len;
+    auto chunk_of = [&](int step) -> int { return REVERSE ? int(N) - 1 - (s0 + step) : s0 + step; };
+    const bool store = sg.store_all || seg == 0;
+    const float* init_s = seg == 0 ? init : (sg.init_seg ? sg.init_seg + seg * sg.stride : nullptr);
+    float* fin_s = fin ? fin + seg * sg.stride : nullptr;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSLOT; ++s) {
@@ -169,8 +227,8 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
         float x[64];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-            const float4 v4 = init ? reinterpret_cast<const float4*>(init + (bh * K + c) * V + v0 + col0)[e]
-                                   : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 v4 = init_s ? reinterpret_cast<const float4*>(init_s + (bh * K + c) * V + v0 + col0)[e]
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
             x[4 * e] = v4.x;
             x[4 * e + 1] = v4.y;
             x[4 * e + 2] = v4.z;
@@ -200,7 +258,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
                                pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]), pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]));
             fence_proxy_async_smem();
             named_sync(1 + grp, 128);
-            if (issuer && ok) {
+            if (issuer && ok && store) {
                 tma_store_3d(&tmS, v0 + col0, kbase, int(bh * N + ci), stg);
                 bulk_commit();
             }
@@ -224,7 +282,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
         if (issuer) bulk_wait_read_all();  // the stores finish on their own; the CTA may exit once they have read smem
         if (ok) {
             for (int w = 0; w < 2; ++w) {
-                float* f = w ? fin2 : fin;
+                float* f = w ? fin2 : fin_s;
                 if (!f) continue;
                 float4* d4 = reinterpret_cast<float4*>(f + (bh * K + c) * V + v0 + col0);
 #pragma unroll
@@ -251,9 +309,16 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
 
 bool tc_states_walk_supported(const Problem& p) { return p.V % 64 == 0; }
 
+size_t tc_walk_seg_floats(const Problem& p) {
+    // only walks whose narrow grid covers few SMs are ever split; the size does not depend on the device
+    const int64_t narrow_ctas = p.BH * (p.K / 128) * (p.V / 64);
+    if (narrow_ctas > 64 || p.N < 12) return 0;
+    return size_t(2) * kMaxSegs * size_t(p.BH * p.K * p.V);
+}
+
 gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
-                                 const float* init, float* fin, float* fin2, __nv_bfloat16* states, bool reverse,
-                                 cudaStream_t s, const char* name) {
+                                 const float* init, float* fin, float* fin2, __nv_bfloat16* states, float* segbuf,
+                                 bool reverse, cudaStream_t s, const char* name) {
     CUtensorMap m[3];
     memset(m, 0, sizeof(m));
     if (!(map3(&m[0], A, uint64_t(p.K), uint64_t(p.L), uint64_t(p.BH)) &&
@@ -262,17 +327,55 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
         return GLA_ERR_CUDA;
     // 128-column tiles halve the re-reads of the key operand through L2 when d_v allows and the grid
     // still covers half of the SMs; otherwise 64-column tiles with more chunks in flight
+    const int64_t sms = sm_count();
     const int64_t wide_ctas = p.BH * (p.K / 128) * (p.V / 128);
-    const bool wide = p.V % 128 == 0 && 2 * wide_ctas >= sm_count();
+    const bool wide = p.V % 128 == 0 && 2 * wide_ctas >= sms;
     const int bvs = wide ? 128 : 64;
     const size_t smem = (wide ? StCfg<128>::smem : StCfg<64>::smem) + sizeof(StBars);
     auto fn = wide ? (reverse ? k_states_walk<128, true> : k_states_walk<128, false>)
                    : (reverse ? k_states_walk<64, true> : k_states_walk<64, false>);
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
         return GLA_ERR_CUDA;
-    const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH));
-    GLA_LAUNCH_PDL(name, fn, grid, wide ? st_threads<128>() : st_threads<64>(), smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N, p.V, p.K,
-               device_error_word());
+    const int64_t ctas = p.BH * (p.K / 128) * (p.V / bvs);
+    // segments: as many as the SMs allow (each at least four chunks); two passes only pay from three
+    int64_t G = 1;
+    if (segbuf) {
+        G = sms / ctas;
+        if (G > kMaxSegs) G = kMaxSegs;
+        if (G > p.N / 4) G = p.N / 4;
+        if (G < 3) G = 1;
+    }
+    const int len = int((p.N + G - 1) / G);
+    G = (p.N + len - 1) / len;
+    const unsigned threads = wide ? st_threads<128>() : st_threads<64>();
+    if (G == 1) {
+        const WalkSegs sg{0, int(p.N), 1, 0, nullptr};
+        const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH));
+        GLA_LAUNCH_PDL(name, fn, grid, threads, smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N,
+                       p.V, p.K, p.BH, sg, device_error_word());
+        return GLA_OK;
+    }
+    const int64_t stride = p.BH * p.K * p.V;
+    float* E = segbuf;                               // end state of every segment walked from zero
+    float* S_in = segbuf + int64_t(kMaxSegs) * stride;  // true state entering every segment
+    {
+        const WalkSegs sg{0, len, 0, stride, nullptr};
+        const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH * G));
+        GLA_LAUNCH_PDL(name, fn, grid, threads, smem, s, m[0], m[1], m[2], gam, init, E, nullptr, states, p.L, p.N,
+                       p.V, p.K, p.BH, sg, device_error_word());
+    }
+    {
+        auto scan = reverse ? k_walk_seg_scan<true> : k_walk_seg_scan<false>;
+        const unsigned threads = unsigned(p.V / 4 < 128 ? p.V / 4 : 128);  // >= 16 >= G
+        GLA_LAUNCH_PDL("tc_walk_seg_scan", scan, dim3(unsigned(p.BH * p.K)), threads, 0, s, E, gam, S_in, fin, fin2,
+                       p.N, p.K, p.V, p.BH, int(G), len);
+    }
+    {
+        const WalkSegs sg{1, len, 1, stride, S_in};
+        const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH * (G - 1)));
+        GLA_LAUNCH_PDL(name, fn, grid, threads, smem, s, m[0], m[1], m[2], gam, init, nullptr, nullptr, states, p.L,
+                       p.N, p.V, p.K, p.BH, sg, device_error_word());
+    }
     return GLA_OK;
 }
 
