@@ -29,6 +29,21 @@ gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const 
 // dv:      A1 = Q~, B1 = dO, A2 = K~, Pm = P^T, reverse order, Y = dv, X0 = dhT.
 enum WalkMode : int { kWalkFused = 0, kWalkStatesOnly = 1, kWalkOutputOnly = 2 };
 
+// A long walk over few heads is split into segments of `len` chunks (walk
+// order) that run in parallel: pass 1 walks every segment from a zero state
+// (segment 0 from the true initial state) and keeps the end states; a scan
+// over the segments turns them into the true state entering each segment
+// (S_in[g+1] = diag(prod of e^{Gamma} over segment g) S_in[g] + E[g], fp32);
+// pass 2 walks the segments again from those states. A plain walk is one
+// segment.
+struct WalkSegs {
+    int first;              // first segment of this launch
+    int len;                // chunks (walk steps) per segment
+    int store_all;          // 1: every segment stores its states, 0: segment 0 only, -1: none
+    int64_t stride;         // elements between the per-segment [BH][K][V] fp32 blocks of init_seg / fin
+    const float* init_seg;  // start states of segments >= 1, indexed by segment (null: zero)
+};
+
 struct WalkArgs {
     const __nv_bfloat16* A1;  // [BH][L][K]
     const __nv_bfloat16* B1;  // [BH][L][V]
@@ -45,6 +60,12 @@ struct WalkArgs {
     int mode;
     bool reverse;
     bool p_transposed;
+    // fused mode: segments (seg_count > 1: every segment in one launch, segment g > 0 starting from
+    // seg_init + g * seg_stride; fin and fin2 are then left to the segment scan)
+    int seg_count = 1;
+    int seg_len = 0;
+    const float* seg_init = nullptr;
+    int64_t seg_stride = 0;
 };
 
 gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, const char* name);
@@ -56,6 +77,12 @@ gla_status tc_walk_launch(const Problem& p, const WalkArgs& a, cudaStream_t s, c
 // holds tc_walk_seg_floats(p) floats of workspace (null: never split).
 bool tc_states_walk_supported(const Problem& p);
 size_t tc_walk_seg_floats(const Problem& p);
+// Pass 1 and the scan of a segmented walk for the fused (non-materialised) walks: returns the
+// number of segments G (1: not split, nothing launched), their length and the entering states;
+// fin / fin2 receive the final state.
+int tc_walk_seg_prepare(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
+                        const float* init, float* fin, float* fin2, float* segbuf, bool reverse, cudaStream_t s,
+                        int* len, const float** S_in, int64_t* stride, gla_status* st);
 gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
                                  const float* init, float* fin, float* fin2, __nv_bfloat16* states, float* segbuf,
                                  bool reverse, cudaStream_t s, const char* name);

@@ -43,11 +43,9 @@ TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
     b.P = a.take<__nv_bfloat16>(size_t(p.BH * p.N * kTcChunk * kTcChunk));
     b.gam = a.take<float>(size_t(p.BH * p.N * p.K));
     b.hT = a.take<float>(size_t(p.BH * p.K * p.V));
-    if (bwd || p.state_mode == GLA_STATE_MATERIALIZED) {
-        b.states = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
-        const size_t nseg = tc_walk_seg_floats(p);
-        if (nseg) b.segbuf = a.take<float>(nseg);
-    }
+    if (bwd || p.state_mode == GLA_STATE_MATERIALIZED) b.states = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
+    const size_t nseg = tc_walk_seg_floats(p);
+    if (nseg) b.segbuf = a.take<float>(nseg);
     if (bwd) b.Dbuf = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
     return b;
 }
@@ -94,6 +92,11 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
     a.Y = static_cast<__nv_bfloat16*>(o);
     if (p.state_mode == GLA_STATE_NONMATERIALIZED) {
         a.mode = kWalkFused;
+        // few heads, many chunks: the walk runs as parallel segments from the entering states that a
+        // zero-start pass and a scan provide (the scan writes hT)
+        a.seg_count = tc_walk_seg_prepare(p, b.Kt, a.B1, b.gam, h0, hT, b.hT, b.segbuf, false, s, &a.seg_len,
+                                          &a.seg_init, &a.seg_stride, &st);
+        if (st != GLA_OK) return st;
         return tc_walk_launch(p, a, s, "tc_walk_fwd");
     }
     a.states = b.states;
@@ -147,6 +150,9 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
         if (p.state_mode == GLA_STATE_NONMATERIALIZED) {
             a.mode = kWalkFused;
             a.p_transposed = true;
+            a.seg_count = tc_walk_seg_prepare(p, b.Qt, a.B1, b.gam, dhT, dh0, nullptr, b.segbuf, true, s,
+                                              &a.seg_len, &a.seg_init, &a.seg_stride, &st);
+            if (st != GLA_OK) return st;
             st = tc_walk_launch(p, a, s, "tc_walk_dv");
             if (st != GLA_OK) return st;
         } else {

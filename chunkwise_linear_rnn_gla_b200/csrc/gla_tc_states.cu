@@ -61,22 +61,7 @@ struct StBars {
     int abort_flag;
 };
 
-// A long walk over few heads is split into segments of sg.len chunks that run
-// in parallel: pass 1 walks every segment from a zero state (segment 0 from
-// the true initial state, storing its states) and keeps the end states;
-// a scan over the segments turns them into the true state entering each
-// segment (S_in[g+1] = diag(prod of e^{Gamma} over segment g) S_in[g] +
-// E[g], all fp32); pass 2 walks segments 1.. again from those states and
-// stores theirs. A plain walk is one segment.
-constexpr int kMaxSegs = 16;
-
-struct WalkSegs {
-    int first;              // first segment of this launch
-    int len;                // chunks (walk steps) per segment
-    int store_all;          // every segment stores its states (else segment 0 only)
-    int64_t stride;         // elements between the per-segment [BH][K][V] fp32 blocks of init_seg / fin
-    const float* init_seg;  // start states of segments >= 1, indexed by segment (null: zero)
-};
+constexpr int kMaxSegs = 16;  // segments of a split walk (WalkSegs, gla_tc.h)
 
 // S_in[g] for g = 1 .. G-1 from the pass-1 end states E[g] (E[0] is exact), and the final state.
 // One block per state row (head, key channel), one thread per four value columns; the first G
@@ -135,7 +120,7 @@ __global__ void __launch_bounds__(st_threads<BVS>(), StCfg<BVS>::min_blocks)
     const int s0 = seg * sg.len;
     const int nsteps = int(N) - s0 < sg.len ? int(N) - s0 : sg.len;
     auto chunk_of = [&](int step) -> int { return REVERSE ? int(N) - 1 - (s0 + step) : s0 + step; };
-    const bool store = sg.store_all || seg == 0;
+    const bool store = sg.store_all > 0 || (sg.store_all == 0 && seg == 0);
     const float* init_s = seg == 0 ? init : (sg.init_seg ? sg.init_seg + seg * sg.stride : nullptr);
     float* fin_s = fin ? fin + seg * sg.stride : nullptr;
 
@@ -305,6 +290,67 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
     return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Tile width and segments of a walk. 128-column tiles halve the re-reads of the key operand through
+// L2 when d_v allows and the grid still covers half of the SMs; otherwise 64-column tiles with more
+// chunks in flight. Segments: as many as the SMs allow for the CTAs of one segment (at most
+// kMaxSegs, each at least four chunks); two passes only pay from three segments on.
+struct WalkPlan {
+    bool wide;
+    int64_t G;
+    int len;
+};
+
+WalkPlan walk_plan(const Problem& p, int64_t ctas_per_segment_narrow, bool may_split) {
+    WalkPlan w{};
+    const int64_t sms = sm_count();
+    const int64_t wide_ctas = p.BH * (p.K / 128) * (p.V / 128);
+    w.wide = p.V % 128 == 0 && 2 * wide_ctas >= sms;
+    const int64_t ctas = w.wide ? wide_ctas : ctas_per_segment_narrow;
+    w.G = 1;
+    if (may_split) {
+        w.G = sms / ctas;
+        if (w.G > kMaxSegs) w.G = kMaxSegs;
+        if (w.G > p.N / 4) w.G = p.N / 4;
+        if (w.G < 3) w.G = 1;
+    }
+    w.len = int((p.N + w.G - 1) / w.G);
+    w.G = (p.N + w.len - 1) / w.len;
+    return w;
+}
+
+gla_status launch_states(const Problem& p, const CUtensorMap* m, bool wide, bool reverse, const float* gam,
+                         const float* init, float* fin, float* fin2, __nv_bfloat16* states, const WalkSegs& sg,
+                         int64_t nseg, cudaStream_t s, const char* name) {
+    const int bvs = wide ? 128 : 64;
+    const size_t smem = (wide ? StCfg<128>::smem : StCfg<64>::smem) + sizeof(StBars);
+    auto fn = wide ? (reverse ? k_states_walk<128, true> : k_states_walk<128, false>)
+                   : (reverse ? k_states_walk<64, true> : k_states_walk<64, false>);
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+        return GLA_ERR_CUDA;
+    const unsigned threads = wide ? st_threads<128>() : st_threads<64>();
+    const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH * nseg));
+    GLA_LAUNCH_PDL(name, fn, grid, threads, smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N, p.V,
+                   p.K, p.BH, sg, device_error_word());
+    return GLA_OK;
+}
+
+gla_status launch_seg_scan(const Problem& p, bool reverse, const float* E, const float* gam, float* S_in, float* fin,
+                           float* fin2, int64_t G, int len, cudaStream_t s) {
+    auto scan = reverse ? k_walk_seg_scan<true> : k_walk_seg_scan<false>;
+    const unsigned threads = unsigned(p.V / 4 < 128 ? p.V / 4 : 128);  // >= 16 >= G
+    GLA_LAUNCH_PDL("tc_walk_seg_scan", scan, dim3(unsigned(p.BH * p.K)), threads, 0, s, E, gam, S_in, fin, fin2, p.N,
+                   p.K, p.V, p.BH, int(G), len);
+    return GLA_OK;
+}
+
+bool make_maps(CUtensorMap* m, const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B,
+               const void* states) {
+    memset(m, 0, 3 * sizeof(CUtensorMap));
+    return map3(&m[0], A, uint64_t(p.K), uint64_t(p.L), uint64_t(p.BH)) &&
+           map3(&m[1], B, uint64_t(p.V), uint64_t(p.L), uint64_t(p.BH)) &&
+           map3(&m[2], states, uint64_t(p.V), uint64_t(p.K), uint64_t(p.BH * p.N));
+}
+
 }  // namespace
 
 bool tc_states_walk_supported(const Problem& p) { return p.V % 64 == 0; }
@@ -320,63 +366,47 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
                                  const float* init, float* fin, float* fin2, __nv_bfloat16* states, float* segbuf,
                                  bool reverse, cudaStream_t s, const char* name) {
     CUtensorMap m[3];
-    memset(m, 0, sizeof(m));
-    if (!(map3(&m[0], A, uint64_t(p.K), uint64_t(p.L), uint64_t(p.BH)) &&
-          map3(&m[1], B, uint64_t(p.V), uint64_t(p.L), uint64_t(p.BH)) &&
-          map3(&m[2], states, uint64_t(p.V), uint64_t(p.K), uint64_t(p.BH * p.N))))
-        return GLA_ERR_CUDA;
-    // 128-column tiles halve the re-reads of the key operand through L2 when d_v allows and the grid
-    // still covers half of the SMs; otherwise 64-column tiles with more chunks in flight
-    const int64_t sms = sm_count();
-    const int64_t wide_ctas = p.BH * (p.K / 128) * (p.V / 128);
-    const bool wide = p.V % 128 == 0 && 2 * wide_ctas >= sms;
-    const int bvs = wide ? 128 : 64;
-    const size_t smem = (wide ? StCfg<128>::smem : StCfg<64>::smem) + sizeof(StBars);
-    auto fn = wide ? (reverse ? k_states_walk<128, true> : k_states_walk<128, false>)
-                   : (reverse ? k_states_walk<64, true> : k_states_walk<64, false>);
-    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
-        return GLA_ERR_CUDA;
-    const int64_t ctas = p.BH * (p.K / 128) * (p.V / bvs);
-    // segments: as many as the SMs allow (each at least four chunks); two passes only pay from three
-    int64_t G = 1;
-    if (segbuf) {
-        G = sms / ctas;
-        if (G > kMaxSegs) G = kMaxSegs;
-        if (G > p.N / 4) G = p.N / 4;
-        if (G < 3) G = 1;
-    }
-    const int len = int((p.N + G - 1) / G);
-    G = (p.N + len - 1) / len;
-    const unsigned threads = wide ? st_threads<128>() : st_threads<64>();
-    if (G == 1) {
-        const WalkSegs sg{0, int(p.N), 1, 0, nullptr};
-        const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH));
-        GLA_LAUNCH_PDL(name, fn, grid, threads, smem, s, m[0], m[1], m[2], gam, init, fin, fin2, states, p.L, p.N,
-                       p.V, p.K, p.BH, sg, device_error_word());
-        return GLA_OK;
+    if (!make_maps(m, p, A, B, states)) return GLA_ERR_CUDA;
+    const WalkPlan w = walk_plan(p, p.BH * (p.K / 128) * (p.V / 64), segbuf != nullptr);
+    if (w.G == 1)
+        return launch_states(p, m, w.wide, reverse, gam, init, fin, fin2, states, WalkSegs{0, int(p.N), 1, 0, nullptr},
+                             1, s, name);
+    const int64_t stride = p.BH * p.K * p.V;
+    float* E = segbuf;                                  // end state of every segment walked from zero
+    float* S_in = segbuf + int64_t(kMaxSegs) * stride;  // true state entering every segment
+    gla_status st = launch_states(p, m, w.wide, reverse, gam, init, E, nullptr, states,
+                                  WalkSegs{0, w.len, 0, stride, nullptr}, w.G, s, name);
+    if (st == GLA_OK) st = launch_seg_scan(p, reverse, E, gam, S_in, fin, fin2, w.G, w.len, s);
+    if (st == GLA_OK)
+        st = launch_states(p, m, w.wide, reverse, gam, init, nullptr, nullptr, states,
+                           WalkSegs{1, w.len, 1, stride, S_in}, w.G - 1, s, name);
+    return st;
+}
+
+int tc_walk_seg_prepare(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
+                        const float* init, float* fin, float* fin2, float* segbuf, bool reverse, cudaStream_t s,
+                        int* len, const float** S_in_out, int64_t* stride_out, gla_status* st) {
+    *st = GLA_OK;
+    if (!segbuf) return 1;
+    // segments sized for the fused walk's grid (one CTA per head and 64 value columns)
+    const WalkPlan w = walk_plan(p, p.BH * (p.V / 64), true);
+    if (w.G == 1) return 1;
+    CUtensorMap m[3];
+    // pass 1 stores nothing; the states map only has to be a valid descriptor
+    if (!make_maps(m, p, A, B, segbuf)) {
+        *st = GLA_ERR_CUDA;
+        return 1;
     }
     const int64_t stride = p.BH * p.K * p.V;
-    float* E = segbuf;                               // end state of every segment walked from zero
-    float* S_in = segbuf + int64_t(kMaxSegs) * stride;  // true state entering every segment
-    {
-        const WalkSegs sg{0, len, 0, stride, nullptr};
-        const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH * G));
-        GLA_LAUNCH_PDL(name, fn, grid, threads, smem, s, m[0], m[1], m[2], gam, init, E, nullptr, states, p.L, p.N,
-                       p.V, p.K, p.BH, sg, device_error_word());
-    }
-    {
-        auto scan = reverse ? k_walk_seg_scan<true> : k_walk_seg_scan<false>;
-        const unsigned threads = unsigned(p.V / 4 < 128 ? p.V / 4 : 128);  // >= 16 >= G
-        GLA_LAUNCH_PDL("tc_walk_seg_scan", scan, dim3(unsigned(p.BH * p.K)), threads, 0, s, E, gam, S_in, fin, fin2,
-                       p.N, p.K, p.V, p.BH, int(G), len);
-    }
-    {
-        const WalkSegs sg{1, len, 1, stride, S_in};
-        const dim3 grid(unsigned(p.V / bvs), unsigned(p.K / 128), unsigned(p.BH * (G - 1)));
-        GLA_LAUNCH_PDL(name, fn, grid, threads, smem, s, m[0], m[1], m[2], gam, init, nullptr, nullptr, states, p.L,
-                       p.N, p.V, p.K, p.BH, sg, device_error_word());
-    }
-    return GLA_OK;
+    float* E = segbuf;
+    float* S_in = segbuf + int64_t(kMaxSegs) * stride;
+    *st = launch_states(p, m, w.wide, reverse, gam, init, E, nullptr, nullptr, WalkSegs{0, w.len, -1, stride, nullptr},
+                        w.G, s, reverse ? "tc_walk_seg_dv" : "tc_walk_seg_fwd");
+    if (*st == GLA_OK) *st = launch_seg_scan(p, reverse, E, gam, S_in, fin, fin2, w.G, w.len, s);
+    *len = w.len;
+    *S_in_out = S_in;
+    *stride_out = stride;
+    return int(w.G);
 }
 
 }  // namespace gla

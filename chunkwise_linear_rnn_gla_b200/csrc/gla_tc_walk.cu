@@ -134,7 +134,8 @@ __global__ void __launch_bounds__(WalkCfg<NH, MODE>::threads, WalkCfg<NH, MODE>:
            const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmP,
            const __grid_constant__ CUtensorMap tmS, const float* __restrict__ gam, const float* __restrict__ init,
            float* __restrict__ fin, float* __restrict__ fin2, __nv_bfloat16* __restrict__ Y,
-           __nv_bfloat16* __restrict__ states, int64_t L, int64_t N, int64_t V, int64_t K, int* err) {
+           __nv_bfloat16* __restrict__ states, int64_t L, int64_t N, int64_t V, int64_t K, int64_t BH, WalkSegs sg,
+           int* err) {
     constexpr int KC = NH * 128;  // key channels owned by this CTA
     using Cfg = WalkCfg<NH, MODE>;
     extern __shared__ uint8_t smem_raw[];
@@ -146,16 +147,20 @@ __global__ void __launch_bounds__(WalkCfg<NH, MODE>::threads, WalkCfg<NH, MODE>:
     volatile int* abort_flag = &bar.abort_flag;
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    const int64_t bh = blockIdx.z;
+    // blockIdx.z = head + BH * (segment - sg.first); a segment is sg.len consecutive walk steps
+    const int64_t bh = blockIdx.z % BH;
+    const int seg = sg.first + int(blockIdx.z / BH);
+    const int s0 = seg * sg.len;
     const int v0 = blockIdx.x * BV;
-    const int nsteps = MODE == kWalkOutputOnly ? 1 : int(N);
+    const int nsteps = MODE == kWalkOutputOnly ? 1 : (int(N) - s0 < sg.len ? int(N) - s0 : sg.len);
     const int first_chunk = MODE == kWalkOutputOnly ? int(blockIdx.y) : 0;
     // states-only walks may split the key channels over blockIdx.y
     const int kbase = MODE == kWalkStatesOnly ? int(blockIdx.y) * KC : 0;
     auto chunk_of = [&](int step) -> int {
         if (MODE == kWalkOutputOnly) return first_chunk;
-        return REVERSE ? int(N) - 1 - step : step;
+        return REVERSE ? int(N) - 1 - (s0 + step) : s0 + step;
     };
+    const float* init_s = seg == 0 ? init : (sg.init_seg ? sg.init_seg + seg * sg.stride : nullptr);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < Cfg::ring; ++s) {
@@ -357,7 +362,7 @@ __global__ void __launch_bounds__(WalkCfg<NH, MODE>::threads, WalkCfg<NH, MODE>:
                     float x[16];
 #pragma unroll
                     for (int e = 0; e < 16; ++e)
-                        x[e] = init ? init[(bh * K + c) * V + v0 + c16 * 16 + e] : 0.f;
+                        x[e] = init_s ? init_s[(bh * K + c) * V + v0 + c16 * 16 + e] : 0.f;
                     tmem_st16(tmem + lane_off + col_S<NH>() + uint32_t(h * BV + c16 * 16), x);
                     if (MODE == kWalkFused) {  // only the fused walk keeps a bf16 copy in smem
                         uint8_t* row = sS + (c - kbase) * 128;
@@ -534,9 +539,13 @@ gla_status launch_walk(const Problem& p, const WalkArgs& a, const CUtensorMap* m
         return GLA_ERR_CUDA;
     const unsigned gy = MODE == kWalkOutputOnly ? unsigned(p.N)
                         : MODE == kWalkStatesOnly ? unsigned(p.K / KC) : 1u;
-    const dim3 grid(unsigned(p.V / BV), gy, unsigned(p.BH));
+    const bool split = MODE == kWalkFused && a.seg_count > 1;
+    const WalkSegs sg = split ? WalkSegs{0, a.seg_len, 1, a.seg_stride, a.seg_init} : WalkSegs{0, int(p.N), 1, 0, nullptr};
+    const dim3 grid(unsigned(p.V / BV), gy, unsigned(p.BH * (split ? a.seg_count : 1)));
+    // a split walk leaves the final state to the segment scan
     GLA_LAUNCH_PDL(name, fn, grid, Cfg::threads, smem, s, maps[0], maps[1], maps[2], maps[3], maps[4], a.gam, a.init,
-               a.fin, a.fin2, a.Y, a.states, p.L, p.N, p.V, p.K, device_error_word());
+                   split ? nullptr : a.fin, split ? nullptr : a.fin2, a.Y, a.states, p.L, p.N, p.V, p.K, p.BH, sg,
+                   device_error_word());
     return GLA_OK;
 }
 

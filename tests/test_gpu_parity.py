@@ -343,12 +343,14 @@ def test_tc_step_replays_from_cuda_graph(mode):
 
 
 
+@pytest.mark.parametrize("mode", ["materialized", "nonmaterialized"])
 @pytest.mark.parametrize("z_mean", [0.0, 2.0])
-def test_tc_segmented_state_walk(z_mean):
-    """Few heads and many chunks: the materialised state walks run as parallel segments (a zero-start
-    pass, a scan over the segment end states, a second pass from the true entering states). Ragged
-    last chunk, nonzero h0 and dhT, slow (z_mean=2) and ordinary gates; fwd and bwd against the oracle."""
+def test_tc_segmented_state_walk(z_mean, mode):
+    """Few heads and many chunks: the state walks (materialised, and the fused non-materialised walks)
+    run as parallel segments (a zero-start pass, a scan over the segment end states, a second pass
+    from the true entering states). Ragged last chunk, nonzero h0 and dhT, slow (z_mean=2) and
+    ordinary gates; fwd and bwd against the oracle."""
     B, H, L, K, V = 1, 2, 128 * 20 + 37, 128, 128
     inp = make_inputs(B, H, L, K, V, "bf16", seed=28, z_mean=z_mean, h0=True, dhT=True)
-    check_fwd(inp, "bf16", "tc", state_mode="materialized")
-    check_bwd(inp, "bf16", "tc", state_mode="materialized")
+    check_fwd(inp, "bf16", "tc", state_mode=mode)
+    check_bwd(inp, "bf16", "tc", state_mode=mode)
