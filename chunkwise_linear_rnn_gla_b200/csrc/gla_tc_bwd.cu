@@ -242,18 +242,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                  mbar_wait(&bar.khat_ready, 0, err, abort_flag) && mbar_wait(&bar.qt_full, 0, err, abort_flag);
             if (ok) {
                 tc_fence_after();
-                const uint32_t idQ = idesc_bf16_f32(128, 128, true, false);
-                const uint32_t idK = idesc_bf16_f32(128, 128, true, true);
                 const uint32_t dpm = smem_u32(base + DPM_OFF), qt = smem_u32(base + QT_OFF);
                 const uint32_t kh0 = smem_u32(base + KH_OFF);
+                // The masked dP is lower triangular (s <= j), so a 16-token slice of the contraction only
+                // reaches part of the output: token slice kk of s feeds the dq columns j >= 16 kk, token
+                // slice kk of j feeds the dk columns s < 16 (kk + 1). The dk slices run from the last,
+                // whose MMA spans (and so initialises) every column.
 #pragma unroll
                 for (int kk = 0; kk < C / 16; ++kk) {
-                    // dQ^T[c][j] += sum_s K^0[s][c] dP[j][s]: A = K^0 (MN-major), B = dP (K-major)
-                    mma_bf16(tmem + 128, sdesc_sw128(kh0 + kk * 2048, PIECE, 1024),
-                             sdesc_sw128(dpm + (kk / 4) * PIECE + (kk % 4) * 32, 16, 1024), idQ, 1u);
-                    // dKi^T[c][s] = sum_j Q~[j][c] dP[j][s]: A = Q~ (MN-major), B = dP (MN-major)
-                    mma_bf16(tmem + 0, sdesc_sw128(qt + kk * 2048, PIECE, 1024),
-                             sdesc_sw128(dpm + kk * 2048, PIECE, 1024), idK, kk > 0 ? 1u : 0u);
+                    // dQ^T[c][j] += sum_s K^0[s][c] dP[j][s] for j >= 16 kk: A = K^0 (MN-major), B = dP
+                    // (K-major) from row j = 16 kk
+                    const int j0 = 16 * kk;
+                    mma_bf16(tmem + 128 + uint32_t(j0), sdesc_sw128(kh0 + kk * 2048, PIECE, 1024),
+                             sdesc_sw128(dpm + (kk / 4) * PIECE + (kk % 4) * 32 + j0 * 128, 16, 1024),
+                             idesc_bf16_f32(128, C - j0, true, false), 1u);
+                    // dKi^T[c][s] = sum_j Q~[j][c] dP[j][s] for s < 16 (k + 1), k = 7 - kk: A = Q~
+                    // (MN-major), B = dP (MN-major)
+                    const int k = C / 16 - 1 - kk;
+                    mma_bf16(tmem + 0, sdesc_sw128(qt + k * 2048, PIECE, 1024),
+                             sdesc_sw128(dpm + k * 2048, PIECE, 1024), idesc_bf16_f32(128, 16 * (k + 1), true, true),
+                             kk > 0 ? 1u : 0u);
                 }
                 mma_commit(&bar.accB);
             }
