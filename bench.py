@@ -151,14 +151,34 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu_index), "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            self.t_start = time.time()
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def wait_first_sample(self, timeout_s=3.0):
+        """Block until nvidia-smi has written its first sample, so that sampling is live before the
+        timed region starts."""
+        if self.proc is None:
+            return
+        t0 = time.time()
+        while time.time() - t0 < timeout_s:
+            try:
+                if os.path.getsize(self.path) > 0:
+                    return
+            except OSError:
+                return
+            time.sleep(0.01)
+
+    def stop(self, keep_busy=None, min_s=0.0):
+        """Stop sampling. `keep_busy` (a callable that enqueues work) keeps the GPU on the same step
+        until `min_s` seconds have passed since start, so that a short timed region still gets
+        samples taken under its own load."""
         if self.proc is None:
             return None
-        time.sleep(0.25)
+        if keep_busy is not None:
+            while time.time() - self.t_start < min_s:
+                keep_busy()
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -356,8 +376,20 @@ def main():
     # pass A: the step as a user runs it (headline time, clocks, launch count)
     clocks = ClockSampler(dev.index if world == 1 else local_rank)
     clocks.start()
+    clocks.wait_first_sample()
     total_ms, launches = timed_pass(False, use_graph=graph is not None)
-    clk = clocks.stop()
+
+    def keep_busy():  # the same step, untimed, so that the clock samples are taken under this load
+        for _ in range(20):
+            if graph is not None:
+                graph.replay()
+            else:
+                step()
+        torch.cuda.synchronize(dev)
+
+    clk = clocks.stop(keep_busy, min_s=0.6)
+    if clk is not None:
+        clk["window"] = "timed pass A, then the same step replayed untimed until 0.6 s of sampling (100 ms period)"
     eager_ms = timed_pass(False)[0] if graph is not None else total_ms
     # pass B: the same K steps with a CUDA event pair around every kernel launch, for the per-kernel
     # durations of the roofline (the events between kernels lengthen the step, so pass A is the headline)
