@@ -220,6 +220,13 @@ def gla_check_device_error(stream=None) -> int:
     return int(load().gla_check_device_error(s))
 
 
+def gla_selftest_wait_timeout(limit_cycles=0, stream=None) -> None:
+    """Run the library's bounded-wait self-test kernel (a wait that nothing completes); the next
+    gla_check_device_error reports GLA_ERR_TIMEOUT."""
+    s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
+    _check(load().gla_selftest_wait_timeout(int(limit_cycles), s), "gla_selftest_wait_timeout")
+
+
 def gla_launch_count() -> int:
     return int(load().gla_launch_count())
 

@@ -24,6 +24,7 @@ EXPORTS = (
     "gla_fwd_workspace_size", "gla_bwd_workspace_size", "gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum",
     "gla_check_device_error", "gla_status_string", "gla_abi_version", "gla_resolve", "gla_launch_count",
     "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset", "gla_fwd_noalloc",
+    "gla_selftest_wait_timeout",
 )
 
 
@@ -61,6 +62,8 @@ def _declare(lib):
     lib.gla_chunk_cumsum.restype = ctypes.c_int
     lib.gla_check_device_error.argtypes = [vp]
     lib.gla_check_device_error.restype = ctypes.c_int
+    lib.gla_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+    lib.gla_selftest_wait_timeout.restype = ctypes.c_int
     lib.gla_status_string.argtypes = [ctypes.c_int]
     lib.gla_status_string.restype = ctypes.c_char_p
     lib.gla_abi_version.restype = ctypes.c_int

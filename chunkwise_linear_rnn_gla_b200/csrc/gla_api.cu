@@ -11,6 +11,7 @@
 #include <vector>
 
 #include "gla_internal.h"
+#include "tc_prims.cuh"
 
 namespace gla {
 namespace {
@@ -311,6 +312,29 @@ gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, 
     p.N = (p.L + C - 1) / C;
     if (p.BH > 65535 || p.N > 65535) return GLA_ERR_UNSUPPORTED;
     return gla::simt_chunk_cumsum(p, log_a, Bcum, static_cast<cudaStream_t>(stream));
+}
+
+namespace {
+// One thread waits on an mbarrier nothing arrives on: the bounded wait must give up, record the
+// timeout and let the kernel finish.
+__global__ void k_selftest_wait_timeout(int* err, long long limit_cycles) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        gla::tc::mbar_init(&bar, 1);
+        abort_flag = 0;
+        gla::tc::fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)gla::tc::mbar_wait(&bar, 0, err, &abort_flag, limit_cycles);
+}
+}  // namespace
+
+gla_status gla_selftest_wait_timeout(long long limit_cycles, void* stream) {
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    GLA_LAUNCH("selftest_wait_timeout", k_selftest_wait_timeout, 1, 32, 0, s, gla::device_error_word(),
+               limit_cycles > 0 ? limit_cycles : 2000000LL);
+    return GLA_OK;
 }
 
 gla_status gla_check_device_error(void* stream) {

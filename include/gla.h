@@ -173,6 +173,15 @@ gla_status gla_fwd_noalloc(const gla_desc* d, const void* q, const void* k, cons
  * the last check, GLA_ERR_CUDA on a sticky CUDA error, else GLA_OK. */
 gla_status gla_check_device_error(void* stream);
 
+/* Self-test of the error path: launches one CTA whose mbarrier wait can never
+ * complete (nothing arrives on the barrier). The bounded wait gives up after
+ * about `limit_cycles` SM cycles (0: 2,000,000, about 1 ms) and records
+ * GLA_ERR_TIMEOUT in the device flag, exactly as a stalled kernel of the path
+ * would; the kernel then exits normally and the context stays usable. The
+ * next gla_check_device_error(stream) reports GLA_ERR_TIMEOUT. Returns
+ * GLA_ERR_CUDA if the launch fails. */
+gla_status gla_selftest_wait_timeout(long long limit_cycles, void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* gla_status_string(gla_status s);
 

@@ -354,3 +354,17 @@ def test_tc_segmented_state_walk(z_mean, mode):
     inp = make_inputs(B, H, L, K, V, "bf16", seed=28, z_mean=z_mean, h0=True, dhT=True)
     check_fwd(inp, "bf16", "tc", state_mode=mode)
     check_bwd(inp, "bf16", "tc", state_mode=mode)
+
+
+def test_bounded_wait_timeout_is_reported_and_the_context_survives():
+    """Failure detection without a GPU fault: a kernel whose mbarrier wait nothing completes gives up
+    after its bound, the host reads GLA_ERR_TIMEOUT (once; the flag is cleared), and the same context
+    then runs the layer correctly."""
+    torch.cuda.synchronize()
+    assert gla.gla_check_device_error() == 0
+    gla.gla_selftest_wait_timeout()
+    assert gla.gla_check_device_error() == 5  # GLA_ERR_TIMEOUT
+    assert gla.gla_check_device_error() == 0
+    inp = make_inputs(1, 2, 300, 128, 128, "bf16", seed=29)
+    check_fwd(inp, "bf16", "tc", state_mode="materialized")
+    assert gla.gla_check_device_error() == 0
