@@ -86,12 +86,18 @@ __global__ void __launch_bounds__(128) k_walk_seg_scan(const float* __restrict__
     const int64_t stride = BH * K * V;
     for (int64_t v4 = t; v4 < V / 4; v4 += blockDim.x) {
         const int64_t e4 = row * (V / 4) + v4;
-        float4 x = reinterpret_cast<const float4*>(E)[e4];
-        for (int g = 1; g < G; ++g) {
+        // every segment's end state first (independent loads), then the recurrence over them
+        float4 u[kMaxSegs];
+#pragma unroll
+        for (int g = 0; g < kMaxSegs; ++g)
+            if (g < G) u[g] = reinterpret_cast<const float4*>(E + g * stride)[e4];
+        float4 x = u[0];
+#pragma unroll
+        for (int g = 1; g < kMaxSegs; ++g) {
+            if (g >= G) break;
             reinterpret_cast<float4*>(S_in + g * stride)[e4] = x;
             const float d = dec[g];
-            const float4 u = reinterpret_cast<const float4*>(E + g * stride)[e4];
-            x = make_float4(fmaf(d, x.x, u.x), fmaf(d, x.y, u.y), fmaf(d, x.z, u.z), fmaf(d, x.w, u.w));
+            x = make_float4(fmaf(d, x.x, u[g].x), fmaf(d, x.y, u[g].y), fmaf(d, x.z, u[g].z), fmaf(d, x.w, u[g].w));
         }
         if (fin) reinterpret_cast<float4*>(fin)[e4] = x;
         if (fin2) reinterpret_cast<float4*>(fin2)[e4] = x;
