@@ -145,7 +145,7 @@ gla_status resolve(const gla_desc* d, Problem& p) {
     p.impl = impl;
     if (impl == GLA_IMPL_SIMT) {
         p.C = d->chunk ? d->chunk : 64;
-        p.c = d->subchunk ? d->subchunk : p.C;
+        p.c = d->subchunk ? d->subchunk : (p.C < 16 ? p.C : 16);  // secondary chunks of 16 rows
         if (d->state_mode == GLA_STATE_NONMATERIALIZED) return GLA_ERR_UNSUPPORTED;
         p.state_mode = GLA_STATE_MATERIALIZED;
     } else {

@@ -8,7 +8,9 @@
 // inter-chunk states). With B the per-chunk inclusive cumsum of log alpha and
 // Gamma = B at the chunk's last row:
 //   o_j     = (q_j * e^{B_j}) S_[i] + sum_{s<=j} P_js v_s,
-//   P_js    = sum_c q_jc k_sc e^{B_jc - B_sc}           (log space, exact)
+//   P_js    = sum_c q_jc k_sc e^{B_jc - B_sc}           (two-level: log space inside
+//                                                        a sub-chunk, rescaled
+//                                                        products across them)
 //   S_[i+1] = diag(e^Gamma) S_[i] + sum_j (k_j * e^{Gamma - B_j})^T v_j
 // and the backward in the same form with D_i = dL/dS_[i+1]; the gate gradient
 // is the closed-form reverse cumsum of q*dq - k*dk plus sum_v dhT*hT.
@@ -40,28 +42,43 @@ __global__ void __launch_bounds__(128) k_chunk_cumsum(const float* __restrict__ 
     float* dst = Bc + (bh * L) * K + c;
     float acc = 0.f;
     for (int64_t t = t0; t < t1; ++t) {
-        acc += src[t * K];
+        acc += la_floor(src[t * K]);
         dst[t * K] = acc;
     }
 }
 
 // ---------------------------------------------------------------------------
 // Intra-chunk scores P_js = sum_c q_jc k_sc exp(B_jc - B_sc) for s <= j < nvalid
-// (zero elsewhere), one exponential per term (log space). Layout P[BH,N,C,C].
+// (zero elsewhere), layout P[BH,N,C,C], with the two-level (secondary)
+// chunking of the chunk form ("Gated Linear Attention Transformers with
+// Hardware-Efficient Training", atlas.scime.ai summary, "Approach"): the rows
+// split into sub-chunks of `csub`. For a key s in sub-chunk J below the query
+// row's sub-chunk I, with rho_J = B at the last row of J,
+//   q_j k_s e^{B_j - B_s} = (q_j e^{B_j - rho_J}) (k_s e^{rho_J - B_s}),
+// both factors <= 1 (B is non-increasing), so the off-diagonal sub-blocks are
+// plain products of rescaled operands: one exponential per (query row, key
+// sub-chunk, channel) and one per key. Pairs inside a diagonal sub-block take
+// one exponential per term (log space). Thread = one query row and SPT keys.
 template <typename T, int C>
 __global__ void __launch_bounds__(kThreads) k_intra_P(const T* __restrict__ q, const T* __restrict__ k,
                                                       const float* __restrict__ Bc, float* __restrict__ P,
-                                                      int64_t L, int64_t K, int64_t N) {
-    constexpr int CT = 16;  // channel tile
-    constexpr int PP = (C * C + kThreads - 1) / kThreads;
-    __shared__ float sq[C][CT + 1], sk[C][CT + 1], sB[C][CT + 1];
+                                                      int64_t L, int64_t K, int64_t N, int csub) {
+    constexpr int CT = 16;                       // channel tile
+    constexpr int SPT = C < 16 ? C : 16;         // keys per thread
+    constexpr int TPR = C / SPT;                 // threads per query row
+    constexpr int RPP = kThreads / TPR;          // query rows per pass
+    constexpr int NPASS = (C + RPP - 1) / RPP;
+    __shared__ float sq[C][CT + 1], sk[C][CT + 1], skr[C][CT + 1], sB[C][CT + 1];
     const int64_t i = blockIdx.x, bh = blockIdx.y;
     const int64_t t0 = i * C;
     const int nvalid = int(L - t0 < C ? L - t0 : C);
     const int tid = threadIdx.x;
-    float acc[PP];
+    const int s0 = (tid % TPR) * SPT;
+    float acc[NPASS][SPT];
 #pragma unroll
-    for (int p = 0; p < PP; ++p) acc[p] = 0.f;
+    for (int ps = 0; ps < NPASS; ++ps)
+#pragma unroll
+        for (int e = 0; e < SPT; ++e) acc[ps][e] = 0.f;
     for (int64_t c0 = 0; c0 < K; c0 += CT) {
         for (int e = tid; e < C * CT; e += kThreads) {
             const int j = e / CT, cc = e % CT;
@@ -78,16 +95,39 @@ __global__ void __launch_bounds__(kThreads) k_intra_P(const T* __restrict__ q, c
             sB[j][cc] = g;
         }
         __syncthreads();
+        // keys rescaled to the end of their sub-chunk (its last valid row): k_s e^{rho_J - B_s}
+        for (int e = tid; e < C * CT; e += kThreads) {
+            const int srow = e / CT, cc = e % CT;
+            int last = (srow / csub + 1) * csub - 1;
+            last = last < nvalid - 1 ? last : nvalid - 1;
+            skr[srow][cc] = srow < nvalid ? sk[srow][cc] * expf(sB[last][cc] - sB[srow][cc]) : 0.f;
+        }
+        __syncthreads();
 #pragma unroll
-        for (int p = 0; p < PP; ++p) {
-            const int pair = tid + p * kThreads;
-            if (pair < C * C) {
-                const int j = pair / C, s = pair % C;
-                if (s <= j && j < nvalid) {
-                    float a = acc[p];
+        for (int ps = 0; ps < NPASS; ++ps) {
+            const int j = tid / TPR + ps * RPP;
+            if (j >= C || j >= nvalid || s0 > j) continue;
+            const int I = j / csub;
+            for (int cc = 0; cc < CT; ++cc) {
+                const float qj = sq[j][cc], bj = sB[j][cc];
+                int Jc = -1;        // key sub-chunk whose factor is cached
+                float qr = 0.f;     // q_j e^{B_j - rho_J}
 #pragma unroll
-                    for (int cc = 0; cc < CT; ++cc) a += sq[j][cc] * sk[s][cc] * expf(sB[j][cc] - sB[s][cc]);
-                    acc[p] = a;
+                for (int e = 0; e < SPT; ++e) {
+                    const int sk_ = s0 + e;
+                    const int J = sk_ / csub;
+                    float term = 0.f;
+                    if (J == I) {
+                        term = qj * sk[sk_][cc] * expf(bj - sB[sk_][cc]);
+                    } else if (J < I) {
+                        if (J != Jc) {
+                            const int last = (J + 1) * csub - 1;  // J < I: its rows are all valid
+                            qr = qj * expf(bj - sB[last][cc]);
+                            Jc = J;
+                        }
+                        term = qr * skr[sk_][cc];
+                    }
+                    acc[ps][e] += sk_ <= j ? term : 0.f;
                 }
             }
         }
@@ -95,9 +135,11 @@ __global__ void __launch_bounds__(kThreads) k_intra_P(const T* __restrict__ q, c
     }
     float* dst = P + (bh * N + i) * C * C;
 #pragma unroll
-    for (int p = 0; p < PP; ++p) {
-        const int pair = tid + p * kThreads;
-        if (pair < C * C) dst[pair] = acc[p];
+    for (int ps = 0; ps < NPASS; ++ps) {
+        const int j = tid / TPR + ps * RPP;
+        if (j >= C) continue;
+#pragma unroll
+        for (int e = 0; e < SPT; ++e) dst[j * C + s0 + e] = (j < nvalid && s0 + e <= j) ? acc[ps][e] : 0.f;
     }
 }
 
@@ -330,7 +372,7 @@ __global__ void __launch_bounds__(kThreads) k_dqdk(const T* __restrict__ q, cons
                                                    const float* __restrict__ Bc, const float* __restrict__ Sbuf,
                                                    const float* __restrict__ Dbuf, const float* __restrict__ dP,
                                                    T* __restrict__ dq, T* __restrict__ dk, float* __restrict__ r,
-                                                   int64_t L, int64_t K, int64_t V, int64_t N) {
+                                                   int64_t L, int64_t K, int64_t V, int64_t N, int csub) {
     constexpr int KT = 32, VT = 32, RPT = C / 8;
     extern __shared__ float smem[];
     float(*sq)[KT + 1] = reinterpret_cast<float(*)[KT + 1]>(smem);
@@ -396,6 +438,10 @@ __global__ void __launch_bounds__(kThreads) k_dqdk(const T* __restrict__ q, cons
     __syncthreads();
     const float Gam = sB[C - 1][cl];  // rows past nvalid hold B of the last valid row
     const float* dPc = dP + (bh * N + i) * C * C;
+    // two-level (secondary) chunking as in the forward scores: a pair in different sub-chunks is the
+    // product of two factors <= 1 through rho = B at the last row of the earlier sub-chunk; a pair
+    // in the same sub-chunk takes one exponential per term (log space)
+    auto rho = [&](int J) { return sB[(J + 1) * csub - 1 < C ? (J + 1) * csub - 1 : C - 1][cl]; };
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {
         const int j = g + 8 * m;
@@ -403,8 +449,24 @@ __global__ void __launch_bounds__(kThreads) k_dqdk(const T* __restrict__ q, cons
         float dqj = aq[m] * expf(bj);
         float dkj = ak[m] * expf(Gam - bj);
         if (j < nvalid) {
-            for (int s = 0; s <= j; ++s) dqj += dPc[j * C + s] * sk[s][cl] * expf(bj - sB[s][cl]);
-            for (int jj = j; jj < nvalid; ++jj) dkj += dPc[jj * C + j] * sq[jj][cl] * expf(sB[jj][cl] - bj);
+            const int I = j / csub;
+            // dq_j: keys s <= j; sub-chunk J < I contributes e^{B_j - rho_J} sum_s dP_js k_s e^{rho_J - B_s}
+            for (int J = 0; J < I; ++J) {
+                const float rJ = rho(J);
+                float part = 0.f;
+                for (int s = J * csub; s < (J + 1) * csub; ++s) part += dPc[j * C + s] * sk[s][cl] * expf(rJ - sB[s][cl]);
+                dqj += expf(bj - rJ) * part;
+            }
+            for (int s = I * csub; s <= j; ++s) dqj += dPc[j * C + s] * sk[s][cl] * expf(bj - sB[s][cl]);
+            // dk_j: queries jj >= j; those past j's sub-chunk I contribute e^{rho_I - B_j} dP q e^{B_jj - rho_I}
+            const int jend = (I + 1) * csub < nvalid ? (I + 1) * csub : nvalid;
+            for (int jj = j; jj < jend; ++jj) dkj += dPc[jj * C + j] * sq[jj][cl] * expf(sB[jj][cl] - bj);
+            if (jend < nvalid) {
+                const float rI = rho(I);
+                float part = 0.f;
+                for (int jj = jend; jj < nvalid; ++jj) part += dPc[jj * C + j] * sq[jj][cl] * expf(sB[jj][cl] - rI);
+                dkj += expf(rI - bj) * part;
+            }
             if (c < K) {
                 const int64_t off = (bh * L + t0 + j) * K + c;
                 stf(dq + off, dqj);
@@ -531,7 +593,7 @@ gla_status fwd_impl(const Problem& p, const T* q, const T* k, const T* v, const 
     const dim3 gc(unsigned(cdiv(p.K, 128)), unsigned(p.N), unsigned(p.BH));
     GLA_LAUNCH("simt_chunk_cumsum", k_chunk_cumsum, gc, 128, 0, s, la, Bc, p.L, p.K, p.C);
     GLA_LAUNCH("simt_intra_P", (k_intra_P<T, C>), dim3(unsigned(p.N), unsigned(p.BH)), kThreads, 0, s, q, k, Bc,
-               P, p.L, p.K, p.N);
+               P, p.L, p.K, p.N, int(p.c));
     const dim3 gw(unsigned(cdiv(p.K, 32)), unsigned(cdiv(p.V, 64)), unsigned(p.BH));
     GLA_LAUNCH("simt_state_walk", (k_state_walk<T, false>), gw, kThreads, 0, s, k, v, Bc, h0, Sbuf, hT, p.L, p.K,
                p.V, p.C, p.N);
@@ -548,7 +610,7 @@ gla_status bwd_impl(const Problem& p, const T* q, const T* k, const T* v, const 
         const dim3 gc(unsigned(cdiv(p.K, 128)), unsigned(p.N), unsigned(p.BH));
         GLA_LAUNCH("simt_chunk_cumsum", k_chunk_cumsum, gc, 128, 0, s, la, Bc, p.L, p.K, p.C);
         GLA_LAUNCH("simt_intra_P", (k_intra_P<T, C>), dim3(unsigned(p.N), unsigned(p.BH)), kThreads, 0, s, q, k,
-                   Bc, P, p.L, p.K, p.N);
+                   Bc, P, p.L, p.K, p.N, int(p.c));
         const dim3 gw(unsigned(cdiv(p.K, 32)), unsigned(cdiv(p.V, 64)), unsigned(p.BH));
         GLA_LAUNCH("simt_state_walk", (k_state_walk<T, false>), gw, kThreads, 0, s, k, v, Bc, h0, Sbuf,
                    (float*)nullptr, p.L, p.K, p.V, p.C, p.N);
@@ -563,7 +625,7 @@ gla_status bwd_impl(const Problem& p, const T* q, const T* k, const T* v, const 
         return GLA_ERR_CUDA;
     const dim3 gq(unsigned(cdiv(p.K, 32)), unsigned(p.N), unsigned(p.BH));
     GLA_LAUNCH("simt_dqdk", (k_dqdk<T, C>), gq, kThreads, sm, s, q, k, v, dO, Bc, Sbuf, Dbuf, dP, dq, dk, r, p.L, p.K,
-               p.V, p.N);
+               p.V, p.N, int(p.c));
     const dim3 gv(unsigned(cdiv(p.V, 64)), unsigned(p.N), unsigned(p.BH));
     GLA_LAUNCH("simt_dv", (k_dv<T, C>), gv, kThreads, 0, s, k, dO, Bc, Dbuf, P, dv, p.L, p.K, p.V, p.N);
     const float* hT = Sbuf + p.N * p.K * p.V;  // slot N of (b,h) = 0; stride below

@@ -355,7 +355,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int r = 0; r < 8; ++r) {
                         const int t = 16 * g + 8 * h + r;
-                        lv[r] = sLA[t * C + c];
+                        lv[r] = la_floor(sLA[t * C + c]);
                         kv[r] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + KH_OFF + tile_off(t, c)));
                     }
 #pragma unroll
@@ -407,12 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int j = t; j >= 0; --j) {
                     eq += dpm(t, j) * ks(j) * __expf(fminf(d, 0.f));
-                    d += j < nvalid ? lap[roff(j)] : 0.f;
+                    d += j < nvalid ? la_floor(lap[roff(j)]) : 0.f;
                 }
                 d = 0.f;
 #pragma unroll 1
                 for (int j = t; j < C; ++j) {
-                    if (j > t) d += j < nvalid ? lap[roff(j)] : 0.f;
+                    if (j > t) d += j < nvalid ? la_floor(lap[roff(j)]) : 0.f;
                     ek += dpm(j, t) * qs(j) * __expf(fminf(d, 0.f));
                 }
                 rbuf[t * C + c] = eq;

@@ -78,7 +78,7 @@ __device__ __forceinline__ void load_rows(const float* lap, const __nv_bfloat16*
         const float2 l2 = *reinterpret_cast<const float2*>(lap + o);
         const uint32_t qq = *reinterpret_cast<const uint32_t*>(qp + o);
         const uint32_t kk = *reinterpret_cast<const uint32_t*>(kp + o);
-        bb[r] = v ? l2 : make_float2(0.f, 0.f);
+        bb[r] = v ? make_float2(la_floor(l2.x), la_floor(l2.y)) : make_float2(0.f, 0.f);
         qv[r] = v ? qq : 0u;
         kv[r] = v ? kk : 0u;
     }
@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                         const int tk = 4 * lane + e;
                         const bool v = tk < nvalid;
                         const int64_t off = (bh * L + t0 + (v ? tk : 0)) * K + ch;
-                        a[e] = v ? la[off] : 0.f;
+                        a[e] = v ? la_floor(la[off]) : 0.f;
                         qa[e] = v ? __bfloat162float(q[off]) : 0.f;
                         ka[e] = v ? __bfloat162float(k[off]) : 0.f;
                     }

@@ -134,10 +134,13 @@ gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void*
                     const float* log_a, float* S, void* o, void* stream);
 
 /* Per-chunk inclusive log-space gate cumsum: for chunk i and row j,
- * Bcum[t = iC + j] = sum_{r=0..j} log_a[iC + r] per key channel, restarting
- * at every chunk boundary (C = the descriptor's chunk). In/out [B,H,L,Dk]
- * fp32. This is the first stage of every chunkwise pass; it is exported so
- * that it can be checked and timed on its own. */
+ * Bcum[t = iC + j] = sum_{r=0..j} max(log_a[iC + r], -200) per key channel,
+ * restarting at every chunk boundary (C = the descriptor's chunk). In/out
+ * [B,H,L,Dk] fp32. The floor changes no decay factor (e^-200 is 0 in fp32)
+ * but keeps a zero gate given as a huge negative number from swallowing the
+ * gates after it in the fp32 sum; every chunkwise pass applies it. This is
+ * the first stage of every chunkwise pass; it is exported so that it can be
+ * checked and timed on its own. */
 gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, void* stream);
 
 /* ---- forward without any allocation ---------------------------------------

@@ -54,7 +54,7 @@ def test_resolve_defaults(lib):
     c, sc, im, sm = (ctypes.c_int32() for _ in range(4))
     assert lib.gla_resolve(ctypes.byref(desc(dtype=0)), ctypes.byref(c), ctypes.byref(sc), ctypes.byref(im),
                            ctypes.byref(sm)) == 0
-    assert (c.value, im.value) == (64, 1)  # fp32 -> CUDA-core path, chunk 64
+    assert (c.value, sc.value, im.value) == (64, 16, 1)  # fp32 -> CUDA-core path, chunk 64, sub-chunks of 16
     # bf16 at a tensor-core shape -> tensor-core path, C = 128, c = 16, materialised states
     assert lib.gla_resolve(ctypes.byref(desc(dtype=1, Dk=256, Dv=512, L=2048)), ctypes.byref(c), ctypes.byref(sc),
                            ctypes.byref(im), ctypes.byref(sm)) == 0

@@ -75,6 +75,21 @@ def test_chunk_size_invariance(impl, chunk):
     check_bwd(inp, "f32", impl, chunk=chunk)
 
 
+@pytest.mark.parametrize("subchunk", [1, 4, 16, 64])
+def test_secondary_chunking_invariance(subchunk):
+    """The CUDA-core path's two-level chunking: pairs in different sub-chunks as products of two
+    factors <= 1 (rescaled at the end of the earlier sub-chunk), pairs inside one in log space. Every
+    sub-chunk length gives the oracle's result (subchunk 64 = one sub-chunk per chunk, all log space),
+    also with strong gates and a zero gate."""
+    inp = make_inputs(1, 2, 300, 64, 128, "f32", seed=6, h0=True, dhT=True)
+    check_fwd(inp, "f32", "simt", chunk=64, subchunk=subchunk)
+    check_bwd(inp, "f32", "simt", chunk=64, subchunk=subchunk)
+    strong = make_inputs(1, 1, 200, 64, 64, "f32", seed=7, gate_scale=1.0)
+    strong["log_a"][0, 0, 100, :] = -1e30  # alpha = 0: exact forgetting
+    check_fwd(strong, "f32", "simt", chunk=64, subchunk=subchunk)
+    check_bwd(strong, "f32", "simt", chunk=64, subchunk=subchunk)
+
+
 @pytest.mark.parametrize("impl", IMPLS)
 @pytest.mark.parametrize("KV", [(32, 48), (128, 256), (96, 64)])
 def test_head_dims(impl, KV):
@@ -368,3 +383,18 @@ def test_bounded_wait_timeout_is_reported_and_the_context_survives():
     inp = make_inputs(1, 2, 300, 128, 128, "bf16", seed=29)
     check_fwd(inp, "bf16", "tc", state_mode="materialized")
     assert gla.gla_check_device_error() == 0
+
+
+@pytest.mark.parametrize("impl", ["simt", "tc"])
+def test_single_zero_gate_mid_chunk(impl):
+    """A zero gate (alpha = 0, log alpha = -1e30) in the middle of a chunk, ordinary gates after it:
+    exact forgetting, and the decay among the later steps of the same chunk must not be lost to the
+    huge cumulative sum."""
+    dt = "f32" if impl == "simt" else "bf16"
+    K, V = (64, 64) if impl == "simt" else (128, 128)
+    inp = make_inputs(1, 2, 300, K, V, dt, seed=30, gate_scale=1.0, h0=True, dhT=True)
+    inp["log_a"][0, 0, 100, :] = -1e30
+    inp["log_a"][0, 1, 170, : K // 2] = -1e30
+    kw = dict(state_mode="materialized") if impl == "tc" else {}
+    check_fwd(inp, dt, impl, **kw)
+    check_bwd(inp, dt, impl, **kw)
