@@ -107,12 +107,12 @@ def kernel_models(w, C):
 # ncu capture of the default workload, with the SHA-1 of the kernel's source
 # file at capture time: a kernel whose source changed since reports null.
 NCU_TRAFFIC = {
-    "tc_prep": (75858688, "gla_tc_prep.cu", "33a8a99db46d13e3db1856e62934183d4c9ac1d7"),
-    "tc_walk_states": (83981056, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
-    "tc_output": (136546816, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
-    "tc_walk_dstates": (76066560, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
-    "tc_output_dv": (136039168, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
-    "tc_bwd_chunk": (333487359, "gla_tc_bwd.cu", "777d3c67271f29ccd44ad8c773dba63a7642c707"),
+    "tc_prep": (74336256, "gla_tc_prep.cu", "13e8d173e1ef24a6ea33660af099850d6e98cfaf"),
+    "tc_walk_states": (82829568, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
+    "tc_output": (135774976, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
+    "tc_walk_dstates": (75097600, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
+    "tc_output_dv": (136403712, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
+    "tc_bwd_chunk": (330472448, "gla_tc_bwd.cu", "a7323768795bc10dcfda90f0f92666b5702b21ef"),
 }
 
 
