@@ -112,7 +112,7 @@ NCU_TRAFFIC = {
     "tc_output": (135774976, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
     "tc_walk_dstates": (75097600, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
     "tc_output_dv": (136403712, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
-    "tc_bwd_chunk": (330472448, "gla_tc_bwd.cu", "a7323768795bc10dcfda90f0f92666b5702b21ef"),
+    "tc_bwd_chunk": (331860736, "gla_tc_bwd.cu", "c2a6f65f16833267640da8c56f1e6da405f4b868"),
 }
 
 

@@ -80,7 +80,7 @@ constexpr int kThreads = 576;
 constexpr int kFinal = 512;  // threads of the final phase: warps 2-17
 constexpr float kSafeDecay = 64.f;
 constexpr float kSafeGam = 1.6038109e-28f;  // e^-64
-constexpr uint32_t kStaggerNs = 8000;       // start offset of every other first-wave CTA
+constexpr uint32_t kStaggerNs = 10000;      // start offset of every other first-wave CTA
 
 struct BwdBars {
     uint64_t full[NSTAGE], empty[NSTAGE];
