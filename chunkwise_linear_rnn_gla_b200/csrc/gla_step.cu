@@ -8,9 +8,12 @@
 // The step is a pure stream over the fp32 state (read + write 8*Dk*Dv bytes
 // per head), so the kernel is laid out for HBM: each thread owns four
 // adjacent state columns (16-byte loads/stores, a warp covers 512 contiguous
-// bytes of one state row), a block covers up to 256 columns of one head, and
+// bytes of one state row), a block covers up to 128 columns of one head, and
 // the Dk rows are split over KS row-slices whose partial q.S sums are reduced
-// in shared memory.
+// in shared memory. Each thread loads a batch of rows before storing any, so
+// that the stream has enough loads in flight when the state comes from HBM.
+
+#include <cstdint>
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -22,12 +25,37 @@ namespace gla {
 namespace {
 
 constexpr int kStepThreads = 256;
+constexpr int kStepBatch = 8;  // state rows a thread has in flight
+
+template <int VEC>
+struct StepVec;
+template <>
+struct StepVec<4> {
+    using type = float4;
+    static __device__ __forceinline__ float get(const float4& x, int e) {
+        return e == 0 ? x.x : e == 1 ? x.y : e == 2 ? x.z : x.w;
+    }
+    static __device__ __forceinline__ void set(float4& x, int e, float y) {
+        if (e == 0) x.x = y;
+        else if (e == 1) x.y = y;
+        else if (e == 2) x.z = y;
+        else x.w = y;
+    }
+};
+template <>
+struct StepVec<1> {
+    using type = float;
+    static __device__ __forceinline__ float get(const float& x, int) { return x; }
+    static __device__ __forceinline__ void set(float& x, int, float y) { x = y; }
+};
 
 template <typename T, int VEC>
 __global__ void __launch_bounds__(kStepThreads) k_step(const T* __restrict__ q, const T* __restrict__ k,
                                                        const T* __restrict__ v, const float* __restrict__ la,
                                                        float* __restrict__ S, T* __restrict__ o, int K, int V,
                                                        int CG) {
+    using SV = StepVec<VEC>;
+    using vec_t = typename SV::type;
     extern __shared__ float sm[];
     float* sq = sm;
     float* sk = sm + K;
@@ -47,32 +75,33 @@ __global__ void __launch_bounds__(kStepThreads) k_step(const T* __restrict__ q, 
     float acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-    if (ks < KS && col0 < V) {
+    if (col0 < V) {
         float vv[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) vv[e] = ldf(v + bh * V + col0 + e);
         float* base = S + bh * int64_t(K) * V + col0;
-        if (VEC == 4) {
-#pragma unroll 4
-            for (int c = ks; c < K; c += KS) {
-                float4 s4 = *reinterpret_cast<const float4*>(base + int64_t(c) * V);
-                const float a = sa[c], kc = sk[c], qc = sq[c];
-                s4.x = a * s4.x + kc * vv[0];
-                s4.y = a * s4.y + kc * vv[VEC > 1 ? 1 : 0];
-                s4.z = a * s4.z + kc * vv[VEC > 2 ? 2 : 0];
-                s4.w = a * s4.w + kc * vv[VEC > 3 ? 3 : 0];
-                *reinterpret_cast<float4*>(base + int64_t(c) * V) = s4;
-                acc[0] += qc * s4.x;
-                acc[VEC > 1 ? 1 : 0] += qc * s4.y;
-                acc[VEC > 2 ? 2 : 0] += qc * s4.z;
-                acc[VEC > 3 ? 3 : 0] += qc * s4.w;
+        // rows ks, ks+KS, ...: a batch of kStepBatch rows is loaded before any of them is stored, so
+        // that every thread keeps that many independent loads in flight
+        for (int c0 = ks; c0 < K; c0 += KS * kStepBatch) {
+            vec_t sv[kStepBatch];
+#pragma unroll
+            for (int u = 0; u < kStepBatch; ++u) {
+                const int c = c0 + u * KS;
+                if (c < K) sv[u] = *reinterpret_cast<const vec_t*>(base + int64_t(c) * V);
             }
-        } else {
-            for (int c = ks; c < K; c += KS) {
-                float s1 = base[int64_t(c) * V];
-                s1 = sa[c] * s1 + sk[c] * vv[0];
-                base[int64_t(c) * V] = s1;
-                acc[0] += sq[c] * s1;
+#pragma unroll
+            for (int u = 0; u < kStepBatch; ++u) {
+                const int c = c0 + u * KS;
+                if (c < K) {
+                    const float a = sa[c], kc = sk[c], qc = sq[c];
+#pragma unroll
+                    for (int e = 0; e < VEC; ++e) {
+                        const float x = a * SV::get(sv[u], e) + kc * vv[e];
+                        SV::set(sv[u], e, x);
+                        acc[e] += qc * x;
+                    }
+                    *reinterpret_cast<vec_t*>(base + int64_t(c) * V) = sv[u];
+                }
             }
         }
     }
@@ -93,10 +122,13 @@ template <typename T>
 gla_status step_typed(const Problem& p, const T* q, const T* k, const T* v, const float* la, float* S, T* o,
                       cudaStream_t s) {
     const int K = int(p.K), V = int(p.V);
-    const bool vec = (V % 4) == 0;
+    // 16-byte state accesses need a 16-byte aligned state and rows of a multiple of 4 floats
+    const bool vec = (V % 4) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;
     const int VEC = vec ? 4 : 1;
-    const int ncols = V / VEC + (vec ? 0 : 0);
-    int CG = ncols < 64 ? ncols : 64;
+    const int ncols = V / VEC;
+    // 32 column groups (512 bytes of a state row per warp) and 8 row-slices per block: several
+    // blocks per head, so that even a small batch fills the SMs
+    int CG = ncols < 32 ? ncols : 32;
     // a power of two that divides the block so that every row-slice is full
     int cg2 = 1;
     while (cg2 * 2 <= CG) cg2 *= 2;

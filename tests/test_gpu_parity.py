@@ -163,6 +163,39 @@ def test_step_matches_oracle(dtype):
     compare("S", Sd, S_ref, "f32" if dtype == "f32" else "bf16")
 
 
+@pytest.mark.parametrize("K,V", [(100, 96), (200, 7), (1, 4)])
+def test_step_ragged_rows_odd_columns(K, V):
+    """Decode step with a row count that leaves the last row batch partial, an odd value width
+    (scalar column path) and a single key channel."""
+    import oracle
+
+    B, H, T = 3, 2, 5
+    st = make_step_inputs(B, H, K, V, T, "bf16", seed=18)
+    S = torch.randn(B, H, K, V, generator=torch.Generator().manual_seed(2)) * 0.1
+    S_ref = S.double().numpy()
+    Sd = S.cuda()
+    for t in range(T):
+        o = gla.gla_step(st["q"][t].cuda(), st["k"][t].cuda(), st["v"][t].cuda(), st["log_a"][t].cuda(), Sd)
+        o_ref, S_ref = oracle.step(to_f64_numpy(st["q"][t]), to_f64_numpy(st["k"][t]), to_f64_numpy(st["v"][t]),
+                                   to_f64_numpy(st["log_a"][t]), S_ref)
+        torch.cuda.synchronize()
+        compare("o_%d" % t, o, o_ref, "bf16")
+    compare("S", Sd, S_ref, "bf16")
+
+
+def test_step_rejects_a_misaligned_state():
+    """A state 4 bytes past a 16-byte boundary is refused before any launch; the state is untouched."""
+    B, H, K, V = 2, 2, 64, 96
+    st = make_step_inputs(B, H, K, V, 1, "bf16", seed=19)
+    buf = torch.ones(B * H * K * V + 4, device="cuda")
+    Sd = buf[1:1 + B * H * K * V].view(B, H, K, V)
+    with pytest.raises(gla.GlaError) as ei:
+        gla.gla_step(st["q"][0].cuda(), st["k"][0].cuda(), st["v"][0].cuda(), st["log_a"][0].cuda(), Sd)
+    assert "INVALID_ARG" in str(ei.value)
+    torch.cuda.synchronize()
+    assert bool((buf == 1).all())
+
+
 def test_step_iterated_equals_fwd():
     B, H, L, K, V = 2, 2, 70, 64, 64
     inp = make_inputs(B, H, L, K, V, "f32", seed=16, h0=True)
