@@ -163,10 +163,11 @@ def test_step_matches_oracle(dtype):
     compare("S", Sd, S_ref, "f32" if dtype == "f32" else "bf16")
 
 
-@pytest.mark.parametrize("K,V", [(100, 96), (200, 7), (1, 4)])
+@pytest.mark.parametrize("K,V", [(100, 96), (200, 7), (1, 4), (200, 104), (8, 32), (256, 40), (64, 36)])
 def test_step_ragged_rows_odd_columns(K, V):
-    """Decode step with a row count that leaves the last row batch partial, an odd value width
-    (scalar column path) and a single key channel."""
+    """Decode step with row counts that leave the last row batch or the last 128-row box partial,
+    value widths that leave the last 32-column tile partial or need the scalar column path, and
+    one or eight key channels."""
     import oracle
 
     B, H, T = 3, 2, 5
@@ -181,6 +182,35 @@ def test_step_ragged_rows_odd_columns(K, V):
         torch.cuda.synchronize()
         compare("o_%d" % t, o, o_ref, "bf16")
     compare("S", Sd, S_ref, "bf16")
+
+
+def test_step_replays_from_cuda_graph():
+    """Eight decode steps captured in a CUDA graph and replayed give the eager steps' outputs and
+    state bit for bit (the steps are chained by programmatic dependent launch)."""
+    B, H, K, V, T = 8, 4, 128, 256, 8
+    st = make_step_inputs(B, H, K, V, T, "bf16", seed=20)
+    q, k, v, la = (st[n].cuda() for n in ("q", "k", "v", "log_a"))
+    S0 = torch.randn(B, H, K, V, generator=torch.Generator().manual_seed(3)).cuda() * 0.1
+    S_e = S0.clone()
+    outs_e = [gla.gla_step(q[t], k[t], v[t], la[t], S_e).clone() for t in range(T)]
+    S_g = S0.clone()
+    outs_g = [torch.empty(B, H, V, dtype=torch.bfloat16, device="cuda") for _ in range(T)]
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        gla.gla_step(q[0], k[0], v[0], la[0], S0.clone(), o=outs_g[0])
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for t in range(T):
+            gla.gla_step(q[t], k[t], v[t], la[t], S_g, o=outs_g[t])
+    S_g.copy_(S0)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(S_g, S_e)
+    for t in range(T):
+        assert torch.equal(outs_g[t], outs_e[t]), t
 
 
 def test_step_rejects_a_misaligned_state():
