@@ -109,10 +109,10 @@ def kernel_models(w, C):
 NCU_TRAFFIC = {
     "tc_prep": (74336256, "gla_tc_prep.cu", "13e8d173e1ef24a6ea33660af099850d6e98cfaf"),
     "tc_walk_states": (82829568, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
-    "tc_output": (135774976, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
+    "tc_output": (135306240, "gla_tc_out.cu", "285ea49a1a538d922b569c6ed2e3ad1ab5af4341"),
     "tc_walk_dstates": (75097600, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
-    "tc_output_dv": (136403712, "gla_tc_out.cu", "0c9f4538a556acc403c249a15df0a55ccfdc8a5c"),
-    "tc_bwd_chunk": (331860736, "gla_tc_bwd.cu", "c2a6f65f16833267640da8c56f1e6da405f4b868"),
+    "tc_output_dv": (132920832, "gla_tc_out.cu", "285ea49a1a538d922b569c6ed2e3ad1ab5af4341"),
+    "tc_bwd_chunk": (327452160, "gla_tc_bwd.cu", "4ebf7e129f463e33f6887504e06f27e8599c0b35"),
 }
 
 

@@ -89,9 +89,12 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
 
 // Chunk-parallel Y_i = A_i X_i + Pm_i B_i from stored bf16 chunk states X
 // (gla_tc_out.cu): forward o (A = Q~, Pm = P) and dv (A = K~, Pm = P^T).
+// late_wait: the kernel follows, by programmatic dependent launch, a kernel that it does not
+// depend on and that triggers its dependents only after its own wait; it then reads its inputs
+// at once and waits for that kernel only before it exits.
 gla_status tc_chunk_out_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* X,
                                const __nv_bfloat16* Pm, const __nv_bfloat16* Bv, bool p_transposed,
-                               __nv_bfloat16* Y, cudaStream_t s, const char* name);
+                               __nv_bfloat16* Y, bool late_wait, cudaStream_t s, const char* name);
 
 // Backward, chunk-parallel part (gla_tc_bwd.cu): dq, dk and dlog a from dO, v,
 // the stored states S_[i] and D_i, Q~ and e^Gamma.

@@ -106,7 +106,7 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
              : tc_walk_launch(p, a, s, "tc_walk_states");
     if (st != GLA_OK) return st;
     return tc_chunk_out_launch(p, b.Qt, b.states, b.P, static_cast<const __nv_bfloat16*>(v), false,
-                               static_cast<__nv_bfloat16*>(o), s, "tc_output");
+                               static_cast<__nv_bfloat16*>(o), false, s, "tc_output");
 }
 
 gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* la, const float* h0,
@@ -161,9 +161,13 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
                                                                      b.segbuf, true, s, "tc_walk_dstates")
                                              : tc_walk_launch(p, a, s, "tc_walk_dstates");
             if (st != GLA_OK) return st;
-            st = tc_chunk_out_launch(p, b.Kt, b.Dbuf, b.P, static_cast<const __nv_bfloat16*>(dO), true,
-                                     static_cast<__nv_bfloat16*>(dv), s, "tc_output_dv");
+            // dv does not depend on the chunk backward, which triggers its dependents only after its
+            // own wait: launched after it, the dv GEMM starts on the SMs that the backward's last
+            // wave leaves idle and waits for the backward only before it exits
+            st = tc_bwd_chunk_launch(p, q, k, la, dO, v, b.Qt, b.gam, b.states, b.Dbuf, dq, dk, dla, s);
             if (st != GLA_OK) return st;
+            return tc_chunk_out_launch(p, b.Kt, b.Dbuf, b.P, static_cast<const __nv_bfloat16*>(dO), true,
+                                       static_cast<__nv_bfloat16*>(dv), true, s, "tc_output_dv");
         }
     }
     return tc_bwd_chunk_launch(p, q, k, la, dO, v, b.Qt, b.gam, b.states, b.Dbuf, dq, dk, dla, s);

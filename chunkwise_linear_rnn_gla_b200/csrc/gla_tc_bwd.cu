@@ -158,8 +158,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         tma_prefetch(&tmK);
         tma_prefetch(&tmLA);
     }
-    pdl_launch_dependents();
+    // dependents are triggered only after the wait, so that a dependent that reads the same inputs
+    // without waiting for this kernel (the dv GEMM) finds them complete
     pdl_wait();
+    pdl_launch_dependents();
 
     if (warp == 0) {
         if (lane == 0) {

@@ -56,7 +56,8 @@ template <int NH, int NQ, bool PT>
 __global__ void __launch_bounds__(kOutThreads, 1)
     k_chunk_out(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmX,
                 const __grid_constant__ CUtensorMap tmP, const __grid_constant__ CUtensorMap tmB,
-                __nv_bfloat16* __restrict__ Y, int64_t L, int64_t N, int64_t V, int64_t BH, int* err) {
+                __nv_bfloat16* __restrict__ Y, int64_t L, int64_t N, int64_t V, int64_t BH, int late_wait,
+                int* err) {
     using Cfg = OutCfg<NQ>;
     constexpr int BVO = Cfg::bvo, G = Cfg::group;
     extern __shared__ uint8_t smem_raw[];
@@ -104,7 +105,10 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         tma_prefetch(&tmB);
     }
     pdl_launch_dependents();
-    pdl_wait();
+    // late_wait: launched after a kernel that it does not depend on (every input was complete before
+    // that kernel passed its own wait); the blocks start on the SMs that kernel leaves idle, and
+    // wait for it only before they exit, so that whatever follows sees both kernels complete
+    if (!late_wait) pdl_wait();
 
     if (warp == 0) {
         if (lane == 0) {
@@ -220,6 +224,7 @@ __global__ void __launch_bounds__(kOutThreads, 1)
         tc_fence_after();
         tmem_dealloc(tmem, Cfg::tmem_cols);
     }
+    if (late_wait) pdl_wait();
 }
 
 bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
@@ -230,7 +235,8 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
 }
 
 template <int NH, int NQ, bool PT>
-gla_status launch_out(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, cudaStream_t s, const char* name) {
+gla_status launch_out(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, bool late_wait, cudaStream_t s,
+                      const char* name) {
     auto fn = k_chunk_out<NH, NQ, PT>;
     const size_t smem = OutCfg<NQ>::smem;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
@@ -239,22 +245,23 @@ gla_status launch_out(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, 
     const int64_t sms = sm_count();
     const unsigned grid = unsigned(items < sms ? items : sms);
     GLA_LAUNCH_PDL(name, fn, dim3(grid), kOutThreads, smem, s, m[0], m[1], m[2], m[3], Y, p.L, p.N, p.V, p.BH,
-               device_error_word());
+                   int(late_wait), device_error_word());
     return GLA_OK;
 }
 
 template <int NH, bool PT>
-gla_status launch_out_nq(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, cudaStream_t s, const char* name) {
-    if (p.V % 256 == 0) return launch_out<NH, 4, PT>(p, m, Y, s, name);
-    if (p.V % 128 == 0) return launch_out<NH, 2, PT>(p, m, Y, s, name);
-    return launch_out<NH, 1, PT>(p, m, Y, s, name);
+gla_status launch_out_nq(const Problem& p, const CUtensorMap* m, __nv_bfloat16* Y, bool lw, cudaStream_t s,
+                         const char* name) {
+    if (p.V % 256 == 0) return launch_out<NH, 4, PT>(p, m, Y, lw, s, name);
+    if (p.V % 128 == 0) return launch_out<NH, 2, PT>(p, m, Y, lw, s, name);
+    return launch_out<NH, 1, PT>(p, m, Y, lw, s, name);
 }
 
 }  // namespace
 
 gla_status tc_chunk_out_launch(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* X,
                                const __nv_bfloat16* Pm, const __nv_bfloat16* Bv, bool p_transposed,
-                               __nv_bfloat16* Y, cudaStream_t s, const char* name) {
+                               __nv_bfloat16* Y, bool late_wait, cudaStream_t s, const char* name) {
     CUtensorMap m[4];
     memset(m, 0, sizeof(m));
     const uint64_t L = uint64_t(p.L), K = uint64_t(p.K), V = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
@@ -262,8 +269,11 @@ gla_status tc_chunk_out_launch(const Problem& p, const __nv_bfloat16* A, const _
           map3(&m[3], Bv, V, L, BH)))
         return GLA_ERR_CUDA;
     const int NH = int(p.K / 128);
-    if (NH == 1) return p_transposed ? launch_out_nq<1, true>(p, m, Y, s, name) : launch_out_nq<1, false>(p, m, Y, s, name);
-    if (NH == 2) return p_transposed ? launch_out_nq<2, true>(p, m, Y, s, name) : launch_out_nq<2, false>(p, m, Y, s, name);
+    const bool lw = late_wait;
+    if (NH == 1)
+        return p_transposed ? launch_out_nq<1, true>(p, m, Y, lw, s, name) : launch_out_nq<1, false>(p, m, Y, lw, s, name);
+    if (NH == 2)
+        return p_transposed ? launch_out_nq<2, true>(p, m, Y, lw, s, name) : launch_out_nq<2, false>(p, m, Y, lw, s, name);
     return GLA_ERR_UNSUPPORTED;
 }
 
