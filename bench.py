@@ -473,6 +473,9 @@ def main():
     layer_roof = {"roofline_ms": round(t_roof * 1e3, 5), "frac": round(t_roof * 1e3 / ms_per_step, 4),
                   "alg_bytes": alg["bytes"], "alg_flops": alg["flops"],
                   "tflops": round(alg["flops"] / (ms_per_step / 1e3) / 1e12, 2),
+                  # the same flops against the sustained (power-capped) bf16 GEMM rate
+                  "tflops_frac_of_sustained_bf16": round(alg["flops"] / (ms_per_step / 1e3) / 1e12
+                                                         / peaks["bf16_tflops_sustained"], 4),
                   "bound": "hbm" if alg["bytes"] / peaks["hbm_gbs"] / 1e9 > alg["flops"] / peaks["bf16_tflops"] / 1e12
                   else "tensor"}
 
