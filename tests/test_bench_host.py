@@ -1,0 +1,95 @@
+"""Host-side checks of the benchmark's accounting (CPU only): the algorithmic byte and flop
+model of one fwd+bwd step, the per-kernel byte models behind the roofline, and the rule that a
+recorded ncu traffic figure is dropped once the kernel's source has changed."""
+import hashlib
+import os
+import sys
+from types import SimpleNamespace
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+
+
+def _shape(B, H, L, K, V):
+    return SimpleNamespace(B=B, H=H, L=L, K=K, V=V)
+
+
+def _io_bytes(B, H, L, K, V):
+    """Every tensor the layer reads or writes once, listed one by one (bf16 q, k, v, o, dO, dq, dk,
+    dv; fp32 log a, dlog a, hT, dh0)."""
+    th, bh = B * H * L, B * H
+    fwd = [("q", th * K, 2), ("k", th * K, 2), ("v", th * V, 2), ("log_a", th * K, 4), ("o", th * V, 2),
+           ("hT", bh * K * V, 4)]
+    bwd = [("q", th * K, 2), ("k", th * K, 2), ("v", th * V, 2), ("dO", th * V, 2), ("log_a", th * K, 4),
+           ("dq", th * K, 2), ("dk", th * K, 2), ("dv", th * V, 2), ("dlog_a", th * K, 4),
+           ("dh0", bh * K * V, 4)]
+    return sum(n * e for _, n, e in fwd), sum(n * e for _, n, e in bwd)
+
+
+def _gemm_flops(B, H, L, K, V, C):
+    """The chunk form's contractions per chunk of C tokens, 2 flops per multiply-add; the
+    intra-chunk products count their causal half."""
+    n_chunks = B * H * (L // C)
+    fwd = [2 * C * K * V,  # state update K~^T V
+           2 * C * K * V,  # inter output Q~ S
+           C * C * K,      # causal half of Q K^T
+           C * C * V]      # causal half of P V
+    bwd = [2 * C * K * V] * 4 + [  # D chain, dO S^T, v D^T, K~ D
+        C * C * V,  # dP = dO V^T
+        C * C * V,  # P^T dO
+        C * C * K,  # dP K
+        C * C * K,  # dP^T Q
+        C * C * K]  # P recomputed
+    return n_chunks * sum(fwd), n_chunks * sum(bwd)
+
+
+def test_layer_model_matches_the_tensor_list():
+    for (B, H, L, K, V) in [(4, 4, 2048, 256, 512), (8, 4, 2048, 128, 256), (1, 4, 16384, 128, 256)]:
+        m = bench.algorithmic_model(_shape(B, H, L, K, V), C=128)
+        bf, bb = _io_bytes(B, H, L, K, V)
+        assert (m["bytes_fwd"], m["bytes_bwd"]) == (bf, bb)
+        ff, fb = _gemm_flops(B, H, L, K, V, 128)
+        assert (m["flops_fwd"], m["flops_bwd"]) == (ff, fb)
+
+
+def test_layer_roofline_of_the_1p3b_shape():
+    m = bench.algorithmic_model(_shape(4, 4, 2048, 256, 512), C=128)
+    assert m["bytes"] == 385875968 and m["flops"] == 62277025792
+    t_hbm = m["bytes"] / 6551e9
+    t_flop = m["flops"] / 1655.1e12
+    assert t_hbm > t_flop  # bound by HBM
+    assert abs(t_hbm * 1e6 - 58.9) < 0.05
+
+
+def test_kernel_byte_models_of_the_1p3b_shape():
+    """Per-launch algorithmic megabytes of the tensor-core kernels at B=4, H=4, L=2048, d_k=256,
+    d_v=512, C=128, as tabulated with the measured kernel times."""
+    m = bench.kernel_models(_shape(4, 4, 2048, 256, 512), 128)
+    want = {"tc_prep": 109.3, "tc_walk_states": 117.4, "tc_output": 159.4, "tc_walk_dstates": 117.4,
+            "tc_output_dv": 159.4, "tc_bwd_chunk": 352.6}
+    for name, mb in want.items():
+        assert abs(m[name]["bytes"] / 1e6 - mb) < 0.05, name
+        assert m[name]["bound"] == "hbm"
+    # the decode step streams the fp32 state once in and once out
+    d = bench.kernel_models(_shape(64, 4, 1, 128, 256), 128)["step"]
+    assert d["bytes"] == 2 * 64 * 4 * 128 * 256 * 4
+
+
+def test_recorded_traffic_is_dropped_when_the_source_changes(monkeypatch):
+    src = "gla_step.cu"
+    with open(os.path.join(ROOT, "chunkwise_linear_rnn_gla_b200", "csrc", src), "rb") as f:
+        sha = hashlib.sha1(f.read()).hexdigest()
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"current": (123, src, sha), "stale": (456, src, "0" * 40),
+                                               "missing": (789, "no_such_file.cu", sha)})
+    assert bench.measured_traffic("current") == 123
+    assert bench.measured_traffic("stale") is None
+    assert bench.measured_traffic("missing") is None
+    assert bench.measured_traffic("unknown") is None
+
+
+def test_recorded_traffic_entries_name_existing_sources():
+    for name, (nbytes, src, sha) in bench.NCU_TRAFFIC.items():
+        assert nbytes > 0 and len(sha) == 40
+        assert os.path.exists(os.path.join(ROOT, "chunkwise_linear_rnn_gla_b200", "csrc", src)), name
