@@ -93,3 +93,15 @@ def test_recorded_traffic_entries_name_existing_sources():
     for name, (nbytes, src, sha) in bench.NCU_TRAFFIC.items():
         assert nbytes > 0 and len(sha) == 40
         assert os.path.exists(os.path.join(ROOT, "chunkwise_linear_rnn_gla_b200", "csrc", src)), name
+
+
+def test_workload_timer_lists_and_validates_without_a_gpu(capsys):
+    import pytest
+
+    from chunkwise_linear_rnn_gla_b200 import time_workloads
+
+    assert time_workloads.main(["--list"]) == 0
+    listed = [line.split(" - ")[0] for line in capsys.readouterr().out.splitlines()]
+    assert "gla1p3b_fwdbwd" in listed and "decode" in listed and "tiny_f32" not in listed
+    with pytest.raises(SystemExit):
+        time_workloads.main(["--only", "no_such_workload"])
