@@ -1,6 +1,6 @@
 #!/usr/bin/env python
-"""Benchmark: GLA layer forward+backward tokens/s on B200 and the roofline
-fraction of the dominant kernel.
+"""Benchmark: GLA layer forward+backward tokens/s on B200 and its fraction of
+the layer roofline.
 
 One step = gla_fwd + gla_bwd (the backward reuses the forward's workspace) on
 the 1.3B-layer shape B=4 H=4 L=2048 d_k=256 d_v=512, bf16 q/k/v/dO with fp32
@@ -17,6 +17,8 @@ from __future__ import annotations
 import argparse
 import json
 import math
+
+import numpy as np
 import os
 import statistics
 import subprocess
@@ -101,6 +103,44 @@ def kernel_models(w, C):
                              + BH * N * K * 4,
                              flops=th * (2 * C * V + 4 * K * V + 4 * C * K), bound="hbm")
     return m
+
+
+def method_bytes(w):
+    """Per kernel: bytes of the LAYER's own inputs that the kernel reads plus the layer's own outputs
+    that it writes (q, k, v, dO, log a, h0/dhT in; o, hT, dq, dk, dv, dlog a, dh0 out), each once.
+    The implementation's intermediates (chunk states, rescaled operands, score blocks) are not
+    counted: this is the figure a kernel's bandwidth fraction is judged on."""
+    BH, L, K, V = w.B * w.H, w.L, w.K, w.V
+    th = BH * L
+    e = 2
+    st = BH * K * V * 4
+    return {
+        "tc_prep": th * (2 * K * e + 4 * K),                      # q, k, log a
+        "tc_walk_states": th * V * e + st,                        # v; hT
+        "tc_output": th * V * e * 2,                              # v; o
+        "tc_walk_dstates": th * V * e + st,                       # dO; dh0
+        "tc_output_dv": th * V * e * 2,                           # dO; dv
+        "tc_bwd_chunk": th * (2 * K * e + 4 * K + 2 * V * e + 2 * K * e + 4 * K),  # q k log a v dO; dq dk dlog a
+        "tc_walk_fwd": th * (2 * V * e) + st,                     # v; o, hT
+        "tc_walk_dv": th * (2 * V * e) + st,                      # dO; dv, dh0
+        "step": 2 * st + BH * (2 * K * e + V * e + 4 * K + V * e),
+    }
+
+
+def fwd_model(w, C=128):
+    """Algorithmic bytes and flops of the forward alone (o and hT from q, k, v, log a)."""
+    m = algorithmic_model(w, C)
+    return {"bytes": m["bytes_fwd"], "flops": m["flops_fwd"]}
+
+
+def layer_roofline(alg_bytes, alg_flops, ms, peaks):
+    """The step against max(algorithmic bytes / measured HBM bandwidth, algorithmic flops / measured
+    bf16 dense peak)."""
+    t_hbm = alg_bytes / (peaks["hbm_gbs"] * 1e9)
+    t_flop = alg_flops / (peaks["bf16_tflops"] * 1e12)
+    t_roof = max(t_hbm, t_flop)
+    return {"roofline_ms": round(t_roof * 1e3, 5), "frac": round(t_roof * 1e3 / ms, 4),
+            "bound": "hbm" if t_hbm >= t_flop else "tensor"}
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one
@@ -241,6 +281,162 @@ def cpu_baseline(w, budget_s=20.0):
                       % (nheads, w.B * w.H, w.L, w.K, w.V, reps, dt)}
 
 
+# ------------------------------------------------------- the other workloads
+def oracle_sample(w, passes, n_heads_max, L_max):
+    """The fp64 oracle as it stands on a bounded sample of a workload: the first n heads (n = host
+    cores, at most B*H) over the first L_max tokens. Returns tokens/s (a token carries H heads)."""
+    import oracle
+    from chunkwise_linear_rnn_gla_b200.inputs import make_inputs, to_f64_numpy
+
+    cores = oracle.num_threads()
+    Ls = min(w.L, L_max)
+    nheads = max(1, min(w.B * w.H, cores, n_heads_max))
+    inp = make_inputs(1, nheads, Ls, w.K, w.V, w.dtype, seed=0, z_mean=w.z_mean, with_grad=(passes != "fwd"))
+    f = {n: to_f64_numpy(t) for n, t in inp.items()}
+    t0 = time.perf_counter()
+    oracle.fwd(f["q"], f["k"], f["v"], f["log_a"])
+    if passes != "fwd":
+        oracle.bwd(f["q"], f["k"], f["v"], f["log_a"], f["dO"])
+    dt = time.perf_counter() - t0
+    return {"value": nheads * Ls / w.H / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": "%d of %d heads, first %d of L=%d tokens, %s fp64 step recurrence, %.2f s"
+                      % (nheads, w.B * w.H, Ls, w.L, passes, dt)}
+
+
+def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
+    """Device time of every other named workload, eager calls with L2 flushed before each (median of
+    `reps` CUDA-event timings after 3 warm-ups): the 340M-layer forward, the long sequence with
+    materialised and non-materialised states (with each mode's workspace bytes: the memory
+    footprint), the fixed-token sweep, and the decode workload with L2 flushed and with the state
+    left in L2."""
+    import torch
+
+    import chunkwise_linear_rnn_gla_b200 as gla
+    from chunkwise_linear_rnn_gla_b200.inputs import DECODE, WORKLOADS, make_inputs, make_step_inputs
+
+    stream = torch.cuda.current_stream(dev)
+
+    def med_ms(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1.0)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            ts.append(a.elapsed_time(b))
+        return sorted(ts)[len(ts) // 2]
+
+    cases = [("gla340m_fwd", "fwd", ("materialized",)), ("long16k", "fwd+bwd", ("materialized", "nonmaterialized"))]
+    cases += [("sweep_L%d" % L, "fwd+bwd", ("materialized",)) for L in (1024, 2048, 4096, 8192, 16384)]
+    out = {}
+    for name, passes, modes in cases:
+        w = WORKLOADS[name]
+        inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=0, z_mean=w.z_mean, with_grad=(passes != "fwd"))
+        d = {k: v.to(dev) for k, v in inp.items()}
+        o = torch.empty_like(d["v"])
+        hT = torch.empty(w.B, w.H, w.K, w.V, device=dev)
+        outs = None
+        if passes != "fwd":
+            outs = {"dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]), "dv": torch.empty_like(d["v"]),
+                    "dlog_a": torch.empty_like(d["log_a"]), "dh0": torch.empty(w.B, w.H, w.K, w.V, device=dev)}
+        alg = algorithmic_model(w) if passes != "fwd" else fwd_model(w)
+        entry = {"B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V, "passes": passes, "modes": {}}
+        for mode in modes:
+            desc = gla.make_desc(w.B, w.H, w.L, w.K, w.V, w.dtype, 0, 0, mode, "auto")
+            ws_f, ws_b = gla.gla_fwd_workspace_size(desc), gla.gla_bwd_workspace_size(desc)
+            ws = torch.empty(ws_b if passes != "fwd" else ws_f, dtype=torch.uint8, device=dev)
+            kw = dict(state_mode=mode)
+
+            def fn():
+                gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], None, o=o, hT=hT, workspace=ws, **kw)
+                if outs is not None:
+                    gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], None, None, workspace=ws,
+                                ws_from_fwd=True, out=outs, **kw)
+
+            ms = med_ms(fn)
+            lr = layer_roofline(alg["bytes"], alg["flops"], ms, peaks)
+            entry["modes"][mode] = {"ms": round(ms, 5), "tokens_per_s": round(w.B * w.L / ms * 1e3, 1),
+                                    "layer_roofline_frac": lr["frac"], "roofline_ms": lr["roofline_ms"],
+                                    "workspace_bytes": {"fwd": ws_f, "fwd+bwd": ws_b}}
+            del ws
+        if with_cpu:
+            entry["cpu_baseline"] = oracle_sample(w, passes, 16, 1024)
+        out[name] = entry
+        del inp, d, o, hT, outs
+        torch.cuda.empty_cache()
+
+    # decode: B=64, H=4, d_k=128, d_v=256, one token per call, fp32 state carried
+    B, H, K, V = (DECODE[n] for n in ("B", "H", "K", "V"))
+    T = 64
+    st = make_step_inputs(B, H, K, V, T, DECODE["dtype"], seed=0)
+    q, k, v, la = (st[n].to(dev) for n in ("q", "k", "v", "log_a"))
+    S = torch.zeros(B, H, K, V, device=dev)
+    ob = torch.empty(T, B, H, V, dtype=q.dtype, device=dev)
+    for t in range(T):
+        gla.gla_step(q[t], k[t], v[t], la[t], S, o=ob[t])
+    torch.cuda.synchronize(dev)
+    flushed = []
+    for t in range(T):
+        flush.fill_(1.0)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        gla.gla_step(q[t], k[t], v[t], la[t], S, o=ob[t])
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        flushed.append(a.elapsed_time(b))
+    ms_flushed = sorted(flushed)[T // 2]
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        gla.gla_step(q[0], k[0], v[0], la[0], S, o=ob[0])
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for t in range(T):
+            gla.gla_step(q[t], k[t], v[t], la[t], S, o=ob[t])
+    g.replay()
+    torch.cuda.synchronize(dev)
+    reps_g = DECODE["steps"] // T
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps_g):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms_res = a.elapsed_time(b) / (reps_g * T)
+    del g
+    state_bytes = 2 * B * H * K * V * 4
+    dec = {"B": B, "H": H, "d_k": K, "d_v": V, "steps": DECODE["steps"],
+           "l2_resident": {"us_per_step": round(ms_res * 1e3, 3), "tokens_per_s": round(B / ms_res * 1e3, 1),
+                           "state_GBps": round(state_bytes / ms_res / 1e6, 1),
+                           "how": "CUDA graph of 64 steps replayed %d times (%d steps); the 33.5 MB state stays in L2"
+                                  % (reps_g, reps_g * T)},
+           "l2_flushed": {"us_per_step": round(ms_flushed * 1e3, 3), "tokens_per_s": round(B / ms_flushed * 1e3, 1),
+                          "state_GBps": round(state_bytes / ms_flushed / 1e6, 1),
+                          "hbm_frac": round(state_bytes / ms_flushed / 1e6 / peaks["hbm_gbs"], 4),
+                          "how": "median of 64 single calls, each after a 512 MB write"}}
+    if with_cpu:
+        import oracle
+        from chunkwise_linear_rnn_gla_b200.inputs import to_f64_numpy
+
+        f = {n: to_f64_numpy(st[n][0]) for n in ("q", "k", "v", "log_a")}
+        S0 = np.zeros((B, H, K, V))
+        t0 = time.perf_counter()
+        nrep = 4
+        for _ in range(nrep):
+            oracle.step(f["q"], f["k"], f["v"], f["log_a"], S0)
+        dt = (time.perf_counter() - t0) / nrep
+        dec["cpu_baseline"] = {"value": B / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+                               "sample": "%d decode steps of the full batch, fp64, %.3f s per step" % (nrep, dt)}
+    out["decode_b64"] = dec
+    return out
+
+
 # --------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -252,6 +448,8 @@ def main():
     ap.add_argument("--kernel-impl", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--state-mode", default="materialized", choices=["auto", "materialized", "nonmaterialized"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the timing of the other named workloads and the decode workload")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-graph", action="store_true",
@@ -407,14 +605,17 @@ def main():
         pin = {k: v.pin_memory() for k, v in inp.items()}
         host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
         host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        host_hT = torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)
         h2d = sum(v.numel() * v.element_size() for v in pin.values())
-        d2h = sum(v.numel() * v.element_size() for v in host_out.values()) + host_o.numel() * host_o.element_size()
+        d2h = (sum(v.numel() * v.element_size() for v in host_out.values()) + host_o.numel() * host_o.element_size()
+               + host_hT.numel() * host_hT.element_size())
 
         def e2e_step():
             for k_, v_ in pin.items():
                 d[k_].copy_(v_, non_blocking=True)
             step()
             host_o.copy_(o, non_blocking=True)
+            host_hT.copy_(hT, non_blocking=True)
             for k_, v_ in outs.items():
                 host_out[k_].copy_(v_, non_blocking=True)
 
@@ -433,51 +634,56 @@ def main():
                "h2d_bytes_per_step": int(h2d),
                "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
 
-    # ---------------- roofline of the dominant kernel
+    # ---------------- roofline of the whole step (the headline) and of the dominant kernel
     peaks, peaks_src = load_peaks()
     models = kernel_models(w, C)
-    roof = None
+    mbytes = method_bytes(w)
+    kroof = None
     kernels = {}
     if prof:
-        top = max(prof.items(), key=lambda kv: kv[1][1])
+        tot = sum(x[1] for x in prof.values())
         for name, (n, ms) in prof.items():
-            kernels[name] = {"launches": n, "total_ms": round(ms, 4), "share": round(ms / sum(x[1] for x in prof.values()), 4)}
-        name, (n, ms) = top
+            kernels[name] = {"launches": n, "total_ms": round(ms, 4), "share": round(ms / tot, 4),
+                             "us_per_launch": round(ms / n * 1e3, 2)}
+            if name in mbytes:
+                kernels[name]["method_frac"] = round(mbytes[name] / (ms / n / 1e3) / 1e9 / peaks["hbm_gbs"], 4)
+        name, (n, ms) = max(prof.items(), key=lambda kv: kv[1][1])
         avg_s = ms / n / 1e3
         mdl = models.get(name)
-        if mdl is not None:
-            if mdl["bound"] == "hbm":
-                ach = mdl["bytes"] / avg_s / 1e9
-                roof = {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
-                        "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "traffic": None}
-            elif mdl["bound"] == "tensor":
-                ach = mdl["flops"] / avg_s / 1e12
-                pk = peaks["bf16_tflops_sustained"]
-                roof = {"kernel": name, "bound": "tensor", "achieved": round(ach, 2), "peak": pk, "unit": "TFLOP/s",
-                        "frac": round(ach / pk, 4), "traffic": None}
-            else:  # fp32 CUDA-core arithmetic: 148 SMs x 128 FMA/clk x 2 flop x max SM clock
-                pk = 148 * 128 * 2 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-                ach = mdl["flops"] / avg_s / 1e12
-                roof = {"kernel": name, "bound": "alu", "achieved": round(ach, 2), "peak": round(pk, 1),
-                        "unit": "TFLOP/s", "frac": round(ach / pk, 4), "traffic": None}
-            roof["peak_source"] = peaks_src
-            roof["timing"] = ("CUDA events around each kernel launch over K further timed steps "
-                              "(pass B, %.4f ms per step with the events; the headline step time is pass A, "
-                              "without them)" % (prof_total_ms / args.steps))
-            roof["launch_ms"] = round(ms / n, 4)
-            roof["traffic"] = measured_traffic(name)
-            roof["alg_bytes"] = mdl["bytes"]
+        if mdl is not None and name in mbytes:
+            ach = mbytes[name] / avg_s / 1e9
+            kroof = {"kernel": name, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": round(ach / peaks["hbm_gbs"], 4), "peak_source": peaks_src,
+                     "alg_bytes_method": mbytes[name], "alg_bytes_impl": mdl["bytes"],
+                     "frac_impl": round(mdl["bytes"] / avg_s / 1e9 / peaks["hbm_gbs"], 4),
+                     "launch_ms": round(ms / n, 4), "traffic": measured_traffic(name),
+                     "timing": ("CUDA events around each kernel launch over K further timed steps (pass B, "
+                                "%.4f ms per step with the events; the headline step time is pass A, without them)"
+                                % (prof_total_ms / args.steps)),
+                     "bytes_note": ("achieved = the layer's own inputs read and outputs written by this kernel "
+                                    "(alg_bytes_method) / its launch time; alg_bytes_impl adds the "
+                                    "implementation's chunk states and operand workspace")}
 
     alg = algorithmic_model(w, C)
-    t_roof = max(alg["bytes"] / (peaks["hbm_gbs"] * 1e9), alg["flops"] / (peaks["bf16_tflops"] * 1e12))
-    layer_roof = {"roofline_ms": round(t_roof * 1e3, 5), "frac": round(t_roof * 1e3 / ms_per_step, 4),
+    lr = layer_roofline(alg["bytes"], alg["flops"], ms_per_step, peaks)
+    step_traffic = None
+    if kernels and all(measured_traffic(k) is not None for k in kernels):
+        step_traffic = sum(measured_traffic(k) * kernels[k]["launches"] for k in kernels) // max(1, args.steps)
+    layer_roof = {"roofline_ms": lr["roofline_ms"], "frac": lr["frac"], "bound": lr["bound"],
+                  "achieved_GBps": round(alg["bytes"] / (ms_per_step / 1e3) / 1e9, 1), "peak_GBps": peaks["hbm_gbs"],
                   "alg_bytes": alg["bytes"], "alg_flops": alg["flops"],
                   "tflops": round(alg["flops"] / (ms_per_step / 1e3) / 1e12, 2),
                   # the same flops against the sustained (power-capped) bf16 GEMM rate
                   "tflops_frac_of_sustained_bf16": round(alg["flops"] / (ms_per_step / 1e3) / 1e12
                                                          / peaks["bf16_tflops_sustained"], 4),
-                  "bound": "hbm" if alg["bytes"] / peaks["hbm_gbs"] / 1e9 > alg["flops"] / peaks["bf16_tflops"] / 1e12
-                  else "tensor"}
+                  "traffic_per_step": step_traffic,
+                  "definition": "the whole fwd+bwd step against max(algorithmic bytes / measured HBM copy "
+                                "bandwidth, algorithmic flops / measured bf16 dense peak); traffic_per_step = "
+                                "summed ncu DRAM bytes of the step's launches (null when any kernel changed since)"}
+
+    workloads = None
+    if rank == 0 and world == 1 and not args.no_workloads:
+        workloads = run_workloads(dev, peaks, flush, with_cpu=not args.no_cpu_baseline)
 
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -489,12 +695,13 @@ def main():
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
                 "data": "synthetic (seeded N(0,1)/sqrt(d_k) q,k,v; log_a = logsigmoid(N(0,1))/16; dO ~ N(0,1))",
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V,
-                           "global_batch": dp.global_batch(w.B, world), "seq_len": w.L, "chunk": C, "subchunk": sc,
+                           "global_batch": dp.global_batch(w.B, world), "seq_len": w.L, "chunk": C,
+                           "subchunk": sc if impl_name == "simt" else None,
                            "kernel_impl": impl_name, "state_mode": mode, "parallelism": "dp%d" % world,
                            "l2": "flushed between timed steps (512 MB write)", "step_launch": graph_note,
                            "eager_ms_per_step": round(eager_ms / args.steps, 5)},
-                "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cb, "e2e": e2e,
-                "gpu_launches": int(launches), "clocks": clk, "kernels": kernels}
+                "roofline": kroof, "layer_roofline": layer_roof, "cpu_baseline": cb,
+                "e2e": e2e, "gpu_launches": int(launches), "clocks": clk, "kernels": kernels, "workloads": workloads}
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.barrier()

@@ -42,20 +42,39 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
+def _compile(cmd):
+    return subprocess.run(cmd, capture_output=True, text=True)
+
+
 def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    """Compile every .cu under csrc/ into libgla.so (no-op when up to date)."""
+    """Compile every .cu under csrc/ into libgla.so (no-op when up to date). Each translation unit is
+    compiled on its own, in parallel, into an object file under _build/ (no device code crosses
+    translation units), then the objects are linked into the shared library."""
     if not force and up_to_date():
         return LIB
+    from concurrent.futures import ThreadPoolExecutor
+
+    objdir = os.path.join(ROOT, "_build", "libgla")
+    os.makedirs(objdir, exist_ok=True)
+    flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
+             "-I", os.path.join(ROOT, "include"), *(["-Xptxas", "-v"] if verbose else []), *(extra or [])]
+    objs, cmds = [], []
+    for src in sources():
+        obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
+        objs.append(obj)
+        cmds.append([nvcc(), *flags, "-c", src, "-o", obj])
+    with ThreadPoolExecutor(max_workers=min(len(cmds), os.cpu_count() or 4)) as ex:
+        results = list(ex.map(_compile, cmds))
+    for r in results:
+        if r.returncode != 0 or verbose:
+            sys.stderr.write(r.stdout + r.stderr)
+    if any(r.returncode != 0 for r in results):
+        raise RuntimeError("nvcc failed building libgla.so")
     tmp = LIB + ".tmp.%d" % os.getpid()
-    cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr",
-           "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
-           *(["-Xptxas", "-v"] if verbose else []), *(extra or []), *sources(), "-o", tmp]
-    r = subprocess.run(cmd, capture_output=True, text=True)
+    r = subprocess.run([nvcc(), *ARCH, "-shared", *objs, "-o", tmp], capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed building libgla.so")
-    if verbose:
-        sys.stderr.write(r.stdout + r.stderr)
+        raise RuntimeError("nvcc failed linking libgla.so")
     os.replace(tmp, LIB)
     return LIB
 

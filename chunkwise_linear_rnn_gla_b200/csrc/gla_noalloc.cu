@@ -23,10 +23,15 @@
 //    array and must be serialised by the caller.
 //  * The device address of the array is looked up (cudaGetSymbolAddress) the
 //    first time the entry point runs on each device, with that device
-//    current. That lookup is host-side set-up and allocates nothing; make
-//    this first call on each device before any stream capture begins.
+//    current, and looked up again if the device's context has changed since
+//    (a device reset replaces the context and moves the array). That lookup
+//    is host-side set-up and allocates nothing; make the first call on each
+//    device, and the first call after a reset, before any stream capture
+//    begins.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 #include <mutex>
 
@@ -38,10 +43,41 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[GLA_NOALLOC_SCR
 
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
+// Per device: the context the address was looked up in (its process-unique id) and the address.
+struct ScratchEntry {
+    unsigned long long ctx_id;
+    void* ptr;
+};
+ScratchEntry g_scratch[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (set-up on first
-// use per device); nullptr if the lookup failed.
+// The current context's process-unique id (cuCtxGetId), or 0 when none is current or the query is
+// unavailable. A device reset destroys the primary context; the next context gets a new id, so an
+// address looked up in the old one is never reused.
+unsigned long long current_context_id() {
+    static std::once_flag once;
+    static PFN_cuCtxGetCurrent_v4000 get_current = nullptr;
+    static PFN_cuCtxGetId_v12000 get_id = nullptr;
+    std::call_once(once, [] {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+        fn = nullptr;
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(fn);
+    });
+    if (!get_current || !get_id) return 0;
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
+
+// Device address of the scratch array in the current device's current context. Set-up (the symbol
+// lookup) runs on the first call per device and again whenever the context has changed since (after
+// a device reset); nullptr if the lookup failed.
 void* scratch_on_current_device(gla_status* st) {
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
@@ -49,17 +85,21 @@ void* scratch_on_current_device(gla_status* st) {
         return nullptr;
     }
     std::lock_guard<std::mutex> lk(g_setup_mu);
-    if (!g_scratch_ptr[dev]) {
+    const unsigned long long id = current_context_id();
+    ScratchEntry& e = g_scratch[dev];
+    if (!e.ptr || id == 0 || id != e.ctx_id) {
         void* ptr = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
-        if (e != cudaSuccess || !ptr) {
+        const cudaError_t err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (err != cudaSuccess || !ptr) {
             *st = GLA_ERR_CUDA;
             return nullptr;
         }
-        g_scratch_ptr[dev] = ptr;
+        // the lookup makes the device's primary context current if none was: take its id now
+        e.ctx_id = id != 0 ? id : current_context_id();
+        e.ptr = ptr;
     }
     *st = GLA_OK;
-    return g_scratch_ptr[dev];
+    return e.ptr;
 }
 
 }  // namespace

@@ -1,8 +1,8 @@
 // Single-token recurrent decode step:
 //   S <- diag(exp(log_a)) S + k^T v   (fp32, in place),   o = q S.
 // The recurrent form of the layer (podcast.app episode page "Gated Linear
-// Attention for Efficient Long Sequences": a gated, recurrent-style memory
-// update; the gate is G = alpha^T 1, "Gated Linear Attention Transformers with
+// Attention for Efficient Long Sequences", summary: a gated memory updated
+// once per token; the gate is G = alpha^T 1, "Gated Linear Attention Transformers with
 // Hardware-Efficient Training", atlas.scime.ai summary, "Approach").
 //
 // The step is a pure stream over the fp32 state (read + write 8*Dk*Dv bytes

@@ -63,8 +63,8 @@ typedef enum gla_dtype {
     GLA_DTYPE_BF16 = 1
 } gla_dtype;
 
-/* How the inter-chunk states are handled ("Approach" section: "materialized
- * or non-materialized inter-chunk states"). */
+/* How the inter-chunk states are handled (the "Approach" section offers both:
+ * the per-chunk states may be stored in memory or kept on chip). */
 typedef enum gla_state_mode {
     GLA_STATE_AUTO = 0,            /* library picks: materialised              */
     GLA_STATE_MATERIALIZED = 1,    /* write S_[i] of every chunk to workspace  */
@@ -118,8 +118,8 @@ gla_status gla_fwd(const gla_desc* d, const void* q, const void* k, const void* 
  * (dtype), dlog_a [B,H,L,Dk] (fp32), dh0 [B,H,Dk,Dv] (fp32, may be NULL).
  * h0 and dhT may be NULL (zero). The gate gradient is the closed form
  *   dlog_a_t = sum_{s>=t} (q_s*dq_s - k_s*dk_s) + sum_v dhT[:,v]*hT[:,v]
- * ("Approach": "a closed-form gradient for the gates that avoids
- * materializing per-step states"). dq, dk, dv are the full gradients. */
+ * (the "Approach" section's closed-form gate gradient, which needs no
+ * per-step state). dq, dk, dv are the full gradients. */
 gla_status gla_bwd(const gla_desc* d, const void* q, const void* k, const void* v,
                    const float* log_a, const float* h0, const void* dO, const float* dhT,
                    void* dq, void* dk, void* dv, float* dlog_a, float* dh0,
@@ -128,8 +128,8 @@ gla_status gla_bwd(const gla_desc* d, const void* q, const void* k, const void* 
 /* One recurrent decode step for B*H independent states (d->L is ignored):
  * S <- diag(exp(log_a)) S + k^T v (in place), then o = q S.
  * q, k, log_a: [B,H,Dk]; v, o: [B,H,Dv]; S: [B,H,Dk,Dv] fp32. The recurrent
- * form of the layer (podcast.app episode page, summary: "a gated,
- * recurrent-style memory update"). */
+ * form of the layer (podcast.app episode page, summary: the layer read as a
+ * gated memory updated once per token). */
 gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void* v,
                     const float* log_a, float* S, void* o, void* stream);
 
@@ -165,8 +165,9 @@ gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, 
  *    contents; nothing in it needs clearing, but calls that overlap on the
  *    GPU (other streams or host threads) race and must be serialised.
  *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current): make that first call
- *    before any stream capture begins. */
+ *    (cudaGetSymbolAddress, with that device current), and so does the first
+ *    call after the device's context was replaced (cudaDeviceReset): make
+ *    those calls before any stream capture begins. */
 #define GLA_NOALLOC_SCRATCH_BYTES (16u << 20)
 gla_status gla_fwd_noalloc(const gla_desc* d, const void* q, const void* k, const void* v,
                            const float* log_a, const float* h0, void* o, float* hT, void* stream);

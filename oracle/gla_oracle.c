@@ -18,9 +18,10 @@
  * Training" (atlas.scime.ai summary of arXiv 2312.06635), section
  * "Approach": the gate is G_t = alpha_t^T 1, i.e. a matrix whose rows are
  * constant along the value dimension, so G_t (.) S = diag(alpha_t) S: a decay
- * of each key channel. The recurrent (one-step) reading of the same layer is
- * the "recurrent-style memory update" of the podcast.app episode page
- * ("Gated Linear Attention for Efficient Long Sequences", summary paragraph).
+ * of each key channel. The recurrent (one-step) reading of the same layer, a
+ * gated memory updated once per token, is the summary paragraph of the
+ * podcast.app episode page ("Gated Linear Attention for Efficient Long
+ * Sequences").
  * Output-after-update (o_t uses S_t, not S_{t-1}) is the plain reading of
  * o_t = q_t S_t; there is no 1/sqrt(d) scale and no normaliser inside the
  * layer (the pages give none).
