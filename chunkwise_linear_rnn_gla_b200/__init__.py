@@ -21,7 +21,7 @@ import torch
 from . import _lib
 from ._lib import GlaDesc, GlaError, load  # noqa: F401
 
-__all__ = ["gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum", "gla_fwd_workspace_size",
+__all__ = ["gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum", "gla_fwd_workspace_size", "gla_last_device_error",
            "gla_bwd_workspace_size", "gla_resolve", "gla_check_device_error", "gla_launch_count",
            "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset",
            "make_desc", "GlaError"]
@@ -95,6 +95,30 @@ def _workspace(nbytes: int, dev, workspace: Optional[torch.Tensor]):
     return workspace, workspace.numel() * workspace.element_size()
 
 
+# ---- checking mode: the library's device-side checks plus host-side canaries around the outputs.
+# Every output the binding allocates is carved from a larger buffer whose margins hold NaN; after the
+# call (which is then synchronous) the margins must still be NaN and the device error flag clear.
+_CANARY = 256  # elements on each side (>= 256 bytes, keeps 16-byte alignment)
+
+
+def _guarded(shape, dtype, dev, guards):
+    n = 1
+    for x in shape:
+        n *= int(x)
+    buf = torch.full((n + 2 * _CANARY,), float("nan"), dtype=dtype, device=dev)
+    guards.append((buf, n))
+    return buf[_CANARY:_CANARY + n].view(*shape)
+
+
+def _finish_checks(guards, what):
+    st = gla_check_device_error()
+    if st != _lib.GLA_OK:
+        raise GlaError(st, what + " (checking mode)")
+    for buf, n in guards:
+        if not (bool(torch.isnan(buf[:_CANARY]).all()) and bool(torch.isnan(buf[_CANARY + n:]).all())):
+            raise GlaError(_lib.GLA_ERR_WORKSPACE, what + " (checking mode: an output canary was overwritten)")
+
+
 def _desc_from(q, v, chunk, subchunk, state_mode, impl, flags=0):
     B, H, L, Dk = q.shape
     Dv = v.shape[-1]
@@ -102,9 +126,12 @@ def _desc_from(q, v, chunk, subchunk, state_mode, impl, flags=0):
 
 
 def gla_fwd(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto", o=None, hT=None,
-            want_hT=True, workspace=None):
+            want_hT=True, workspace=None, checks=False):
     """Forward. Returns (o, hT); hT is None when want_hT is False and no hT
-    buffer is given. `workspace` (uint8 tensor) may be passed to reuse it."""
+    buffer is given. `workspace` (uint8 tensor) may be passed to reuse it.
+    checks=True runs the library's checking mode (gate domain, finite
+    outputs, workspace guards) with canaries around the outputs allocated
+    here; the call then synchronises and raises GlaError on any failure."""
     load()
     dev = q.device
     B, H, L, Dk = q.shape
@@ -115,12 +142,15 @@ def gla_fwd(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", 
     _need(log_a, "log_a", q.shape, torch.float32, dev)
     if h0 is not None:
         _need(h0, "h0", (B, H, Dk, Dv), torch.float32, dev)
-    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl)
+    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, _lib.FLAG_CHECKS if checks else 0)
+    guards = []
+    alloc = (lambda shp, t: _guarded(shp, t, dev, guards)) if checks else \
+        (lambda shp, t: torch.empty(*shp, dtype=t, device=dev))
     if o is None:
-        o = torch.empty(B, H, L, Dv, dtype=dt, device=dev)
+        o = alloc((B, H, L, Dv), dt)
     _need(o, "o", (B, H, L, Dv), dt, dev)
     if hT is None and want_hT:
-        hT = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+        hT = alloc((B, H, Dk, Dv), torch.float32)
     if hT is not None:
         _need(hT, "hT", (B, H, Dk, Dv), torch.float32, dev)
     ws, nbytes = _workspace(gla_fwd_workspace_size(desc), dev, workspace)
@@ -128,14 +158,17 @@ def gla_fwd(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", 
         st = load().gla_fwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(h0), _ptr(o),
                             _ptr(hT), _ptr(ws), nbytes, _stream(dev))
     _check(st, "gla_fwd")
+    if checks:
+        _finish_checks(guards, "gla_fwd")
     return o, hT
 
 
 def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto",
-            want_dh0=True, workspace=None, ws_from_fwd=False, out=None):
+            want_dh0=True, workspace=None, ws_from_fwd=False, out=None, checks=False):
     """Backward of <dO, o> + <dhT, hT>. Returns a dict with dq, dk, dv,
     dlog_a and dh0. With ws_from_fwd=True the workspace must be the one the
-    matching gla_fwd call used (same inputs, same options)."""
+    matching gla_fwd call used (same inputs, same options, checks included).
+    checks=True: as for gla_fwd."""
     load()
     dev = q.device
     B, H, L, Dk = q.shape
@@ -149,37 +182,44 @@ def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state
         _need(h0, "h0", (B, H, Dk, Dv), torch.float32, dev)
     if dhT is not None:
         _need(dhT, "dhT", (B, H, Dk, Dv), torch.float32, dev)
-    flags = _lib.FLAG_WS_FROM_FWD if ws_from_fwd else 0
+    flags = (_lib.FLAG_WS_FROM_FWD if ws_from_fwd else 0) | (_lib.FLAG_CHECKS if checks else 0)
     desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, flags)
     if ws_from_fwd and workspace is None:
         raise ValueError("ws_from_fwd needs the forward's workspace")
+    guards = []
+    alloc = (lambda shp, t: _guarded(shp, t, dev, guards)) if checks else \
+        (lambda shp, t: torch.empty(*shp, dtype=t, device=dev))
     out = dict(out or {})
     dq = out.get("dq")
     if dq is None:
-        dq = torch.empty_like(q)
+        dq = alloc(q.shape, dt)
     dk = out.get("dk")
     if dk is None:
-        dk = torch.empty_like(k)
+        dk = alloc(k.shape, dt)
     dv = out.get("dv")
     if dv is None:
-        dv = torch.empty_like(v)
+        dv = alloc(v.shape, dt)
     dla = out.get("dlog_a")
     if dla is None:
-        dla = torch.empty_like(log_a)
+        dla = alloc(log_a.shape, torch.float32)
     dh0 = out.get("dh0")
     if dh0 is None and want_dh0:
-        dh0 = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+        dh0 = alloc((B, H, Dk, Dv), torch.float32)
     ws, nbytes = _workspace(gla_bwd_workspace_size(desc), dev, workspace)
     with torch.cuda.device(dev):
         st = load().gla_bwd(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(h0), _ptr(dO),
                             _ptr(dhT), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dla), _ptr(dh0), _ptr(ws), nbytes,
                             _stream(dev))
     _check(st, "gla_bwd")
+    if checks:
+        _finish_checks(guards, "gla_bwd")
     return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dh0": dh0}
 
 
-def gla_step(q, k, v, log_a, S, o=None):
-    """One decode step; S [B,H,Dk,Dv] fp32 is updated in place. Returns o [B,H,Dv]."""
+def gla_step(q, k, v, log_a, S, o=None, checks=False):
+    """One decode step; S [B,H,Dk,Dv] fp32 is updated in place. Returns o [B,H,Dv].
+    checks=True: the library's checking mode (gate domain, finite o and S), synchronous, raises on a
+    failure."""
     load()
     dev = q.device
     B, H, Dk = q.shape
@@ -189,14 +229,17 @@ def gla_step(q, k, v, log_a, S, o=None):
     _need(v, "v", (B, H, Dv), dt, dev)
     _need(log_a, "log_a", q.shape, torch.float32, dev)
     _need(S, "S", (B, H, Dk, Dv), torch.float32, dev)
+    guards = []
     if o is None:
-        o = torch.empty(B, H, Dv, dtype=dt, device=dev)
+        o = _guarded((B, H, Dv), dt, dev, guards) if checks else torch.empty(B, H, Dv, dtype=dt, device=dev)
     _need(o, "o", (B, H, Dv), dt, dev)
-    desc = make_desc(B, H, 1, Dk, Dv, _dt(q))
+    desc = make_desc(B, H, 1, Dk, Dv, _dt(q), flags=_lib.FLAG_CHECKS if checks else 0)
     with torch.cuda.device(dev):
         st = load().gla_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(S), _ptr(o),
                              _stream(dev))
     _check(st, "gla_step")
+    if checks:
+        _finish_checks(guards, "gla_step")
     return o
 
 
@@ -218,6 +261,12 @@ def gla_chunk_cumsum(log_a, chunk=64, out=None):
 def gla_check_device_error(stream=None) -> int:
     s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
     return int(load().gla_check_device_error(s))
+
+
+def gla_last_device_error(stream=None) -> int:
+    """The same report as gla_check_device_error (the name the layer's scope table uses)."""
+    s = ctypes.c_void_p(stream if stream is not None else torch.cuda.current_stream().cuda_stream)
+    return int(load().gla_last_device_error(s))
 
 
 def gla_selftest_wait_timeout(limit_cycles=0, stream=None) -> None:

@@ -9,22 +9,27 @@ import os
 import threading
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libgla.so")
+# GLA_CHECKS=1 in the environment selects the checking build (every call runs the library's checks).
+LIB_PATH = os.path.join(HERE, "libgla_checks.so" if os.environ.get("GLA_CHECKS") == "1" else "libgla.so")
 
 GLA_OK = 0
+GLA_ERR_INVALID_ARG = 1
+GLA_ERR_WORKSPACE = 3
+GLA_ERR_TIMEOUT = 5
 STATUS_NAMES = {0: "GLA_OK", 1: "GLA_ERR_INVALID_ARG", 2: "GLA_ERR_UNSUPPORTED", 3: "GLA_ERR_WORKSPACE",
                 4: "GLA_ERR_CUDA", 5: "GLA_ERR_TIMEOUT"}
 DTYPE = {"f32": 0, "bf16": 1}
 STATE_MODE = {"auto": 0, "materialized": 1, "nonmaterialized": 2}
 IMPL = {"auto": 0, "simt": 1, "tc": 2}
 FLAG_WS_FROM_FWD = 0x1
+FLAG_CHECKS = 0x2
 
 # Every function the header declares, for the ABI-completeness test.
 EXPORTS = (
     "gla_fwd_workspace_size", "gla_bwd_workspace_size", "gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum",
     "gla_check_device_error", "gla_status_string", "gla_abi_version", "gla_resolve", "gla_launch_count",
     "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset", "gla_fwd_noalloc",
-    "gla_selftest_wait_timeout",
+    "gla_selftest_wait_timeout", "gla_last_device_error", "gla_fwd_workspace_bytes", "gla_bwd_workspace_bytes",
 )
 
 
@@ -62,6 +67,12 @@ def _declare(lib):
     lib.gla_chunk_cumsum.restype = ctypes.c_int
     lib.gla_check_device_error.argtypes = [vp]
     lib.gla_check_device_error.restype = ctypes.c_int
+    lib.gla_last_device_error.argtypes = [vp]
+    lib.gla_last_device_error.restype = ctypes.c_int
+    lib.gla_fwd_workspace_bytes.argtypes = [dp]
+    lib.gla_fwd_workspace_bytes.restype = sz
+    lib.gla_bwd_workspace_bytes.argtypes = [dp]
+    lib.gla_bwd_workspace_bytes.restype = sz
     lib.gla_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
     lib.gla_selftest_wait_timeout.restype = ctypes.c_int
     lib.gla_status_string.argtypes = [ctypes.c_int]

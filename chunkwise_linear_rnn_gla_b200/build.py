@@ -1,6 +1,9 @@
 """Build libgla.so in-tree with nvcc for sm_100a.
 
-    python -m chunkwise_linear_rnn_gla_b200.build [--force] [--verbose]
+    python -m chunkwise_linear_rnn_gla_b200.build [--force] [--verbose] [--checks]
+
+--checks builds the checking library libgla_checks.so instead (-DGLA_CHECKS: every call runs the
+checks of GLA_FLAG_CHECKS); the binding loads it when the environment sets GLA_CHECKS=1.
 
 The library is a plain shared object (C ABI, no torch or Python types in its
 signatures); the binding in this package loads it with ctypes.
@@ -16,6 +19,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libgla.so")
+LIB_CHECKS = os.path.join(HERE, "libgla_checks.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -35,10 +39,10 @@ def _deps():
         os.path.join(ROOT, "include", "gla.h")]
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in _deps())
 
 
@@ -46,18 +50,21 @@ def _compile(cmd):
     return subprocess.run(cmd, capture_output=True, text=True)
 
 
-def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    """Compile every .cu under csrc/ into libgla.so (no-op when up to date). Each translation unit is
-    compiled on its own, in parallel, into an object file under _build/ (no device code crosses
-    translation units), then the objects are linked into the shared library."""
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra=None, checks: bool = False) -> str:
+    """Compile every .cu under csrc/ into libgla.so (libgla_checks.so with checks=True; no-op when up
+    to date). Each translation unit is compiled on its own, in parallel, into an object file under
+    _build/ (no device code crosses translation units), then the objects are linked into the shared
+    library."""
+    lib = LIB_CHECKS if checks else LIB
+    if not force and up_to_date(lib):
+        return lib
     from concurrent.futures import ThreadPoolExecutor
 
-    objdir = os.path.join(ROOT, "_build", "libgla")
+    objdir = os.path.join(ROOT, "_build", "libgla_checks" if checks else "libgla")
     os.makedirs(objdir, exist_ok=True)
     flags = [*ARCH, "-O3", "-lineinfo", "-std=c++17", "--expt-relaxed-constexpr", "-Xcompiler", "-fPIC",
-             "-I", os.path.join(ROOT, "include"), *(["-Xptxas", "-v"] if verbose else []), *(extra or [])]
+             "-I", os.path.join(ROOT, "include"), *(["-Xptxas", "-v"] if verbose else []), *(extra or []),
+             *(["-DGLA_CHECKS"] if checks else [])]
     objs, cmds = [], []
     for src in sources():
         obj = os.path.join(objdir, os.path.basename(src)[:-3] + ".o")
@@ -70,15 +77,14 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
             sys.stderr.write(r.stdout + r.stderr)
     if any(r.returncode != 0 for r in results):
         raise RuntimeError("nvcc failed building libgla.so")
-    tmp = LIB + ".tmp.%d" % os.getpid()
+    tmp = lib + ".tmp.%d" % os.getpid()
     r = subprocess.run([nvcc(), *ARCH, "-shared", *objs, "-o", tmp], capture_output=True, text=True)
     if r.returncode != 0:
         sys.stderr.write(r.stdout + r.stderr)
-        raise RuntimeError("nvcc failed linking libgla.so")
-    os.replace(tmp, LIB)
-    return LIB
+        raise RuntimeError("nvcc failed linking " + os.path.basename(lib))
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="--verbose" in sys.argv)
-    print(LIB)
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, checks="--checks" in sys.argv))

@@ -122,7 +122,7 @@ gla_status resolve(const gla_desc* d, Problem& p) {
     if (d->subchunk < 0) return GLA_ERR_INVALID_ARG;
     if (d->state_mode < GLA_STATE_AUTO || d->state_mode > GLA_STATE_NONMATERIALIZED) return GLA_ERR_INVALID_ARG;
     if (d->impl < GLA_IMPL_AUTO || d->impl > GLA_IMPL_TC) return GLA_ERR_INVALID_ARG;
-    if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD)) return GLA_ERR_INVALID_ARG;
+    if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
     p.B = d->B;
     p.H = d->H;
     p.L = d->L;
@@ -238,10 +238,23 @@ gla_status gla_fwd(const gla_desc* d, const void* q, const void* k, const void* 
     const size_t need = fwd_ws(p);
     st = check_ws(workspace, workspace_bytes, need);
     if (st != GLA_OK) return st;
-    gla::Arena a{static_cast<char*>(workspace), workspace_bytes, 0};
+    gla::Arena a = gla::make_arena(p, workspace, workspace_bytes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p.impl == GLA_IMPL_TC) return gla::tc_fwd(p, q, k, v, log_a, h0, o, hT, a, s);
-    return gla::simt_fwd(p, q, k, v, log_a, h0, o, hT, a, s);
+    const bool chk = gla::checks_on(p);
+    gla::Arena layout = gla::make_arena(p, workspace, workspace_bytes);
+    if (chk) {
+        (p.impl == GLA_IMPL_TC ? gla::tc_layout : gla::simt_layout)(p, layout, false);
+        st = gla::check_gates(log_a, p.BH * p.L * p.K, s);
+        if (st == GLA_OK) st = gla::guards_fill(layout, s);
+        if (st != GLA_OK) return st;
+    }
+    st = p.impl == GLA_IMPL_TC ? gla::tc_fwd(p, q, k, v, log_a, h0, o, hT, a, s)
+                               : gla::simt_fwd(p, q, k, v, log_a, h0, o, hT, a, s);
+    if (st != GLA_OK || !chk) return st;
+    st = gla::check_finite(o, p.BH * p.L * p.V, p.bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(hT, p.BH * p.K * p.V, false, s);
+    if (st == GLA_OK) st = gla::guards_check(layout, s);
+    return st;
 }
 
 gla_status gla_bwd(const gla_desc* d, const void* q, const void* k, const void* v, const float* log_a,
@@ -265,10 +278,27 @@ gla_status gla_bwd(const gla_desc* d, const void* q, const void* k, const void* 
     const size_t need = bwd_ws(p);
     st = check_ws(workspace, workspace_bytes, need);
     if (st != GLA_OK) return st;
-    gla::Arena a{static_cast<char*>(workspace), workspace_bytes, 0};
+    gla::Arena a = gla::make_arena(p, workspace, workspace_bytes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (p.impl == GLA_IMPL_TC) return gla::tc_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s);
-    return gla::simt_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s);
+    const bool chk = gla::checks_on(p);
+    gla::Arena layout = gla::make_arena(p, workspace, workspace_bytes);
+    if (chk) {
+        (p.impl == GLA_IMPL_TC ? gla::tc_layout : gla::simt_layout)(p, layout, true);
+        st = gla::check_gates(log_a, p.BH * p.L * p.K, s);
+        if (st == GLA_OK) st = gla::guards_fill(layout, s);
+        if (st != GLA_OK) return st;
+    }
+    st = p.impl == GLA_IMPL_TC ? gla::tc_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s)
+                               : gla::simt_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s);
+    if (st != GLA_OK || !chk) return st;
+    const int64_t nk = p.BH * p.L * p.K, nv = p.BH * p.L * p.V;
+    st = gla::check_finite(dq, nk, p.bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(dk, nk, p.bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(dv, nv, p.bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(dlog_a, nk, false, s);
+    if (st == GLA_OK) st = gla::check_finite(dh0, p.BH * p.K * p.V, false, s);
+    if (st == GLA_OK) st = gla::guards_check(layout, s);
+    return st;
 }
 
 gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void* v, const float* log_a, float* S,
@@ -283,6 +313,7 @@ gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void*
     GLA_REQUIRE_PTR(S);
     GLA_REQUIRE_PTR(o);
     if (d->B * d->H > 65535 || d->Dk > 8192) return GLA_ERR_UNSUPPORTED;
+    if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
     Problem p{};
     p.B = d->B;
     p.H = d->H;
@@ -291,7 +322,15 @@ gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void*
     p.V = d->Dv;
     p.BH = d->B * d->H;
     p.bf16 = d->dtype == GLA_DTYPE_BF16;
-    return gla::step_launch(p, q, k, v, log_a, S, o, static_cast<cudaStream_t>(stream));
+    p.flags = d->flags;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool chk = gla::checks_on(p);
+    gla_status st = chk ? gla::check_gates(log_a, p.BH * p.K, s) : GLA_OK;
+    if (st == GLA_OK) st = gla::step_launch(p, q, k, v, log_a, S, o, s);
+    if (st != GLA_OK || !chk) return st;
+    st = gla::check_finite(o, p.BH * p.V, p.bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(S, p.BH * p.K * p.V, false, s);
+    return st;
 }
 
 gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, void* stream) {
@@ -346,10 +385,18 @@ gla_status gla_check_device_error(void* stream) {
     if (h != 0) {
         const int zero = 0;
         if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return GLA_ERR_CUDA;
-        return GLA_ERR_TIMEOUT;
+        if (h & gla::tc::kErrWaitTimeout) return GLA_ERR_TIMEOUT;
+        if (h & (gla::kErrBadGate | gla::kErrNonFinite)) return GLA_ERR_INVALID_ARG;
+        if (h & gla::kErrGuard) return GLA_ERR_WORKSPACE;
+        return GLA_ERR_CUDA;
     }
     return GLA_OK;
 }
+
+gla_status gla_last_device_error(void* stream) { return gla_check_device_error(stream); }
+
+size_t gla_fwd_workspace_bytes(const gla_desc* d) { return gla_fwd_workspace_size(d); }
+size_t gla_bwd_workspace_bytes(const gla_desc* d) { return gla_bwd_workspace_size(d); }
 
 uint64_t gla_launch_count(void) { return gla::g_launches.load(); }
 void gla_launch_count_reset(void) { gla::g_launches.store(0); }

@@ -24,18 +24,36 @@ struct Problem {
 };
 
 // Bump allocator over the caller's workspace; every slice is 256-B aligned.
+// With guards on (GLA_FLAG_CHECKS), every slice is followed by a 256-byte guard
+// block that the checking build fills with a pattern before the kernels run
+// and verifies after them, so a kernel writing past the end of its slice is
+// reported (gla_check_device_error -> GLA_ERR_WORKSPACE).
+constexpr int kMaxGuards = 32;
+constexpr size_t kGuardBytes = 256;
 struct Arena {
     char* base;
     size_t cap;
     size_t used;
+    bool guard = false;
+    int nguard = 0;
+    char* guards[kMaxGuards] = {};
     template <typename T>
     T* take(size_t count) {
         size_t off = (used + 255) & ~size_t(255);
         size_t bytes = count * sizeof(T);
         used = off + bytes;
+        if (guard && nguard < kMaxGuards) {
+            const size_t g = (used + 255) & ~size_t(255);
+            if (base) guards[nguard] = base + g;
+            ++nguard;
+            used = g + kGuardBytes;
+        }
         return base ? reinterpret_cast<T*>(base + off) : nullptr;
     }
 };
+
+// Arena over a workspace (base may be null for size queries); guards follow the problem's flags.
+Arena make_arena(const Problem& p, void* base, size_t cap);
 
 // ---- launch bookkeeping (gla_api.cu) ------------------------------------
 // Every kernel launch goes through launch_begin/launch_end so that the
@@ -43,12 +61,26 @@ struct Arena {
 void launch_begin(const char* name, cudaStream_t s);
 gla_status launch_end(const char* name, cudaStream_t s);
 
-// Device-side error word (set by kernels whose bounded waits run out).
+// Device-side error word (set by kernels whose bounded waits run out, and by
+// the checking build's checks). Bits: tc::kErrWaitTimeout, kErrBadGate,
+// kErrNonFinite, kErrGuard.
 int* device_error_word();
+enum : int { kErrBadGate = 2, kErrNonFinite = 4, kErrGuard = 8 };
+
+// ---- checking build (gla_checks.cu) ------------------------------------------
+// Before a pass: every gate must be finite and <= 0 (kErrBadGate); the workspace
+// guards are filled. After it: every output element must be finite
+// (kErrNonFinite) and every guard intact (kErrGuard).
+gla_status check_gates(const float* log_a, int64_t n, cudaStream_t s);
+gla_status check_finite(const void* p, int64_t n, bool bf16, cudaStream_t s);
+gla_status guards_fill(const Arena& a, cudaStream_t s);
+gla_status guards_check(const Arena& a, cudaStream_t s);
+bool checks_on(const Problem& p);
 
 // ---- SIMT path (gla_simt.cu) ---------------------------------------------
 size_t simt_fwd_workspace(const Problem& p);
 size_t simt_bwd_workspace(const Problem& p);
+void simt_layout(const Problem& p, Arena& a, bool bwd);  // carve `a` as the pass would (guard positions)
 gla_status simt_chunk_cumsum(const Problem& p, const float* log_a, float* Bc, cudaStream_t s);
 gla_status simt_fwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
                     const float* h0, void* o, float* hT, Arena& ws, cudaStream_t s);
@@ -64,6 +96,7 @@ gla_status step_launch(const Problem& p, const void* q, const void* k, const voi
 bool tc_supported(const Problem& p);
 size_t tc_fwd_workspace(const Problem& p);
 size_t tc_bwd_workspace(const Problem& p);
+void tc_layout(const Problem& p, Arena& a, bool bwd);
 gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
                   const float* h0, void* o, float* hT, Arena& ws, cudaStream_t s);
 gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,

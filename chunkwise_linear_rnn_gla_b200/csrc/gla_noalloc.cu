@@ -112,7 +112,7 @@ extern "C" gla_status gla_fwd_noalloc(const gla_desc* d, const void* q, const vo
     // entry point runs), then the ordinary argument checks.
     gla_desc dd = *d;
     dd.impl = GLA_IMPL_SIMT;
-    dd.flags = 0;
+    dd.flags = d->flags & GLA_FLAG_CHECKS;  // a forward has nothing to reuse
     const size_t need = gla_fwd_workspace_size(&dd);
     if (need == 0) {
         int32_t c = 0;

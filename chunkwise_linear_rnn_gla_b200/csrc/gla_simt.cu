@@ -695,16 +695,18 @@ gla_status bwd_dispatch(const Problem& p, const void* q, const void* k, const vo
 }  // namespace
 
 size_t simt_fwd_workspace(const Problem& p) {
-    Arena a{nullptr, 0, 0};
+    Arena a = make_arena(p, nullptr, 0);
     carve(p, a, false);
     return a.used;
 }
 
 size_t simt_bwd_workspace(const Problem& p) {
-    Arena a{nullptr, 0, 0};
+    Arena a = make_arena(p, nullptr, 0);
     carve(p, a, true);
     return a.used;
 }
+
+void simt_layout(const Problem& p, Arena& a, bool bwd) { carve(p, a, bwd); }
 
 gla_status simt_chunk_cumsum(const Problem& p, const float* log_a, float* Bc, cudaStream_t s) {
     const dim3 gc(unsigned(cdiv(p.K, 128)), unsigned(p.N), unsigned(p.BH));

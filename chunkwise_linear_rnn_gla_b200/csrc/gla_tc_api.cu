@@ -63,16 +63,18 @@ bool tc_supported(const Problem& p) {
 }
 
 size_t tc_fwd_workspace(const Problem& p) {
-    Arena a{nullptr, 0, 0};
+    Arena a = make_arena(p, nullptr, 0);
     carve(p, a, false);
     return a.used;
 }
 
 size_t tc_bwd_workspace(const Problem& p) {
-    Arena a{nullptr, 0, 0};
+    Arena a = make_arena(p, nullptr, 0);
     carve(p, a, true);
     return a.used;
 }
+
+void tc_layout(const Problem& p, Arena& a, bool bwd) { carve(p, a, bwd); }
 
 gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v, const float* la, const float* h0,
                   void* o, float* hT, Arena& ws, cudaStream_t s) {

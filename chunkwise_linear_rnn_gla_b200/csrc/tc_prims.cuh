@@ -93,7 +93,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
         if (*abort) return false;
         if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
         if (clock64() - t0 > limit_cycles) {
-            if (err) atomicExch(err, kErrWaitTimeout);
+            if (err) atomicOr(err, kErrWaitTimeout);
             *abort = 1;
             return false;
         }

@@ -99,6 +99,21 @@ typedef struct gla_desc {
  * workspace or the inputs in between. */
 #define GLA_FLAG_WS_FROM_FWD 0x1
 
+/* Checking mode (the same as building the library with -DGLA_CHECKS, which
+ * turns it on for every call). Each call then also enqueues:
+ *  - before the pass, a check that every log_a element is finite and <= 0;
+ *  - before the pass, a fill of guard blocks (256 bytes) placed after every
+ *    workspace slice, and after the pass a check that they are intact;
+ *  - after the pass, a check that every output element is finite.
+ * A failed check does not stop the call or trap: it sets the device error
+ * flag, and the next gla_check_device_error reports GLA_ERR_INVALID_ARG (a
+ * gate outside its domain, or a non-finite output, e.g. from a NaN input) or
+ * GLA_ERR_WORKSPACE (a guard block was overwritten: a kernel wrote outside
+ * its slice). The workspace sizes include the guard blocks when the flag is
+ * set, so a forward and the backward that reuses its workspace must agree on
+ * it. Off by default: the checks read every gate and output once more. */
+#define GLA_FLAG_CHECKS 0x2
+
 /* Workspace bytes gla_fwd / gla_bwd need for `d` (0 when `d` is invalid).
  * A buffer of gla_bwd_workspace_size bytes also serves gla_fwd, so one
  * workspace can be shared by a forward and the following backward. */
@@ -174,8 +189,19 @@ gla_status gla_fwd_noalloc(const gla_desc* d, const void* q, const void* k, cons
 
 /* Blocks until `stream` is idle, then reports (and clears) the device-side
  * error flag: GLA_ERR_TIMEOUT if a bounded wait ran out in any kernel since
- * the last check, GLA_ERR_CUDA on a sticky CUDA error, else GLA_OK. */
+ * the last check; else, for calls made in checking mode (GLA_FLAG_CHECKS),
+ * GLA_ERR_INVALID_ARG if a gate was outside its domain or an output was not
+ * finite, GLA_ERR_WORKSPACE if a workspace guard block was overwritten;
+ * GLA_ERR_CUDA on a sticky CUDA error; else GLA_OK. */
 gla_status gla_check_device_error(void* stream);
+
+/* The same report under the name the scope table of this layer gives it. */
+gla_status gla_last_device_error(void* stream);
+
+/* gla_fwd_workspace_size / gla_bwd_workspace_size under the names the scope
+ * table of this layer gives them (identical results). */
+size_t gla_fwd_workspace_bytes(const gla_desc* d);
+size_t gla_bwd_workspace_bytes(const gla_desc* d);
 
 /* Self-test of the error path: launches one CTA whose mbarrier wait can never
  * complete (nothing arrives on the barrier). The bounded wait gives up after
