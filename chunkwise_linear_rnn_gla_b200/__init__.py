@@ -62,9 +62,19 @@ def _need(t, name, shape, dtype, dev):
 
 
 def make_desc(B, H, L, Dk, Dv, dtype="bf16", chunk=0, subchunk=0, state_mode="auto", impl="auto",
-              flags=0) -> GlaDesc:
+              flags=0, gate="channel", tau=0.0) -> GlaDesc:
+    """Problem descriptor. gate: what log_a holds -- "channel" (log alpha [B,H,L,Dk]), "scalar"
+    (one log decay per head and step, [B,H,L]), "head" (one fixed log decay per head, [H]) or
+    "preact" (the gate's argument z [B,H,L,Dk], log alpha = logsigmoid(z) / tau)."""
     return GlaDesc(B, H, L, Dk, Dv, _lib.DTYPE[dtype], chunk, subchunk, _lib.STATE_MODE[state_mode],
-                   _lib.IMPL[impl], flags)
+                   _lib.IMPL[impl], flags, _lib.GATE[gate], float(tau))
+
+
+def gate_shape(gate, B, H, L, Dk):
+    """Shape of the log_a argument (and of dlog_a) for a gate kind; L=None for the decode step."""
+    steps = () if L is None else (L,)
+    return {"channel": (B, H) + steps + (Dk,), "scalar": (B, H) + steps, "head": (H,),
+            "preact": (B, H) + steps + (Dk,)}[gate]
 
 
 def gla_fwd_workspace_size(desc: GlaDesc) -> int:
@@ -119,14 +129,14 @@ def _finish_checks(guards, what):
             raise GlaError(_lib.GLA_ERR_WORKSPACE, what + " (checking mode: an output canary was overwritten)")
 
 
-def _desc_from(q, v, chunk, subchunk, state_mode, impl, flags=0):
+def _desc_from(q, v, chunk, subchunk, state_mode, impl, flags=0, gate="channel", tau=0.0):
     B, H, L, Dk = q.shape
     Dv = v.shape[-1]
-    return make_desc(B, H, L, Dk, Dv, _dt(q), chunk, subchunk, state_mode, impl, flags)
+    return make_desc(B, H, L, Dk, Dv, _dt(q), chunk, subchunk, state_mode, impl, flags, gate, tau)
 
 
 def gla_fwd(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto", o=None, hT=None,
-            want_hT=True, workspace=None, checks=False):
+            want_hT=True, workspace=None, checks=False, gate="channel", tau=0.0):
     """Forward. Returns (o, hT); hT is None when want_hT is False and no hT
     buffer is given. `workspace` (uint8 tensor) may be passed to reuse it.
     checks=True runs the library's checking mode (gate domain, finite
@@ -139,10 +149,10 @@ def gla_fwd(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", 
     dt = q.dtype
     _need(k, "k", q.shape, dt, dev)
     _need(v, "v", (B, H, L, Dv), dt, dev)
-    _need(log_a, "log_a", q.shape, torch.float32, dev)
+    _need(log_a, "log_a", gate_shape(gate, B, H, L, Dk), torch.float32, dev)
     if h0 is not None:
         _need(h0, "h0", (B, H, Dk, Dv), torch.float32, dev)
-    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, _lib.FLAG_CHECKS if checks else 0)
+    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, _lib.FLAG_CHECKS if checks else 0, gate, tau)
     guards = []
     alloc = (lambda shp, t: _guarded(shp, t, dev, guards)) if checks else \
         (lambda shp, t: torch.empty(*shp, dtype=t, device=dev))
@@ -164,7 +174,7 @@ def gla_fwd(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", 
 
 
 def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto",
-            want_dh0=True, workspace=None, ws_from_fwd=False, out=None, checks=False):
+            want_dh0=True, workspace=None, ws_from_fwd=False, out=None, checks=False, gate="channel", tau=0.0):
     """Backward of <dO, o> + <dhT, hT>. Returns a dict with dq, dk, dv,
     dlog_a and dh0. With ws_from_fwd=True the workspace must be the one the
     matching gla_fwd call used (same inputs, same options, checks included).
@@ -176,14 +186,14 @@ def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state
     dt = q.dtype
     _need(k, "k", q.shape, dt, dev)
     _need(v, "v", (B, H, L, Dv), dt, dev)
-    _need(log_a, "log_a", q.shape, torch.float32, dev)
+    _need(log_a, "log_a", gate_shape(gate, B, H, L, Dk), torch.float32, dev)
     _need(dO, "dO", (B, H, L, Dv), dt, dev)
     if h0 is not None:
         _need(h0, "h0", (B, H, Dk, Dv), torch.float32, dev)
     if dhT is not None:
         _need(dhT, "dhT", (B, H, Dk, Dv), torch.float32, dev)
     flags = (_lib.FLAG_WS_FROM_FWD if ws_from_fwd else 0) | (_lib.FLAG_CHECKS if checks else 0)
-    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, flags)
+    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, flags, gate, tau)
     if ws_from_fwd and workspace is None:
         raise ValueError("ws_from_fwd needs the forward's workspace")
     guards = []
@@ -202,6 +212,7 @@ def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state
     dla = out.get("dlog_a")
     if dla is None:
         dla = alloc(log_a.shape, torch.float32)
+    _need(dla, "dlog_a", log_a.shape, torch.float32, dev)
     dh0 = out.get("dh0")
     if dh0 is None and want_dh0:
         dh0 = alloc((B, H, Dk, Dv), torch.float32)
@@ -216,7 +227,7 @@ def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state
     return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dh0": dh0}
 
 
-def gla_step(q, k, v, log_a, S, o=None, checks=False):
+def gla_step(q, k, v, log_a, S, o=None, checks=False, gate="channel", tau=0.0):
     """One decode step; S [B,H,Dk,Dv] fp32 is updated in place. Returns o [B,H,Dv].
     checks=True: the library's checking mode (gate domain, finite o and S), synchronous, raises on a
     failure."""
@@ -227,13 +238,13 @@ def gla_step(q, k, v, log_a, S, o=None, checks=False):
     dt = q.dtype
     _need(k, "k", q.shape, dt, dev)
     _need(v, "v", (B, H, Dv), dt, dev)
-    _need(log_a, "log_a", q.shape, torch.float32, dev)
+    _need(log_a, "log_a", gate_shape(gate, B, H, None, Dk), torch.float32, dev)
     _need(S, "S", (B, H, Dk, Dv), torch.float32, dev)
     guards = []
     if o is None:
         o = _guarded((B, H, Dv), dt, dev, guards) if checks else torch.empty(B, H, Dv, dtype=dt, device=dev)
     _need(o, "o", (B, H, Dv), dt, dev)
-    desc = make_desc(B, H, 1, Dk, Dv, _dt(q), flags=_lib.FLAG_CHECKS if checks else 0)
+    desc = make_desc(B, H, 1, Dk, Dv, _dt(q), flags=_lib.FLAG_CHECKS if checks else 0, gate=gate, tau=tau)
     with torch.cuda.device(dev):
         st = load().gla_step(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(S), _ptr(o),
                              _stream(dev))

@@ -21,6 +21,7 @@ STATUS_NAMES = {0: "GLA_OK", 1: "GLA_ERR_INVALID_ARG", 2: "GLA_ERR_UNSUPPORTED",
 DTYPE = {"f32": 0, "bf16": 1}
 STATE_MODE = {"auto": 0, "materialized": 1, "nonmaterialized": 2}
 IMPL = {"auto": 0, "simt": 1, "tc": 2}
+GATE = {"channel": 0, "scalar": 1, "head": 2, "preact": 3}
 FLAG_WS_FROM_FWD = 0x1
 FLAG_CHECKS = 0x2
 
@@ -30,6 +31,7 @@ EXPORTS = (
     "gla_check_device_error", "gla_status_string", "gla_abi_version", "gla_resolve", "gla_launch_count",
     "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset", "gla_fwd_noalloc",
     "gla_selftest_wait_timeout", "gla_last_device_error", "gla_fwd_workspace_bytes", "gla_bwd_workspace_bytes",
+    "gla_segment_decay", "gla_state_combine",
 )
 
 
@@ -37,7 +39,7 @@ class GlaDesc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("L", ctypes.c_int64), ("Dk", ctypes.c_int64),
                 ("Dv", ctypes.c_int64), ("dtype", ctypes.c_int32), ("chunk", ctypes.c_int32),
                 ("subchunk", ctypes.c_int32), ("state_mode", ctypes.c_int32), ("impl", ctypes.c_int32),
-                ("flags", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("gate", ctypes.c_int32), ("gate_tau", ctypes.c_float)]
 
 
 _lock = threading.Lock()
@@ -91,6 +93,11 @@ def _declare(lib):
     lib.gla_profile_reset.restype = None
     lib.gla_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.gla_fwd_noalloc.restype = ctypes.c_int
+    lib.gla_segment_decay.argtypes = [dp, vp, vp, vp]
+    lib.gla_segment_decay.restype = ctypes.c_int
+    i64 = ctypes.c_int64
+    lib.gla_state_combine.argtypes = [i64, i64, i64, i64, vp, vp, vp, i32, i32, vp, vp]
+    lib.gla_state_combine.restype = ctypes.c_int
 
 
 def load(path: str = LIB_PATH):

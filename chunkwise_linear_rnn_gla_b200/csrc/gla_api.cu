@@ -112,6 +112,18 @@ namespace {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Gate kind and temperature (include/gla.h, gla_gate).
+bool gate_ok(const gla_desc* d, Problem& p) {
+    if (d->gate < GLA_GATE_CHANNEL || d->gate > GLA_GATE_PREACT) return false;
+    p.gate = d->gate;
+    p.inv_tau = 0.f;
+    if (d->gate == GLA_GATE_PREACT) {
+        if (!(d->gate_tau > 0.f) || !(d->gate_tau < 3.0e38f)) return false;
+        p.inv_tau = 1.f / d->gate_tau;
+    }
+    return true;
+}
+
 // Fill `p` from `d` (defaults applied). Returns GLA_OK or an error status.
 gla_status resolve(const gla_desc* d, Problem& p) {
     if (!d) return GLA_ERR_INVALID_ARG;
@@ -123,6 +135,7 @@ gla_status resolve(const gla_desc* d, Problem& p) {
     if (d->state_mode < GLA_STATE_AUTO || d->state_mode > GLA_STATE_NONMATERIALIZED) return GLA_ERR_INVALID_ARG;
     if (d->impl < GLA_IMPL_AUTO || d->impl > GLA_IMPL_TC) return GLA_ERR_INVALID_ARG;
     if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
+    if (!gate_ok(d, p)) return GLA_ERR_INVALID_ARG;
     p.B = d->B;
     p.H = d->H;
     p.L = d->L;
@@ -163,8 +176,48 @@ gla_status resolve(const gla_desc* d, Problem& p) {
     return GLA_OK;
 }
 
-size_t fwd_ws(const Problem& p) { return p.impl == GLA_IMPL_TC ? gla::tc_fwd_workspace(p) : gla::simt_fwd_workspace(p); }
-size_t bwd_ws(const Problem& p) { return p.impl == GLA_IMPL_TC ? gla::tc_bwd_workspace(p) : gla::simt_bwd_workspace(p); }
+// Workspace layout of a pass: [per-channel log alpha when the gate kind is not per channel] [the
+// path's own slices] [backward of a scalar or head gate: the per-channel gate gradient]. The
+// forward's part is a prefix of the backward's, so a backward can reuse a forward's workspace.
+struct Layout {
+    float* la_pc = nullptr;   // expanded per-channel log alpha (null: the caller's log_a is per channel)
+    float* dla_pc = nullptr;  // per-channel gate gradient (backward, scalar and head kinds)
+};
+
+// The tensor-core path reads every gate kind natively; the CUDA-core path works on the expansion.
+Layout carve_all(const Problem& p, gla::Arena& a, bool bwd, bool path_too) {
+    Layout l;
+    if (p.gate != GLA_GATE_CHANNEL && p.impl == GLA_IMPL_SIMT) l.la_pc = a.take<float>(size_t(p.BH * p.L * p.K));
+    if (path_too) {
+        if (bwd) (p.impl == GLA_IMPL_TC ? gla::tc_layout : gla::simt_layout)(p, a, true);
+        else (p.impl == GLA_IMPL_TC ? gla::tc_layout : gla::simt_layout)(p, a, false);
+    }
+    return l;
+}
+
+float* carve_dla_pc(const Problem& p, gla::Arena& a) {
+    return (p.impl == GLA_IMPL_SIMT && (p.gate == GLA_GATE_SCALAR || p.gate == GLA_GATE_HEAD))
+               ? a.take<float>(size_t(p.BH * p.L * p.K))
+               : nullptr;
+}
+
+size_t ws_size(const Problem& p, bool bwd) {
+    gla::Arena a = gla::make_arena(p, nullptr, 0);
+    carve_all(p, a, bwd, true);
+    if (bwd) carve_dla_pc(p, a);
+    return a.used;
+}
+
+size_t fwd_ws(const Problem& p) { return ws_size(p, false); }
+size_t bwd_ws(const Problem& p) { return ws_size(p, true); }
+
+int64_t gate_elems(const Problem& p, int64_t steps) {
+    switch (p.gate) {
+        case GLA_GATE_SCALAR: return p.BH * steps;
+        case GLA_GATE_HEAD: return p.H;
+        default: return p.BH * steps * p.K;
+    }
+}
 
 gla_status check_ws(void* ws, size_t bytes, size_t need) {
     if (need == 0) return GLA_OK;
@@ -241,15 +294,22 @@ gla_status gla_fwd(const gla_desc* d, const void* q, const void* k, const void* 
     gla::Arena a = gla::make_arena(p, workspace, workspace_bytes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool chk = gla::checks_on(p);
+    const Layout l = carve_all(p, a, false, false);  // gate slices; the path carves the rest itself
+    const float* la = log_a;
+    if (l.la_pc) {
+        st = gla::gate_expand(p, log_a, l.la_pc, s);
+        if (st != GLA_OK) return st;
+        la = l.la_pc;
+    }
     gla::Arena layout = gla::make_arena(p, workspace, workspace_bytes);
     if (chk) {
-        (p.impl == GLA_IMPL_TC ? gla::tc_layout : gla::simt_layout)(p, layout, false);
-        st = gla::check_gates(log_a, p.BH * p.L * p.K, s);
+        carve_all(p, layout, false, true);
+        st = p.gate == GLA_GATE_PREACT ? GLA_OK : gla::check_gates(log_a, gate_elems(p, p.L), s);
         if (st == GLA_OK) st = gla::guards_fill(layout, s);
         if (st != GLA_OK) return st;
     }
-    st = p.impl == GLA_IMPL_TC ? gla::tc_fwd(p, q, k, v, log_a, h0, o, hT, a, s)
-                               : gla::simt_fwd(p, q, k, v, log_a, h0, o, hT, a, s);
+    st = p.impl == GLA_IMPL_TC ? gla::tc_fwd(p, q, k, v, la, h0, o, hT, a, s)
+                               : gla::simt_fwd(p, q, k, v, la, h0, o, hT, a, s);
     if (st != GLA_OK || !chk) return st;
     st = gla::check_finite(o, p.BH * p.L * p.V, p.bf16, s);
     if (st == GLA_OK) st = gla::check_finite(hT, p.BH * p.K * p.V, false, s);
@@ -281,21 +341,44 @@ gla_status gla_bwd(const gla_desc* d, const void* q, const void* k, const void* 
     gla::Arena a = gla::make_arena(p, workspace, workspace_bytes);
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool chk = gla::checks_on(p);
+    const Layout l = carve_all(p, a, true, false);
+    const float* la = log_a;
+    if (l.la_pc) {
+        // a forward's workspace holds the expansion already, unless the caller says nothing of it
+        if (!(p.flags & GLA_FLAG_WS_FROM_FWD)) {
+            st = gla::gate_expand(p, log_a, l.la_pc, s);
+            if (st != GLA_OK) return st;
+        }
+        la = l.la_pc;
+    }
     gla::Arena layout = gla::make_arena(p, workspace, workspace_bytes);
     if (chk) {
-        (p.impl == GLA_IMPL_TC ? gla::tc_layout : gla::simt_layout)(p, layout, true);
-        st = gla::check_gates(log_a, p.BH * p.L * p.K, s);
+        carve_all(p, layout, true, true);
+        carve_dla_pc(p, layout);
+        st = p.gate == GLA_GATE_PREACT ? GLA_OK : gla::check_gates(log_a, gate_elems(p, p.L), s);
         if (st == GLA_OK) st = gla::guards_fill(layout, s);
         if (st != GLA_OK) return st;
     }
-    st = p.impl == GLA_IMPL_TC ? gla::tc_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s)
-                               : gla::simt_bwd(p, q, k, v, log_a, h0, dO, dhT, dq, dk, dv, dlog_a, dh0, a, s);
+    // the per-channel gate gradient goes to the workspace (scalar, head) or to dlog_a itself (channel,
+    // preact: scaled in place afterwards)
+    float* dla_pc = dlog_a;
+    {
+        gla::Arena tail = gla::make_arena(p, workspace, workspace_bytes);
+        carve_all(p, tail, true, true);
+        float* w = carve_dla_pc(p, tail);
+        if (tail.used > tail.cap) return GLA_ERR_WORKSPACE;
+        if (w) dla_pc = w;
+    }
+    st = p.impl == GLA_IMPL_TC ? gla::tc_bwd(p, q, k, v, la, h0, dO, dhT, dq, dk, dv, dla_pc, dh0, a, s)
+                               : gla::simt_bwd(p, q, k, v, la, h0, dO, dhT, dq, dk, dv, dla_pc, dh0, a, s);
+    if (st == GLA_OK && p.gate != GLA_GATE_CHANNEL && p.impl == GLA_IMPL_SIMT)
+        st = gla::gate_grad(p, log_a, dla_pc, dlog_a, s);
     if (st != GLA_OK || !chk) return st;
     const int64_t nk = p.BH * p.L * p.K, nv = p.BH * p.L * p.V;
     st = gla::check_finite(dq, nk, p.bf16, s);
     if (st == GLA_OK) st = gla::check_finite(dk, nk, p.bf16, s);
     if (st == GLA_OK) st = gla::check_finite(dv, nv, p.bf16, s);
-    if (st == GLA_OK) st = gla::check_finite(dlog_a, nk, false, s);
+    if (st == GLA_OK) st = gla::check_finite(dlog_a, gate_elems(p, p.L), false, s);
     if (st == GLA_OK) st = gla::check_finite(dh0, p.BH * p.K * p.V, false, s);
     if (st == GLA_OK) st = gla::guards_check(layout, s);
     return st;
@@ -315,6 +398,7 @@ gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void*
     if (d->B * d->H > 65535 || d->Dk > 8192) return GLA_ERR_UNSUPPORTED;
     if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
     Problem p{};
+    if (!gate_ok(d, p)) return GLA_ERR_INVALID_ARG;
     p.B = d->B;
     p.H = d->H;
     p.L = 1;
@@ -325,7 +409,7 @@ gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void*
     p.flags = d->flags;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool chk = gla::checks_on(p);
-    gla_status st = chk ? gla::check_gates(log_a, p.BH * p.K, s) : GLA_OK;
+    gla_status st = chk && p.gate != GLA_GATE_PREACT ? gla::check_gates(log_a, gate_elems(p, 1), s) : GLA_OK;
     if (st == GLA_OK) st = gla::step_launch(p, q, k, v, log_a, S, o, s);
     if (st != GLA_OK || !chk) return st;
     st = gla::check_finite(o, p.BH * p.V, p.bf16, s);
@@ -338,6 +422,7 @@ gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, 
     if (d->B < 1 || d->H < 1 || d->L < 1 || d->Dk < 1) return GLA_ERR_INVALID_ARG;
     const int C = d->chunk ? d->chunk : 64;
     if (C != 16 && C != 32 && C != 64 && C != 128) return GLA_ERR_INVALID_ARG;
+    if (d->gate != GLA_GATE_CHANNEL) return GLA_ERR_UNSUPPORTED;
     GLA_REQUIRE_PTR(log_a);
     GLA_REQUIRE_PTR(Bcum);
     Problem p{};
@@ -351,6 +436,27 @@ gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, 
     p.N = (p.L + C - 1) / C;
     if (p.BH > 65535 || p.N > 65535) return GLA_ERR_UNSUPPORTED;
     return gla::simt_chunk_cumsum(p, log_a, Bcum, static_cast<cudaStream_t>(stream));
+}
+
+gla_status gla_segment_decay(const gla_desc* d, const float* log_a, float* a, void* stream) {
+    Problem p{};
+    gla_status st = resolve(d, p);
+    if (st != GLA_OK) return st;
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(a);
+    return gla::segment_decay(p, log_a, a, static_cast<cudaStream_t>(stream));
+}
+
+gla_status gla_state_combine(int64_t G, int64_t BH, int64_t Dk, int64_t Dv, const float* a, const float* U,
+                             const float* init, int32_t r, int32_t reverse, float* out, void* stream) {
+    if (G < 1 || BH < 1 || Dk < 1 || Dv < 1 || Dv % 4 != 0 || r < 0 || r >= G) return GLA_ERR_INVALID_ARG;
+    if (reverse != 0 && reverse != 1) return GLA_ERR_INVALID_ARG;
+    if (BH * Dk * (Dv / 4) > (int64_t(1) << 31) - 1) return GLA_ERR_UNSUPPORTED;
+    GLA_REQUIRE_PTR(a);
+    GLA_REQUIRE_PTR(U);
+    GLA_OPTIONAL_PTR(init);
+    GLA_REQUIRE_PTR(out);
+    return gla::state_combine(G, BH, Dk, Dv, a, U, init, r, reverse, out, static_cast<cudaStream_t>(stream));
 }
 
 namespace {

@@ -21,6 +21,8 @@ struct Problem {
     int impl;        // GLA_IMPL_SIMT or GLA_IMPL_TC (never AUTO)
     int state_mode;  // never AUTO
     int flags;
+    int gate = 0;         // gla_gate: what the caller's log_a holds
+    float inv_tau = 0.f;  // GLA_GATE_PREACT: 1 / gate_tau
 };
 
 // Bump allocator over the caller's workspace; every slice is 256-B aligned.
@@ -76,6 +78,18 @@ gla_status check_finite(const void* p, int64_t n, bool bf16, cudaStream_t s);
 gla_status guards_fill(const Arena& a, cudaStream_t s);
 gla_status guards_check(const Arena& a, cudaStream_t s);
 bool checks_on(const Problem& p);
+
+// ---- gate kinds (gla_gates.cu) ------------------------------------------------
+// Per-channel log alpha [B,H,L,K] from the caller's gate argument, and the caller's gate gradient
+// from the per-channel one (scalar / head: sums; preact: dpc and dla are the same buffer, scaled in
+// place by sigmoid(-z)/tau).
+gla_status gate_expand(const Problem& p, const float* g, float* out, cudaStream_t s);
+gla_status gate_grad(const Problem& p, const float* g, const float* dpc, float* dla, cudaStream_t s);
+
+// ---- sequence-sharded evaluation (gla_seq.cu) ---------------------------------
+gla_status segment_decay(const Problem& p, const float* log_a, float* a, cudaStream_t s);
+gla_status state_combine(int64_t G, int64_t BH, int64_t K, int64_t V, const float* a, const float* U,
+                         const float* init, int r, int reverse, float* out, cudaStream_t s);
 
 // ---- SIMT path (gla_simt.cu) ---------------------------------------------
 size_t simt_fwd_workspace(const Problem& p);

@@ -19,6 +19,7 @@
 #include <cuda_runtime.h>
 
 #include "gla_common.cuh"
+#include "gla_gate.cuh"
 #include "gla_internal.h"
 
 namespace gla {
@@ -51,7 +52,7 @@ struct StepVec<1> {
 
 template <typename T, int VEC>
 __global__ void __launch_bounds__(kStepThreads) k_step(const T* __restrict__ q, const T* __restrict__ k,
-                                                       const T* __restrict__ v, const float* __restrict__ la,
+                                                       const T* __restrict__ v, GateArgs la,
                                                        float* __restrict__ S, T* __restrict__ o, int K, int V,
                                                        int CG) {
     using SV = StepVec<VEC>;
@@ -67,7 +68,7 @@ __global__ void __launch_bounds__(kStepThreads) k_step(const T* __restrict__ q, 
     for (int c = tid; c < K; c += kStepThreads) {
         sq[c] = ldf(q + bh * K + c);
         sk[c] = ldf(k + bh * K + c);
-        sa[c] = expf(la[bh * K + c]);
+        sa[c] = expf(gate_log_alpha(la, bh, 0, c, 1, K));
     }
     __syncthreads();
     const int cg = tid % CG, ks = tid / CG;
@@ -119,8 +120,9 @@ __global__ void __launch_bounds__(kStepThreads) k_step(const T* __restrict__ q, 
 }
 
 template <typename T>
-gla_status step_typed(const Problem& p, const T* q, const T* k, const T* v, const float* la, float* S, T* o,
+gla_status step_typed(const Problem& p, const T* q, const T* k, const T* v, const float* g, float* S, T* o,
                       cudaStream_t s) {
+    const GateArgs la{g, p.gate, p.inv_tau, p.H};
     const int K = int(p.K), V = int(p.V);
     // 16-byte state accesses need a 16-byte aligned state and rows of a multiple of 4 floats
     const bool vec = (V % 4) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;

@@ -18,8 +18,9 @@ constexpr int kTcBV = 64;      // value columns per walk CTA
 
 // Chunk-parallel gate preparation (gla_tc_prep.cu): Q~, K~, e^Gamma and the
 // masked intra-chunk scores P.
+// `la` is the gate argument of kind `gate_kind` (gla_gate.cuh): the kernel reads every kind natively.
 gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const float* la, __nv_bfloat16* Qt,
-                          __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, cudaStream_t s);
+                          __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, int gate_kind, cudaStream_t s);
 
 // Row-gated chunk walk (gla_tc_walk.cu). State X [K x 64-column tile] with the
 // gate on its rows. Per chunk i (in walk order):
@@ -98,8 +99,14 @@ gla_status tc_chunk_out_launch(const Problem& p, const __nv_bfloat16* A, const _
 
 // Backward, chunk-parallel part (gla_tc_bwd.cu): dq, dk and dlog a from dO, v,
 // the stored states S_[i] and D_i, Q~ and e^Gamma.
+// `la` is the gate argument of kind p.gate. Per-channel kinds write dla (dL/dlog alpha, or dL/dz for
+// preact) directly; the scalar kinds write per-CTA partial sums over their 128 channels to
+// gpart[(bh * N + i) * (K / 128) + kh][token] (zero past the end of the sequence), which
+// tc_gate_grad_partials reduces into the caller's gradient.
 gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
                                const void* v, const __nv_bfloat16* Qt, const float* gam, const __nv_bfloat16* Sbuf,
-                               const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, cudaStream_t s);
+                               const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, float* gpart,
+                               cudaStream_t s);
+gla_status tc_gate_grad_partials(const Problem& p, const float* gpart, float* dla, cudaStream_t s);
 
 }  // namespace gla

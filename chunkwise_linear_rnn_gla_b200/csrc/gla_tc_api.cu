@@ -15,6 +15,8 @@
 //                      chunk-parallel tc_output_dv computes dv)
 //   tc_bwd_chunk       dP = dO v^T, dQ~ = dO S_[i]^T, dK~ = v D_i^T and the
 //                      intra-chunk terms on tcgen05, dq, dk, closed-form dlog a
+//   [gate_grad_partials] scalar gate kinds: the gate gradient summed over channels
+// Every kernel reads the caller's gate argument natively (gla_gate.cuh).
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -32,6 +34,7 @@ struct TcBuffers {
     __nv_bfloat16* states;
     float* segbuf;  // segmented state walks: end states and entering states per segment
     __nv_bfloat16* Dbuf;
+    float* gpart;   // scalar gate kinds: per-CTA partial sums of the gate gradient
 };
 
 // The backward layout extends the forward's, so a forward workspace can be
@@ -47,6 +50,8 @@ TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
     const size_t nseg = tc_walk_seg_floats(p);
     if (nseg) b.segbuf = a.take<float>(nseg);
     if (bwd) b.Dbuf = a.take<__nv_bfloat16>(size_t(p.BH * p.N * p.K * p.V));
+    if (bwd && (p.gate == GLA_GATE_SCALAR || p.gate == GLA_GATE_HEAD))
+        b.gpart = a.take<float>(size_t(p.BH * p.N * (p.K / 128) * kTcChunk));
     return b;
 }
 
@@ -80,7 +85,7 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
                   void* o, float* hT, Arena& ws, cudaStream_t s) {
     TcBuffers b = carve(p, ws, false);
     if (ws.used > ws.cap) return GLA_ERR_WORKSPACE;
-    gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, s);
+    gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, p.gate, s);
     if (st != GLA_OK) return st;
     WalkArgs a{};
     a.A1 = b.Kt;
@@ -119,7 +124,7 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
     const bool reuse = (p.flags & GLA_FLAG_WS_FROM_FWD) != 0;
     gla_status st;
     if (!reuse) {
-        st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, s);
+        st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, p.gate, s);
         if (st != GLA_OK) return st;
     }
     if (!(reuse && p.state_mode == GLA_STATE_MATERIALIZED)) {
@@ -166,13 +171,18 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
             // dv does not depend on the chunk backward, which triggers its dependents only after its
             // own wait: launched after it, the dv GEMM starts on the SMs that the backward's last
             // wave leaves idle and waits for the backward only before it exits
-            st = tc_bwd_chunk_launch(p, q, k, la, dO, v, b.Qt, b.gam, b.states, b.Dbuf, dq, dk, dla, s);
+            st = tc_bwd_chunk_launch(p, q, k, la, dO, v, b.Qt, b.gam, b.states, b.Dbuf, dq, dk, dla, b.gpart, s);
             if (st != GLA_OK) return st;
-            return tc_chunk_out_launch(p, b.Kt, b.Dbuf, b.P, static_cast<const __nv_bfloat16*>(dO), true,
-                                       static_cast<__nv_bfloat16*>(dv), true, s, "tc_output_dv");
+            st = tc_chunk_out_launch(p, b.Kt, b.Dbuf, b.P, static_cast<const __nv_bfloat16*>(dO), true,
+                                     static_cast<__nv_bfloat16*>(dv), true, s, "tc_output_dv");
+            // the dv GEMM waits for the chunk backward before it exits: the partials are complete
+            if (st == GLA_OK && b.gpart) st = tc_gate_grad_partials(p, b.gpart, dla, s);
+            return st;
         }
     }
-    return tc_bwd_chunk_launch(p, q, k, la, dO, v, b.Qt, b.gam, b.states, b.Dbuf, dq, dk, dla, s);
+    st = tc_bwd_chunk_launch(p, q, k, la, dO, v, b.Qt, b.gam, b.states, b.Dbuf, dq, dk, dla, b.gpart, s);
+    if (st == GLA_OK && b.gpart) st = tc_gate_grad_partials(p, b.gpart, dla, s);
+    return st;
 }
 
 }  // namespace gla

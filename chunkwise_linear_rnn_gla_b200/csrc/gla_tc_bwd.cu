@@ -53,6 +53,7 @@
 #include <type_traits>
 
 #include "gla_common.cuh"
+#include "gla_gate.cuh"
 #include "gla_internal.h"
 #include "gla_tc.h"
 #include "tc_host.h"
@@ -89,7 +90,10 @@ struct BwdBars {
     int abort_flag;
     int any_exact;  // some key channel of this CTA is beyond the bound
     float xd[128];  // sum_v D_i[c,v] S_[i][c,v]
+    float btab[128];  // scalar gate kinds: the per-token cumsum b_t in base-2 units
 };
+
+constexpr bool scalar_kind(int GK) { return GK == kGateScalar || GK == kGateHead; }
 
 // byte offset of element (row, col) in a [128 x 128] bf16 tile stored as two
 // SW128 pieces of 64 columns
@@ -99,6 +103,7 @@ __device__ __forceinline__ uint32_t tile_off(int row, int col) {
            uint32_t(c64 & 7) * 2u;
 }
 
+template <int GK>
 __global__ void __launch_bounds__(kThreads, 1)
     k_bwd_chunk(const __grid_constant__ CUtensorMap tmDO, const __grid_constant__ CUtensorMap tmV,
                 const __grid_constant__ CUtensorMap tmS, const __grid_constant__ CUtensorMap tmD,
@@ -107,8 +112,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const __grid_constant__ CUtensorMap tmDK,
                 const __grid_constant__ CUtensorMap tmLA,
                 const __nv_bfloat16* __restrict__ q,
-                const __nv_bfloat16* __restrict__ k, const float* __restrict__ la, const float* __restrict__ gam,
-                __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, float* __restrict__ dla, int64_t L,
+                const __nv_bfloat16* __restrict__ k, GateArgs ga, const float* __restrict__ gam,
+                __nv_bfloat16* __restrict__ dq, __nv_bfloat16* __restrict__ dk, float* __restrict__ dla,
+                float* __restrict__ gpart, int64_t L,
                 int64_t N, int64_t K, int64_t V, uint32_t stagger_ns, uint32_t n_first, int* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -175,8 +181,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (global_ns() < until) __nanosleep(256);
             }
             // the gate prologue's inputs first: log a (dense fp32) and k (into the K^0 operand area)
-            mbar_arrive_expect_tx(&bar.pro_full, 4 * PIECE + 2 * PIECE);
-            tma_load_3d(base + LA_OFF, &tmLA, 128 * kh, i * C, int(bh), &bar.pro_full);
+            mbar_arrive_expect_tx(&bar.pro_full, (scalar_kind(GK) ? 0u : 4 * PIECE) + 2 * PIECE);
+            if (!scalar_kind(GK)) tma_load_3d(base + LA_OFF, &tmLA, 128 * kh, i * C, int(bh), &bar.pro_full);
             tma_load_3d(base + KH_OFF, &tmK, 128 * kh, i * C, int(bh), &bar.pro_full);
             tma_load_3d(base + KH_OFF + PIECE, &tmK, 128 * kh + 64, i * C, int(bh), &bar.pro_full);
             bool ok = true;
@@ -254,10 +260,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int kk = 0; kk < C / 16; ++kk) {
                     // dQ^T[c][j] += sum_s K^0[s][c] dP[j][s] for j >= 16 kk: A = K^0 (MN-major), B = dP
                     // (K-major) from row j = 16 kk
+                    // scalar gate kinds: A = the raw k tile and a decay-weighted dP, into its own accumulator
+                    // (columns 384.., initialised by the first slice, which spans every column)
                     const int j0 = 16 * kk;
-                    mma_bf16(tmem + 128 + uint32_t(j0), sdesc_sw128(kh0 + kk * 2048, PIECE, 1024),
+                    mma_bf16(tmem + (scalar_kind(GK) ? 384u : 128u) + uint32_t(j0), sdesc_sw128(kh0 + kk * 2048, PIECE, 1024),
                              sdesc_sw128(dpm + (kk / 4) * PIECE + (kk % 4) * 32 + j0 * 128, 16, 1024),
-                             idesc_bf16_f32(128, C - j0, true, false), 1u);
+                             idesc_bf16_f32(128, C - j0, true, false), (scalar_kind(GK) && kk == 0) ? 0u : 1u);
                     // dKi^T[c][s] = sum_j Q~[j][c] dP[j][s] for s < 16 (k + 1), k = 7 - kk: A = Q~
                     // (MN-major), B = dP (MN-major)
                     const int k = C / 16 - 1 - kk;
@@ -281,11 +289,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int fgrp = (warp - 2) >> 2;  // final-phase group: tokens 32 fgrp .. 32 fgrp + 31
         const uint32_t lane_off = uint32_t(32 * q4) << 16;
         const int64_t chg = int64_t(128) * kh + c;
-        const bool safe = gam[(bh * N + i) * K + chg] >= kSafeGam;
-        // rows past the end of the sequence (last chunk) read the last valid row and are zeroed
+        // scalar gate kinds have no range bound: their intra terms are weighted by the decay in fp32
+        const bool safe = scalar_kind(GK) || gam[(bh * N + i) * K + chg] >= kSafeGam;
         const int64_t rb = (bh * L + t0) * K + chg;
-        const float* lap = la + rb;
-        auto roff = [&](int t) -> uint32_t { return uint32_t(t < nvalid ? t : nvalid - 1) * uint32_t(K); };
+        // log alpha of token t (< nvalid) of this thread's channel, for the exact path
+        auto gate_t = [&](int t) -> float { return la_floor(gate_log_alpha(ga, bh, t0 + t, chg, L, K)); };
         if (row_warp) {
             // x_c = sum_v D_i[c,v] S_[i][c,v] from the staged tiles
             float x = 0.f;
@@ -314,18 +322,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             bar.xd[c] = x;
             mbar_arrive(&bar.xd_ready);
-            // dP epilogue: thread = token row r (= c), mask s > r, bf16, swizzled tile
+            // dP epilogue: thread = token row r (= c), mask s > r, bf16, swizzled tile; scalar gate kinds
+            // weight each term by its decay e^{b_r - b_s} (<= 1), so that the intra products take the raw
+            // q and k
             const int r = c;
             // tcgen05.ld is warp-collective: the condition must be the same for the whole warp
-            if (__all_sync(0xffffffffu, ok && mbar_wait(&bar.accA, 0, err, abort_flag))) {
+            if (__all_sync(0xffffffffu, ok && mbar_wait(&bar.accA, 0, err, abort_flag) &&
+                                            (!scalar_kind(GK) || mbar_wait(&bar.khat_ready, 0, err, abort_flag)))) {
                 tc_fence_after();
+                const float br = scalar_kind(GK) ? bar.btab[r] : 0.f;
 #pragma unroll 1
                 for (int c16 = 0; c16 < C / 16; ++c16) {
                     float y[16];
                     tmem_ld16(tmem + lane_off + uint32_t(16 * c16), y);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) y[e] = (16 * c16 + e <= r) ? y[e] : 0.f;
+                    for (int e = 0; e < 16; ++e) {
+                        const int sc = 16 * c16 + e;
+                        float w = y[e];
+                        if (scalar_kind(GK)) w *= exp2_ftz(fminf(br - bar.btab[sc], 0.f));
+                        y[e] = sc <= r ? w : 0.f;
+                    }
 #pragma unroll
                     for (int hh = 0; hh < 2; ++hh) {
                         const int c8 = 2 * (c16 & 3) + hh;  // 16-byte chunk within the 64-column piece
@@ -357,22 +374,35 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int r = 0; r < 8; ++r) {
                         const int t = 16 * g + 8 * h + r;
-                        lv[r] = la_floor(sLA[t * C + c]);
-                        kv[r] = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + KH_OFF + tile_off(t, c)));
+                        if (scalar_kind(GK)) {  // one decay per token (or per head) for every channel
+                            lv[r] = t < nvalid ? la_floor(GK == kGateScalar ? ga.g[bh * L + t0 + t] : ga.g[bh % ga.H])
+                                               : 0.f;
+                        } else {
+                            const float x = sLA[t * C + c];  // zero past the end of the sequence (TMA fill)
+                            lv[r] = t < nvalid ? la_floor(GK == kGatePreact ? logsigmoid_f(x) * ga.inv_tau : x) : 0.f;
+                            kv[r] = __bfloat162float(
+                                *reinterpret_cast<const __nv_bfloat16*>(base + KH_OFF + tile_off(t, c)));
+                        }
                     }
 #pragma unroll
                     for (int r = 0; r < 8; ++r) {
                         B += lv[r] * kLog2e;
-                        const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; used when safe
-                        tb[8 * h + r] = safe ? e : B;
-                        kv[r] = safe ? kv[r] * e : 0.f;
+                        if (scalar_kind(GK)) {
+                            if (c == 0) bar.btab[16 * g + 8 * h + r] = B;
+                        } else {
+                            const float e = exp2_ftz(fminf(-B, (kSafeDecay + 1.f) * kLog2e));  // e^{-B}; used when safe
+                            tb[8 * h + r] = safe ? e : B;
+                            kv[r] = safe ? kv[r] * e : 0.f;
+                        }
                     }
+                    if (!scalar_kind(GK)) {
 #pragma unroll
-                    for (int r = 0; r < 8; ++r)  // K^0 in place of k
-                        *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(16 * g + 8 * h + r, c)) =
-                            __float2bfloat16_rn(kv[r]);
+                        for (int r = 0; r < 8; ++r)  // K^0 in place of k
+                            *reinterpret_cast<__nv_bfloat16*>(base + KH_OFF + tile_off(16 * g + 8 * h + r, c)) =
+                                __float2bfloat16_rn(kv[r]);
+                    }
                 }
-                tmem_st16(tmem + lane_off + 384u + uint32_t(16 * g), tb);
+                if (!scalar_kind(GK)) tmem_st16(tmem + lane_off + 384u + uint32_t(16 * g), tb);
             }
             if (__any_sync(0xffffffffu, !safe) && lane == 0) atomicOr(&bar.any_exact, 1);
             tmem_wait_st();
@@ -409,12 +439,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll 1
                 for (int j = t; j >= 0; --j) {
                     eq += dpm(t, j) * ks(j) * __expf(fminf(d, 0.f));
-                    d += j < nvalid ? la_floor(lap[roff(j)]) : 0.f;
+                    d += j < nvalid ? gate_t(j) : 0.f;
                 }
                 d = 0.f;
 #pragma unroll 1
                 for (int j = t; j < C; ++j) {
-                    if (j > t) d += j < nvalid ? la_floor(lap[roff(j)]) : 0.f;
+                    if (j > t) d += j < nvalid ? gate_t(j) : 0.f;
                     ek += dpm(j, t) * qs(j) * __expf(fminf(d, 0.f));
                 }
                 rbuf[t * C + c] = eq;
@@ -435,7 +465,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         float eGam = 0.f, Gam = 0.f;  // Gamma in base-2 units
         if (ok) {
             tc_fence_after();
-            {
+            if (scalar_kind(GK)) {
+                // Gamma = b at the chunk's last row (rows past the end of the sequence add nothing)
+                Gam = bar.btab[C - 1];
+                eGam = exp2_ftz(fminf(Gam, 0.f));
+            } else {
                 // Gamma from the last column of the gate table (e^{-Gamma}, or Gamma itself)
                 float v8[8];
                 tmem_ld8(tmem + lane_off + 504u, v8);
@@ -465,7 +499,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int r = 7; r >= 0; --r) {
                         const int t = 8 * g + r;
                         float eGB, dqv, dkv;
-                        if (decltype(all_safe)::value || safe) {
+                        if (scalar_kind(GK)) {
+                            // inter parts carry the decay factors, the intra accumulators (raw q, k and a
+                            // decay-weighted dP) none: vT holds the intra part of dq
+                            const float b2 = bar.btab[t];
+                            eGB = exp2_ftz(fminf(Gam - b2, 0.f));
+                            dqv = fmaf(exp2_ftz(fminf(b2, 0.f)), vQ[r], vT[r]);
+                            dkv = fmaf(eGB, vJ[r], vI[r]);
+                        } else if (decltype(all_safe)::value || safe) {
                             const float e = vT[r];  // e^{-B_t}
                             eGB = eGam * e;
                             dqv = __fdividef(vQ[r], e);
@@ -515,10 +556,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int f = 0; f < 4; ++f) carry += xch[128 * f + c] + (f > fgrp ? xch[512 + 128 * f + c] : 0.f);
             float dv[32];
 #pragma unroll
-            for (int u = 0; u < 32; ++u) dv[u] = rbuf[(tlo + u) * C + c] + carry;
+            for (int u = 0; u < 32; ++u) dv[u] = tlo + u < nvalid ? rbuf[(tlo + u) * C + c] + carry : 0.f;
+            if (scalar_kind(GK)) {
+                // sum over this CTA's 128 channels per token: across the warp's 32 lanes by a butterfly that
+                // leaves token tlo + l's sum in lane l, then over the group's 4 warps in fixed order
 #pragma unroll
-            for (int u = 0; u < 32; ++u)
-                if (tlo + u < nvalid) dla[rb + int64_t(tlo + u) * K] = dv[u];
+                for (int kb = 16; kb >= 1; kb >>= 1) {
+#pragma unroll
+                    for (int j = 0; j < kb; ++j) {
+                        const bool hi = (lane & kb) != 0;
+                        const float give = hi ? dv[j] : dv[j + kb];
+                        const float got = __shfl_xor_sync(0xffffffffu, give, kb);
+                        dv[j] = (hi ? dv[j + kb] : dv[j]) + got;
+                    }
+                }
+                xch[2048 + (4 * fgrp + q4) * 32 + lane] = dv[0];
+            } else {
+#pragma unroll
+                for (int u = 0; u < 32; ++u)
+                    if (tlo + u < nvalid) {
+                        const int64_t o = rb + int64_t(tlo + u) * K;
+                        // preact: dL/dz = dL/dlog alpha * sigmoid(-z) / tau
+                        dla[o] = GK == kGatePreact ? dv[u] * sigmoid_neg_f(ga.g[o]) * ga.inv_tau : dv[u];
+                    }
+            }
+        }
+        if (scalar_kind(GK)) {
+            named_sync(4 + fgrp, 128);
+            if (ok && q4 == 0) {  // one warp per group: this CTA's partial of the gradient of tokens tlo ..
+                const float* red = xch + 2048 + 4 * fgrp * 32;  // [quadrant][token] after the group sums
+                const float v = red[lane] + red[32 + lane] + red[64 + lane] + red[96 + lane];
+                gpart[((bh * N + i) * (K / 128) + kh) * C + tlo + lane] = v;
+            }
         }
         if (issuer) bulk_wait_read_all();  // the stores finish on their own; the CTA may exit once they have read smem
     }
@@ -550,31 +619,47 @@ bool map_f32_tile(CUtensorMap* m, const void* base, uint64_t inner, uint64_t row
 constexpr size_t kSmem = 1024 + KH_OFF + 2 * PIECE + sizeof(BwdBars);
 static_assert(kSmem <= 232448, "shared memory");
 
-}  // namespace
-
-gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
-                               const void* v, const __nv_bfloat16* Qt, const float* gam, const __nv_bfloat16* Sbuf,
-                               const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, cudaStream_t s) {
-    CUtensorMap m[10];
-    memset(m, 0, sizeof(m));
-    const uint64_t L = uint64_t(p.L), K = uint64_t(p.K), V = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
-    if (!(map_sw128(&m[0], dO, V, L, BH) && map_sw128(&m[1], v, V, L, BH) && map_sw128(&m[2], Sbuf, V, K, BH * N) &&
-          map_sw128(&m[3], Dbuf, V, K, BH * N) && map_sw128(&m[4], Qt, K, L, BH) && map_sw128(&m[5], q, K, L, BH) &&
-          map_sw128(&m[6], k, K, L, BH) && map_sw128(&m[7], dq, K, L, BH, 32) && map_sw128(&m[8], dk, K, L, BH, 32) &&
-          map_f32_tile(&m[9], la, K, L, BH)))
-        return GLA_ERR_CUDA;
-    if (cudaFuncSetAttribute(k_bwd_chunk, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
+template <int GK>
+gla_status launch_bwd_gk(const Problem& p, const CUtensorMap* m, const void* q, const void* k, const GateArgs& ga,
+                         const float* gam, void* dq, void* dk, float* dla, float* gpart, cudaStream_t s) {
+    auto fn = k_bwd_chunk<GK>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.K / 128), unsigned(p.BH));
     // one CTA per SM: stagger the first wave only when there are later waves for it to shape
     const int64_t sms = sm_count();
     const uint32_t stagger = int64_t(grid.x) * grid.y * grid.z > sms ? kStaggerNs : 0u;
-    GLA_LAUNCH_PDL("tc_bwd_chunk", k_bwd_chunk, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7],
-               m[8], m[9],
-               static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), la, gam,
-               static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, p.L, p.N, p.K, p.V, stagger,
-               unsigned(sms), device_error_word());
+    GLA_LAUNCH_PDL("tc_bwd_chunk", fn, grid, kThreads, kSmem, s, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], m[8],
+                   m[9], static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k), ga, gam,
+                   static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk), dla, gpart, p.L, p.N, p.K, p.V,
+                   stagger, unsigned(sms), device_error_word());
     return GLA_OK;
+}
+
+}  // namespace
+
+gla_status tc_bwd_chunk_launch(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
+                               const void* v, const __nv_bfloat16* Qt, const float* gam, const __nv_bfloat16* Sbuf,
+                               const __nv_bfloat16* Dbuf, void* dq, void* dk, float* dla, float* gpart,
+                               cudaStream_t s) {
+    CUtensorMap m[10];
+    memset(m, 0, sizeof(m));
+    const uint64_t L = uint64_t(p.L), K = uint64_t(p.K), V = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
+    const bool sk = p.gate == kGateScalar || p.gate == kGateHead;
+    // scalar gate kinds: the intra dK~ product takes the raw q tile (decay in the dP weights), and there
+    // is no per-channel gate tile (its map is never used; any valid descriptor stands in)
+    if (!(map_sw128(&m[0], dO, V, L, BH) && map_sw128(&m[1], v, V, L, BH) && map_sw128(&m[2], Sbuf, V, K, BH * N) &&
+          map_sw128(&m[3], Dbuf, V, K, BH * N) && map_sw128(&m[4], sk ? q : static_cast<const void*>(Qt), K, L, BH) &&
+          map_sw128(&m[5], q, K, L, BH) && map_sw128(&m[6], k, K, L, BH) && map_sw128(&m[7], dq, K, L, BH, 32) &&
+          map_sw128(&m[8], dk, K, L, BH, 32) && (sk ? map_sw128(&m[9], k, K, L, BH) : map_f32_tile(&m[9], la, K, L, BH))))
+        return GLA_ERR_CUDA;
+    const GateArgs ga{la, p.gate, p.inv_tau, p.H};
+    switch (p.gate) {
+        case kGateScalar: return launch_bwd_gk<kGateScalar>(p, m, q, k, ga, gam, dq, dk, dla, gpart, s);
+        case kGateHead: return launch_bwd_gk<kGateHead>(p, m, q, k, ga, gam, dq, dk, dla, gpart, s);
+        case kGatePreact: return launch_bwd_gk<kGatePreact>(p, m, q, k, ga, gam, dq, dk, dla, gpart, s);
+        default: return launch_bwd_gk<kGateChannel>(p, m, q, k, ga, gam, dq, dk, dla, gpart, s);
+    }
 }
 
 }  // namespace gla

@@ -47,7 +47,7 @@
 extern "C" {
 #endif
 
-#define GLA_ABI_VERSION 1
+#define GLA_ABI_VERSION 2
 
 typedef enum gla_status {
     GLA_OK = 0,
@@ -78,11 +78,36 @@ typedef enum gla_impl {
     GLA_IMPL_TC = 2     /* bf16 tensor-core kernels (tcgen05/TMEM/TMA)         */
 } gla_impl;
 
+/* What the `log_a` argument of every entry point holds, and what the
+ * backward returns in `dlog_a`. The pages compare the per-channel gate with
+ * two coarser decays ("Measured effects" ablations of "Gated Linear Attention
+ * Transformers with Hardware-Efficient Training", atlas.scime.ai summary): a
+ * decay that depends on the data but is one scalar per head and step, and a
+ * fixed decay per head that does not depend on the data. The "Approach"
+ * section makes the gate a function of the input; GLA_GATE_PREACT takes that
+ * function's argument and applies it inside the kernels.
+ *   kind                log_a (fwd/bwd)   log_a (step)   dlog_a (bwd)
+ *   GLA_GATE_CHANNEL    [B,H,L,Dk]        [B,H,Dk]       [B,H,L,Dk] dL/dlog_a
+ *   GLA_GATE_SCALAR     [B,H,L]           [B,H]          [B,H,L]    dL/dlog_a (summed over channels)
+ *   GLA_GATE_HEAD       [H]               [H]            [H]        dL/dlog_a (summed over b, t, channels)
+ *   GLA_GATE_PREACT     z [B,H,L,Dk]      z [B,H,Dk]     [B,H,L,Dk] dL/dz
+ * CHANNEL, SCALAR and HEAD take log alpha itself (finite, <= 0). PREACT takes
+ * any finite z and uses log alpha = logsigmoid(z) / gate_tau (gate_tau > 0),
+ * so dL/dz = dL/dlog_alpha * sigmoid(-z) / gate_tau. */
+typedef enum gla_gate {
+    GLA_GATE_CHANNEL = 0,
+    GLA_GATE_SCALAR = 1,
+    GLA_GATE_HEAD = 2,
+    GLA_GATE_PREACT = 3
+} gla_gate;
+
 /* Problem descriptor. B, H, L >= 1; Dk, Dv >= 1 (each path states its own
  * supported set and returns GLA_ERR_UNSUPPORTED outside it). chunk = 0 and
  * subchunk = 0 pick defaults; otherwise chunk must be one of 16, 32, 64, 128
  * and subchunk must divide chunk. The result does not depend on chunk or
- * subchunk beyond rounding. */
+ * subchunk beyond rounding. gate = GLA_GATE_CHANNEL and gate_tau = 0 are the
+ * per-channel gate of earlier versions of this ABI; gate_tau is read only for
+ * GLA_GATE_PREACT. */
 typedef struct gla_desc {
     int64_t B, H, L, Dk, Dv;
     int32_t dtype;      /* gla_dtype                                   */
@@ -91,6 +116,8 @@ typedef struct gla_desc {
     int32_t state_mode; /* gla_state_mode                              */
     int32_t impl;       /* gla_impl                                    */
     int32_t flags;      /* GLA_FLAG_* bits                             */
+    int32_t gate;       /* gla_gate: what log_a holds                  */
+    float gate_tau;     /* GLA_GATE_PREACT: log alpha = logsigmoid(z) / gate_tau */
 } gla_desc;
 
 /* gla_bwd: the workspace still holds what gla_fwd left in it for the same
@@ -157,6 +184,31 @@ gla_status gla_step(const gla_desc* d, const void* q, const void* k, const void*
  * the first stage of every chunkwise pass; it is exported so that it can be
  * checked and timed on its own. */
 gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, void* stream);
+
+/* ---- sequence-sharded evaluation --------------------------------------------
+ * The state recurrence is affine in the entering state, so a segment of steps
+ * maps an entering state X to diag(a) X + U, with a = exp(sum of log alpha over
+ * the segment) per key channel and U the segment's end state from a zero start
+ * (gla_fwd with h0 = NULL). Segments of one sequence held by different devices
+ * exchange (a, U) and combine them; the backward exchanges (a, W) with W the dh0
+ * of the segment's gla_bwd with dhT = NULL. The pages carry the recurrent state
+ * across training segments ("Gated Linear Attention Transformers with
+ * Hardware-Efficient Training", atlas.scime.ai summary, "Measured effects":
+ * truncated BPTT); here the segments are shards of one sequence. */
+
+/* a[B,H,Dk] = exp(sum over the descriptor's L steps of log alpha) for the
+ * gate argument log_a of kind d->gate (fp32, device). */
+gla_status gla_segment_decay(const gla_desc* d, const float* log_a, float* a, void* stream);
+
+/* Combine the summaries of G segments (one after another in a [G][BH][Dk] and
+ * U [G][BH][Dk][Dv], fp32, device):
+ *   reverse = 0: out = X_r with X_0 = init (NULL: zero), X_{g+1} = diag(a_g) X_g + U_g
+ *                (the state entering segment r);
+ *   reverse = 1: out = Y_r with Y_{G-1} = init (NULL: zero), Y_{g-1} = diag(a_g) Y_g + U_g
+ *                (the gradient arriving at the end of segment r, with U_g = W_g).
+ * init and out are [BH][Dk][Dv]; Dv must be a multiple of 4; 0 <= r < G. */
+gla_status gla_state_combine(int64_t G, int64_t BH, int64_t Dk, int64_t Dv, const float* a, const float* U,
+                             const float* init, int32_t r, int32_t reverse, float* out, void* stream);
 
 /* ---- forward without any allocation ---------------------------------------
  * The paper has no counterpart to this entry point; it exists for callers

@@ -35,7 +35,7 @@ def test_exports_every_declared_symbol(lib):
 
 
 def test_abi_version(lib):
-    assert lib.gla_abi_version() == 1
+    assert lib.gla_abi_version() == 2
 
 
 def test_status_strings(lib):
