@@ -330,10 +330,14 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
             ts.append(a.elapsed_time(b))
         return sorted(ts)[len(ts) // 2]
 
-    cases = [("gla340m_fwd", "fwd", ("materialized",)), ("long16k", "fwd+bwd", ("materialized", "nonmaterialized"))]
-    cases += [("sweep_L%d" % L, "fwd+bwd", ("materialized",)) for L in (1024, 2048, 4096, 8192, 16384)]
+    cases = [("gla340m_fwd", "fwd", ("materialized",), {}, "gla340m_fwd"),
+             ("long16k", "fwd+bwd", ("materialized", "nonmaterialized"), {}, "long16k")]
+    cases += [("sweep_L%d" % L, "fwd+bwd", ("materialized",), {}, "sweep_L%d" % L) for L in (1024, 2048, 4096, 8192, 16384)]
+    # the intra-chunk scores by two-level chunking (sub-chunks of 16) against the default single GEMM
+    cases += [("gla1p3b_fwdbwd", "fwd+bwd", ("materialized",), {"subchunk": sc}, "gla1p3b_subchunk%d" % sc)
+              for sc in (128, 16)]
     out = {}
-    for name, passes, modes in cases:
+    for name, passes, modes, extra, label in cases:
         w = WORKLOADS[name]
         inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=0, z_mean=w.z_mean, with_grad=(passes != "fwd"))
         d = {k: v.to(dev) for k, v in inp.items()}
@@ -344,12 +348,12 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
             outs = {"dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]), "dv": torch.empty_like(d["v"]),
                     "dlog_a": torch.empty_like(d["log_a"]), "dh0": torch.empty(w.B, w.H, w.K, w.V, device=dev)}
         alg = algorithmic_model(w) if passes != "fwd" else fwd_model(w)
-        entry = {"B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V, "passes": passes, "modes": {}}
+        entry = {"B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V, "passes": passes, "modes": {}, **extra}
         for mode in modes:
-            desc = gla.make_desc(w.B, w.H, w.L, w.K, w.V, w.dtype, 0, 0, mode, "auto")
+            desc = gla.make_desc(w.B, w.H, w.L, w.K, w.V, w.dtype, 0, extra.get("subchunk", 0), mode, "auto")
             ws_f, ws_b = gla.gla_fwd_workspace_size(desc), gla.gla_bwd_workspace_size(desc)
             ws = torch.empty(ws_b if passes != "fwd" else ws_f, dtype=torch.uint8, device=dev)
-            kw = dict(state_mode=mode)
+            kw = dict(state_mode=mode, **extra)
 
             def fn():
                 gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], None, o=o, hT=hT, workspace=ws, **kw)
@@ -363,9 +367,9 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
                                     "layer_roofline_frac": lr["frac"], "roofline_ms": lr["roofline_ms"],
                                     "workspace_bytes": {"fwd": ws_f, "fwd+bwd": ws_b}}
             del ws
-        if with_cpu:
+        if with_cpu and not extra:
             entry["cpu_baseline"] = oracle_sample(w, passes, 16, 1024)
-        out[name] = entry
+        out[label] = entry
         del inp, d, o, hT, outs
         torch.cuda.empty_cache()
 
@@ -696,7 +700,9 @@ def main():
                 "data": "synthetic (seeded N(0,1)/sqrt(d_k) q,k,v; log_a = logsigmoid(N(0,1))/16; dO ~ N(0,1))",
                 "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V,
                            "global_batch": dp.global_batch(w.B, world), "seq_len": w.L, "chunk": C,
-                           "subchunk": sc if impl_name == "simt" else None,
+                           # sub-chunk length of the intra-chunk scores: equal to the chunk on the tensor-core
+                           # path means one GEMM per chunk (no secondary chunking); 16 is the two-level form
+                           "subchunk": sc,
                            "kernel_impl": impl_name, "state_mode": mode, "parallelism": "dp%d" % world,
                            "l2": "flushed between timed steps (512 MB write)", "step_launch": graph_note,
                            "eager_ms_per_step": round(eager_ms / args.steps, 5)},

@@ -149,7 +149,7 @@ gla_status resolve(const gla_desc* d, Problem& p) {
     if (impl == GLA_IMPL_AUTO) {
         Problem probe = p;
         probe.C = d->chunk ? d->chunk : 128;
-        probe.c = d->subchunk ? d->subchunk : 16;
+        probe.c = d->subchunk ? d->subchunk : 128;
         probe.N = (p.L + probe.C - 1) / probe.C;
         probe.impl = GLA_IMPL_TC;
         probe.state_mode = d->state_mode;
@@ -164,7 +164,7 @@ gla_status resolve(const gla_desc* d, Problem& p) {
     } else {
         if (!p.bf16) return GLA_ERR_UNSUPPORTED;
         p.C = d->chunk ? d->chunk : 128;
-        p.c = d->subchunk ? d->subchunk : 16;
+        p.c = d->subchunk ? d->subchunk : 128;  // one GEMM per chunk; 16 selects two-level chunking
         // materialised states are the faster mode on this path (the backward needs the stored states in
         // either mode); non-materialised keeps the forward's footprint free of them
         p.state_mode = d->state_mode == GLA_STATE_AUTO ? GLA_STATE_MATERIALIZED : d->state_mode;

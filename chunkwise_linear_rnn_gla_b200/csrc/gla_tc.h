@@ -13,7 +13,7 @@ namespace gla {
 __device__ __forceinline__ uint32_t tc_smem_u32(const void* p) { return tc::smem_u32(p); }
 
 constexpr int kTcChunk = 128;  // C on the tensor-core path
-constexpr int kTcSub = 16;     // secondary chunk c
+constexpr int kTcSub = 128;    // secondary chunk c: the default, one GEMM per chunk (16: two-level)
 constexpr int kTcBV = 64;      // value columns per walk CTA
 
 // Chunk-parallel gate preparation (gla_tc_prep.cu): Q~, K~, e^Gamma and the
@@ -21,6 +21,10 @@ constexpr int kTcBV = 64;      // value columns per walk CTA
 // `la` is the gate argument of kind `gate_kind` (gla_gate.cuh): the kernel reads every kind natively.
 gla_status tc_prep_launch(const Problem& p, const void* q, const void* k, const float* la, __nv_bfloat16* Qt,
                           __nv_bfloat16* Kt, __nv_bfloat16* P, float* gam, int gate_kind, cudaStream_t s);
+
+// Two-level intra-chunk scores (gla_tc_twolevel.cu), sub-chunk length 16: overwrites P.
+gla_status tc_intra_twolevel_launch(const Problem& p, const void* q, const void* k, const float* la,
+                                    __nv_bfloat16* P, cudaStream_t s);
 
 // Row-gated chunk walk (gla_tc_walk.cu). State X [K x 64-column tile] with the
 // gate on its rows. Per chunk i (in walk order):

@@ -55,11 +55,17 @@ TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
     return b;
 }
 
+// Sub-chunk length 16 with a per-channel gate: the intra-chunk scores by two-level chunking (the
+// scalar kinds' scores are exact decay-weighted products already).
+bool two_level(const Problem& p) {
+    return p.c == 16 && (p.gate == GLA_GATE_CHANNEL || p.gate == GLA_GATE_PREACT);
+}
+
 }  // namespace
 
 bool tc_supported(const Problem& p) {
     if (!p.bf16) return false;
-    if (p.C != kTcChunk || p.c != kTcSub) return false;
+    if (p.C != kTcChunk || (p.c != kTcSub && p.c != 16)) return false;
     if (p.K != 128 && p.K != 256) return false;
     if (p.V < 64 || p.V % 64 != 0 || p.V / 64 > 65535) return false;
     if (p.BH > 65535 || p.N > 65535) return false;
@@ -86,6 +92,7 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
     TcBuffers b = carve(p, ws, false);
     if (ws.used > ws.cap) return GLA_ERR_WORKSPACE;
     gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, p.gate, s);
+    if (st == GLA_OK && two_level(p)) st = tc_intra_twolevel_launch(p, q, k, la, b.P, s);
     if (st != GLA_OK) return st;
     WalkArgs a{};
     a.A1 = b.Kt;
@@ -125,6 +132,7 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
     gla_status st;
     if (!reuse) {
         st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, p.gate, s);
+        if (st == GLA_OK && two_level(p)) st = tc_intra_twolevel_launch(p, q, k, la, b.P, s);
         if (st != GLA_OK) return st;
     }
     if (!(reuse && p.state_mode == GLA_STATE_MATERIALIZED)) {

@@ -292,8 +292,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // scalar gate kinds have no range bound: their intra terms are weighted by the decay in fp32
         const bool safe = scalar_kind(GK) || gam[(bh * N + i) * K + chg] >= kSafeGam;
         const int64_t rb = (bh * L + t0) * K + chg;
-        // log alpha of token t (< nvalid) of this thread's channel, for the exact path
-        auto gate_t = [&](int t) -> float { return la_floor(gate_log_alpha(ga, bh, t0 + t, chg, L, K)); };
+        // log alpha of token t (< nvalid) of this thread's channel, for the exact path (per-channel kinds)
+        const float* lap = ga.g + rb;
+        auto gate_t = [&](int t) -> float {
+            const float x = lap[int64_t(t) * K];
+            return la_floor(GK == kGatePreact ? logsigmoid_f(x) * ga.inv_tau : x);
+        };
         if (row_warp) {
             // x_c = sum_v D_i[c,v] S_[i][c,v] from the staged tiles
             float x = 0.f;
@@ -378,8 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                             lv[r] = t < nvalid ? la_floor(GK == kGateScalar ? ga.g[bh * L + t0 + t] : ga.g[bh % ga.H])
                                                : 0.f;
                         } else {
-                            const float x = sLA[t * C + c];  // zero past the end of the sequence (TMA fill)
-                            lv[r] = t < nvalid ? la_floor(GK == kGatePreact ? logsigmoid_f(x) * ga.inv_tau : x) : 0.f;
+                            // zero past the end of the sequence (TMA fill): a zero log alpha, except that the
+                            // pre-activation's zero must be masked explicitly
+                            const float x = sLA[t * C + c];
+                            if (GK == kGatePreact) lv[r] = t < nvalid ? la_floor(logsigmoid_f(x) * ga.inv_tau) : 0.f;
+                            else lv[r] = la_floor(x);
                             kv[r] = __bfloat162float(
                                 *reinterpret_cast<const __nv_bfloat16*>(base + KH_OFF + tile_off(t, c)));
                         }
@@ -556,7 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int f = 0; f < 4; ++f) carry += xch[128 * f + c] + (f > fgrp ? xch[512 + 128 * f + c] : 0.f);
             float dv[32];
 #pragma unroll
-            for (int u = 0; u < 32; ++u) dv[u] = tlo + u < nvalid ? rbuf[(tlo + u) * C + c] + carry : 0.f;
+            for (int u = 0; u < 32; ++u) {
+                dv[u] = rbuf[(tlo + u) * C + c] + carry;
+                if (scalar_kind(GK) && tlo + u >= nvalid) dv[u] = 0.f;  // rows past the end add nothing
+            }
             if (scalar_kind(GK)) {
                 // sum over this CTA's 128 channels per token: across the warp's 32 lanes by a butterfly that
                 // leaves token tlo + l's sum in lane l, then over the group's 4 warps in fixed order

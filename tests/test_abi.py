@@ -55,10 +55,10 @@ def test_resolve_defaults(lib):
     assert lib.gla_resolve(ctypes.byref(desc(dtype=0)), ctypes.byref(c), ctypes.byref(sc), ctypes.byref(im),
                            ctypes.byref(sm)) == 0
     assert (c.value, sc.value, im.value) == (64, 16, 1)  # fp32 -> CUDA-core path, chunk 64, sub-chunks of 16
-    # bf16 at a tensor-core shape -> tensor-core path, C = 128, c = 16, materialised states
+    # bf16 at a tensor-core shape -> tensor-core path, C = 128, one sub-chunk per chunk (single GEMM), materialised
     assert lib.gla_resolve(ctypes.byref(desc(dtype=1, Dk=256, Dv=512, L=2048)), ctypes.byref(c), ctypes.byref(sc),
                            ctypes.byref(im), ctypes.byref(sm)) == 0
-    assert (c.value, sc.value, im.value, sm.value) == (128, 16, 2, 1)
+    assert (c.value, sc.value, im.value, sm.value) == (128, 128, 2, 1)
 
 
 @pytest.mark.parametrize("bad", [dict(B=0), dict(L=0), dict(Dk=0), dict(dtype=7), dict(chunk=48), dict(chunk=-1),

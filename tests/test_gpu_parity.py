@@ -509,3 +509,50 @@ def test_single_zero_gate_mid_chunk(impl):
     kw = dict(state_mode="materialized") if impl == "tc" else {}
     check_fwd(inp, dt, impl, **kw)
     check_bwd(inp, dt, impl, **kw)
+
+
+# ------------------------------------ two-level (secondary) chunking on the tensor-core path
+@pytest.mark.parametrize("shape", [(1, 2, 129, 128, 64), (1, 1, 300, 256, 128), (2, 2, 512, 128, 64)])
+def test_tc_two_level_intra_chunks(shape):
+    """Sub-chunk length 16 on the tensor-core path: off-diagonal 16-row blocks as bf16 tcgen05 GEMMs
+    with both factors rescaled to <= 1 against each key sub-chunk's last row, diagonal blocks in fp32
+    log space; forward and backward against the oracle, with strong gates, a zero gate and ragged L."""
+    B, H, L, K, V = shape
+    inp = make_inputs(B, H, L, K, V, "bf16", seed=L + K + 7, h0=True, dhT=True, gate_scale=1.0)
+    inp["log_a"][0, 0, L // 2, : K // 2] = -1e30
+    check_fwd(inp, "bf16", "tc", subchunk=16)
+    check_bwd(inp, "bf16", "tc", subchunk=16)
+
+
+def _straddling_gates(B, H, L, K, seed):
+    """Gates whose decay over a 128-step chunk, Gamma_c, is spread over [-70, -58] across the key
+    channels: both sides of the -64 bound of the single-GEMM form."""
+    g = torch.Generator().manual_seed(seed)
+    target = -58.0 - 12.0 * torch.rand(B, H, 1, K, generator=g)  # chunk decay per channel
+    jitter = 1.0 + 0.5 * (torch.rand(B, H, L, K, generator=g) - 0.5)
+    return (target / 128.0 * jitter).float().contiguous()
+
+
+def test_two_level_vs_single_gemm_accuracy():
+    """The accuracy side of the comparison of the two intra-chunk forms on the 1.3B layer shape (one
+    batch row): gates straddling the single-GEMM form's range bound. Both forms meet the tolerance;
+    the errors against the oracle are printed for the comparison table."""
+    w = WORKLOADS["gla1p3b_fwdbwd"]
+    B, H, L, K, V = 1, w.H, w.L, w.K, w.V
+    inp = make_inputs(B, H, L, K, V, "bf16", seed=70, with_grad=True)
+    inp["log_a"] = _straddling_gates(B, H, L, K, seed=71)
+    o_ref, hT_ref = oracle_fwd(inp)
+    ref = oracle_bwd(inp)
+    d = to_dev(inp)
+    errs = {}
+    for sc in (128, 16):
+        o, hT = run_fwd(d, "tc", subchunk=sc)
+        g = run_bwd(d, "tc", subchunk=sc)
+        e = {"o": compare("o (subchunk %d)" % sc, o, o_ref, "bf16"),
+             "hT": compare("hT (subchunk %d)" % sc, hT, hT_ref, "bf16")}
+        for n in ("dq", "dk", "dv", "dlog_a", "dh0"):
+            e[n] = compare("%s (subchunk %d)" % (n, sc), g[n], ref[n], "bf16")
+        errs[sc] = e
+    print("\nmax |gpu - oracle| / max |oracle| with straddling gates:")
+    for sc, e in errs.items():
+        print("  subchunk %3d: " % sc + "  ".join("%s %.3e" % kv for kv in e.items()))
