@@ -147,12 +147,13 @@ def layer_roofline(alg_bytes, alg_flops, ms, peaks):
 # ncu capture of the default workload, with the SHA-1 of the kernel's source
 # file at capture time: a kernel whose source changed since reports null.
 NCU_TRAFFIC = {
-    "tc_prep": (74336256, "gla_tc_prep.cu", "13e8d173e1ef24a6ea33660af099850d6e98cfaf"),
-    "tc_walk_states": (82829568, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
-    "tc_output": (135306240, "gla_tc_out.cu", "285ea49a1a538d922b569c6ed2e3ad1ab5af4341"),
-    "tc_walk_dstates": (75097600, "gla_tc_states.cu", "bb8f83f1545289b859a5164c6b67cdc98e708734"),
-    "tc_output_dv": (132920832, "gla_tc_out.cu", "285ea49a1a538d922b569c6ed2e3ad1ab5af4341"),
-    "tc_bwd_chunk": (327452160, "gla_tc_bwd.cu", "4ebf7e129f463e33f6887504e06f27e8599c0b35"),
+    "tc_prep": (74451200, "gla_tc_prep.cu", "50bba1f6b1363e821086631a7d2d5c1d3a961acc"),
+    "tc_walk_states": (82471424, "gla_tc_states.cu", "2412bcc17a256403d58ee52850586d71ceeb4601"),
+    "tc_output": (132055552, "gla_tc_out.cu", "285ea49a1a538d922b569c6ed2e3ad1ab5af4341"),
+    "tc_walk_dstates": (72099328, "gla_tc_states.cu", "2412bcc17a256403d58ee52850586d71ceeb4601"),
+    "tc_output_dv": (132318208, "gla_tc_out.cu", "285ea49a1a538d922b569c6ed2e3ad1ab5af4341"),
+    "tc_bwd_chunk": (331208960, "gla_tc_bwd.cu", "7a225b8667dab37de39518c25b00451539497f35"),
+    "tc_intra_twolevel": (68345344, "gla_tc_twolevel.cu", "a3457917f64458551c35f0e9c74e355a0ad1a3a5"),
 }
 
 
@@ -451,6 +452,9 @@ def main():
     ap.add_argument("--workload", default="gla1p3b_fwdbwd")
     ap.add_argument("--kernel-impl", default="auto", choices=["auto", "simt", "tc"])
     ap.add_argument("--state-mode", default="materialized", choices=["auto", "materialized", "nonmaterialized"])
+    ap.add_argument("--subchunk", type=int, default=0,
+                    help="sub-chunk length of the intra-chunk scores (0: the default single GEMM per chunk; "
+                         "16: two-level chunking on the tensor-core path)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the timing of the other named workloads and the decode workload")
@@ -502,14 +506,14 @@ def main():
 
     inp = make_inputs(w.B, w.H, w.L, w.K, w.V, w.dtype, seed=dp.shard_seed(0, rank))
     d = {k: v.to(dev) for k, v in inp.items()}
-    desc = gla.make_desc(w.B, w.H, w.L, w.K, w.V, w.dtype, 0, 0, args.state_mode, args.kernel_impl)
+    desc = gla.make_desc(w.B, w.H, w.L, w.K, w.V, w.dtype, 0, args.subchunk, args.state_mode, args.kernel_impl)
     C, sc, impl_name, mode = gla.gla_resolve(desc)
     ws = torch.empty(gla.gla_bwd_workspace_size(desc), dtype=torch.uint8, device=dev)
     o = torch.empty_like(d["v"])
     hT = torch.empty(w.B, w.H, w.K, w.V, dtype=torch.float32, device=dev)
     outs = {"dq": torch.empty_like(d["q"]), "dk": torch.empty_like(d["k"]), "dv": torch.empty_like(d["v"]),
             "dlog_a": torch.empty_like(d["log_a"]), "dh0": torch.empty(w.B, w.H, w.K, w.V, device=dev)}
-    kw = dict(impl=args.kernel_impl, state_mode=args.state_mode)
+    kw = dict(impl=args.kernel_impl, state_mode=args.state_mode, subchunk=args.subchunk)
 
     def step():
         gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], None, o=o, hT=hT, workspace=ws, **kw)

@@ -22,6 +22,7 @@ from . import _lib
 from ._lib import GlaDesc, GlaError, load  # noqa: F401
 
 __all__ = ["gla_fwd", "gla_bwd", "gla_step", "gla_chunk_cumsum", "gla_fwd_workspace_size", "gla_last_device_error",
+           "gla_fwd_final_state", "gla_bwd_initial_grad",
            "gla_bwd_workspace_size", "gla_resolve", "gla_check_device_error", "gla_launch_count",
            "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset",
            "make_desc", "GlaError"]
@@ -225,6 +226,55 @@ def gla_bwd(q, k, v, log_a, dO, h0=None, dhT=None, *, chunk=0, subchunk=0, state
     if checks:
         _finish_checks(guards, "gla_bwd")
     return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dh0": dh0}
+
+
+def gla_fwd_final_state(q, k, v, log_a, h0=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto",
+                        hT=None, workspace=None, gate="channel", tau=0.0):
+    """hT of gla_fwd without o (tensor-core path; GlaError GLA_ERR_UNSUPPORTED elsewhere)."""
+    load()
+    dev = q.device
+    B, H, L, Dk = q.shape
+    Dv = v.shape[-1]
+    _need(k, "k", q.shape, q.dtype, dev)
+    _need(v, "v", (B, H, L, Dv), q.dtype, dev)
+    _need(log_a, "log_a", gate_shape(gate, B, H, L, Dk), torch.float32, dev)
+    if h0 is not None:
+        _need(h0, "h0", (B, H, Dk, Dv), torch.float32, dev)
+    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, 0, gate, tau)
+    if hT is None:
+        hT = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+    _need(hT, "hT", (B, H, Dk, Dv), torch.float32, dev)
+    ws, nbytes = _workspace(gla_fwd_workspace_size(desc), dev, workspace)
+    with torch.cuda.device(dev):
+        st = load().gla_fwd_final_state(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(h0),
+                                        _ptr(hT), _ptr(ws), nbytes, _stream(dev))
+    _check(st, "gla_fwd_final_state")
+    return hT
+
+
+def gla_bwd_initial_grad(q, k, v, log_a, dO, dhT=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto",
+                         dh0=None, workspace=None, gate="channel", tau=0.0):
+    """dh0 of gla_bwd without the other gradients (tensor-core path; GlaError GLA_ERR_UNSUPPORTED
+    elsewhere). v only gives the value width."""
+    load()
+    dev = q.device
+    B, H, L, Dk = q.shape
+    Dv = v.shape[-1]
+    _need(k, "k", q.shape, q.dtype, dev)
+    _need(log_a, "log_a", gate_shape(gate, B, H, L, Dk), torch.float32, dev)
+    _need(dO, "dO", (B, H, L, Dv), q.dtype, dev)
+    if dhT is not None:
+        _need(dhT, "dhT", (B, H, Dk, Dv), torch.float32, dev)
+    desc = _desc_from(q, v, chunk, subchunk, state_mode, impl, 0, gate, tau)
+    if dh0 is None:
+        dh0 = torch.empty(B, H, Dk, Dv, dtype=torch.float32, device=dev)
+    _need(dh0, "dh0", (B, H, Dk, Dv), torch.float32, dev)
+    ws, nbytes = _workspace(gla_bwd_workspace_size(desc), dev, workspace)
+    with torch.cuda.device(dev):
+        st = load().gla_bwd_initial_grad(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(log_a), _ptr(dO), _ptr(dhT),
+                                         _ptr(dh0), _ptr(ws), nbytes, _stream(dev))
+    _check(st, "gla_bwd_initial_grad")
+    return dh0
 
 
 def gla_step(q, k, v, log_a, S, o=None, checks=False, gate="channel", tau=0.0):

@@ -14,6 +14,7 @@ LIB_PATH = os.path.join(HERE, "libgla_checks.so" if os.environ.get("GLA_CHECKS")
 
 GLA_OK = 0
 GLA_ERR_INVALID_ARG = 1
+GLA_ERR_UNSUPPORTED = 2
 GLA_ERR_WORKSPACE = 3
 GLA_ERR_TIMEOUT = 5
 STATUS_NAMES = {0: "GLA_OK", 1: "GLA_ERR_INVALID_ARG", 2: "GLA_ERR_UNSUPPORTED", 3: "GLA_ERR_WORKSPACE",
@@ -31,7 +32,7 @@ EXPORTS = (
     "gla_check_device_error", "gla_status_string", "gla_abi_version", "gla_resolve", "gla_launch_count",
     "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset", "gla_fwd_noalloc",
     "gla_selftest_wait_timeout", "gla_last_device_error", "gla_fwd_workspace_bytes", "gla_bwd_workspace_bytes",
-    "gla_segment_decay", "gla_state_combine",
+    "gla_segment_decay", "gla_state_combine", "gla_fwd_final_state", "gla_bwd_initial_grad",
 )
 
 
@@ -93,6 +94,10 @@ def _declare(lib):
     lib.gla_profile_reset.restype = None
     lib.gla_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp]
     lib.gla_fwd_noalloc.restype = ctypes.c_int
+    lib.gla_fwd_final_state.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gla_fwd_final_state.restype = ctypes.c_int
+    lib.gla_bwd_initial_grad.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gla_bwd_initial_grad.restype = ctypes.c_int
     lib.gla_segment_decay.argtypes = [dp, vp, vp, vp]
     lib.gla_segment_decay.restype = ctypes.c_int
     i64 = ctypes.c_int64

@@ -438,6 +438,42 @@ gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, 
     return gla::simt_chunk_cumsum(p, log_a, Bcum, static_cast<cudaStream_t>(stream));
 }
 
+gla_status gla_fwd_final_state(const gla_desc* d, const void* q, const void* k, const void* v, const float* log_a,
+                               const float* h0, float* hT, void* workspace, size_t workspace_bytes, void* stream) {
+    Problem p{};
+    gla_status st = resolve(d, p);
+    if (st != GLA_OK) return st;
+    if (p.impl != GLA_IMPL_TC || p.state_mode != GLA_STATE_MATERIALIZED) return GLA_ERR_UNSUPPORTED;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(v);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(hT);
+    GLA_OPTIONAL_PTR(h0);
+    st = check_ws(workspace, workspace_bytes, fwd_ws(p));
+    if (st != GLA_OK) return st;
+    gla::Arena a = gla::make_arena(p, workspace, workspace_bytes);
+    return gla::tc_fwd_final_state(p, q, k, v, log_a, h0, hT, a, static_cast<cudaStream_t>(stream));
+}
+
+gla_status gla_bwd_initial_grad(const gla_desc* d, const void* q, const void* k, const float* log_a, const void* dO,
+                                const float* dhT, float* dh0, void* workspace, size_t workspace_bytes, void* stream) {
+    Problem p{};
+    gla_status st = resolve(d, p);
+    if (st != GLA_OK) return st;
+    if (p.impl != GLA_IMPL_TC || p.state_mode != GLA_STATE_MATERIALIZED) return GLA_ERR_UNSUPPORTED;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(dO);
+    GLA_REQUIRE_PTR(dh0);
+    GLA_OPTIONAL_PTR(dhT);
+    st = check_ws(workspace, workspace_bytes, bwd_ws(p));
+    if (st != GLA_OK) return st;
+    gla::Arena a = gla::make_arena(p, workspace, workspace_bytes);
+    return gla::tc_bwd_initial_grad(p, q, k, log_a, dO, dhT, dh0, a, static_cast<cudaStream_t>(stream));
+}
+
 gla_status gla_segment_decay(const gla_desc* d, const float* log_a, float* a, void* stream) {
     Problem p{};
     gla_status st = resolve(d, p);

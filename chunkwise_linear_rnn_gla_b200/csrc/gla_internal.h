@@ -113,6 +113,12 @@ size_t tc_bwd_workspace(const Problem& p);
 void tc_layout(const Problem& p, Arena& a, bool bwd);
 gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
                   const float* h0, void* o, float* hT, Arena& ws, cudaStream_t s);
+// Only the end state of a forward (prep and a walk that stores nothing), and only the gradient at the
+// entering state of a backward (prep and the reverse walk): the summaries of sequence-sharded evaluation.
+gla_status tc_fwd_final_state(const Problem& p, const void* q, const void* k, const void* v, const float* la,
+                              const float* h0, float* hT, Arena& ws, cudaStream_t s);
+gla_status tc_bwd_initial_grad(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
+                               const float* dhT, float* dh0, Arena& ws, cudaStream_t s);
 gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* log_a,
                   const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
                   float* dlog_a, float* dh0, Arena& ws, cudaStream_t s);

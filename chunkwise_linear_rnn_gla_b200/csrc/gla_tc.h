@@ -92,6 +92,11 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
                                  const float* init, float* fin, float* fin2, __nv_bfloat16* states, float* segbuf,
                                  bool reverse, cudaStream_t s, const char* name);
 
+// The final state of the walk only (nothing stored; few heads: parallel segments and a scan).
+gla_status tc_states_walk_final(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
+                                const float* init, float* fin, float* segbuf, bool reverse, cudaStream_t s,
+                                const char* name);
+
 // Chunk-parallel Y_i = A_i X_i + Pm_i B_i from stored bf16 chunk states X
 // (gla_tc_out.cu): forward o (A = Q~, Pm = P) and dv (A = K~, Pm = P^T).
 // late_wait: the kernel follows, by programmatic dependent launch, a kernel that it does not

@@ -123,6 +123,26 @@ gla_status tc_fwd(const Problem& p, const void* q, const void* k, const void* v,
                                static_cast<__nv_bfloat16*>(o), false, s, "tc_output");
 }
 
+gla_status tc_fwd_final_state(const Problem& p, const void* q, const void* k, const void* v, const float* la,
+                              const float* h0, float* hT, Arena& ws, cudaStream_t s) {
+    TcBuffers b = carve(p, ws, false);
+    if (ws.used > ws.cap) return GLA_ERR_WORKSPACE;
+    gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, p.gate, s);
+    if (st != GLA_OK) return st;
+    return tc_states_walk_final(p, b.Kt, static_cast<const __nv_bfloat16*>(v), b.gam, h0, hT, b.segbuf, false, s,
+                                "tc_walk_final");
+}
+
+gla_status tc_bwd_initial_grad(const Problem& p, const void* q, const void* k, const float* la, const void* dO,
+                               const float* dhT, float* dh0, Arena& ws, cudaStream_t s) {
+    TcBuffers b = carve(p, ws, true);
+    if (ws.used > ws.cap) return GLA_ERR_WORKSPACE;
+    gla_status st = tc_prep_launch(p, q, k, la, b.Qt, b.Kt, b.P, b.gam, p.gate, s);
+    if (st != GLA_OK) return st;
+    return tc_states_walk_final(p, b.Qt, static_cast<const __nv_bfloat16*>(dO), b.gam, dhT, dh0, b.segbuf, true, s,
+                                "tc_walk_dfinal");
+}
+
 gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v, const float* la, const float* h0,
                   const void* dO, const float* dhT, void* dq, void* dk, void* dv, float* dla, float* dh0, Arena& ws,
                   cudaStream_t s) {

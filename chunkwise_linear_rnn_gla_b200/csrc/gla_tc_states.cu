@@ -389,6 +389,25 @@ gla_status tc_states_walk_launch(const Problem& p, const __nv_bfloat16* A, const
     return st;
 }
 
+gla_status tc_states_walk_final(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
+                                const float* init, float* fin, float* segbuf, bool reverse, cudaStream_t s,
+                                const char* name) {
+    CUtensorMap m[3];
+    // nothing is stored: the states map only has to be a valid descriptor
+    if (!make_maps(m, p, A, B, A)) return GLA_ERR_CUDA;
+    const WalkPlan w = walk_plan(p, p.BH * (p.K / 128) * (p.V / 64), segbuf != nullptr);
+    if (w.G == 1)
+        return launch_states(p, m, w.wide, reverse, gam, init, fin, nullptr, nullptr,
+                             WalkSegs{0, int(p.N), -1, 0, nullptr}, 1, s, name);
+    const int64_t stride = p.BH * p.K * p.V;
+    float* E = segbuf;
+    float* S_in = segbuf + int64_t(kMaxSegs) * stride;
+    gla_status st = launch_states(p, m, w.wide, reverse, gam, init, E, nullptr, nullptr,
+                                  WalkSegs{0, w.len, -1, stride, nullptr}, w.G, s, name);
+    if (st == GLA_OK) st = launch_seg_scan(p, reverse, E, gam, S_in, fin, nullptr, w.G, w.len, s);
+    return st;
+}
+
 int tc_walk_seg_prepare(const Problem& p, const __nv_bfloat16* A, const __nv_bfloat16* B, const float* gam,
                         const float* init, float* fin, float* fin2, float* segbuf, bool reverse, cudaStream_t s,
                         int* len, const float** S_in_out, int64_t* stride_out, gla_status* st) {

@@ -16,9 +16,10 @@ Attention Transformers with Hardware-Efficient Training", atlas.scime.ai
 summary, "Measured effects": truncated BPTT over 2K segments); here the
 segments are shards of one sequence on different devices.
 
-Every arithmetic step runs in the library's kernels (gla_fwd, gla_bwd,
-gla_segment_decay, gla_state_combine); this module moves tensors and calls the
-collective. The phases are separate functions so that a caller (or a test) can
+Every arithmetic step runs in the library's kernels (gla_fwd_final_state and
+gla_bwd_initial_grad for the summaries where the tensor-core path serves them,
+else gla_fwd and gla_bwd; gla_segment_decay; gla_state_combine); this module
+moves tensors and calls the collective. The phases are separate functions so that a caller (or a test) can
 run several shards on one device in turn.
 """
 from __future__ import annotations
@@ -28,7 +29,7 @@ from typing import Callable, List, Optional, Sequence
 
 import torch
 
-from . import _lib, gla_bwd, gla_fwd, gate_shape, make_desc
+from . import _lib, gla_bwd, gla_bwd_initial_grad, gla_fwd, gla_fwd_final_state, gate_shape, make_desc
 from ._lib import load
 
 __all__ = ["segment_decay", "state_combine", "summary_fwd", "finish_fwd", "summary_bwd", "finish_bwd",
@@ -83,9 +84,15 @@ def state_combine(a_all: torch.Tensor, U_all: torch.Tensor, r: int, init: Option
 
 # ---- the phases of one rank ---------------------------------------------------------------------
 def summary_fwd(q, k, v, log_a, gate="channel", tau=0.0, **kw):
-    """(a, U) of this segment: its decay and its end state from a zero start."""
+    """(a, U) of this segment: its decay and its end state from a zero start (the state walk alone where
+    the library has it, else a full forward)."""
     B, H, L, Dk = q.shape
-    _, U = gla_fwd(q, k, v, log_a, None, gate=gate, tau=tau, **kw)
+    try:
+        U = gla_fwd_final_state(q, k, v, log_a, None, gate=gate, tau=tau, **kw)
+    except _lib.GlaError as e:
+        if e.status != _lib.GLA_ERR_UNSUPPORTED:
+            raise
+        _, U = gla_fwd(q, k, v, log_a, None, gate=gate, tau=tau, **kw)
     return segment_decay(log_a, B, H, L, Dk, gate, tau), U
 
 
@@ -100,8 +107,13 @@ def summary_bwd(q, k, v, log_a, dO, gate="channel", tau=0.0, **kw):
     """(a, W) of this segment: its decay and the gradient it sends to its entering state when nothing
     arrives at its end (that gradient does not depend on the entering state)."""
     B, H, L, Dk = q.shape
-    g = gla_bwd(q, k, v, log_a, dO, None, None, gate=gate, tau=tau, **kw)
-    return segment_decay(log_a, B, H, L, Dk, gate, tau), g["dh0"]
+    try:
+        W = gla_bwd_initial_grad(q, k, v, log_a, dO, None, gate=gate, tau=tau, **kw)
+    except _lib.GlaError as e:
+        if e.status != _lib.GLA_ERR_UNSUPPORTED:
+            raise
+        W = gla_bwd(q, k, v, log_a, dO, None, None, gate=gate, tau=tau, **kw)["dh0"]
+    return segment_decay(log_a, B, H, L, Dk, gate, tau), W
 
 
 def finish_bwd(q, k, v, log_a, dO, h0_r, a_all, W_all, r, dhT=None, gate="channel", tau=0.0, **kw):

@@ -196,6 +196,21 @@ gla_status gla_chunk_cumsum(const gla_desc* d, const float* log_a, float* Bcum, 
  * Hardware-Efficient Training", atlas.scime.ai summary, "Measured effects":
  * truncated BPTT); here the segments are shards of one sequence. */
 
+/* The summaries alone, cheaper than the full passes (tensor-core path with
+ * materialised states; GLA_ERR_UNSUPPORTED otherwise, and the full pass then
+ * gives the same result):
+ *  - gla_fwd_final_state: hT of gla_fwd (h0 may be NULL) without computing o
+ *    (the preparation and a state walk that stores nothing);
+ *  - gla_bwd_initial_grad: dh0 of gla_bwd (dhT may be NULL) without the other
+ *    gradients (the preparation and the reverse walk).
+ * Workspace: as gla_fwd / gla_bwd for the same descriptor. */
+gla_status gla_fwd_final_state(const gla_desc* d, const void* q, const void* k, const void* v,
+                               const float* log_a, const float* h0, float* hT,
+                               void* workspace, size_t workspace_bytes, void* stream);
+gla_status gla_bwd_initial_grad(const gla_desc* d, const void* q, const void* k, const float* log_a,
+                                const void* dO, const float* dhT, float* dh0,
+                                void* workspace, size_t workspace_bytes, void* stream);
+
 /* a[B,H,Dk] = exp(sum over the descriptor's L steps of log alpha) for the
  * gate argument log_a of kind d->gate (fp32, device). */
 gla_status gla_segment_decay(const gla_desc* d, const float* log_a, float* a, void* stream);

@@ -175,3 +175,26 @@ def test_sequence_shards_on_one_gpu(impl, dtype, K, V):
     for n in ("dq", "dk", "dv", "dlog_a"):
         compare(n, torch.cat([g[n] for g in grads], dim=2), ref[n], dtype)
     compare("dh0", grads[0]["dh0"], ref["dh0"], dtype)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("L", [300, 128 * 20 + 37])
+def test_summary_entry_points_match_the_full_passes(L):
+    """gla_fwd_final_state / gla_bwd_initial_grad (the state walks alone) give the hT / dh0 of the full
+    gla_fwd / gla_bwd bit for bit (the same walk kernels; the long case runs the segmented walks), and
+    the oracle's."""
+    import chunkwise_linear_rnn_gla_b200 as gla
+    from tests.parity import compare, oracle_bwd, oracle_fwd
+
+    B, H, K, V = 1, 2, 128, 128
+    inp = make_inputs(B, H, L, K, V, "bf16", seed=62, h0=True, dhT=True)
+    d = {n: t.cuda() for n, t in inp.items()}
+    _, hT = gla.gla_fwd(d["q"], d["k"], d["v"], d["log_a"], d["h0"], impl="tc")
+    hT2 = gla.gla_fwd_final_state(d["q"], d["k"], d["v"], d["log_a"], d["h0"], impl="tc")
+    g = gla.gla_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d["h0"], d["dhT"], impl="tc")
+    dh02 = gla.gla_bwd_initial_grad(d["q"], d["k"], d["v"], d["log_a"], d["dO"], d["dhT"], impl="tc")
+    torch.cuda.synchronize()
+    assert torch.equal(hT, hT2)
+    assert torch.equal(g["dh0"], dh02)
+    compare("hT", hT2, oracle_fwd(inp)[1], "bf16")
+    compare("dh0", dh02, oracle_bwd(inp)["dh0"], "bf16")
