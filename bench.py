@@ -442,6 +442,15 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
     return out
 
 
+def workload_config(w, world):
+    """The workload both arms of the benchmark run (identical keys and values in both JSON lines)."""
+    from chunkwise_linear_rnn_gla_b200 import dp
+
+    return {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V,
+            "global_batch": dp.global_batch(w.B, world), "seq_len": w.L, "parallelism": "dp%d" % world,
+            "passes": w.passes, "gate": "per key channel, log alpha = logsigmoid(z)/16, z ~ N(%g, 1)" % w.z_mean}
+
+
 # --------------------------------------------------------------------- main
 def main():
     ap = argparse.ArgumentParser()
@@ -459,7 +468,7 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the timing of the other named workloads and the decode workload")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=8)
     ap.add_argument("--no-graph", action="store_true",
                     help="launch the timed step eagerly instead of replaying it from a CUDA graph")
     args = ap.parse_args()
@@ -484,7 +493,7 @@ def main():
         line = {"impl": "reference", "metric": metric, "value": cb["value"], "unit": "tokens/s", "n_gpus": args.gpus,
                 "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V},
+                "config": workload_config(w, args.gpus),
                 "cpu_baseline": cb,
                 "e2e": {"value": cb["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -608,39 +617,65 @@ def main():
     value = dp.job_throughput(w.B * w.L, world, ms_per_step)
 
     # ---------------- end to end through the public API, host buffers
+    # Every step copies its inputs from pinned host memory and reads every result back. The copies are
+    # pipelined across steps as an input pipeline would run them: step i+1's inputs go host -> device on
+    # one stream and step i-1's results device -> host on another while step i computes (PCIe carries
+    # both directions at once); inputs and outputs are double-buffered on the device and on the host.
     e2e = None
     if not args.no_e2e:
         pin = {k: v.pin_memory() for k, v in inp.items()}
-        host_out = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs.items()}
-        host_o = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        host_hT = torch.empty(hT.shape, dtype=hT.dtype, pin_memory=True)
+        outs_all = {"o": o, "hT": hT, **outs}
+        dins = [d, {k: torch.empty_like(v) for k, v in d.items()}]
+        douts = [outs_all, {k: torch.empty_like(v) for k, v in outs_all.items()}]
+        hosts = [{k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in outs_all.items()} for _ in range(2)]
         h2d = sum(v.numel() * v.element_size() for v in pin.values())
-        d2h = (sum(v.numel() * v.element_size() for v in host_out.values()) + host_o.numel() * host_o.element_size()
-               + host_hT.numel() * host_hT.element_size())
+        d2h = sum(v.numel() * v.element_size() for v in outs_all.values())
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
 
-        def e2e_step():
-            for k_, v_ in pin.items():
-                d[k_].copy_(v_, non_blocking=True)
-            step()
-            host_o.copy_(o, non_blocking=True)
-            host_hT.copy_(hT, non_blocking=True)
-            for k_, v_ in outs.items():
-                host_out[k_].copy_(v_, non_blocking=True)
+        def e2e_run(n):
+            for j in range(n):
+                b = j % 2
+                din, dout, host = dins[b], douts[b], hosts[b]
+                if j >= 2:
+                    s_in.wait_event(ev_comp[b])  # step j-2 has finished reading this input set
+                with torch.cuda.stream(s_in):
+                    for k_, v_ in pin.items():
+                        din[k_].copy_(v_, non_blocking=True)
+                    ev_in[b].record(s_in)
+                stream.wait_event(ev_in[b])
+                if j >= 2:
+                    stream.wait_event(ev_out[b])  # step j-2's results have been read out of this output set
+                gla.gla_fwd(din["q"], din["k"], din["v"], din["log_a"], None, o=dout["o"], hT=dout["hT"],
+                            workspace=ws, **kw)
+                gla.gla_bwd(din["q"], din["k"], din["v"], din["log_a"], din["dO"], None, None, workspace=ws,
+                            ws_from_fwd=True, out={n_: dout[n_] for n_ in outs}, **kw)
+                ev_comp[b].record(stream)
+                s_out.wait_event(ev_comp[b])
+                with torch.cuda.stream(s_out):
+                    for k_, v_ in dout.items():
+                        host[k_].copy_(v_, non_blocking=True)
+                    ev_out[b].record(s_out)
 
-        e2e_step()
+        e2e_run(2)
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
         a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a_.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        b_.record(stream)
+        a_.record(s_in)
+        e2e_run(args.e2e_steps)
+        s_out.wait_stream(s_in)
+        s_out.wait_stream(stream)
+        b_.record(s_out)
         torch.cuda.synchronize(dev)
         e2e_ms = dp.max_over_ranks(a_.elapsed_time(b_) / args.e2e_steps)
         e2e = {"value": dp.job_throughput(w.B * w.L, world, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d),
-               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms}
+               "d2h_bytes_per_step": int(d2h), "ms_per_step": e2e_ms,
+               "how": ("%d steps, inputs host->device and results device->host pipelined across steps on two "
+                       "copy streams, double-buffered" % args.e2e_steps)}
 
     # ---------------- roofline of the whole step (the headline) and of the dominant kernel
     peaks, peaks_src = load_peaks()
@@ -702,12 +737,12 @@ def main():
                 "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5), "higher_is_better": True,
                 "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.dtype == "bf16" else "f32",
                 "data": "synthetic (seeded N(0,1)/sqrt(d_k) q,k,v; log_a = logsigmoid(N(0,1))/16; dO ~ N(0,1))",
-                "config": {"workload": w.name, "B": w.B, "H": w.H, "L": w.L, "d_k": w.K, "d_v": w.V,
-                           "global_batch": dp.global_batch(w.B, world), "seq_len": w.L, "chunk": C,
+                "config": workload_config(w, world),
+                "impl_config": {"chunk": C,
                            # sub-chunk length of the intra-chunk scores: equal to the chunk on the tensor-core
                            # path means one GEMM per chunk (no secondary chunking); 16 is the two-level form
                            "subchunk": sc,
-                           "kernel_impl": impl_name, "state_mode": mode, "parallelism": "dp%d" % world,
+                           "kernel_impl": impl_name, "state_mode": mode,
                            "l2": "flushed between timed steps (512 MB write)", "step_launch": graph_note,
                            "eager_ms_per_step": round(eager_ms / args.steps, 5)},
                 "roofline": kroof, "layer_roofline": layer_roof, "cpu_baseline": cb,

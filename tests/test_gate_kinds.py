@@ -186,3 +186,32 @@ def test_scalar_gates_beyond_the_range_bound(kind):
     for n in ("dq", "dk", "dv", "dh0"):
         compare(n, gr[n], ref[n], "bf16")
     compare("dlog_a (%s)" % kind, gr["dlog_a"], grad_of_kind(kind, arg, ref["dlog_a"]), "bf16")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("kind", ["scalar", "head", "preact", "channel"])
+@pytest.mark.parametrize("L", [1, 131])
+def test_gate_kinds_short_and_ragged(kind, L):
+    """Every gate kind on the tensor-core path at L = 1 (one partial chunk) and a ragged L, with h0 and
+    dhT; the pre-activation and the per-channel kinds also with two-level chunking."""
+    B, H, K, V = 1, 2, 128, 64
+    inp = make_inputs(B, H, L, K, V, "bf16", seed=58 + L, h0=True, dhT=True)
+    if kind == "channel":
+        arg = inp["log_a"]
+        pc = to_f64_numpy(arg)
+    else:
+        arg, pc = gate_inputs(kind, B, H, L, K, seed=59 + L)
+    o_ref, hT_ref, ref = _oracle(inp, np.ascontiguousarray(pc))
+    d = {n: t.cuda() for n, t in inp.items()}
+    a = arg.contiguous().cuda()
+    for sc in ((0, 16) if kind in ("preact", "channel") else (0,)):
+        kw = dict(impl="tc", gate=kind, tau=TAU, subchunk=sc)
+        o, hT = gla.gla_fwd(d["q"], d["k"], d["v"], a, d["h0"], **kw)
+        g = gla.gla_bwd(d["q"], d["k"], d["v"], a, d["dO"], d["h0"], d["dhT"], **kw)
+        torch.cuda.synchronize()
+        compare("o", o, o_ref, "bf16")
+        compare("hT", hT, hT_ref, "bf16")
+        for n in ("dq", "dk", "dv", "dh0"):
+            compare(n, g[n], ref[n], "bf16")
+        compare("dlog_a (%s)" % kind, g["dlog_a"], grad_of_kind(kind, arg, ref["dlog_a"]) if kind != "channel"
+                else ref["dlog_a"], "bf16")
