@@ -20,6 +20,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "gla_oracle.c")
+_SRC_GSA = os.path.join(_HERE, "gsa_oracle.c")
 _LIB = os.path.join(_HERE, "libgla_oracle.so")
 _lock = threading.Lock()
 _lib = None
@@ -29,10 +30,11 @@ _i64 = ctypes.c_int64
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with gcc (OpenMP) into ``oracle/libgla_oracle.so``."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+    """Compile the oracle (both C files) with gcc (OpenMP) into ``oracle/libgla_oracle.so``."""
+    newest = max(os.path.getmtime(_SRC), os.path.getmtime(_SRC_GSA))
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
         tmp = _LIB + ".tmp.%d" % os.getpid()
-        cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c99", _SRC, "-o", tmp, "-lm"]
+        cmd = ["gcc", "-O2", "-fopenmp", "-shared", "-fPIC", "-std=c99", _SRC, _SRC_GSA, "-o", tmp, "-lm"]
         subprocess.run(cmd, check=True)
         os.replace(tmp, _LIB)
     return _LIB
@@ -50,6 +52,10 @@ def _load():
             lib.gla_oracle_step.restype = None
             lib.gla_oracle_bwd.argtypes = [_i64] * 5 + [_dp] * 13 + [_i64]
             lib.gla_oracle_bwd.restype = None
+            lib.gsa_oracle_fwd.argtypes = [_i64] * 6 + [_dp] * 10
+            lib.gsa_oracle_fwd.restype = None
+            lib.gsa_oracle_bwd.argtypes = [_i64] * 6 + [_dp] * 15 + [_i64]
+            lib.gsa_oracle_bwd.restype = None
             lib.gla_oracle_num_threads.restype = ctypes.c_int
             lib.gla_oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -126,3 +132,48 @@ def step(q, k, v, log_a, S):
     o = np.zeros((B, H, V))
     lib.gla_oracle_step(B, H, K, V, _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(S), _ptr(o))
     return o, S
+
+
+# ---- gated slot attention (gsa_oracle.c) ------------------------------------------------------------
+def gsa_fwd(q, k, v, log_a, hk0=None, hv0=None):
+    """Gated slot attention forward, step by step in fp64.
+
+    q, k [B,H,L,K]; v [B,H,L,V]; log_a [B,H,L,m]; hk0 [B,H,m,K], hv0 [B,H,m,V] (None = zero).
+    Returns (o [B,H,L,V], s [B,H,L,m] read weights, hkT [B,H,m,K], hvT [B,H,m,V]).
+    """
+    lib = _load()
+    q, k, v, log_a = _c(q), _c(k), _c(v), _c(log_a)
+    B, H, L, K = q.shape
+    V, m = v.shape[-1], log_a.shape[-1]
+    assert k.shape == q.shape and v.shape == (B, H, L, V) and log_a.shape == (B, H, L, m)
+    hk0c = None if hk0 is None else _c(hk0)
+    hv0c = None if hv0 is None else _c(hv0)
+    o = np.zeros((B, H, L, V))
+    s = np.zeros((B, H, L, m))
+    hkT = np.zeros((B, H, m, K))
+    hvT = np.zeros((B, H, m, V))
+    lib.gsa_oracle_fwd(B, H, L, K, V, m, _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(hk0c), _ptr(hv0c), _ptr(o),
+                       _ptr(s), _ptr(hkT), _ptr(hvT))
+    return o, s, hkT, hvT
+
+
+def gsa_bwd(q, k, v, log_a, dO, hk0=None, hv0=None, dhkT=None, dhvT=None, seg: int = 64):
+    """Reverse-mode gradients of <dO, o> + <dhkT, hkT> + <dhvT, hvT> for gated slot attention.
+
+    Returns a dict with dq, dk, dv, dlog_a, dhk0, dhv0.
+    """
+    lib = _load()
+    q, k, v, log_a, dO = _c(q), _c(k), _c(v), _c(log_a), _c(dO)
+    B, H, L, K = q.shape
+    V, m = v.shape[-1], log_a.shape[-1]
+    opt = [None if t is None else _c(t) for t in (hk0, hv0, dhkT, dhvT)]
+    dq = np.zeros((B, H, L, K))
+    dk = np.zeros((B, H, L, K))
+    dv = np.zeros((B, H, L, V))
+    dla = np.zeros((B, H, L, m))
+    dhk0 = np.zeros((B, H, m, K))
+    dhv0 = np.zeros((B, H, m, V))
+    lib.gsa_oracle_bwd(B, H, L, K, V, m, _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(opt[0]), _ptr(opt[1]),
+                       _ptr(dO), _ptr(opt[2]), _ptr(opt[3]), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(dla), _ptr(dhk0),
+                       _ptr(dhv0), int(seg))
+    return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dhk0": dhk0, "dhv0": dhv0}
