@@ -33,6 +33,7 @@ EXPORTS = (
     "gla_launch_count_reset", "gla_profile_enable", "gla_profile_read", "gla_profile_reset", "gla_fwd_noalloc",
     "gla_selftest_wait_timeout", "gla_last_device_error", "gla_fwd_workspace_bytes", "gla_bwd_workspace_bytes",
     "gla_segment_decay", "gla_state_combine", "gla_fwd_final_state", "gla_bwd_initial_grad",
+    "gla_gsa_resolve", "gla_gsa_fwd_workspace_size", "gla_gsa_bwd_workspace_size", "gla_gsa_fwd", "gla_gsa_bwd",
 )
 
 
@@ -98,6 +99,16 @@ def _declare(lib):
     lib.gla_fwd_final_state.restype = ctypes.c_int
     lib.gla_bwd_initial_grad.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.gla_bwd_initial_grad.restype = ctypes.c_int
+    lib.gla_gsa_resolve.argtypes = [dp, i32, ctypes.POINTER(i32)]
+    lib.gla_gsa_resolve.restype = ctypes.c_int
+    lib.gla_gsa_fwd_workspace_size.argtypes = [dp, i32]
+    lib.gla_gsa_fwd_workspace_size.restype = sz
+    lib.gla_gsa_bwd_workspace_size.argtypes = [dp, i32]
+    lib.gla_gsa_bwd_workspace_size.restype = sz
+    lib.gla_gsa_fwd.argtypes = [dp, i32] + [vp] * 9 + [vp, sz, vp]
+    lib.gla_gsa_fwd.restype = ctypes.c_int
+    lib.gla_gsa_bwd.argtypes = [dp, i32] + [vp] * 15 + [vp, sz, vp]
+    lib.gla_gsa_bwd.restype = ctypes.c_int
     lib.gla_segment_decay.argtypes = [dp, vp, vp, vp]
     lib.gla_segment_decay.restype = ctypes.c_int
     i64 = ctypes.c_int64

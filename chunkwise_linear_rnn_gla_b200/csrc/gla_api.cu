@@ -225,6 +225,47 @@ gla_status check_ws(void* ws, size_t bytes, size_t need) {
     return GLA_OK;
 }
 
+// The two GLA passes of gated slot attention (include/gla.h): layer one has GLA key width `slots` and
+// value width Dk, layer two key width `slots` and value width Dv. bf16 with 128 slots takes the
+// tensor-core route when both passes resolve to the tensor-core path; everything else runs both passes
+// on the CUDA-core path in fp32.
+gla_status resolve_gsa(const gla_desc* d, int32_t slots, gla::GsaProblem& g) {
+    if (!d || slots < 1) return GLA_ERR_INVALID_ARG;
+    if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
+    if (d->gate != GLA_GATE_CHANNEL) return d->gate < GLA_GATE_CHANNEL || d->gate > GLA_GATE_PREACT
+                                                ? GLA_ERR_INVALID_ARG
+                                                : GLA_ERR_UNSUPPORTED;
+    if (d->dtype != GLA_DTYPE_F32 && d->dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+    gla_desc da = *d, db = *d;
+    da.Dk = slots;
+    da.Dv = d->Dk;
+    da.flags = 0;
+    db.Dk = slots;
+    db.Dv = d->Dv;
+    db.flags = 0;
+    g.m = slots;
+    g.io_bf16 = d->dtype == GLA_DTYPE_BF16;
+    g.tc = false;
+    if (g.io_bf16 && d->impl != GLA_IMPL_SIMT && (d->subchunk == 0 || d->subchunk == 128) &&
+        d->state_mode != GLA_STATE_NONMATERIALIZED) {
+        gla_desc ta = da, tb = db;
+        ta.state_mode = tb.state_mode = GLA_STATE_MATERIALIZED;
+        gla::GsaProblem t{};
+        if (resolve(&ta, t.A) == GLA_OK && resolve(&tb, t.B) == GLA_OK && gla::gsa_tc_route(t.A, t.B, slots)) {
+            g.A = t.A;
+            g.B = t.B;
+            g.tc = true;
+            return GLA_OK;
+        }
+    }
+    if (d->impl == GLA_IMPL_TC) return GLA_ERR_UNSUPPORTED;
+    da.dtype = db.dtype = GLA_DTYPE_F32;
+    da.impl = db.impl = GLA_IMPL_SIMT;
+    gla_status st = resolve(&da, g.A);
+    if (st == GLA_OK) st = resolve(&db, g.B);
+    return st;
+}
+
 #define GLA_REQUIRE_PTR(ptr) \
     do {                     \
         if (!(ptr) || !aligned((ptr), 16)) return GLA_ERR_INVALID_ARG; \
@@ -493,6 +534,100 @@ gla_status gla_state_combine(int64_t G, int64_t BH, int64_t Dk, int64_t Dv, cons
     GLA_OPTIONAL_PTR(init);
     GLA_REQUIRE_PTR(out);
     return gla::state_combine(G, BH, Dk, Dv, a, U, init, r, reverse, out, static_cast<cudaStream_t>(stream));
+}
+
+gla_status gla_gsa_resolve(const gla_desc* d, int32_t slots, int32_t* impl) {
+    gla::GsaProblem g{};
+    const gla_status st = resolve_gsa(d, slots, g);
+    if (st == GLA_OK && impl) *impl = g.tc ? GLA_IMPL_TC : GLA_IMPL_SIMT;
+    return st;
+}
+
+size_t gla_gsa_fwd_workspace_size(const gla_desc* d, int32_t slots) {
+    gla::GsaProblem g{};
+    if (resolve_gsa(d, slots, g) != GLA_OK) return 0;
+    return gla::gsa_workspace(g, false);
+}
+
+size_t gla_gsa_bwd_workspace_size(const gla_desc* d, int32_t slots) {
+    gla::GsaProblem g{};
+    if (resolve_gsa(d, slots, g) != GLA_OK) return 0;
+    return gla::gsa_workspace(g, true);
+}
+
+gla_status gla_gsa_fwd(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
+                       const float* log_a, const float* hk0, const float* hv0, void* o, float* hkT, float* hvT,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    gla::GsaProblem g{};
+    gla_status st = resolve_gsa(d, slots, g);
+    if (st != GLA_OK) return st;
+    if (d->flags & GLA_FLAG_WS_FROM_FWD) return GLA_ERR_INVALID_ARG;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(v);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(o);
+    GLA_OPTIONAL_PTR(hk0);
+    GLA_OPTIONAL_PTR(hv0);
+    GLA_OPTIONAL_PTR(hkT);
+    GLA_OPTIONAL_PTR(hvT);
+    st = check_ws(workspace, workspace_bytes, gla::gsa_workspace(g, false));
+    if (st != GLA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Problem pc = g.B;
+    pc.flags = d->flags;
+    const bool chk = gla::checks_on(pc);
+    const int64_t nm = g.B.BH * g.B.L * g.m;
+    if (chk && (st = gla::check_gates(log_a, nm, s)) != GLA_OK) return st;
+    st = gla::gsa_fwd(g, q, k, v, log_a, hk0, hv0, o, hkT, hvT, workspace, workspace_bytes, s);
+    if (st != GLA_OK || !chk) return st;
+    st = gla::check_finite(o, g.B.BH * g.B.L * g.B.V, g.io_bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(hkT, g.A.BH * g.m * g.A.V, false, s);
+    if (st == GLA_OK) st = gla::check_finite(hvT, g.B.BH * g.m * g.B.V, false, s);
+    return st;
+}
+
+gla_status gla_gsa_bwd(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
+                       const float* log_a, const float* hk0, const float* hv0, const void* dO, const float* dhkT,
+                       const float* dhvT, void* dq, void* dk, void* dv, float* dlog_a, float* dhk0, float* dhv0,
+                       void* workspace, size_t workspace_bytes, void* stream) {
+    gla::GsaProblem g{};
+    gla_status st = resolve_gsa(d, slots, g);
+    if (st != GLA_OK) return st;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(v);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(dO);
+    GLA_REQUIRE_PTR(dq);
+    GLA_REQUIRE_PTR(dk);
+    GLA_REQUIRE_PTR(dv);
+    GLA_REQUIRE_PTR(dlog_a);
+    GLA_OPTIONAL_PTR(hk0);
+    GLA_OPTIONAL_PTR(hv0);
+    GLA_OPTIONAL_PTR(dhkT);
+    GLA_OPTIONAL_PTR(dhvT);
+    GLA_OPTIONAL_PTR(dhk0);
+    GLA_OPTIONAL_PTR(dhv0);
+    st = check_ws(workspace, workspace_bytes, gla::gsa_workspace(g, true));
+    if (st != GLA_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    Problem pc = g.B;
+    pc.flags = d->flags;
+    const bool chk = gla::checks_on(pc);
+    const int64_t nm = g.B.BH * g.B.L * g.m;
+    if (chk && (st = gla::check_gates(log_a, nm, s)) != GLA_OK) return st;
+    st = gla::gsa_bwd(g, q, k, v, log_a, hk0, hv0, dO, dhkT, dhvT, dq, dk, dv, dlog_a, dhk0, dhv0,
+                      (d->flags & GLA_FLAG_WS_FROM_FWD) != 0, workspace, workspace_bytes, s);
+    if (st != GLA_OK || !chk) return st;
+    const int64_t nk = g.B.BH * g.B.L * g.A.V, nv = g.B.BH * g.B.L * g.B.V;
+    st = gla::check_finite(dq, nk, g.io_bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(dk, nk, g.io_bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(dv, nv, g.io_bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(dlog_a, nm, false, s);
+    if (st == GLA_OK) st = gla::check_finite(dhk0, g.A.BH * g.m * g.A.V, false, s);
+    if (st == GLA_OK) st = gla::check_finite(dhv0, g.B.BH * g.m * g.B.V, false, s);
+    return st;
 }
 
 namespace {

@@ -1,0 +1,384 @@
+// Gated slot attention: the read of a slot memory from its value side, on tcgen05.
+//
+// Both memories of gated slot attention are GLA states over the slots (mlsanity
+// card for "Gated Slot Attention for Efficient Linear-Time Sequence Modeling",
+// abstract: two GLA layers joined by a softmax over the slots). With the slot
+// gate's per-chunk cumsum B (one column per slot), the write weights w and the
+// memory M_[i] entering chunk i ([m slots x D], a stored bf16 chunk state of the
+// GLA walk with key w), the memory seen by token j of the chunk, read with a
+// D-vector x_j, is
+//   r_j = e^{B_j} * ( M_[i] x_j^T + sum_{s<=j} (x_j . y_s) w_s e^{-B_s} )      [m]
+// (y the memory's value rows). Layer one's logits are this read with x = q,
+// y = k, M = the key memory; the softmax backward needs the same read of the
+// value memory with x = dO, y = v (the gradient of the read weights). Both stay
+// in fp32 up to the softmax (forward) or its backward (the kernel's epilogue).
+//
+// One CTA per (chunk, head); m = 128 slots. Over D in 64-wide pieces:
+//   TMEM cols [0,128)   A1 = x y^T          (M=128 tokens, N=128 tokens)
+//   TMEM cols [128,256) L  = x M_[i]^T      (N=128 slots)
+// as ONE N=256 tcgen05.mma per 16-wide k step (the y piece and the M piece sit
+// side by side in shared memory). The epilogue masks A1 (s <= j) into bf16 P1,
+// and L += P1 Phi with Phi = w e^{-B} (token x slot, MN-major operand built by
+// the CUDA cores from the gate while the loads run). A slot whose chunk decay
+// passes the range bound (Gamma < -64) gets a zero Phi column and exact
+// log-space intra terms. Roles (192 threads): warp 0 TMA, warp 1 TMEM owner and
+// MMA issuer, warps 2-5 the gate cumsum (thread = slot), then the epilogue
+// (thread = token row).
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstring>
+
+#include "gla_common.cuh"
+#include "gla_internal.h"
+#include "gla_tc.h"
+#include "tc_host.h"
+
+namespace gla {
+namespace {
+
+using namespace tc;
+
+constexpr int C = kTcChunk;  // 128 tokens per chunk
+constexpr int kSlots = 128;
+constexpr uint32_t PIECE = 16384;  // [128 rows x 64 bf16] with the 128-byte swizzle
+constexpr int kThreadsSR = 192;
+constexpr uint32_t kTmemCols = 256;
+constexpr float kBound2 = 64.f * kLog2e;  // range bound in base-2 units
+
+struct SRBars {
+    uint64_t full[2], empty[2];
+    uint64_t a_full, p_ready, phi_ready, l_full, drain;
+    uint32_t tmem_slot;
+    int abort_flag;
+    uint32_t flag[kSlots];  // 1: the slot's chunk decay passes the range bound
+};
+
+constexpr size_t kRing = size_t(2) * 3 * PIECE;          // x, y, M pieces, two stages
+constexpr size_t kPhi = size_t(2) * PIECE;               // Phi [128 tokens x 128 slots] bf16
+constexpr size_t kBs = size_t(C) * kSlots * sizeof(float);  // B (base 2) [128 x 128] fp32
+constexpr size_t kSmem = 1024 + kRing + kPhi + kBs + sizeof(SRBars);
+
+// B2[t][c] lives at t * 128 + (c ^ (t & 31)): a warp reading one column over 32 rows (epilogue) or one
+// row over 32 columns (cumsum) touches 32 different banks.
+__device__ __forceinline__ int bs_idx(int t, int c) { return t * kSlots + (c ^ (t & 31)); }
+
+// bf16 write weight, exactly as the elementwise kernel that feeds the GLA passes rounds it
+__device__ __forceinline__ float write_weight(float la) { return __bfloat162float(__float2bfloat16_rn(1.f - __expf(la))); }
+
+// Exact intra-chunk term of a slot beyond the range bound: sum_{s<=r} P1[r][s] w_s e^{B_r - B_s}
+__device__ __noinline__ float exact_intra(const uint8_t* p1, const float* Bs, const float* la_c, int64_t m, int r,
+                                          int c, float b2r) {
+    float acc = 0.f;
+    for (int s = 0; s <= r; ++s) {
+        const uint32_t off = uint32_t(s >> 6) * PIECE + sw128_offset(uint32_t(r), uint32_t(s & 63));
+        const float pv = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(p1 + off));
+        const float w = write_weight(la_c[int64_t(s) * m]);
+        acc = fmaf(pv * w, exp2_ftz(b2r - Bs[bs_idx(s, c)]), acc);
+    }
+    return acc;
+}
+
+// one TMEM column of the warp's 32 lanes
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return __uint_as_float(r);
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(__float_as_uint(v)) : "memory");
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(kThreadsSR, 1)
+    k_gsa_slot_read(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
+                    const __grid_constant__ CUtensorMap tmM, const float* __restrict__ la,
+                    const float* __restrict__ s_in, __nv_bfloat16* __restrict__ s_b, float* __restrict__ s_f,
+                    int64_t L, int64_t N, int64_t D, int* err) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* phi = ring + kRing;
+    float* Bs = reinterpret_cast<float*>(phi + kPhi);
+    SRBars& bar = *reinterpret_cast<SRBars*>(reinterpret_cast<uint8_t*>(Bs) + kBs);
+    volatile int* abort_flag = &bar.abort_flag;
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    const int i = int(blockIdx.x);
+    const int64_t bh = blockIdx.y;
+    const int64_t t0 = int64_t(i) * C;
+    const int np = int(D / 64);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&bar.full[s], 1);
+            mbar_init(&bar.empty[s], 1);
+        }
+        mbar_init(&bar.a_full, 1);
+        mbar_init(&bar.p_ready, 128);
+        mbar_init(&bar.phi_ready, 128);
+        mbar_init(&bar.l_full, 1);
+        mbar_init(&bar.drain, 1);
+        bar.abort_flag = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&bar.tmem_slot, kTmemCols);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = bar.tmem_slot;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch(&tmX);
+            tma_prefetch(&tmY);
+            tma_prefetch(&tmM);
+            int pc = 0;
+            for (; pc < np; ++pc) {
+                const int s = pc & 1;
+                if (!mbar_wait(&bar.empty[s], uint32_t(((pc >> 1) & 1) ^ 1), err, abort_flag)) break;
+                uint8_t* st = ring + s * 3 * PIECE;
+                mbar_arrive_expect_tx(&bar.full[s], 3 * PIECE);
+                tma_load_3d(st, &tmX, 64 * pc, int(t0), int(bh), &bar.full[s]);
+                tma_load_3d(st + PIECE, &tmY, 64 * pc, int(t0), int(bh), &bar.full[s]);
+                tma_load_3d(st + 2 * PIECE, &tmM, 64 * pc, 0, int(bh * N + i), &bar.full[s]);
+            }
+            if (pc < np)  // gave up: let the copies already issued land before the block exits
+                for (int w = pc - 2; w < pc; ++w)
+                    if (w >= 0) mbar_drain(&bar.full[w & 1], uint32_t((w >> 1) & 1));
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            const uint32_t id1 = idesc_bf16_f32(128, 256, false, false);
+            const uint32_t id3 = idesc_bf16_f32(128, kSlots, false, true);
+            bool ok = true;
+            for (int pc = 0; pc < np && ok; ++pc) {
+                const int s = pc & 1;
+                ok = mbar_wait(&bar.full[s], uint32_t((pc >> 1) & 1), err, abort_flag);
+                if (!ok) break;
+                tc_fence_after();
+                const uint32_t st = smem_u32(ring + s * 3 * PIECE);
+#pragma unroll
+                for (int kk = 0; kk < 4; ++kk)
+                    mma_bf16(tmem, sdesc_sw128(st + kk * 32, 16, 1024), sdesc_sw128(st + PIECE + kk * 32, 16, 1024),
+                             id1, (pc > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(&bar.empty[s]);
+            }
+            if (ok) mma_commit(&bar.a_full);
+            ok = ok && mbar_wait(&bar.p_ready, 0, err, abort_flag) && mbar_wait(&bar.phi_ready, 0, err, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t p1 = smem_u32(ring), ph = smem_u32(phi);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem + 128, sdesc_sw128(p1 + (kk / 4) * PIECE + (kk % 4) * 32, 16, 1024),
+                             sdesc_sw128(ph + kk * 2048, PIECE, 1024), id3, 1u);
+                mma_commit(&bar.l_full);
+            }
+            mma_commit(&bar.drain);
+            mbar_drain(&bar.drain, 0);
+        }
+    } else {
+        const int tid = threadIdx.x - 64;  // 0..127
+        const int64_t nvalid = L - t0 < C ? L - t0 : C;
+        // ---- gate cumsum (thread = slot c) and Phi = w e^{-B} ----
+        {
+            const int c = tid;
+            const float* lac = la + (bh * L + t0) * kSlots + c;
+            float run = 0.f;
+            for (int tb = 0; tb < C; tb += 16) {
+                float v[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) v[e] = (tb + e < nvalid) ? lac[int64_t(tb + e) * kSlots] : 0.f;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    run = fmaf(la_floor(v[e]), kLog2e, run);
+                    Bs[bs_idx(tb + e, c)] = run;
+                }
+            }
+            const bool beyond = run < -kBound2;
+            bar.flag[c] = beyond ? 1u : 0u;
+            uint8_t* pp = phi + (c >> 6) * PIECE;
+            for (int t = 0; t < C; ++t) {
+                float f = 0.f;
+                if (!beyond && t < nvalid) f = write_weight(lac[int64_t(t) * kSlots]) * exp2_ftz(-Bs[bs_idx(t, c)]);
+                *reinterpret_cast<__nv_bfloat16*>(pp + sw128_offset(uint32_t(t), uint32_t(c & 63))) =
+                    __float2bfloat16_rn(f);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&bar.phi_ready);
+        }
+        named_sync(1, 128);  // B and the flags are complete for every slot
+        // ---- epilogue: thread = token row r ----
+        const int q4 = warp & 3;
+        const int r = 32 * q4 + lane;
+        const uint32_t lane_off = uint32_t(32 * q4) << 16;
+        const int64_t t = t0 + r;
+        const bool valid = r < nvalid;
+        if (__all_sync(0xffffffffu, mbar_wait(&bar.a_full, 0, err, abort_flag))) {
+            tc_fence_after();
+            // P1 = A1 masked to s <= r, bf16, into the ring's first stage (every MMA reading the ring is done)
+#pragma unroll 1
+            for (int cb = 0; cb < C / 16; ++cb) {
+                float a[16];
+                tmem_ld16(tmem + lane_off + uint32_t(16 * cb), a);
+                tmem_wait_ld();
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int s0 = 16 * cb + 8 * h;
+                    uint32_t pk[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float lo = (s0 + 2 * e <= r) ? a[8 * h + 2 * e] : 0.f;
+                        const float hi = (s0 + 2 * e + 1 <= r) ? a[8 * h + 2 * e + 1] : 0.f;
+                        pk[e] = pack_bf16x2(lo, hi);
+                    }
+                    uint8_t* dst = ring + (s0 >> 6) * PIECE + sw128_offset(uint32_t(r), uint32_t(s0 & 63));
+                    *reinterpret_cast<uint4*>(dst) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                }
+            }
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar.p_ready);
+            if (__all_sync(0xffffffffu, mbar_wait(&bar.l_full, 0, err, abort_flag))) {
+                tc_fence_after();
+                // slots beyond the range bound get their final value here (the flags are the same for every
+                // thread, so the single-column TMEM accesses stay warp-uniform)
+#pragma unroll 1
+                for (int c = 0; c < kSlots; ++c) {
+                    if (!bar.flag[c]) continue;
+                    const uint32_t col = tmem + lane_off + uint32_t(128 + c);
+                    float x = tmem_ld1(col);
+                    tmem_wait_ld();
+                    const float b2 = Bs[bs_idx(r, c)];
+                    // the column holds the inter part only (zero Phi column): store the final value, inter part
+                    // times e^{B_r} plus the exact sum (dividing the sum by e^{B_r} instead could overflow)
+                    x = valid ? fmaf(x, exp2_ftz(b2),
+                                     exact_intra(ring, Bs, la + (bh * L + t0) * kSlots + c, kSlots, r, c, b2))
+                              : 0.f;
+                    tmem_st1(col, x);
+                    tmem_wait_st();
+                }
+                // r_c for 16 columns: flagged slots hold their final value already
+                auto read16 = [&](int cb, float* v) {
+                    tmem_ld16(tmem + lane_off + uint32_t(128 + 16 * cb), v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int c = 16 * cb + e;
+                        if (!bar.flag[c]) v[e] *= exp2_ftz(Bs[bs_idx(r, c)]);
+                    }
+                };
+                if (MODE == 0) {
+                    float rr[kSlots];
+#pragma unroll
+                    for (int cb = 0; cb < kSlots / 16; ++cb) read16(cb, rr + 16 * cb);
+                    if (valid) {
+                        float mx = rr[0];
+#pragma unroll
+                        for (int c = 1; c < kSlots; ++c) mx = fmaxf(mx, rr[c]);
+                        float sum = 0.f;
+#pragma unroll
+                        for (int c = 0; c < kSlots; ++c) {
+                            rr[c] = __expf(rr[c] - mx);
+                            sum += rr[c];
+                        }
+                        const float inv = 1.f / sum;
+                        float* df = s_f + (bh * L + t) * kSlots;
+                        __nv_bfloat16* db = s_b + (bh * L + t) * kSlots;
+#pragma unroll
+                        for (int c8 = 0; c8 < kSlots / 8; ++c8) {
+                            uint32_t wf[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                rr[8 * c8 + e] *= inv;
+                                wf[e] = __float_as_uint(rr[8 * c8 + e]);
+                            }
+                            st_global_v8(df + 8 * c8, wf);
+                        }
+#pragma unroll
+                        for (int c16 = 0; c16 < kSlots / 16; ++c16) {
+                            uint32_t wb[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) wb[e] = pack_bf16x2(rr[16 * c16 + 2 * e], rr[16 * c16 + 2 * e + 1]);
+                            st_global_v8(db + 16 * c16, wb);
+                        }
+                    }
+                } else {
+                    // G = s * (r - <s, r>): one pass for <s, r>, a second one for G (TMEM and s read twice)
+                    const float4* sr = reinterpret_cast<const float4*>(s_in + (bh * L + (valid ? t : t0)) * kSlots);
+                    float dot = 0.f;
+#pragma unroll 1
+                    for (int cb = 0; cb < kSlots / 16; ++cb) {
+                        float v[16];
+                        read16(cb, v);
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const float4 sv = sr[4 * cb + e4];
+                            dot = fmaf(sv.x, v[4 * e4], dot);
+                            dot = fmaf(sv.y, v[4 * e4 + 1], dot);
+                            dot = fmaf(sv.z, v[4 * e4 + 2], dot);
+                            dot = fmaf(sv.w, v[4 * e4 + 3], dot);
+                        }
+                    }
+                    __nv_bfloat16* db = s_b + (bh * L + t) * kSlots;
+#pragma unroll 1
+                    for (int cb = 0; cb < kSlots / 16; ++cb) {
+                        float v[16];
+                        read16(cb, v);
+                        uint32_t wb[8];
+#pragma unroll
+                        for (int e4 = 0; e4 < 4; ++e4) {
+                            const float4 sv = sr[4 * cb + e4];
+                            wb[2 * e4] = pack_bf16x2(sv.x * (v[4 * e4] - dot), sv.y * (v[4 * e4 + 1] - dot));
+                            wb[2 * e4 + 1] = pack_bf16x2(sv.z * (v[4 * e4 + 2] - dot), sv.w * (v[4 * e4 + 3] - dot));
+                        }
+                        if (valid) st_global_v8(db + 16 * cb, wb);
+                    }
+                }
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
+    const uint64_t dims[3] = {inner, rows, outer};
+    const uint64_t strides[2] = {inner * 2, inner * rows * 2};
+    const uint32_t box[3] = {64, 128, 1};
+    return encode_tmap(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+bool tc_gsa_slot_read_supported(const Problem& p) {
+    return p.bf16 && p.K == kSlots && p.V >= 64 && p.V % 64 == 0 && p.V <= 4096 && p.N <= 65535 && p.BH <= 65535;
+}
+
+gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* y, const __nv_bfloat16* M,
+                                   const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f, int mode,
+                                   cudaStream_t s) {
+    if (!tc_gsa_slot_read_supported(p)) return GLA_ERR_UNSUPPORTED;
+    CUtensorMap m[3];
+    memset(m, 0, sizeof(m));
+    const uint64_t L = uint64_t(p.L), D = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
+    if (!(map3(&m[0], x, D, L, BH) && map3(&m[1], y, D, L, BH) && map3(&m[2], M, D, kSlots, BH * N)))
+        return GLA_ERR_CUDA;
+    auto fn = mode == 0 ? k_gsa_slot_read<0> : k_gsa_slot_read<1>;
+    if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
+        return GLA_ERR_CUDA;
+    const dim3 grid(unsigned(p.N), unsigned(p.BH));
+    GLA_LAUNCH(mode == 0 ? "gsa_slot_read" : "gsa_slot_read_bwd", fn, grid, kThreadsSR, kSmem, s, m[0], m[1], m[2],
+               la, s_in, s_b, s_f, p.L, p.N, p.V, device_error_word());
+    return GLA_OK;
+}
+
+}  // namespace gla

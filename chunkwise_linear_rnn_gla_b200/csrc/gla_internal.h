@@ -123,6 +123,28 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
                   const float* h0, const void* dO, const float* dhT, void* dq, void* dk, void* dv,
                   float* dlog_a, float* dh0, Arena& ws, cudaStream_t s);
 
+// ---- gated slot attention (gla_gsa.cu) -------------------------------------------
+// The two GLA passes of the method, resolved like any GLA call: A = layer one (GLA key width m, value
+// width Dk: the key memory), B = layer two (key width m, value width Dv: the value memory).
+// tc: the tensor-core route (bf16, m = 128, both passes on the tensor-core path, materialised states);
+// otherwise both passes run on the CUDA-core path in fp32 and io_bf16 says whether the caller's q, k, v,
+// o, dO and gradients are bf16 (converted at the boundary).
+struct GsaProblem {
+    Problem A, B;
+    int64_t m;
+    bool tc;
+    bool io_bf16;
+};
+bool gsa_tc_route(const Problem& A, const Problem& B, int64_t m);
+size_t gsa_workspace(const GsaProblem& g, bool bwd);
+gla_status gsa_fwd(const GsaProblem& g, const void* q, const void* k, const void* v, const float* la,
+                   const float* hk0, const float* hv0, void* o, float* hkT, float* hvT, void* ws, size_t cap,
+                   cudaStream_t s);
+gla_status gsa_bwd(const GsaProblem& g, const void* q, const void* k, const void* v, const float* la,
+                   const float* hk0, const float* hv0, const void* dO, const float* dhkT, const float* dhvT, void* dq,
+                   void* dk, void* dv, float* dla, float* dhk0, float* dhv0, bool reuse, void* ws, size_t cap,
+                   cudaStream_t s);
+
 }  // namespace gla
 
 // Launch helper: bracket a <<<>>> launch with the bookkeeping hooks and return

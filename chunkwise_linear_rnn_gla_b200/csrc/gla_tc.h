@@ -16,6 +16,30 @@ constexpr int kTcChunk = 128;  // C on the tensor-core path
 constexpr int kTcSub = 128;    // secondary chunk c: the default, one GEMM per chunk (16: two-level)
 constexpr int kTcBV = 64;      // value columns per walk CTA
 
+// Workspace slices of a tensor-core pass (gla_tc_api.cu). The backward's layout extends the
+// forward's, so a forward workspace can be handed to the backward unchanged.
+struct TcBuffers {
+    __nv_bfloat16 *Qt, *Kt, *P;  // Q~, K~ [BH][L][K]; masked intra-chunk scores [BH][N][128][128]
+    float *gam, *hT;             // e^Gamma [BH][N][K]; a copy of the final state
+    __nv_bfloat16* states;       // state entering each chunk [BH][N][K][V] (materialised mode, backward)
+    float* segbuf;               // segmented state walks: end states and entering states per segment
+    __nv_bfloat16* Dbuf;         // backward: D_i [BH][N][K][V]
+    float* gpart;                // scalar gate kinds: per-CTA partial sums of the gate gradient
+};
+TcBuffers tc_carve(const Problem& p, Arena& a, bool bwd);
+
+// Gated slot attention, tensor-core path (gla_gsa_read.cu). For the GLA pass problem p (key width
+// m = p.K = 128 slots, value width D = p.V) and chunk states M_[i] [BH][N][m][D] (the slot memory
+// entering chunk i), the read of the memory from its value side, in fp32:
+//   r_j = e^{B_j} * ( M_[i] x_j^T + sum_{s<=j} (x_j . y_s) w_s e^{-B_s} ),  w = bf16(1 - e^{log a}),
+// with B the per-chunk cumsum of log a over the slots (exact log-space terms for a slot whose chunk
+// decay passes the range bound). mode 0 (x = q, y = k): s = softmax(r) into s_b (bf16) and s_f
+// (fp32). mode 1 (x = dO, y = v): G = s * (r - <s, r>) into s_b (bf16), s read from s_in (fp32).
+gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* y, const __nv_bfloat16* M,
+                                   const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f, int mode,
+                                   cudaStream_t s);
+bool tc_gsa_slot_read_supported(const Problem& p);
+
 // Chunk-parallel gate preparation (gla_tc_prep.cu): Q~, K~, e^Gamma and the
 // masked intra-chunk scores P.
 // `la` is the gate argument of kind `gate_kind` (gla_gate.cuh): the kernel reads every kind natively.

@@ -26,20 +26,9 @@
 
 namespace gla {
 
-namespace {
-
-struct TcBuffers {
-    __nv_bfloat16 *Qt, *Kt, *P;
-    float *gam, *hT;
-    __nv_bfloat16* states;
-    float* segbuf;  // segmented state walks: end states and entering states per segment
-    __nv_bfloat16* Dbuf;
-    float* gpart;   // scalar gate kinds: per-CTA partial sums of the gate gradient
-};
-
 // The backward layout extends the forward's, so a forward workspace can be
 // handed to the backward unchanged.
-TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
+TcBuffers tc_carve(const Problem& p, Arena& a, bool bwd) {
     TcBuffers b{};
     b.Qt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
     b.Kt = a.take<__nv_bfloat16>(size_t(p.BH * p.L * p.K));
@@ -54,6 +43,10 @@ TcBuffers carve(const Problem& p, Arena& a, bool bwd) {
         b.gpart = a.take<float>(size_t(p.BH * p.N * (p.K / 128) * kTcChunk));
     return b;
 }
+
+namespace {
+
+TcBuffers carve(const Problem& p, Arena& a, bool bwd) { return tc_carve(p, a, bwd); }
 
 // Sub-chunk length 16 with a per-channel gate: the intra-chunk scores by two-level chunking (the
 // scalar kinds' scores are exact decay-weighted products already).

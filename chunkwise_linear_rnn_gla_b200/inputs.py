@@ -61,6 +61,13 @@ for _L in (1024, 2048, 4096, 8192, 16384):
 DECODE = dict(name="decode_b64", B=64, H=4, K=128, V=256, steps=4096, dtype="bf16")
 
 
+# Gated slot attention: the 1.3B-layer shape with m = 128 slots (the pages give no slot count; 128 keeps
+# the compact per-head memory of the method, 128 x (d_k + d_v), and is a width the tensor-core GLA passes
+# take).
+GSA_WORKLOAD = dict(name="gsa1p3b_fwdbwd", B=4, H=4, L=2048, K=256, V=512, m=128, dtype="bf16",
+                    note="gated slot attention, 1.3B-layer shape B=4 H=4 L=2048 d_k=256 d_v=512, 128 slots, fwd+bwd")
+
+
 def torch_dtype(name: str) -> torch.dtype:
     return {"f32": torch.float32, "bf16": torch.bfloat16}[name]
 
@@ -115,3 +122,31 @@ def to_f64_numpy(t: Optional[torch.Tensor]):
     if t is None:
         return None
     return t.detach().to("cpu").to(torch.float64).numpy()
+
+
+def make_gsa_inputs(B: int, H: int, L: int, K: int, V: int, m: int, dtype: str = "bf16", seed: int = 0,
+                    q_scale: float = 1.0, z_mean: float = 0.0, gate_scale: float = 1.0 / 16.0, h0: bool = False,
+                    dhT: bool = False):
+    """Gated slot attention inputs (CPU tensors): q ~ N(0,1) * q_scale (no 1/sqrt(d_k), so that the slot
+    logits spread), k, v ~ N(0,1)/sqrt(d_k), per-slot gate log_a = logsigmoid(z) * gate_scale with
+    z ~ N(z_mean, 1) [B,H,L,m], dO ~ N(0,1); optional initial memories hk0 [B,H,m,K], hv0 [B,H,m,V] and
+    final-memory gradients dhkT, dhvT (N(0,1) * 0.1, fp32). Draw order q, k, v, z, dO, hk0, hv0, dhkT,
+    dhvT; bf16 rounds q, k, v and dO."""
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    s = 1.0 / math.sqrt(K)
+    out = {"q": torch.randn(B, H, L, K, generator=g) * q_scale,
+           "k": torch.randn(B, H, L, K, generator=g) * s,
+           "v": torch.randn(B, H, L, V, generator=g) * s}
+    z = torch.randn(B, H, L, m, generator=g) + z_mean
+    out["log_a"] = (torch.nn.functional.logsigmoid(z) * gate_scale).float().contiguous()
+    out["dO"] = torch.randn(B, H, L, V, generator=g)
+    if h0:
+        out["hk0"] = torch.randn(B, H, m, K, generator=g) * 0.1
+        out["hv0"] = torch.randn(B, H, m, V, generator=g) * 0.1
+    if dhT:
+        out["dhkT"] = torch.randn(B, H, m, K, generator=g) * 0.1
+        out["dhvT"] = torch.randn(B, H, m, V, generator=g) * 0.1
+    td = torch_dtype(dtype)
+    for name in ("q", "k", "v", "dO"):
+        out[name] = out[name].to(td).contiguous()
+    return out

@@ -225,6 +225,61 @@ gla_status gla_segment_decay(const gla_desc* d, const float* log_a, float* a, vo
 gla_status gla_state_combine(int64_t G, int64_t BH, int64_t Dk, int64_t Dv, const float* a, const float* U,
                              const float* init, int32_t r, int32_t reverse, float* out, void* stream);
 
+/* ---- gated slot attention ---------------------------------------------------
+ * The method of the mlsanity card for "Gated Slot Attention for Efficient
+ * Linear-Time Sequence Modeling" (abstract): a bounded memory of `slots` (m)
+ * slots that a GLA-style data-dependent gate forgets, read by two GLA layers
+ * joined by a softmax over the slots. The card prints no equations; the
+ * reading built here gives each slot the write weight w_t = 1 - a_t (a slot
+ * writes in proportion to what it forgets). Per batch b and head h, with
+ * a_t = exp(log_a_t) in (0,1]^m:
+ *
+ *     Kmem_t = diag(a_t) Kmem_{t-1} + w_t^T k_t        [m x Dk]
+ *     Vmem_t = diag(a_t) Vmem_{t-1} + w_t^T v_t        [m x Dv]
+ *     s_t    = softmax over the m slots of Kmem_t q_t^T
+ *     o_t    = s_t Vmem_t
+ *
+ * Kmem_{-1} = hk0 and Vmem_{-1} = hv0 (NULL: zero); hkT, hvT are the final
+ * memories. Both memories are GLA states over the slot dimension, and the
+ * library evaluates the method as GLA passes of its own kernels (layer one's
+ * read as the query gradient of a GLA with key w and value k; layer two as a
+ * GLA with query s, key w and value v) plus elementwise kernels for w, the
+ * softmax, its backward and the gate gradient.
+ *
+ * Descriptor: B, H, L, Dk (width of q and k), Dv (width of v and o), dtype,
+ * chunk, subchunk, impl and state_mode apply to the GLA passes (GLA key width
+ * m); `gate` must be GLA_GATE_CHANNEL (log_a is the per-slot gate,
+ * GLA_ERR_UNSUPPORTED otherwise); flags: GLA_FLAG_WS_FROM_FWD (backward only:
+ * `workspace` holds the matching gla_gsa_fwd's workspace, same inputs and
+ * options) and GLA_FLAG_CHECKS (gate domain and finite outputs, reported by
+ * gla_check_device_error). bf16 with m = 128 and Dk, Dv multiples of 64 takes
+ * the tensor-core route; every other case the CUDA-core route (gla_gsa_resolve).
+ * Layouts (row-major, contiguous, device):
+ *     q, k, dq, dk            : [B, H, L, Dk]   (dtype)
+ *     v, o, dO, dv            : [B, H, L, Dv]   (dtype)
+ *     log_a, dlog_a           : [B, H, L, m]    (fp32)
+ *     hk0, hkT, dhkT, dhk0    : [B, H, m, Dk]   (fp32, nullable)
+ *     hv0, hvT, dhvT, dhv0    : [B, H, m, Dv]   (fp32, nullable)
+ * The backward returns the gradients of <dO, o> + <dhkT, hkT> + <dhvT, hvT>.
+ * Errors and ownership as for gla_fwd / gla_bwd; the workspace (caller
+ * allocated, 256-byte aligned) holds the two GLA passes' workspaces and the
+ * per-slot intermediates (w, s and, in the backward, their gradients). */
+/* The route gla_gsa_fwd / gla_gsa_bwd take for (d, slots): *impl = GLA_IMPL_TC (tensor cores:
+ * bf16, slots = 128, both GLA passes on the tensor-core path with materialised states, the logits and
+ * the read gradient by a fused fp32 slot-read kernel) or GLA_IMPL_SIMT (both GLA passes on the CUDA
+ * cores in fp32; bf16 tensors are converted at the boundary). Returns GLA_ERR_INVALID_ARG /
+ * GLA_ERR_UNSUPPORTED like the compute calls. */
+gla_status gla_gsa_resolve(const gla_desc* d, int32_t slots, int32_t* impl);
+size_t gla_gsa_fwd_workspace_size(const gla_desc* d, int32_t slots);
+size_t gla_gsa_bwd_workspace_size(const gla_desc* d, int32_t slots);
+gla_status gla_gsa_fwd(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
+                       const float* log_a, const float* hk0, const float* hv0, void* o, float* hkT,
+                       float* hvT, void* workspace, size_t workspace_bytes, void* stream);
+gla_status gla_gsa_bwd(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
+                       const float* log_a, const float* hk0, const float* hv0, const void* dO,
+                       const float* dhkT, const float* dhvT, void* dq, void* dk, void* dv, float* dlog_a,
+                       float* dhk0, float* dhv0, void* workspace, size_t workspace_bytes, void* stream);
+
 /* ---- forward without any allocation ---------------------------------------
  * The paper has no counterpart to this entry point; it exists for callers
  * that cannot allocate device memory or provide a workspace: a plugin under
