@@ -304,6 +304,90 @@ def oracle_sample(w, passes, n_heads_max, L_max):
                       % (nheads, w.B * w.H, Ls, w.L, passes, dt)}
 
 
+def gsa_model(B, H, L, K, V, m, C=128):
+    """Algorithmic work of gated slot attention fwd+bwd (the method's own tensors and the chunk form's
+    arithmetic, no state materialisation). Bytes per token-head: forward reads q, k, v (bf16), the gate
+    (fp32, m) and writes o; the backward reads q, k, v, dO and the gate and writes dq, dk, dv and the
+    gate gradient. FLOPs per token-head: both memories' state updates and reads (4m(d_k + d_v)), the
+    causal halves of the intra-chunk products, and in the backward the two GLA backward passes
+    (8 K V + C(3K + 2V) each, K = m), the read of the value memory for the softmax backward and layer
+    one's forward for dq."""
+    th = B * H * L
+    e = 2
+    fwd_b = e * (2 * K + V) + 4 * m + e * V
+    bwd_b = e * (2 * K + 2 * V) + 4 * m + e * (2 * K + V) + 4 * m
+    f_fwd = 4 * m * (K + V) + C * (K + 2 * m + V)
+    f_bwd = (8 * m * V + C * (3 * m + 2 * V)) + (2 * m * V + C * (V + m)) + (2 * m * K + C * (m + K)) \
+        + (8 * m * K + C * (3 * m + 2 * K))
+    return {"bytes": th * (fwd_b + bwd_b), "flops": th * (f_fwd + f_bwd),
+            "per_token_head": {"bytes": fwd_b + bwd_b, "flops": f_fwd + f_bwd}}
+
+
+def run_gsa(dev, peaks, med_ms, with_cpu=True):
+    """Gated slot attention, 1.3B-layer shape with 128 slots: device time of fwd+bwd (the backward
+    reusing the forward's workspace), the layer roofline of the method's own bytes and FLOPs, the
+    per-kernel breakdown from the library's event hooks, and the fp64 oracle on a bounded sample."""
+    import torch
+
+    import chunkwise_linear_rnn_gla_b200 as gla
+    from chunkwise_linear_rnn_gla_b200 import gsa
+    from chunkwise_linear_rnn_gla_b200.inputs import GSA_WORKLOAD as W, make_gsa_inputs
+
+    B, H, L, K, V, m = (W[n] for n in ("B", "H", "L", "K", "V", "m"))
+    inp = make_gsa_inputs(B, H, L, K, V, m, W["dtype"], seed=0)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    desc = gla.make_desc(B, H, L, K, V, W["dtype"])
+    ws_f, ws_b = gsa.gsa_fwd_workspace_size(desc, m), gsa.gsa_bwd_workspace_size(desc, m)
+    ws = torch.empty(ws_b, dtype=torch.uint8, device=dev)
+
+    def fn():
+        gsa.gsa_fwd(d["q"], d["k"], d["v"], d["log_a"], workspace=ws)
+        gsa.gsa_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], workspace=ws, ws_from_fwd=True)
+
+    ms = med_ms(fn)
+    alg = gsa_model(B, H, L, K, V, m)
+    lr = layer_roofline(alg["bytes"], alg["flops"], ms, peaks)
+    # per-kernel device time (an event pair around every launch; shares, not the headline)
+    fn()
+    torch.cuda.synchronize(dev)
+    gla.gla_profile_reset()
+    gla.gla_profile_enable(True)
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize(dev)
+    gla.gla_profile_enable(False)
+    prof = gla.gla_profile_read()
+    gla.gla_profile_reset()
+    tot = sum(x[1] for x in prof.values()) or 1.0
+    kernels = {n_: {"launches_per_step": c // 3, "us_per_step": round(t / 3 * 1e3, 2), "share": round(t / tot, 4)}
+               for n_, (c, t) in sorted(prof.items(), key=lambda kv: -kv[1][1])}
+    entry = {"B": B, "H": H, "L": L, "d_k": K, "d_v": V, "slots": m, "passes": "fwd+bwd",
+             "route": gsa.gsa_route(desc, m), "ms": round(ms, 5), "tokens_per_s": round(B * L / ms * 1e3, 1),
+             "layer_roofline_frac": lr["frac"], "roofline_ms": lr["roofline_ms"], "bound": lr["bound"],
+             "alg_bytes": alg["bytes"], "alg_flops": alg["flops"], "per_token_head": alg["per_token_head"],
+             "workspace_bytes": {"fwd": ws_f, "fwd+bwd": ws_b}, "kernels": kernels,
+             "note": W["note"]}
+    if with_cpu:
+        import oracle
+        from chunkwise_linear_rnn_gla_b200.inputs import to_f64_numpy
+
+        cores = oracle.num_threads()
+        nh = max(1, min(B * H, cores, 16))
+        Ls = min(L, 512)
+        smp = make_gsa_inputs(1, nh, Ls, K, V, m, W["dtype"], seed=0)
+        f = {n_: to_f64_numpy(t) for n_, t in smp.items()}
+        t0 = time.perf_counter()
+        oracle.gsa_fwd(f["q"], f["k"], f["v"], f["log_a"])
+        oracle.gsa_bwd(f["q"], f["k"], f["v"], f["log_a"], f["dO"])
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": nh * Ls / H / dt, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                                 "sample": "%d of %d heads, first %d of L=%d tokens, fwd+bwd fp64 step recurrence, "
+                                           "%.2f s" % (nh, B * H, Ls, L, dt)}
+    del d, ws
+    torch.cuda.empty_cache()
+    return entry
+
+
 def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
     """Device time of every other named workload, eager calls with L2 flushed before each (median of
     `reps` CUDA-event timings after 3 warm-ups): the 340M-layer forward, the long sequence with
@@ -373,6 +457,8 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
         out[label] = entry
         del inp, d, o, hT, outs
         torch.cuda.empty_cache()
+
+    out["gsa1p3b_fwdbwd"] = run_gsa(dev, peaks, med_ms, with_cpu)
 
     # decode: B=64, H=4, d_k=128, d_v=256, one token per call, fp32 state carried
     B, H, K, V = (DECODE[n] for n in ("B", "H", "K", "V"))

@@ -50,11 +50,19 @@ unsigned grid_for(int64_t n) {
     return unsigned(b);
 }
 
-// w = 1 - exp(log a)
+// w = 1 - exp(log a); four elements per thread (n4 = n / 4 groups), the tail one by one
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_write_weight(const float* __restrict__ la, T* __restrict__ w,
                                                            int64_t n) {
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+    const int64_t n4 = n / 4, stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+        const float4 x = reinterpret_cast<const float4*>(la)[i];
+        stf(w + 4 * i, 1.f - __expf(x.x));
+        stf(w + 4 * i + 1, 1.f - __expf(x.y));
+        stf(w + 4 * i + 2, 1.f - __expf(x.z));
+        stf(w + 4 * i + 3, 1.f - __expf(x.w));
+    }
+    for (int64_t i = 4 * n4 + int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
         stf(w + i, 1.f - __expf(la[i]));
 }
 
@@ -95,12 +103,25 @@ __global__ void __launch_bounds__(kThreads) k_softmax_bwd(const T* __restrict__ 
     }
 }
 
-// dla += dla1 - a * (dw1 + dw2)   (dla holds layer two's gate gradient on entry)
+// dla += dla1 - a * (dw1 + dw2)   (dla holds layer two's gate gradient on entry); four elements per
+// thread, the tail one by one
 template <typename T>
 __global__ void __launch_bounds__(kThreads) k_gate_grad(const float* __restrict__ la, const float* __restrict__ dla1,
                                                         const T* __restrict__ dw1, const T* __restrict__ dw2,
                                                         float* __restrict__ dla, int64_t n) {
-    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += int64_t(gridDim.x) * blockDim.x)
+    const int64_t n4 = n / 4, stride = int64_t(gridDim.x) * blockDim.x;
+    for (int64_t i = int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n4; i += stride) {
+        const float4 x = reinterpret_cast<const float4*>(la)[i];
+        const float4 g1 = reinterpret_cast<const float4*>(dla1)[i];
+        float4 g = reinterpret_cast<const float4*>(dla)[i];
+        const int64_t e = 4 * i;
+        g.x += g1.x - __expf(x.x) * (ldf(dw1 + e) + ldf(dw2 + e));
+        g.y += g1.y - __expf(x.y) * (ldf(dw1 + e + 1) + ldf(dw2 + e + 1));
+        g.z += g1.z - __expf(x.z) * (ldf(dw1 + e + 2) + ldf(dw2 + e + 2));
+        g.w += g1.w - __expf(x.w) * (ldf(dw1 + e + 3) + ldf(dw2 + e + 3));
+        reinterpret_cast<float4*>(dla)[i] = g;
+    }
+    for (int64_t i = 4 * n4 + int64_t(blockIdx.x) * blockDim.x + threadIdx.x; i < n; i += stride)
         dla[i] = dla[i] + dla1[i] - __expf(la[i]) * (ldf(dw1 + i) + ldf(dw2 + i));
 }
 
@@ -112,14 +133,14 @@ __global__ void __launch_bounds__(kThreads) k_convert(const Tin* __restrict__ x,
 
 template <typename T>
 gla_status write_weight(int64_t n, const float* la, T* w, cudaStream_t s) {
-    GLA_LAUNCH("gsa_write_weight", k_write_weight<T>, grid_for(n), kThreads, 0, s, la, w, n);
+    GLA_LAUNCH("gsa_write_weight", k_write_weight<T>, grid_for(cdiv(n, 4)), kThreads, 0, s, la, w, n);
     return GLA_OK;
 }
 
 template <typename T>
 gla_status gate_grad_sum(int64_t n, const float* la, const float* dla1, const T* dw1, const T* dw2, float* dla,
                          cudaStream_t s) {
-    GLA_LAUNCH("gsa_gate_grad", k_gate_grad<T>, grid_for(n), kThreads, 0, s, la, dla1, dw1, dw2, dla, n);
+    GLA_LAUNCH("gsa_gate_grad", k_gate_grad<T>, grid_for(cdiv(n, 4)), kThreads, 0, s, la, dla1, dw1, dw2, dla, n);
     return GLA_OK;
 }
 
@@ -175,10 +196,8 @@ TcRoute carve_tc(const GsaProblem& g, Arena& a, bool bwd) {
 gla_status tc_forward_state(const GsaProblem& g, const void* q, const void* k, const void* v, const float* la,
                             const float* hk0, const float* hv0, float* hkT, float* hvT, const TcRoute& r,
                             TcBuffers& A, TcBuffers& B, cudaStream_t s) {
-    const int64_t nm = g.B.BH * g.B.L * g.m;
-    gla_status st = write_weight<__nv_bfloat16>(nm, la, r.w, s);
-    // K~ = w e^{Gamma - B} and e^Gamma (the walks' operands; the query side of this preparation is unused)
-    if (st == GLA_OK) st = tc_prep_launch(g.A, r.w, r.w, la, A.Qt, A.Kt, A.P, A.gam, GLA_GATE_CHANNEL, s);
+    // w, and the walks' operands K~ = w e^{Gamma - B} and e^Gamma
+    gla_status st = tc_gsa_gate_prep_launch(g.A, la, r.w, A.Kt, A.gam, s);
     if (st == GLA_OK)
         st = tc_states_walk_launch(g.A, A.Kt, static_cast<const __nv_bfloat16*>(k), A.gam, hk0, hkT, A.hT, A.states,
                                    A.segbuf, false, s, "tc_walk_states");

@@ -21,9 +21,10 @@
 // and L += P1 Phi with Phi = w e^{-B} (token x slot, MN-major operand built by
 // the CUDA cores from the gate while the loads run). A slot whose chunk decay
 // passes the range bound (Gamma < -64) gets a zero Phi column and exact
-// log-space intra terms. Roles (192 threads): warp 0 TMA, warp 1 TMEM owner and
-// MMA issuer, warps 2-5 the gate cumsum (thread = slot), then the epilogue
-// (thread = token row).
+// log-space intra terms. Roles (576 threads): warp 0 TMA, warp 1 TMEM owner and
+// MMA issuer, 16 compute warps: the gate cumsum (4 threads per slot, 32 rows
+// each), then the epilogue (4 threads per token row, 32 slot columns each; the
+// softmax and <s, r> combine the four partial results through shared memory).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -44,7 +45,11 @@ using namespace tc;
 constexpr int C = kTcChunk;  // 128 tokens per chunk
 constexpr int kSlots = 128;
 constexpr uint32_t PIECE = 16384;  // [128 rows x 64 bf16] with the 128-byte swizzle
-constexpr int kThreadsSR = 192;
+constexpr int kCW = 16;                    // compute warps
+constexpr int kNT = 32 * kCW;              // compute threads
+constexpr int kQ = kCW / 4;                // compute threads per slot (cumsum) and per token row (epilogue)
+constexpr int kPart = C / kQ;              // rows per cumsum thread, columns per epilogue thread
+constexpr int kThreadsSR = 64 + kNT;
 constexpr uint32_t kTmemCols = 256;
 constexpr float kBound2 = 64.f * kLog2e;  // range bound in base-2 units
 
@@ -53,7 +58,9 @@ struct SRBars {
     uint64_t a_full, p_ready, phi_ready, l_full, drain;
     uint32_t tmem_slot;
     int abort_flag;
-    uint32_t flag[kSlots];  // 1: the slot's chunk decay passes the range bound
+    uint32_t flag[kSlots];     // 1: the slot's chunk decay passes the range bound
+    float tot[kQ][kSlots];     // cumsum: each thread's partial sum over its rows
+    float red[2][kQ][C];       // epilogue: per-row partial reductions of the column groups
 };
 
 constexpr size_t kRing = size_t(2) * 3 * PIECE;          // x, y, M pieces, two stages
@@ -115,8 +122,8 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             mbar_init(&bar.empty[s], 1);
         }
         mbar_init(&bar.a_full, 1);
-        mbar_init(&bar.p_ready, 128);
-        mbar_init(&bar.phi_ready, 128);
+        mbar_init(&bar.p_ready, kNT);
+        mbar_init(&bar.phi_ready, kNT);
         mbar_init(&bar.l_full, 1);
         mbar_init(&bar.drain, 1);
         bar.abort_flag = 0;
@@ -182,53 +189,67 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             mbar_drain(&bar.drain, 0);
         }
     } else {
-        const int tid = threadIdx.x - 64;  // 0..127
+        // compute warps: kQ threads per slot in the cumsum, kQ threads per token row (one column group
+        // each) in the epilogue. Every named barrier below is reached by every compute thread, whatever
+        // a bounded wait returned, so that no thread can wait at one for a thread that gave up.
+        const int tid = threadIdx.x - 64;
         const int64_t nvalid = L - t0 < C ? L - t0 : C;
-        // ---- gate cumsum (thread = slot c) and Phi = w e^{-B} ----
+        // ---- gate cumsum: thread (slot c, part) over rows [kPart part, kPart (part + 1)); Phi = w e^{-B} ----
         {
-            const int c = tid;
+            const int c = tid % kSlots, part = tid / kSlots;
+            const int r0 = part * kPart;
             const float* lac = la + (bh * L + t0) * kSlots + c;
+            float v[kPart];
+#pragma unroll
+            for (int e = 0; e < kPart; ++e) v[e] = (r0 + e < nvalid) ? lac[int64_t(r0 + e) * kSlots] : 0.f;
             float run = 0.f;
-            for (int tb = 0; tb < C; tb += 16) {
-                float v[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = (tb + e < nvalid) ? lac[int64_t(tb + e) * kSlots] : 0.f;
+            for (int e = 0; e < kPart; ++e) run = fmaf(la_floor(v[e]), kLog2e, run);
+            bar.tot[part][c] = run;
+            named_sync(1, kNT);
+            float off = 0.f, gamma = 0.f;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    run = fmaf(la_floor(v[e]), kLog2e, run);
-                    Bs[bs_idx(tb + e, c)] = run;
-                }
+            for (int p2 = 0; p2 < kQ; ++p2) {
+                const float x = bar.tot[p2][c];
+                if (p2 < part) off += x;
+                gamma += x;
             }
-            const bool beyond = run < -kBound2;
-            bar.flag[c] = beyond ? 1u : 0u;
+            const bool beyond = gamma < -kBound2;  // the same for the kQ threads of the slot
+            if (part == 0) bar.flag[c] = beyond ? 1u : 0u;
             uint8_t* pp = phi + (c >> 6) * PIECE;
-            for (int t = 0; t < C; ++t) {
-                float f = 0.f;
-                if (!beyond && t < nvalid) f = write_weight(lac[int64_t(t) * kSlots]) * exp2_ftz(-Bs[bs_idx(t, c)]);
+            run = off;
+#pragma unroll
+            for (int e = 0; e < kPart; ++e) {
+                const int t = r0 + e;
+                run = fmaf(la_floor(v[e]), kLog2e, run);
+                Bs[bs_idx(t, c)] = run;
+                const float f = (!beyond && t < nvalid) ? write_weight(v[e]) * exp2_ftz(-run) : 0.f;
                 *reinterpret_cast<__nv_bfloat16*>(pp + sw128_offset(uint32_t(t), uint32_t(c & 63))) =
                     __float2bfloat16_rn(f);
             }
             fence_proxy_async_smem();
             mbar_arrive(&bar.phi_ready);
         }
-        named_sync(1, 128);  // B and the flags are complete for every slot
-        // ---- epilogue: thread = token row r ----
-        const int q4 = warp & 3;
+        named_sync(1, kNT);  // B and the flags are complete for every slot
+        // ---- epilogue: thread = token row r, column group cg ----
+        const int q4 = warp & 3, cg = (warp - 2) / 4;
         const int r = 32 * q4 + lane;
+        const int c0 = cg * kPart;
         const uint32_t lane_off = uint32_t(32 * q4) << 16;
         const int64_t t = t0 + r;
         const bool valid = r < nvalid;
-        if (__all_sync(0xffffffffu, mbar_wait(&bar.a_full, 0, err, abort_flag))) {
+        const bool ok_a = __all_sync(0xffffffffu, mbar_wait(&bar.a_full, 0, err, abort_flag));
+        if (ok_a) {
             tc_fence_after();
             // P1 = A1 masked to s <= r, bf16, into the ring's first stage (every MMA reading the ring is done)
-#pragma unroll 1
-            for (int cb = 0; cb < C / 16; ++cb) {
+#pragma unroll
+            for (int cb = 0; cb < kPart / 16; ++cb) {
                 float a[16];
-                tmem_ld16(tmem + lane_off + uint32_t(16 * cb), a);
+                tmem_ld16(tmem + lane_off + uint32_t(c0 + 16 * cb), a);
                 tmem_wait_ld();
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    const int s0 = 16 * cb + 8 * h;
+                    const int s0 = c0 + 16 * cb + 8 * h;
                     uint32_t pk[4];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
@@ -242,102 +263,112 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             }
             fence_proxy_async_smem();
             tc_fence_before();
-            mbar_arrive(&bar.p_ready);
-            if (__all_sync(0xffffffffu, mbar_wait(&bar.l_full, 0, err, abort_flag))) {
-                tc_fence_after();
-                // slots beyond the range bound get their final value here (the flags are the same for every
-                // thread, so the single-column TMEM accesses stay warp-uniform)
+        }
+        mbar_arrive(&bar.p_ready);
+        const bool ok = ok_a && __all_sync(0xffffffffu, mbar_wait(&bar.l_full, 0, err, abort_flag));
+        float rr[kPart];
+#pragma unroll
+        for (int e = 0; e < kPart; ++e) rr[e] = 0.f;
+        if (ok) {
+            tc_fence_after();
+            // slots beyond the range bound get their final value first (warp-uniform single-column accesses):
+            // the inter part times e^{B_r} plus the exact intra-chunk sum
 #pragma unroll 1
-                for (int c = 0; c < kSlots; ++c) {
-                    if (!bar.flag[c]) continue;
-                    const uint32_t col = tmem + lane_off + uint32_t(128 + c);
-                    float x = tmem_ld1(col);
-                    tmem_wait_ld();
-                    const float b2 = Bs[bs_idx(r, c)];
-                    // the column holds the inter part only (zero Phi column): store the final value, inter part
-                    // times e^{B_r} plus the exact sum (dividing the sum by e^{B_r} instead could overflow)
-                    x = valid ? fmaf(x, exp2_ftz(b2),
-                                     exact_intra(ring, Bs, la + (bh * L + t0) * kSlots + c, kSlots, r, c, b2))
-                              : 0.f;
-                    tmem_st1(col, x);
-                    tmem_wait_st();
+            for (int c = c0; c < c0 + kPart; ++c) {
+                if (!bar.flag[c]) continue;
+                const uint32_t col = tmem + lane_off + uint32_t(128 + c);
+                float x = tmem_ld1(col);
+                tmem_wait_ld();
+                const float b2 = Bs[bs_idx(r, c)];
+                x = valid ? fmaf(x, exp2_ftz(b2),
+                                 exact_intra(ring, Bs, la + (bh * L + t0) * kSlots + c, kSlots, r, c, b2))
+                          : 0.f;
+                tmem_st1(col, x);
+                tmem_wait_st();
+            }
+#pragma unroll
+            for (int cb = 0; cb < kPart / 16; ++cb) {
+                tmem_ld16(tmem + lane_off + uint32_t(128 + c0 + 16 * cb), rr + 16 * cb);
+                tmem_wait_ld();
+            }
+#pragma unroll
+            for (int e = 0; e < kPart; ++e)
+                if (!bar.flag[c0 + e]) rr[e] *= exp2_ftz(Bs[bs_idx(r, c0 + e)]);
+        }
+        if (MODE == 0) {
+            // softmax over the row's 128 slots, spread over kQ threads
+            float mx = rr[0];
+#pragma unroll
+            for (int e = 1; e < kPart; ++e) mx = fmaxf(mx, rr[e]);
+            bar.red[0][cg][r] = mx;
+            named_sync(1, kNT);
+#pragma unroll
+            for (int g2 = 0; g2 < kQ; ++g2) mx = fmaxf(mx, bar.red[0][g2][r]);
+            float sum = 0.f;
+#pragma unroll
+            for (int e = 0; e < kPart; ++e) {
+                rr[e] = __expf(rr[e] - mx);
+                sum += rr[e];
+            }
+            bar.red[1][cg][r] = sum;
+            named_sync(1, kNT);
+            sum = 0.f;
+#pragma unroll
+            for (int g2 = 0; g2 < kQ; ++g2) sum += bar.red[1][g2][r];
+            if (ok && valid) {
+                const float inv = 1.f / sum;
+                float* df = s_f + (bh * L + t) * kSlots + c0;
+                __nv_bfloat16* db = s_b + (bh * L + t) * kSlots + c0;
+#pragma unroll
+                for (int c8 = 0; c8 < kPart / 8; ++c8) {
+                    uint32_t wf[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        rr[8 * c8 + e] *= inv;
+                        wf[e] = __float_as_uint(rr[8 * c8 + e]);
+                    }
+                    st_global_v8(df + 8 * c8, wf);
                 }
-                // r_c for 16 columns: flagged slots hold their final value already
-                auto read16 = [&](int cb, float* v) {
-                    tmem_ld16(tmem + lane_off + uint32_t(128 + 16 * cb), v);
-                    tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int c = 16 * cb + e;
-                        if (!bar.flag[c]) v[e] *= exp2_ftz(Bs[bs_idx(r, c)]);
+                for (int c16 = 0; c16 < kPart / 16; ++c16) {
+                    uint32_t wb[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) wb[e] = pack_bf16x2(rr[16 * c16 + 2 * e], rr[16 * c16 + 2 * e + 1]);
+                    st_global_v8(db + 16 * c16, wb);
+                }
+            }
+        } else {
+            // G = s * (r - <s, r>)
+            const float4* sr = reinterpret_cast<const float4*>(s_in + (bh * L + (valid ? t : t0)) * kSlots + c0);
+            float4 sv[kPart / 4];
+#pragma unroll
+            for (int e4 = 0; e4 < kPart / 4; ++e4) sv[e4] = sr[e4];
+            float dot = 0.f;
+#pragma unroll
+            for (int e4 = 0; e4 < kPart / 4; ++e4) {
+                dot = fmaf(sv[e4].x, rr[4 * e4], dot);
+                dot = fmaf(sv[e4].y, rr[4 * e4 + 1], dot);
+                dot = fmaf(sv[e4].z, rr[4 * e4 + 2], dot);
+                dot = fmaf(sv[e4].w, rr[4 * e4 + 3], dot);
+            }
+            bar.red[0][cg][r] = dot;
+            named_sync(1, kNT);
+            dot = 0.f;
+#pragma unroll
+            for (int g2 = 0; g2 < kQ; ++g2) dot += bar.red[0][g2][r];
+            if (ok && valid) {
+                __nv_bfloat16* db = s_b + (bh * L + t) * kSlots + c0;
+#pragma unroll
+                for (int c16 = 0; c16 < kPart / 16; ++c16) {
+                    uint32_t wb[8];
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const float4 x = sv[4 * c16 + e4];
+                        const float* y = rr + 16 * c16 + 4 * e4;
+                        wb[2 * e4] = pack_bf16x2(x.x * (y[0] - dot), x.y * (y[1] - dot));
+                        wb[2 * e4 + 1] = pack_bf16x2(x.z * (y[2] - dot), x.w * (y[3] - dot));
                     }
-                };
-                if (MODE == 0) {
-                    float rr[kSlots];
-#pragma unroll
-                    for (int cb = 0; cb < kSlots / 16; ++cb) read16(cb, rr + 16 * cb);
-                    if (valid) {
-                        float mx = rr[0];
-#pragma unroll
-                        for (int c = 1; c < kSlots; ++c) mx = fmaxf(mx, rr[c]);
-                        float sum = 0.f;
-#pragma unroll
-                        for (int c = 0; c < kSlots; ++c) {
-                            rr[c] = __expf(rr[c] - mx);
-                            sum += rr[c];
-                        }
-                        const float inv = 1.f / sum;
-                        float* df = s_f + (bh * L + t) * kSlots;
-                        __nv_bfloat16* db = s_b + (bh * L + t) * kSlots;
-#pragma unroll
-                        for (int c8 = 0; c8 < kSlots / 8; ++c8) {
-                            uint32_t wf[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) {
-                                rr[8 * c8 + e] *= inv;
-                                wf[e] = __float_as_uint(rr[8 * c8 + e]);
-                            }
-                            st_global_v8(df + 8 * c8, wf);
-                        }
-#pragma unroll
-                        for (int c16 = 0; c16 < kSlots / 16; ++c16) {
-                            uint32_t wb[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) wb[e] = pack_bf16x2(rr[16 * c16 + 2 * e], rr[16 * c16 + 2 * e + 1]);
-                            st_global_v8(db + 16 * c16, wb);
-                        }
-                    }
-                } else {
-                    // G = s * (r - <s, r>): one pass for <s, r>, a second one for G (TMEM and s read twice)
-                    const float4* sr = reinterpret_cast<const float4*>(s_in + (bh * L + (valid ? t : t0)) * kSlots);
-                    float dot = 0.f;
-#pragma unroll 1
-                    for (int cb = 0; cb < kSlots / 16; ++cb) {
-                        float v[16];
-                        read16(cb, v);
-#pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const float4 sv = sr[4 * cb + e4];
-                            dot = fmaf(sv.x, v[4 * e4], dot);
-                            dot = fmaf(sv.y, v[4 * e4 + 1], dot);
-                            dot = fmaf(sv.z, v[4 * e4 + 2], dot);
-                            dot = fmaf(sv.w, v[4 * e4 + 3], dot);
-                        }
-                    }
-                    __nv_bfloat16* db = s_b + (bh * L + t) * kSlots;
-#pragma unroll 1
-                    for (int cb = 0; cb < kSlots / 16; ++cb) {
-                        float v[16];
-                        read16(cb, v);
-                        uint32_t wb[8];
-#pragma unroll
-                        for (int e4 = 0; e4 < 4; ++e4) {
-                            const float4 sv = sr[4 * cb + e4];
-                            wb[2 * e4] = pack_bf16x2(sv.x * (v[4 * e4] - dot), sv.y * (v[4 * e4 + 1] - dot));
-                            wb[2 * e4 + 1] = pack_bf16x2(sv.z * (v[4 * e4 + 2] - dot), sv.w * (v[4 * e4 + 3] - dot));
-                        }
-                        if (valid) st_global_v8(db + 16 * cb, wb);
-                    }
+                    st_global_v8(db + 16 * c16, wb);
                 }
             }
         }
@@ -348,6 +379,56 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
         tc_fence_after();
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// Gate preparation of the slot memories' walks, per (chunk, head), thread = slot: the write weight
+// w = bf16(1 - e^{log a}), the walk operand K~ = w e^{Gamma - B} (B the per-chunk cumsum of log a,
+// Gamma its last row) and e^Gamma, as the GLA preparation kernel forms them for a GLA key w.
+constexpr int kGateThreads = kSlots;
+constexpr size_t kGateSmem = size_t(C) * kSlots * (sizeof(float) + sizeof(__nv_bfloat16));
+
+__global__ void __launch_bounds__(kGateThreads) k_gsa_gate_prep(const float* __restrict__ la,
+                                                                __nv_bfloat16* __restrict__ w,
+                                                                __nv_bfloat16* __restrict__ Kt,
+                                                                float* __restrict__ gam, int64_t L, int64_t N) {
+    extern __shared__ uint8_t smem_raw[];
+    float* Bn = reinterpret_cast<float*>(smem_raw);                         // [t][c], nats
+    __nv_bfloat16* ws = reinterpret_cast<__nv_bfloat16*>(Bn + C * kSlots);  // [t][c]
+    const int c = threadIdx.x, i = blockIdx.x;
+    const int64_t bh = blockIdx.y, t0 = int64_t(i) * C;
+    const int64_t nvalid = L - t0 < C ? L - t0 : C;
+    const int64_t base = (bh * L + t0) * kSlots + c;
+    constexpr int kBatch = 32;
+    float cur[kBatch], nxt[kBatch];
+#pragma unroll
+    for (int e = 0; e < kBatch; ++e) cur[e] = e < nvalid ? la[base + int64_t(e) * kSlots] : 0.f;
+    float run = 0.f;
+#pragma unroll 1
+    for (int tb = 0; tb < C; tb += kBatch) {
+        if (tb + kBatch < C) {
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e)
+                nxt[e] = tb + kBatch + e < nvalid ? la[base + int64_t(tb + kBatch + e) * kSlots] : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < kBatch; ++e) {
+            const int t = tb + e;
+            run += la_floor(cur[e]);
+            Bn[t * kSlots + c] = run;
+            const __nv_bfloat16 wb = __float2bfloat16_rn(1.f - __expf(cur[e]));
+            ws[t * kSlots + c] = wb;
+            if (t < nvalid) w[base + int64_t(t) * kSlots] = wb;
+        }
+        if (tb + kBatch < C) {
+#pragma unroll
+            for (int e = 0; e < kBatch; ++e) cur[e] = nxt[e];
+        }
+    }
+    // exponents are <= 0 in exact arithmetic; the clamps absorb cumsum rounding
+    gam[(bh * N + i) * kSlots + c] = __expf(fminf(run, 0.f));
+    for (int t = 0; t < nvalid; ++t)
+        Kt[base + int64_t(t) * kSlots] =
+            __float2bfloat16_rn(__bfloat162float(ws[t * kSlots + c]) * __expf(fminf(run - Bn[t * kSlots + c], 0.f)));
 }
 
 bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
@@ -361,6 +442,17 @@ bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint6
 
 bool tc_gsa_slot_read_supported(const Problem& p) {
     return p.bf16 && p.K == kSlots && p.V >= 64 && p.V % 64 == 0 && p.V <= 4096 && p.N <= 65535 && p.BH <= 65535;
+}
+
+gla_status tc_gsa_gate_prep_launch(const Problem& p, const float* la, __nv_bfloat16* w, __nv_bfloat16* Kt,
+                                   float* gam, cudaStream_t s) {
+    if (p.K != kSlots || p.N > 65535 || p.BH > 65535) return GLA_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(k_gsa_gate_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGateSmem)) !=
+        cudaSuccess)
+        return GLA_ERR_CUDA;
+    GLA_LAUNCH("gsa_gate_prep", k_gsa_gate_prep, dim3(unsigned(p.N), unsigned(p.BH)), kGateThreads, kGateSmem, s, la,
+               w, Kt, gam, p.L, p.N);
+    return GLA_OK;
 }
 
 gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* y, const __nv_bfloat16* M,

@@ -39,6 +39,10 @@ gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* 
                                    const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f, int mode,
                                    cudaStream_t s);
 bool tc_gsa_slot_read_supported(const Problem& p);
+// The slot gate's preparation for the memories' walks (p: key width m = 128): w = bf16(1 - e^{log a})
+// [BH][L][m], the walk operand K~ = w e^{Gamma - B} [BH][L][m] and e^Gamma [BH][N][m].
+gla_status tc_gsa_gate_prep_launch(const Problem& p, const float* la, __nv_bfloat16* w, __nv_bfloat16* Kt,
+                                   float* gam, cudaStream_t s);
 
 // Chunk-parallel gate preparation (gla_tc_prep.cu): Q~, K~, e^Gamma and the
 // masked intra-chunk scores P.
