@@ -8,6 +8,9 @@ case is called eagerly with L2 flushed before every call (a 512 MB write); the f
 of 10 CUDA-event timings around the call, after 3 warm-up calls, followed by the per-kernel split
 from the library's own launch timing over 3 more calls.
 
+For gated slot attention (`inputs.GSA_WORKLOAD`, name "gsa1p3b_fwdbwd"): the forward and the forward +
+backward the same way (`--reps 1` makes one timed call of each, for a profiler).
+
 For the decode step (`inputs.DECODE`, and the same shape with B=256 whose 134 MB state exceeds L2):
 the median of 20 calls with L2 flushed before each, and a CUDA graph of 64 calls replayed 5 times
 with the state left in L2 between calls.
@@ -21,7 +24,7 @@ import torch
 
 from . import gla_bwd, gla_bwd_workspace_size, gla_fwd, gla_profile_enable, gla_profile_read, gla_profile_reset
 from . import gla_step, make_desc
-from .inputs import DECODE, WORKLOADS, make_inputs, make_step_inputs
+from .inputs import DECODE, GSA_WORKLOAD, WORKLOADS, make_gsa_inputs, make_inputs, make_step_inputs
 
 FLUSH_BYTES = 512 * 1024 * 1024
 
@@ -71,6 +74,40 @@ def time_layer(w, flush):
                   % (w.name, mode, tag, ms * 1000, w.B * w.L / ms / 1e3, per), flush=True)
 
 
+def time_gsa(flush, reps=10):
+    from . import gsa
+
+    W = GSA_WORKLOAD
+    inp = make_gsa_inputs(W["B"], W["H"], W["L"], W["K"], W["V"], W["m"], W["dtype"], seed=0)
+    d = {k: v.cuda() for k, v in inp.items()}
+    desc = make_desc(W["B"], W["H"], W["L"], W["K"], W["V"], W["dtype"])
+    ws = torch.empty(gsa.gsa_bwd_workspace_size(desc, W["m"]), dtype=torch.uint8, device="cuda")
+
+    def fwd():
+        gsa.gsa_fwd(d["q"], d["k"], d["v"], d["log_a"], workspace=ws)
+
+    def both():
+        fwd()
+        gsa.gsa_bwd(d["q"], d["k"], d["v"], d["log_a"], d["dO"], workspace=ws, ws_from_fwd=True)
+
+    for tag, fn in (("fwd", fwd), ("fwd+bwd", both)):
+        for _ in range(3 if reps > 1 else 1):
+            fn()
+        ms = _median_ms(fn, flush, reps)
+        per = {}
+        if reps > 1:
+            gla_profile_enable(True)
+            gla_profile_reset()
+            for _ in range(3):
+                flush.zero_()
+                fn()
+            torch.cuda.synchronize()
+            gla_profile_enable(False)
+            per = {k: round(v[1] / v[0] * 1000, 1) for k, v in gla_profile_read().items()}
+        print("%-16s %-15s %-8s %8.1f us  %8.2f Mtok/s  per kernel (us): %s"
+              % (W["name"], gsa.gsa_route(desc, W["m"]), tag, ms * 1000, W["B"] * W["L"] / ms / 1e3, per), flush=True)
+
+
 def time_decode(B, H, K, V, flush):
     st = make_step_inputs(B, H, K, V, 1, DECODE["dtype"], seed=0)
     q, k, v, la = (st[n][0].cuda() for n in ("q", "k", "v", "log_a"))
@@ -110,11 +147,13 @@ def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--only", nargs="*", default=None, help="workload names (and/or 'decode') to time")
     ap.add_argument("--list", action="store_true", help="list the workloads and exit")
+    ap.add_argument("--reps", type=int, default=10, help="timed calls per case (gated slot attention)")
     args = ap.parse_args(argv)
-    names = [n for n, w in WORKLOADS.items() if w.dtype == "bf16"] + ["decode"]
+    names = [n for n, w in WORKLOADS.items() if w.dtype == "bf16"] + [GSA_WORKLOAD["name"], "decode"]
     if args.list:
         for n in names:
-            print(n, "-", WORKLOADS[n].note if n in WORKLOADS else "decode step, B=64 and B=256")
+            print(n, "-", WORKLOADS[n].note if n in WORKLOADS else
+                  GSA_WORKLOAD["note"] if n == GSA_WORKLOAD["name"] else "decode step, B=64 and B=256")
         return 0
     if args.only:
         unknown = [n for n in args.only if n not in names]
@@ -129,6 +168,8 @@ def main(argv=None):
         if n == "decode":
             for B in (DECODE["B"], 4 * DECODE["B"]):
                 time_decode(B, DECODE["H"], DECODE["K"], DECODE["V"], flush)
+        elif n == GSA_WORKLOAD["name"]:
+            time_gsa(flush, max(1, args.reps))
         else:
             time_layer(WORKLOADS[n], flush)
     return 0
