@@ -381,54 +381,50 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
     }
 }
 
-// Gate preparation of the slot memories' walks, per (chunk, head), thread = slot: the write weight
-// w = bf16(1 - e^{log a}), the walk operand K~ = w e^{Gamma - B} (B the per-chunk cumsum of log a,
-// Gamma its last row) and e^Gamma, as the GLA preparation kernel forms them for a GLA key w.
-constexpr int kGateThreads = kSlots;
-constexpr size_t kGateSmem = size_t(C) * kSlots * (sizeof(float) + sizeof(__nv_bfloat16));
+// Gate preparation of the slot memories' walks, per (chunk, head): the write weight
+// w = bf16(1 - e^{log a}), the walk operand K~ = w e^{Gamma - B} (B the per-chunk cumsum of log a, Gamma
+// its last row) and e^Gamma, as the GLA preparation kernel forms them for a GLA key w. kQ threads per slot
+// (32 rows each): partial sums, a prefix over them through shared memory, then every row's values.
+constexpr int kGateThreads = kSlots * kQ;
 
-__global__ void __launch_bounds__(kGateThreads) k_gsa_gate_prep(const float* __restrict__ la,
+__global__ void __launch_bounds__(kGateThreads, 2) k_gsa_gate_prep(const float* __restrict__ la,
                                                                 __nv_bfloat16* __restrict__ w,
                                                                 __nv_bfloat16* __restrict__ Kt,
                                                                 float* __restrict__ gam, int64_t L, int64_t N) {
-    extern __shared__ uint8_t smem_raw[];
-    float* Bn = reinterpret_cast<float*>(smem_raw);                         // [t][c], nats
-    __nv_bfloat16* ws = reinterpret_cast<__nv_bfloat16*>(Bn + C * kSlots);  // [t][c]
-    const int c = threadIdx.x, i = blockIdx.x;
+    __shared__ float tot[kQ][kSlots];
+    const int c = threadIdx.x % kSlots, part = threadIdx.x / kSlots, i = blockIdx.x;
+    const int r0 = part * kPart;
     const int64_t bh = blockIdx.y, t0 = int64_t(i) * C;
     const int64_t nvalid = L - t0 < C ? L - t0 : C;
     const int64_t base = (bh * L + t0) * kSlots + c;
-    constexpr int kBatch = 32;
-    float cur[kBatch], nxt[kBatch];
+    float v[kPart];
 #pragma unroll
-    for (int e = 0; e < kBatch; ++e) cur[e] = e < nvalid ? la[base + int64_t(e) * kSlots] : 0.f;
+    for (int e = 0; e < kPart; ++e) v[e] = r0 + e < nvalid ? la[base + int64_t(r0 + e) * kSlots] : 0.f;
     float run = 0.f;
-#pragma unroll 1
-    for (int tb = 0; tb < C; tb += kBatch) {
-        if (tb + kBatch < C) {
 #pragma unroll
-            for (int e = 0; e < kBatch; ++e)
-                nxt[e] = tb + kBatch + e < nvalid ? la[base + int64_t(tb + kBatch + e) * kSlots] : 0.f;
-        }
+    for (int e = 0; e < kPart; ++e) run += la_floor(v[e]);
+    tot[part][c] = run;
+    __syncthreads();
+    float off = 0.f, gamma = 0.f;
 #pragma unroll
-        for (int e = 0; e < kBatch; ++e) {
-            const int t = tb + e;
-            run += la_floor(cur[e]);
-            Bn[t * kSlots + c] = run;
-            const __nv_bfloat16 wb = __float2bfloat16_rn(1.f - __expf(cur[e]));
-            ws[t * kSlots + c] = wb;
-            if (t < nvalid) w[base + int64_t(t) * kSlots] = wb;
-        }
-        if (tb + kBatch < C) {
-#pragma unroll
-            for (int e = 0; e < kBatch; ++e) cur[e] = nxt[e];
-        }
+    for (int p2 = 0; p2 < kQ; ++p2) {
+        const float x = tot[p2][c];
+        if (p2 < part) off += x;
+        gamma += x;
     }
     // exponents are <= 0 in exact arithmetic; the clamps absorb cumsum rounding
-    gam[(bh * N + i) * kSlots + c] = __expf(fminf(run, 0.f));
-    for (int t = 0; t < nvalid; ++t)
-        Kt[base + int64_t(t) * kSlots] =
-            __float2bfloat16_rn(__bfloat162float(ws[t * kSlots + c]) * __expf(fminf(run - Bn[t * kSlots + c], 0.f)));
+    if (part == 0) gam[(bh * N + i) * kSlots + c] = __expf(fminf(gamma, 0.f));
+    run = off;
+#pragma unroll
+    for (int e = 0; e < kPart; ++e) {
+        const int t = r0 + e;
+        run += la_floor(v[e]);
+        if (t < nvalid) {
+            const __nv_bfloat16 wb = __float2bfloat16_rn(1.f - __expf(v[e]));
+            w[base + int64_t(t) * kSlots] = wb;
+            Kt[base + int64_t(t) * kSlots] = __float2bfloat16_rn(__bfloat162float(wb) * __expf(fminf(gamma - run, 0.f)));
+        }
+    }
 }
 
 bool map3(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint64_t outer) {
@@ -447,11 +443,8 @@ bool tc_gsa_slot_read_supported(const Problem& p) {
 gla_status tc_gsa_gate_prep_launch(const Problem& p, const float* la, __nv_bfloat16* w, __nv_bfloat16* Kt,
                                    float* gam, cudaStream_t s) {
     if (p.K != kSlots || p.N > 65535 || p.BH > 65535) return GLA_ERR_UNSUPPORTED;
-    if (cudaFuncSetAttribute(k_gsa_gate_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kGateSmem)) !=
-        cudaSuccess)
-        return GLA_ERR_CUDA;
-    GLA_LAUNCH("gsa_gate_prep", k_gsa_gate_prep, dim3(unsigned(p.N), unsigned(p.BH)), kGateThreads, kGateSmem, s, la,
-               w, Kt, gam, p.L, p.N);
+    GLA_LAUNCH("gsa_gate_prep", k_gsa_gate_prep, dim3(unsigned(p.N), unsigned(p.BH)), kGateThreads, 0, s, la, w, Kt,
+               gam, p.L, p.N);
     return GLA_OK;
 }
 
