@@ -367,6 +367,20 @@ def run_gsa(dev, peaks, med_ms, with_cpu=True):
              "alg_bytes": alg["bytes"], "alg_flops": alg["flops"], "per_token_head": alg["per_token_head"],
              "workspace_bytes": {"fwd": ws_f, "fwd+bwd": ws_b}, "kernels": kernels,
              "note": W["note"]}
+    # decode: one token per call for a batch of 64 sequences, both memories (fp32) updated in place
+    Bd = 64
+    st = make_gsa_inputs(Bd, H, 1, K, V, m, W["dtype"], seed=1)
+    sd = {n_: st[n_][:, :, 0].contiguous().to(dev) for n_ in ("q", "k", "v", "log_a")}
+    hk = torch.zeros(Bd, H, m, K, device=dev)
+    hv = torch.zeros(Bd, H, m, V, device=dev)
+    step_ms = med_ms(lambda: gsa.gsa_step(sd["q"], sd["k"], sd["v"], sd["log_a"], hk, hv))
+    mem_bytes = 2 * Bd * H * m * (K + V) * 4  # both memories read and written
+    entry["decode"] = {"B": Bd, "us_per_step": round(step_ms * 1e3, 2), "tokens_per_s": round(Bd / step_ms * 1e3, 1),
+                       "memory_GBps": round(mem_bytes / step_ms / 1e6, 1),
+                       "hbm_frac": round(mem_bytes / step_ms / 1e6 / peaks["hbm_gbs"], 4),
+                       "how": "median of single calls, L2 flushed before each; %.1f MB of memories read and "
+                              "written per step" % (mem_bytes / 1e6)}
+    del hk, hv, sd
     if with_cpu:
         import oracle
         from chunkwise_linear_rnn_gla_b200.inputs import to_f64_numpy

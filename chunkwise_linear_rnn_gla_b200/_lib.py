@@ -34,6 +34,7 @@ EXPORTS = (
     "gla_selftest_wait_timeout", "gla_last_device_error", "gla_fwd_workspace_bytes", "gla_bwd_workspace_bytes",
     "gla_segment_decay", "gla_state_combine", "gla_fwd_final_state", "gla_bwd_initial_grad",
     "gla_gsa_resolve", "gla_gsa_fwd_workspace_size", "gla_gsa_bwd_workspace_size", "gla_gsa_fwd", "gla_gsa_bwd",
+    "gla_gsa_step",
 )
 
 
@@ -109,6 +110,8 @@ def _declare(lib):
     lib.gla_gsa_fwd.restype = ctypes.c_int
     lib.gla_gsa_bwd.argtypes = [dp, i32] + [vp] * 15 + [vp, sz, vp]
     lib.gla_gsa_bwd.restype = ctypes.c_int
+    lib.gla_gsa_step.argtypes = [dp, i32] + [vp] * 7 + [vp]
+    lib.gla_gsa_step.restype = ctypes.c_int
     lib.gla_segment_decay.argtypes = [dp, vp, vp, vp]
     lib.gla_segment_decay.restype = ctypes.c_int
     i64 = ctypes.c_int64

@@ -587,6 +587,43 @@ gla_status gla_gsa_fwd(const gla_desc* d, int32_t slots, const void* q, const vo
     return st;
 }
 
+gla_status gla_gsa_step(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
+                        const float* log_a, float* Kmem, float* Vmem, void* o, void* stream) {
+    if (!d || slots < 1) return GLA_ERR_INVALID_ARG;
+    if (d->B < 1 || d->H < 1 || d->Dk < 1 || d->Dv < 1) return GLA_ERR_INVALID_ARG;
+    if (d->dtype != GLA_DTYPE_F32 && d->dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+    if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
+    if (d->gate != GLA_GATE_CHANNEL) return d->gate < GLA_GATE_CHANNEL || d->gate > GLA_GATE_PREACT
+                                                ? GLA_ERR_INVALID_ARG
+                                                : GLA_ERR_UNSUPPORTED;
+    GLA_REQUIRE_PTR(q);
+    GLA_REQUIRE_PTR(k);
+    GLA_REQUIRE_PTR(v);
+    GLA_REQUIRE_PTR(log_a);
+    GLA_REQUIRE_PTR(Kmem);
+    GLA_REQUIRE_PTR(Vmem);
+    GLA_REQUIRE_PTR(o);
+    if (!gla::gsa_step_supported(slots, d->Dk, d->Dv)) return GLA_ERR_UNSUPPORTED;
+    Problem p{};
+    p.B = d->B;
+    p.H = d->H;
+    p.L = 1;
+    p.K = d->Dk;
+    p.V = d->Dv;
+    p.BH = d->B * d->H;
+    p.flags = d->flags;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool chk = gla::checks_on(p);
+    const bool bf16 = d->dtype == GLA_DTYPE_BF16;
+    gla_status st = chk ? gla::check_gates(log_a, p.BH * slots, s) : GLA_OK;
+    if (st == GLA_OK) st = gla::gsa_step(p.BH, slots, d->Dk, d->Dv, bf16, q, k, v, log_a, Kmem, Vmem, o, s);
+    if (st != GLA_OK || !chk) return st;
+    st = gla::check_finite(o, p.BH * d->Dv, bf16, s);
+    if (st == GLA_OK) st = gla::check_finite(Kmem, p.BH * slots * d->Dk, false, s);
+    if (st == GLA_OK) st = gla::check_finite(Vmem, p.BH * slots * d->Dv, false, s);
+    return st;
+}
+
 gla_status gla_gsa_bwd(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
                        const float* log_a, const float* hk0, const float* hv0, const void* dO, const float* dhkT,
                        const float* dhvT, void* dq, void* dk, void* dv, float* dlog_a, float* dhk0, float* dhv0,

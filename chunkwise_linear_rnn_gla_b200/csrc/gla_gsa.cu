@@ -405,6 +405,141 @@ gla_status simt_route_bwd(const GsaProblem& g, const void* q, const void* k, con
     return st;
 }
 
+// ================================================================ decode step
+// One token per head, both memories updated in place (fp32), one block per head:
+//   keys:   Kmem[c] <- a_c Kmem[c] + w_c k,  z_c = Kmem[c] . q      (w = 1 - a, exact in fp32)
+//   read:   s = softmax(z)
+//   values: Vmem[c] <- a_c Vmem[c] + w_c v,  o = sum_c s_c Vmem[c]
+// A warp takes four slot rows at a time (their loads issued together, 16 bytes per lane); the row dot
+// products reduce by shuffles, the softmax runs in one warp, and o sums the warps' partial rows through
+// shared memory in a fixed order.
+constexpr int kStepThreads = 512;
+constexpr int kStepRows = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kStepThreads) k_gsa_step(const T* __restrict__ q, const T* __restrict__ k,
+                                                           const T* __restrict__ v, const float* __restrict__ la,
+                                                           float* __restrict__ Km, float* __restrict__ Vm,
+                                                           T* __restrict__ o, int m, int Dk, int Dv) {
+    extern __shared__ float sh[];
+    float* qs = sh;
+    float* ks = qs + Dk;
+    float* vs = ks + Dk;
+    float* as = vs + Dv;
+    float* ws = as + m;
+    float* zs = ws + m;
+    float* op = zs + m;  // [warps][Dv]
+    const int64_t bh = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5, nw = blockDim.x >> 5;
+    for (int i = tid; i < Dk; i += blockDim.x) {
+        qs[i] = ldf(q + bh * Dk + i);
+        ks[i] = ldf(k + bh * Dk + i);
+    }
+    for (int i = tid; i < Dv; i += blockDim.x) vs[i] = ldf(v + bh * Dv + i);
+    for (int c = tid; c < m; c += blockDim.x) {
+        const float a = __expf(la[bh * m + c]);
+        as[c] = a;
+        ws[c] = 1.f - a;
+    }
+    for (int i = tid; i < nw * Dv; i += blockDim.x) op[i] = 0.f;
+    __syncthreads();
+    const int dk4 = Dk / 4, dv4 = Dv / 4;
+    float4* K4 = reinterpret_cast<float4*>(Km + bh * int64_t(m) * Dk);
+    float4* V4 = reinterpret_cast<float4*>(Vm + bh * int64_t(m) * Dv);
+    const float4* q4 = reinterpret_cast<const float4*>(qs);
+    const float4* k4 = reinterpret_cast<const float4*>(ks);
+    const float4* v4 = reinterpret_cast<const float4*>(vs);
+    // ---- keys and logits
+    for (int c0 = wp * kStepRows; c0 < m; c0 += nw * kStepRows) {
+        float dot[kStepRows];
+#pragma unroll
+        for (int u = 0; u < kStepRows; ++u) dot[u] = 0.f;
+        for (int d4 = lane; d4 < dk4; d4 += 32) {
+            float4 r[kStepRows];
+#pragma unroll
+            for (int u = 0; u < kStepRows; ++u)
+                if (c0 + u < m) r[u] = K4[int64_t(c0 + u) * dk4 + d4];
+            const float4 kk = k4[d4], qq = q4[d4];
+#pragma unroll
+            for (int u = 0; u < kStepRows; ++u) {
+                if (c0 + u >= m) continue;
+                const float a = as[c0 + u], w = ws[c0 + u];
+                float4 x = r[u];
+                x.x = fmaf(a, x.x, w * kk.x);
+                x.y = fmaf(a, x.y, w * kk.y);
+                x.z = fmaf(a, x.z, w * kk.z);
+                x.w = fmaf(a, x.w, w * kk.w);
+                K4[int64_t(c0 + u) * dk4 + d4] = x;
+                dot[u] = fmaf(x.x, qq.x, fmaf(x.y, qq.y, fmaf(x.z, qq.z, fmaf(x.w, qq.w, dot[u]))));
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kStepRows; ++u) {
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) dot[u] += __shfl_xor_sync(0xffffffffu, dot[u], off);
+            if (lane == 0 && c0 + u < m) zs[c0 + u] = dot[u];
+        }
+    }
+    __syncthreads();
+    // ---- softmax over the slots (warp 0)
+    if (wp == 0) {
+        float mx = -INFINITY;
+        for (int c = lane; c < m; c += 32) mx = fmaxf(mx, zs[c]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        float sum = 0.f;
+        for (int c = lane; c < m; c += 32) {
+            const float e = __expf(zs[c] - mx);
+            zs[c] = e;
+            sum += e;
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const float inv = 1.f / sum;
+        __syncwarp();
+        for (int c = lane; c < m; c += 32) zs[c] *= inv;
+    }
+    __syncthreads();
+    // ---- values and the read
+    float4* o4 = reinterpret_cast<float4*>(op + wp * Dv);
+    for (int c0 = wp * kStepRows; c0 < m; c0 += nw * kStepRows) {
+        for (int d4 = lane; d4 < dv4; d4 += 32) {
+            float4 r[kStepRows];
+#pragma unroll
+            for (int u = 0; u < kStepRows; ++u)
+                if (c0 + u < m) r[u] = V4[int64_t(c0 + u) * dv4 + d4];
+            const float4 vv = v4[d4];
+            float4 acc = o4[d4];
+#pragma unroll
+            for (int u = 0; u < kStepRows; ++u) {
+                if (c0 + u >= m) continue;
+                const float a = as[c0 + u], w = ws[c0 + u], sc = zs[c0 + u];
+                float4 y = r[u];
+                y.x = fmaf(a, y.x, w * vv.x);
+                y.y = fmaf(a, y.y, w * vv.y);
+                y.z = fmaf(a, y.z, w * vv.z);
+                y.w = fmaf(a, y.w, w * vv.w);
+                V4[int64_t(c0 + u) * dv4 + d4] = y;
+                acc.x = fmaf(sc, y.x, acc.x);
+                acc.y = fmaf(sc, y.y, acc.y);
+                acc.z = fmaf(sc, y.z, acc.z);
+                acc.w = fmaf(sc, y.w, acc.w);
+            }
+            o4[d4] = acc;
+        }
+    }
+    __syncthreads();
+    for (int x = tid; x < Dv; x += blockDim.x) {
+        float acc = 0.f;
+        for (int w2 = 0; w2 < nw; ++w2) acc += op[w2 * Dv + x];
+        stf(o + bh * Dv + x, acc);
+    }
+}
+
+size_t step_smem(int64_t m, int64_t Dk, int64_t Dv) {
+    return sizeof(float) * size_t(2 * Dk + Dv + 3 * m + (kStepThreads / 32) * Dv);
+}
+
 }  // namespace
 
 bool gsa_tc_route(const Problem& A, const Problem& B, int64_t m) {
@@ -449,6 +584,37 @@ gla_status gsa_bwd(const GsaProblem& g, const void* q, const void* k, const void
     const SimtRoute r = carve_simt(g, a, true);
     if (a.used > a.cap) return GLA_ERR_WORKSPACE;
     return simt_route_bwd(g, q, k, v, la, hk0, hv0, dO, dhkT, dhvT, dq, dk, dv, dla, dhk0, dhv0, reuse, r, s);
+}
+
+}  // namespace gla
+
+namespace gla {
+
+bool gsa_step_supported(int64_t m, int64_t Dk, int64_t Dv) {
+    return m >= 1 && Dk >= 4 && Dv >= 4 && Dk % 4 == 0 && Dv % 4 == 0 && step_smem(m, Dk, Dv) <= 200 * 1024;
+}
+
+gla_status gsa_step(int64_t BH, int64_t m, int64_t Dk, int64_t Dv, bool bf16, const void* q, const void* k,
+                    const void* v, const float* la, float* Km, float* Vm, void* o, cudaStream_t s) {
+    if (!gsa_step_supported(m, Dk, Dv) || BH > 2147483647) return GLA_ERR_UNSUPPORTED;
+    const size_t smem = step_smem(m, Dk, Dv);
+    if (bf16) {
+        if (smem > 48 * 1024 && cudaFuncSetAttribute(k_gsa_step<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     int(smem)) != cudaSuccess)
+            return GLA_ERR_CUDA;
+        GLA_LAUNCH("gsa_step", k_gsa_step<__nv_bfloat16>, unsigned(BH), kStepThreads, smem, s,
+                   static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                   static_cast<const __nv_bfloat16*>(v), la, Km, Vm, static_cast<__nv_bfloat16*>(o), int(m), int(Dk),
+                   int(Dv));
+    } else {
+        if (smem > 48 * 1024 &&
+            cudaFuncSetAttribute(k_gsa_step<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
+            return GLA_ERR_CUDA;
+        GLA_LAUNCH("gsa_step", k_gsa_step<float>, unsigned(BH), kStepThreads, smem, s, static_cast<const float*>(q),
+                   static_cast<const float*>(k), static_cast<const float*>(v), la, Km, Vm, static_cast<float*>(o),
+                   int(m), int(Dk), int(Dv));
+    }
+    return GLA_OK;
 }
 
 }  // namespace gla

@@ -136,6 +136,10 @@ struct GsaProblem {
     bool io_bf16;
 };
 bool gsa_tc_route(const Problem& A, const Problem& B, int64_t m);
+// Decode step: both memories Km [BH][m][Dk], Vm [BH][m][Dv] (fp32) updated in place, o [BH][Dv].
+bool gsa_step_supported(int64_t m, int64_t Dk, int64_t Dv);
+gla_status gsa_step(int64_t BH, int64_t m, int64_t Dk, int64_t Dv, bool bf16, const void* q, const void* k,
+                    const void* v, const float* la, float* Km, float* Vm, void* o, cudaStream_t s);
 size_t gsa_workspace(const GsaProblem& g, bool bwd);
 gla_status gsa_fwd(const GsaProblem& g, const void* q, const void* k, const void* v, const float* la,
                    const float* hk0, const float* hv0, void* o, float* hkT, float* hvT, void* ws, size_t cap,

@@ -19,7 +19,7 @@ import torch
 from . import _lib, _need, _ptr, _stream, _check, _workspace, make_desc, _dt
 from ._lib import load
 
-__all__ = ["gsa_fwd", "gsa_bwd", "gsa_fwd_workspace_size", "gsa_bwd_workspace_size", "gsa_route"]
+__all__ = ["gsa_fwd", "gsa_bwd", "gsa_step", "gsa_fwd_workspace_size", "gsa_bwd_workspace_size", "gsa_route"]
 
 
 def _desc(q, v, chunk, subchunk, state_mode, impl, flags):
@@ -108,3 +108,33 @@ def gsa_bwd(q, k, v, log_a, dO, hk0=None, hv0=None, dhkT=None, dhvT=None, *, chu
     if checks:
         _check(load().gla_check_device_error(_stream(dev)), "gla_gsa_bwd (checking mode)")
     return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dhk0": dhk0, "dhv0": dhv0}
+
+
+def gsa_step(q, k, v, log_a, hk, hv, o=None, checks=False):
+    """One decode step: q, k [B,H,Dk], v [B,H,Dv], log_a [B,H,m] fp32; the memories hk [B,H,m,Dk] and
+    hv [B,H,m,Dv] (fp32) are updated in place. Returns o [B,H,Dv]."""
+    load()
+    dev, dt = q.device, q.dtype
+    B, H, Dk = q.shape
+    _need(k, "k", q.shape, dt, dev)
+    if v.dim() != 3 or tuple(v.shape[:2]) != (B, H):
+        raise ValueError("v has shape %s, expected [%d, %d, Dv]" % (tuple(v.shape), B, H))
+    _need(v, "v", v.shape, dt, dev)
+    Dv = v.shape[-1]
+    if log_a.dim() != 3 or tuple(log_a.shape[:2]) != (B, H):
+        raise ValueError("log_a has shape %s, expected [%d, %d, slots]" % (tuple(log_a.shape), B, H))
+    _need(log_a, "log_a", log_a.shape, torch.float32, dev)
+    m = log_a.shape[-1]
+    _need(hk, "hk", (B, H, m, Dk), torch.float32, dev)
+    _need(hv, "hv", (B, H, m, Dv), torch.float32, dev)
+    if o is None:
+        o = torch.empty(B, H, Dv, dtype=dt, device=dev)
+    _need(o, "o", (B, H, Dv), dt, dev)
+    desc = make_desc(B, H, 1, Dk, Dv, _dt(q), flags=_lib.FLAG_CHECKS if checks else 0)
+    with torch.cuda.device(dev):
+        st = load().gla_gsa_step(ctypes.byref(desc), m, _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(hk), _ptr(hv),
+                                 _ptr(o), _stream(dev))
+    _check(st, "gla_gsa_step")
+    if checks:
+        _check(load().gla_check_device_error(_stream(dev)), "gla_gsa_step (checking mode)")
+    return o

@@ -275,6 +275,14 @@ size_t gla_gsa_bwd_workspace_size(const gla_desc* d, int32_t slots);
 gla_status gla_gsa_fwd(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
                        const float* log_a, const float* hk0, const float* hv0, void* o, float* hkT,
                        float* hvT, void* workspace, size_t workspace_bytes, void* stream);
+/* One decode step of gated slot attention for a batch of single tokens: q, k [B,H,Dk], v [B,H,Dv]
+ * (d->dtype), log_a [B,H,slots] (fp32), the memories Kmem [B,H,slots,Dk] and Vmem [B,H,slots,Dv] (fp32,
+ * updated in place: the step's hkT / hvT), o [B,H,Dv] (d->dtype). d->L is ignored; d->gate must be
+ * GLA_GATE_CHANNEL; Dk and Dv multiples of 4. Applied L times from hk0 / hv0 it gives what gla_gsa_fwd
+ * gives for those L tokens. GLA_FLAG_CHECKS checks the gate domain and that o and both memories are
+ * finite. */
+gla_status gla_gsa_step(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
+                        const float* log_a, float* Kmem, float* Vmem, void* o, void* stream);
 gla_status gla_gsa_bwd(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,
                        const float* log_a, const float* hk0, const float* hv0, const void* dO,
                        const float* dhkT, const float* dhvT, void* dq, void* dk, void* dv, float* dlog_a,

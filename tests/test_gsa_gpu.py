@@ -127,3 +127,40 @@ def test_gsa_workload_full_size():
     assert route_of(inp) == "tc"
     errs = check_all(inp, "bf16", names=("o", "dq", "dk", "dv", "dlog_a"))
     print("gsa workload relative errors", {k: "%.2e" % v for k, v in errs.items()})
+
+
+# ---------------------------------------------------------------- decode step
+@pytest.mark.parametrize("dtype,Dk,Dv,m", [("f32", 64, 32, 16), ("f32", 96, 40, 24), ("bf16", 128, 256, 128),
+                                           ("bf16", 256, 512, 128)])
+def test_gsa_step_matches_oracle(dtype, Dk, Dv, m):
+    """T single-token steps from given memories equal the oracle over those T tokens (o at every step, the
+    final memories)."""
+    B, H, T = 2, 2, 12
+    inp = make_gsa_inputs(B, H, T, Dk, Dv, m, dtype, seed=9, q_scale=4.0, h0=True)
+    d = to_dev(inp)
+    hk, hv = d["hk0"].clone(), d["hv0"].clone()
+    outs = [gsa.gsa_step(*(d[n][:, :, t].contiguous() for n in ("q", "k", "v", "log_a")), hk, hv) for t in range(T)]
+    torch.cuda.synchronize()
+    ref = run_oracle(inp, fwd_only=True)
+    compare("o", torch.stack(outs, dim=2), ref["o"], dtype)
+    compare("hkT", hk, ref["hkT"], dtype)
+    compare("hvT", hv, ref["hvT"], dtype)
+
+
+def test_gsa_step_continues_the_forward():
+    """The forward's final memories (tensor-core route) continued by decode steps give the oracle's outputs
+    and memories over the whole sequence."""
+    B, H, L, T, Dk, Dv, m = 1, 2, 300, 5, 128, 128, 128
+    inp = make_gsa_inputs(B, H, L + T, Dk, Dv, m, "bf16", seed=10, q_scale=4.0)
+    d = to_dev(inp)
+    pre = {n: d[n][:, :, :L].contiguous() for n in ("q", "k", "v", "log_a")}
+    assert route_of(pre) == "tc"
+    o, hk, hv = gsa.gsa_fwd(pre["q"], pre["k"], pre["v"], pre["log_a"], want_state=True)
+    outs = [gsa.gsa_step(*(d[n][:, :, L + t].contiguous() for n in ("q", "k", "v", "log_a")), hk, hv)
+            for t in range(T)]
+    torch.cuda.synchronize()
+    ref = run_oracle(inp, fwd_only=True)
+    compare("o (forward)", o, ref["o"][:, :, :L], "bf16")
+    compare("o (steps)", torch.stack(outs, dim=2), ref["o"][:, :, L:], "bf16")
+    compare("hkT", hk, ref["hkT"], "bf16")
+    compare("hvT", hv, ref["hvT"], "bf16")
