@@ -108,3 +108,63 @@ def test_simt_rejects_nonmaterialized(lib):
 def test_launch_counter_host_only(lib):
     lib.gla_launch_count_reset()
     assert lib.gla_launch_count() == 0
+
+
+# ---------------------------------------------------------------- gated slot attention (host logic only)
+def gsa_route(lib, slots, **kw):
+    im = ctypes.c_int32(-1)
+    st = lib.gla_gsa_resolve(ctypes.byref(desc(**kw)), slots, ctypes.byref(im))
+    return st, im.value
+
+
+def test_gsa_route_selection(lib):
+    tc, simt = _lib.IMPL["tc"], _lib.IMPL["simt"]
+    # bf16, 128 slots, widths that the tensor-core passes take -> tensor cores
+    assert gsa_route(lib, 128, dtype=1, L=2048, Dk=256, Dv=512) == (0, tc)
+    assert gsa_route(lib, 128, dtype=1, L=300, Dk=64, Dv=192) == (0, tc)
+    # other slot counts, fp32, widths off the 64 grid, a two-level sub-chunk or an explicit CUDA-core request
+    for slots, kw in ((64, dict(dtype=1, Dk=128, Dv=128)), (256, dict(dtype=1, Dk=128, Dv=128)),
+                      (128, dict(dtype=0, Dk=128, Dv=128)), (128, dict(dtype=1, Dk=96, Dv=128)),
+                      (128, dict(dtype=1, Dk=128, Dv=128, subchunk=16)), (128, dict(dtype=1, Dk=128, Dv=128, impl=1))):
+        assert gsa_route(lib, slots, L=300, **kw) == (0, simt), (slots, kw)
+    # an explicit tensor-core request that the route cannot serve
+    assert gsa_route(lib, 64, dtype=1, L=300, Dk=128, Dv=128, impl=2)[0] == _lib.GLA_ERR_UNSUPPORTED
+
+
+def test_gsa_rejects_bad_arguments(lib):
+    assert gsa_route(lib, 0, dtype=1)[0] == _lib.GLA_ERR_INVALID_ARG
+    assert gsa_route(lib, 128, dtype=1, gate=1)[0] == _lib.GLA_ERR_UNSUPPORTED  # slot gates are per slot
+    assert gsa_route(lib, 128, dtype=1, gate=9)[0] == _lib.GLA_ERR_INVALID_ARG
+    assert gsa_route(lib, 128, dtype=1, flags=0x40)[0] == _lib.GLA_ERR_INVALID_ARG
+    d = desc(dtype=1, L=64, Dk=128, Dv=128)
+    ptr = ctypes.c_void_p(256)
+    # a null required pointer is rejected on the host, before any launch
+    assert lib.gla_gsa_fwd(ctypes.byref(d), 128, None, ptr, ptr, ptr, None, None, ptr, None, None, ptr, 1 << 30,
+                           None) == _lib.GLA_ERR_INVALID_ARG
+    assert lib.gla_gsa_step(ctypes.byref(d), 128, ptr, ptr, ptr, ptr, ptr, None, ptr, None) == _lib.GLA_ERR_INVALID_ARG
+    # misaligned pointers
+    bad = ctypes.c_void_p(258)
+    assert lib.gla_gsa_step(ctypes.byref(d), 128, bad, ptr, ptr, ptr, ptr, ptr, ptr, None) == _lib.GLA_ERR_INVALID_ARG
+    # a step whose widths are not multiples of 4
+    d3 = desc(dtype=1, L=1, Dk=130, Dv=128)
+    assert lib.gla_gsa_step(ctypes.byref(d3), 128, ptr, ptr, ptr, ptr, ptr, ptr, ptr, None) == _lib.GLA_ERR_UNSUPPORTED
+    # the forward's workspace check runs before any launch
+    assert lib.gla_gsa_fwd(ctypes.byref(d), 128, ptr, ptr, ptr, ptr, None, None, ptr, None, None, ptr, 16,
+                           None) == _lib.GLA_ERR_WORKSPACE
+    # a forward cannot take the forward's workspace
+    dr = desc(dtype=1, L=64, Dk=128, Dv=128, flags=_lib.FLAG_WS_FROM_FWD)
+    assert lib.gla_gsa_fwd(ctypes.byref(dr), 128, ptr, ptr, ptr, ptr, None, None, ptr, None, None, ptr, 1 << 30,
+                           None) == _lib.GLA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("dtype,slots", [(1, 128), (1, 64), (0, 32)])
+def test_gsa_workspace_prefix(lib, dtype, slots):
+    """The backward's workspace extends the forward's (the backward may take the forward's), and both
+    grow with the sequence."""
+    sizes = []
+    for L in (300, 600):
+        d = desc(dtype=dtype, L=L, Dk=128, Dv=256)
+        f, b = lib.gla_gsa_fwd_workspace_size(ctypes.byref(d), slots), lib.gla_gsa_bwd_workspace_size(ctypes.byref(d), slots)
+        assert 0 < f <= b
+        sizes.append(b)
+    assert sizes[1] > sizes[0]
