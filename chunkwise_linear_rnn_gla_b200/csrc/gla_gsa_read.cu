@@ -55,7 +55,7 @@ constexpr float kBound2 = 64.f * kLog2e;  // range bound in base-2 units
 
 struct SRBars {
     uint64_t full[2], empty[2];
-    uint64_t a_full, p_ready, phi_ready, l_full, drain;
+    uint64_t a_full, p_ready, phi_ready, l_full, s_full, drain;
     uint32_t tmem_slot;
     int abort_flag;
     uint32_t flag[kSlots];     // 1: the slot's chunk decay passes the range bound
@@ -67,6 +67,10 @@ constexpr size_t kRing = size_t(2) * 3 * PIECE;          // x, y, M pieces, two 
 constexpr size_t kPhi = size_t(2) * PIECE;               // Phi [128 tokens x 128 slots] bf16
 constexpr size_t kBs = size_t(C) * kSlots * sizeof(float);  // B (base 2) [128 x 128] fp32
 constexpr size_t kSmem = 1024 + kRing + kPhi + kBs + sizeof(SRBars);
+
+// The read gradient's s tile (fp32 [128 rows x 128 slots], four TMA boxes of 32 columns with the 128-byte
+// swizzle) goes to the ring once the D loop is done, into the four 16 KB pieces that P1 does not use.
+__device__ __forceinline__ uint32_t s_piece(int p) { return uint32_t(2 + p) * PIECE; }
 
 // B2[t][c] lives at t * 128 + (c ^ (t & 31)): a warp reading one column over 32 rows (epilogue) or one
 // row over 32 columns (cumsum) touches 32 different banks.
@@ -101,7 +105,8 @@ __device__ __forceinline__ void tmem_st1(uint32_t taddr, float v) {
 template <int MODE>
 __global__ void __launch_bounds__(kThreadsSR, 1)
     k_gsa_slot_read(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY,
-                    const __grid_constant__ CUtensorMap tmM, const float* __restrict__ la,
+                    const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmS,
+                    const float* __restrict__ la,
                     const float* __restrict__ s_in, __nv_bfloat16* __restrict__ s_b, float* __restrict__ s_f,
                     int64_t L, int64_t N, int64_t D, int* err) {
     extern __shared__ uint8_t smem_raw[];
@@ -125,6 +130,7 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
         mbar_init(&bar.p_ready, kNT);
         mbar_init(&bar.phi_ready, kNT);
         mbar_init(&bar.l_full, 1);
+        mbar_init(&bar.s_full, 1);
         mbar_init(&bar.drain, 1);
         bar.abort_flag = 0;
         fence_barrier_init();
@@ -153,9 +159,18 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
                 tma_load_3d(st + PIECE, &tmY, 64 * pc, int(t0), int(bh), &bar.full[s]);
                 tma_load_3d(st + 2 * PIECE, &tmM, 64 * pc, 0, int(bh * N + i), &bar.full[s]);
             }
-            if (pc < np)  // gave up: let the copies already issued land before the block exits
+            if (pc < np) {  // gave up: let the copies already issued land before the block exits
                 for (int w = pc - 2; w < pc; ++w)
                     if (w >= 0) mbar_drain(&bar.full[w & 1], uint32_t((w >> 1) & 1));
+            } else if (MODE == 1 && mbar_wait(&bar.a_full, 0, err, abort_flag)) {
+                // every MMA reading the ring is done: the fp32 s tile of the chunk into the pieces P1 leaves free
+                tma_prefetch(&tmS);
+                mbar_arrive_expect_tx(&bar.s_full, 4 * PIECE);
+#pragma unroll
+                for (int p2 = 0; p2 < 4; ++p2)
+                    tma_load_3d(ring + s_piece(p2), &tmS, 32 * p2, int(t0), int(bh), &bar.s_full);
+                if (!mbar_wait(&bar.s_full, 0, err, abort_flag)) mbar_drain(&bar.s_full, 0);
+            }
         }
     } else if (warp == 1) {
         if (lane == 0) {
@@ -238,6 +253,9 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
         const uint32_t lane_off = uint32_t(32 * q4) << 16;
         const int64_t t = t0 + r;
         const bool valid = r < nvalid;
+        uint32_t fmask = 0;  // slots of the column group beyond the range bound (the same across the warp)
+#pragma unroll
+        for (int e = 0; e < kPart; ++e) fmask |= bar.flag[c0 + e] ? (1u << e) : 0u;
         const bool ok_a = __all_sync(0xffffffffu, mbar_wait(&bar.a_full, 0, err, abort_flag));
         if (ok_a) {
             tc_fence_after();
@@ -274,8 +292,8 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             // slots beyond the range bound get their final value first (warp-uniform single-column accesses):
             // the inter part times e^{B_r} plus the exact intra-chunk sum
 #pragma unroll 1
-            for (int c = c0; c < c0 + kPart; ++c) {
-                if (!bar.flag[c]) continue;
+            for (uint32_t f = fmask; f; f &= f - 1) {
+                const int c = c0 + __ffs(int(f)) - 1;
                 const uint32_t col = tmem + lane_off + uint32_t(128 + c);
                 float x = tmem_ld1(col);
                 tmem_wait_ld();
@@ -293,7 +311,7 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             }
 #pragma unroll
             for (int e = 0; e < kPart; ++e)
-                if (!bar.flag[c0 + e]) rr[e] *= exp2_ftz(Bs[bs_idx(r, c0 + e)]);
+                if (!((fmask >> e) & 1u)) rr[e] *= exp2_ftz(Bs[bs_idx(r, c0 + e)]);
         }
         if (MODE == 0) {
             // softmax over the row's 128 slots, spread over kQ threads
@@ -315,34 +333,40 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             sum = 0.f;
 #pragma unroll
             for (int g2 = 0; g2 < kQ; ++g2) sum += bar.red[1][g2][r];
-            if (ok && valid) {
-                const float inv = 1.f / sum;
-                float* df = s_f + (bh * L + t) * kSlots + c0;
-                __nv_bfloat16* db = s_b + (bh * L + t) * kSlots + c0;
+            // s staged in the ring (free: the second GEMM has read P1; the exact terms above are done, every
+            // thread having passed the first exchange) with a row stride of 129 floats, so that a warp writing
+            // one column over 32 rows, and one reading a row, touch 32 banks; then whole rows are stored
+            float* stg = reinterpret_cast<float*>(ring);
+            constexpr int kStride = kSlots + 1;
+            const float inv = 1.f / sum;
+            if (ok) {
 #pragma unroll
-                for (int c8 = 0; c8 < kPart / 8; ++c8) {
-                    uint32_t wf[8];
+                for (int e = 0; e < kPart; ++e) stg[r * kStride + c0 + e] = rr[e] * inv;
+            }
+            named_sync(1, kNT);
+            if (ok) {
+                for (int rho = warp - 2; rho < nvalid; rho += kCW) {
+                    const float* srow = stg + rho * kStride;
+                    float* df = s_f + (bh * L + t0 + rho) * kSlots;
+                    __nv_bfloat16* db = s_b + (bh * L + t0 + rho) * kSlots;
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        rr[8 * c8 + e] *= inv;
-                        wf[e] = __float_as_uint(rr[8 * c8 + e]);
+                    for (int k4 = 0; k4 < kSlots / 32; ++k4) df[32 * k4 + lane] = srow[32 * k4 + lane];
+#pragma unroll
+                    for (int k2 = 0; k2 < kSlots / 64; ++k2) {
+                        const int c = 64 * k2 + 2 * lane;
+                        *reinterpret_cast<uint32_t*>(db + c) = pack_bf16x2(srow[c], srow[c + 1]);
                     }
-                    st_global_v8(df + 8 * c8, wf);
-                }
-#pragma unroll
-                for (int c16 = 0; c16 < kPart / 16; ++c16) {
-                    uint32_t wb[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) wb[e] = pack_bf16x2(rr[16 * c16 + 2 * e], rr[16 * c16 + 2 * e + 1]);
-                    st_global_v8(db + 16 * c16, wb);
                 }
             }
         } else {
-            // G = s * (r - <s, r>)
-            const float4* sr = reinterpret_cast<const float4*>(s_in + (bh * L + (valid ? t : t0)) * kSlots + c0);
+            // G = s * (r - <s, r>), s from the tile in shared memory (piece cg: this thread's 32 columns;
+            // 16-byte chunk j of row r at (j ^ (r % 8)) * 16)
+            const bool ok_s = ok && __all_sync(0xffffffffu, mbar_wait(&bar.s_full, 0, err, abort_flag));
+            const uint8_t* sp = ring + s_piece(cg) + r * 128;
             float4 sv[kPart / 4];
 #pragma unroll
-            for (int e4 = 0; e4 < kPart / 4; ++e4) sv[e4] = sr[e4];
+            for (int e4 = 0; e4 < kPart / 4; ++e4)
+                sv[e4] = ok_s ? *reinterpret_cast<const float4*>(sp + ((e4 ^ (r & 7)) << 4)) : make_float4(0.f, 0.f, 0.f, 0.f);
             float dot = 0.f;
 #pragma unroll
             for (int e4 = 0; e4 < kPart / 4; ++e4) {
@@ -356,7 +380,7 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             dot = 0.f;
 #pragma unroll
             for (int g2 = 0; g2 < kQ; ++g2) dot += bar.red[0][g2][r];
-            if (ok && valid) {
+            if (ok_s && valid) {
                 __nv_bfloat16* db = s_b + (bh * L + t) * kSlots + c0;
 #pragma unroll
                 for (int c16 = 0; c16 < kPart / 16; ++c16) {
@@ -452,17 +476,26 @@ gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* 
                                    const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f, int mode,
                                    cudaStream_t s) {
     if (!tc_gsa_slot_read_supported(p)) return GLA_ERR_UNSUPPORTED;
-    CUtensorMap m[3];
+    CUtensorMap m[4];
     memset(m, 0, sizeof(m));
     const uint64_t L = uint64_t(p.L), D = uint64_t(p.V), BH = uint64_t(p.BH), N = uint64_t(p.N);
     if (!(map3(&m[0], x, D, L, BH) && map3(&m[1], y, D, L, BH) && map3(&m[2], M, D, kSlots, BH * N)))
         return GLA_ERR_CUDA;
+    if (mode == 1) {
+        const uint64_t dims[3] = {uint64_t(kSlots), L, BH};
+        const uint64_t strides[2] = {uint64_t(kSlots) * 4, uint64_t(kSlots) * L * 4};
+        const uint32_t box[3] = {32, 128, 1};
+        if (!encode_tmap(&m[3], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, s_in, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B))
+            return GLA_ERR_CUDA;
+    } else {
+        m[3] = m[0];  // unused: any valid descriptor
+    }
     auto fn = mode == 0 ? k_gsa_slot_read<0> : k_gsa_slot_read<1>;
     if (cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, int(kSmem)) != cudaSuccess)
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.BH));
     GLA_LAUNCH(mode == 0 ? "gsa_slot_read" : "gsa_slot_read_bwd", fn, grid, kThreadsSR, kSmem, s, m[0], m[1], m[2],
-               la, s_in, s_b, s_f, p.L, p.N, p.V, device_error_word());
+               m[3], la, s_in, s_b, s_f, p.L, p.N, p.V, device_error_word());
     return GLA_OK;
 }
 
