@@ -232,11 +232,16 @@ gla_status check_ws(void* ws, size_t bytes, size_t need) {
 gla_status resolve_gsa(const gla_desc* d, int32_t slots, gla::GsaProblem& g) {
     if (!d || slots < 1) return GLA_ERR_INVALID_ARG;
     if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
-    if (d->gate != GLA_GATE_CHANNEL) return d->gate < GLA_GATE_CHANNEL || d->gate > GLA_GATE_PREACT
-                                                ? GLA_ERR_INVALID_ARG
-                                                : GLA_ERR_UNSUPPORTED;
+    Problem gp{};
+    if (!gate_ok(d, gp)) return GLA_ERR_INVALID_ARG;
+    if (d->gate != GLA_GATE_CHANNEL && d->gate != GLA_GATE_PREACT) return GLA_ERR_UNSUPPORTED;
     if (d->dtype != GLA_DTYPE_F32 && d->dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
+    g.preact = d->gate == GLA_GATE_PREACT;
+    g.inv_tau = gp.inv_tau;
     gla_desc da = *d, db = *d;
+    // the passes take the expanded per-slot log a
+    da.gate = db.gate = GLA_GATE_CHANNEL;
+    da.gate_tau = db.gate_tau = 0.f;
     da.Dk = slots;
     da.Dv = d->Dk;
     da.flags = 0;
@@ -578,7 +583,7 @@ gla_status gla_gsa_fwd(const gla_desc* d, int32_t slots, const void* q, const vo
     pc.flags = d->flags;
     const bool chk = gla::checks_on(pc);
     const int64_t nm = g.B.BH * g.B.L * g.m;
-    if (chk && (st = gla::check_gates(log_a, nm, s)) != GLA_OK) return st;
+    if (chk && !g.preact && (st = gla::check_gates(log_a, nm, s)) != GLA_OK) return st;
     st = gla::gsa_fwd(g, q, k, v, log_a, hk0, hv0, o, hkT, hvT, workspace, workspace_bytes, s);
     if (st != GLA_OK || !chk) return st;
     st = gla::check_finite(o, g.B.BH * g.B.L * g.B.V, g.io_bf16, s);
@@ -593,9 +598,9 @@ gla_status gla_gsa_step(const gla_desc* d, int32_t slots, const void* q, const v
     if (d->B < 1 || d->H < 1 || d->Dk < 1 || d->Dv < 1) return GLA_ERR_INVALID_ARG;
     if (d->dtype != GLA_DTYPE_F32 && d->dtype != GLA_DTYPE_BF16) return GLA_ERR_INVALID_ARG;
     if (d->flags & ~int32_t(GLA_FLAG_WS_FROM_FWD | GLA_FLAG_CHECKS)) return GLA_ERR_INVALID_ARG;
-    if (d->gate != GLA_GATE_CHANNEL) return d->gate < GLA_GATE_CHANNEL || d->gate > GLA_GATE_PREACT
-                                                ? GLA_ERR_INVALID_ARG
-                                                : GLA_ERR_UNSUPPORTED;
+    Problem gp{};
+    if (!gate_ok(d, gp)) return GLA_ERR_INVALID_ARG;
+    if (d->gate != GLA_GATE_CHANNEL && d->gate != GLA_GATE_PREACT) return GLA_ERR_UNSUPPORTED;
     GLA_REQUIRE_PTR(q);
     GLA_REQUIRE_PTR(k);
     GLA_REQUIRE_PTR(v);
@@ -615,8 +620,9 @@ gla_status gla_gsa_step(const gla_desc* d, int32_t slots, const void* q, const v
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const bool chk = gla::checks_on(p);
     const bool bf16 = d->dtype == GLA_DTYPE_BF16;
-    gla_status st = chk ? gla::check_gates(log_a, p.BH * slots, s) : GLA_OK;
-    if (st == GLA_OK) st = gla::gsa_step(p.BH, slots, d->Dk, d->Dv, bf16, q, k, v, log_a, Kmem, Vmem, o, s);
+    gla_status st = chk && d->gate == GLA_GATE_CHANNEL ? gla::check_gates(log_a, p.BH * slots, s) : GLA_OK;
+    if (st == GLA_OK)
+        st = gla::gsa_step(p.BH, slots, d->Dk, d->Dv, bf16, q, k, v, log_a, gp.inv_tau, Kmem, Vmem, o, s);
     if (st != GLA_OK || !chk) return st;
     st = gla::check_finite(o, p.BH * d->Dv, bf16, s);
     if (st == GLA_OK) st = gla::check_finite(Kmem, p.BH * slots * d->Dk, false, s);
@@ -653,7 +659,7 @@ gla_status gla_gsa_bwd(const gla_desc* d, int32_t slots, const void* q, const vo
     pc.flags = d->flags;
     const bool chk = gla::checks_on(pc);
     const int64_t nm = g.B.BH * g.B.L * g.m;
-    if (chk && (st = gla::check_gates(log_a, nm, s)) != GLA_OK) return st;
+    if (chk && !g.preact && (st = gla::check_gates(log_a, nm, s)) != GLA_OK) return st;
     st = gla::gsa_bwd(g, q, k, v, log_a, hk0, hv0, dO, dhkT, dhvT, dq, dk, dv, dlog_a, dhk0, dhv0,
                       (d->flags & GLA_FLAG_WS_FROM_FWD) != 0, workspace, workspace_bytes, s);
     if (st != GLA_OK || !chk) return st;

@@ -35,6 +35,7 @@
 #include <cuda_runtime.h>
 
 #include "gla_common.cuh"
+#include "gla_gate.cuh"
 #include "gla_internal.h"
 #include "gla_tc.h"
 
@@ -419,8 +420,9 @@ constexpr int kStepRows = 4;
 template <typename T>
 __global__ void __launch_bounds__(kStepThreads) k_gsa_step(const T* __restrict__ q, const T* __restrict__ k,
                                                            const T* __restrict__ v, const float* __restrict__ la,
-                                                           float* __restrict__ Km, float* __restrict__ Vm,
-                                                           T* __restrict__ o, int m, int Dk, int Dv) {
+                                                           float inv_tau, float* __restrict__ Km,
+                                                           float* __restrict__ Vm, T* __restrict__ o, int m, int Dk,
+                                                           int Dv) {
     extern __shared__ float sh[];
     float* qs = sh;
     float* ks = qs + Dk;
@@ -437,7 +439,8 @@ __global__ void __launch_bounds__(kStepThreads) k_gsa_step(const T* __restrict__
     }
     for (int i = tid; i < Dv; i += blockDim.x) vs[i] = ldf(v + bh * Dv + i);
     for (int c = tid; c < m; c += blockDim.x) {
-        const float a = __expf(la[bh * m + c]);
+        const float g = la[bh * m + c];
+        const float a = __expf(inv_tau > 0.f ? logsigmoid_f(g) * inv_tau : g);
         as[c] = a;
         ws[c] = 1.f - a;
     }
@@ -547,9 +550,23 @@ bool gsa_tc_route(const Problem& A, const Problem& B, int64_t m) {
            B.state_mode == GLA_STATE_MATERIALIZED && tc_gsa_slot_read_supported(A) && tc_gsa_slot_read_supported(B);
 }
 
+// The pre-activation gate's expansion, log a = logsigmoid(z) / tau, in front of either route's layout (the
+// backward reuses the forward's with the rest of its workspace).
+float* carve_gate(const GsaProblem& g, Arena& a) {
+    return g.preact ? a.take<float>(size_t(g.B.BH * g.B.L * g.m)) : nullptr;
+}
+
+gla_status expand_gate(const GsaProblem& g, const float* z, float* la, cudaStream_t s) {
+    Problem p = g.A;  // key width m: the gate's layout [BH][L][m]
+    p.gate = GLA_GATE_PREACT;
+    p.inv_tau = g.inv_tau;
+    return gate_expand(p, z, la, s);
+}
+
 size_t gsa_workspace(const GsaProblem& g, bool bwd) {
     Arena a = make_arena(g.B, nullptr, 0);
     a.guard = false;
+    carve_gate(g, a);
     if (g.tc) carve_tc(g, a, bwd);
     else carve_simt(g, a, bwd);
     return a.used;
@@ -560,13 +577,24 @@ gla_status gsa_fwd(const GsaProblem& g, const void* q, const void* k, const void
                    cudaStream_t s) {
     Arena a = make_arena(g.B, ws, cap);
     a.guard = false;
+    float* la_x = carve_gate(g, a);
     if (g.tc) {
         const TcRoute r = carve_tc(g, a, false);
         if (a.used > a.cap) return GLA_ERR_WORKSPACE;
+        if (la_x) {
+            const gla_status st = expand_gate(g, la, la_x, s);
+            if (st != GLA_OK) return st;
+            la = la_x;
+        }
         return tc_route_fwd(g, q, k, v, la, hk0, hv0, o, hkT, hvT, r, s);
     }
     const SimtRoute r = carve_simt(g, a, false);
     if (a.used > a.cap) return GLA_ERR_WORKSPACE;
+    if (la_x) {
+        const gla_status st = expand_gate(g, la, la_x, s);
+        if (st != GLA_OK) return st;
+        la = la_x;
+    }
     return simt_route_fwd(g, q, k, v, la, hk0, hv0, o, hkT, hvT, r, s);
 }
 
@@ -576,14 +604,35 @@ gla_status gsa_bwd(const GsaProblem& g, const void* q, const void* k, const void
                    cudaStream_t s) {
     Arena a = make_arena(g.B, ws, cap);
     a.guard = false;
+    float* la_x = carve_gate(g, a);
+    const float* z = la;
+    gla_status st = GLA_OK;
     if (g.tc) {
         const TcRoute r = carve_tc(g, a, true);
         if (a.used > a.cap) return GLA_ERR_WORKSPACE;
-        return tc_route_bwd(g, q, k, v, la, hk0, hv0, dO, dhkT, dhvT, dq, dk, dv, dla, dhk0, dhv0, reuse, r, s);
+        if (la_x) {
+            // a forward's workspace holds the expansion already
+            if (!reuse) st = expand_gate(g, z, la_x, s);
+            if (st != GLA_OK) return st;
+            la = la_x;
+        }
+        st = tc_route_bwd(g, q, k, v, la, hk0, hv0, dO, dhkT, dhvT, dq, dk, dv, dla, dhk0, dhv0, reuse, r, s);
+    } else {
+        const SimtRoute r = carve_simt(g, a, true);
+        if (a.used > a.cap) return GLA_ERR_WORKSPACE;
+        if (la_x) {
+            if (!reuse) st = expand_gate(g, z, la_x, s);
+            if (st != GLA_OK) return st;
+            la = la_x;
+        }
+        st = simt_route_bwd(g, q, k, v, la, hk0, hv0, dO, dhkT, dhvT, dq, dk, dv, dla, dhk0, dhv0, reuse, r, s);
     }
-    const SimtRoute r = carve_simt(g, a, true);
-    if (a.used > a.cap) return GLA_ERR_WORKSPACE;
-    return simt_route_bwd(g, q, k, v, la, hk0, hv0, dO, dhkT, dhvT, dq, dk, dv, dla, dhk0, dhv0, reuse, r, s);
+    if (st != GLA_OK || !g.preact) return st;
+    // dL/dz = dL/dlog a * sigmoid(-z) / tau, in place
+    Problem p = g.A;
+    p.gate = GLA_GATE_PREACT;
+    p.inv_tau = g.inv_tau;
+    return gate_grad(p, z, dla, dla, s);
 }
 
 }  // namespace gla
@@ -595,7 +644,7 @@ bool gsa_step_supported(int64_t m, int64_t Dk, int64_t Dv) {
 }
 
 gla_status gsa_step(int64_t BH, int64_t m, int64_t Dk, int64_t Dv, bool bf16, const void* q, const void* k,
-                    const void* v, const float* la, float* Km, float* Vm, void* o, cudaStream_t s) {
+                    const void* v, const float* la, float inv_tau, float* Km, float* Vm, void* o, cudaStream_t s) {
     if (!gsa_step_supported(m, Dk, Dv) || BH > 2147483647) return GLA_ERR_UNSUPPORTED;
     const size_t smem = step_smem(m, Dk, Dv);
     if (bf16) {
@@ -604,15 +653,15 @@ gla_status gsa_step(int64_t BH, int64_t m, int64_t Dk, int64_t Dv, bool bf16, co
             return GLA_ERR_CUDA;
         GLA_LAUNCH("gsa_step", k_gsa_step<__nv_bfloat16>, unsigned(BH), kStepThreads, smem, s,
                    static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-                   static_cast<const __nv_bfloat16*>(v), la, Km, Vm, static_cast<__nv_bfloat16*>(o), int(m), int(Dk),
-                   int(Dv));
+                   static_cast<const __nv_bfloat16*>(v), la, inv_tau, Km, Vm, static_cast<__nv_bfloat16*>(o), int(m),
+                   int(Dk), int(Dv));
     } else {
         if (smem > 48 * 1024 &&
             cudaFuncSetAttribute(k_gsa_step<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) != cudaSuccess)
             return GLA_ERR_CUDA;
         GLA_LAUNCH("gsa_step", k_gsa_step<float>, unsigned(BH), kStepThreads, smem, s, static_cast<const float*>(q),
-                   static_cast<const float*>(k), static_cast<const float*>(v), la, Km, Vm, static_cast<float*>(o),
-                   int(m), int(Dk), int(Dv));
+                   static_cast<const float*>(k), static_cast<const float*>(v), la, inv_tau, Km, Vm,
+                   static_cast<float*>(o), int(m), int(Dk), int(Dv));
     }
     return GLA_OK;
 }

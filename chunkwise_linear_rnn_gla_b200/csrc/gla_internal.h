@@ -129,17 +129,22 @@ gla_status tc_bwd(const Problem& p, const void* q, const void* k, const void* v,
 // tc: the tensor-core route (bf16, m = 128, both passes on the tensor-core path, materialised states);
 // otherwise both passes run on the CUDA-core path in fp32 and io_bf16 says whether the caller's q, k, v,
 // o, dO and gradients are bf16 (converted at the boundary).
+// preact: the caller's gate argument is z, log a = logsigmoid(z) * inv_tau (expanded into the workspace
+// first; the gate gradient is scaled by sigmoid(-z) * inv_tau at the end).
 struct GsaProblem {
     Problem A, B;
     int64_t m;
     bool tc;
     bool io_bf16;
+    bool preact = false;
+    float inv_tau = 0.f;
 };
 bool gsa_tc_route(const Problem& A, const Problem& B, int64_t m);
 // Decode step: both memories Km [BH][m][Dk], Vm [BH][m][Dv] (fp32) updated in place, o [BH][Dv].
 bool gsa_step_supported(int64_t m, int64_t Dk, int64_t Dv);
+// inv_tau > 0: la holds the pre-activation z, log a = logsigmoid(z) * inv_tau.
 gla_status gsa_step(int64_t BH, int64_t m, int64_t Dk, int64_t Dv, bool bf16, const void* q, const void* k,
-                    const void* v, const float* la, float* Km, float* Vm, void* o, cudaStream_t s);
+                    const void* v, const float* la, float inv_tau, float* Km, float* Vm, void* o, cudaStream_t s);
 size_t gsa_workspace(const GsaProblem& g, bool bwd);
 gla_status gsa_fwd(const GsaProblem& g, const void* q, const void* k, const void* v, const float* la,
                    const float* hk0, const float* hv0, void* o, float* hkT, float* hvT, void* ws, size_t cap,

@@ -22,9 +22,9 @@ from ._lib import load
 __all__ = ["gsa_fwd", "gsa_bwd", "gsa_step", "gsa_fwd_workspace_size", "gsa_bwd_workspace_size", "gsa_route"]
 
 
-def _desc(q, v, chunk, subchunk, state_mode, impl, flags):
+def _desc(q, v, chunk, subchunk, state_mode, impl, flags, gate="channel", tau=0.0):
     B, H, L, Dk = q.shape
-    return make_desc(B, H, L, Dk, v.shape[-1], _dt(q), chunk, subchunk, state_mode, impl, flags)
+    return make_desc(B, H, L, Dk, v.shape[-1], _dt(q), chunk, subchunk, state_mode, impl, flags, gate, tau)
 
 
 def gsa_route(desc, slots: int) -> str:
@@ -56,16 +56,17 @@ def _check_inputs(q, k, v, log_a):
 
 
 def gsa_fwd(q, k, v, log_a, hk0=None, hv0=None, *, chunk=0, subchunk=0, state_mode="auto", impl="auto",
-            want_state=False, workspace=None, checks=False):
+            want_state=False, workspace=None, checks=False, gate="channel", tau=0.0):
     """Forward. Returns (o, hkT, hvT); the final memories are None unless want_state. Pass the same
-    `workspace` to gsa_bwd(ws_from_fwd=True) to reuse the read weights and layer two's states."""
+    `workspace` to gsa_bwd(ws_from_fwd=True) to reuse the read weights and layer two's states.
+    gate="preact": log_a holds the gate's argument z, log a = logsigmoid(z) / tau."""
     load()
     dev, dt, B, H, L, Dk, Dv, m = _check_inputs(q, k, v, log_a)
     if hk0 is not None:
         _need(hk0, "hk0", (B, H, m, Dk), torch.float32, dev)
     if hv0 is not None:
         _need(hv0, "hv0", (B, H, m, Dv), torch.float32, dev)
-    desc = _desc(q, v, chunk, subchunk, state_mode, impl, _lib.FLAG_CHECKS if checks else 0)
+    desc = _desc(q, v, chunk, subchunk, state_mode, impl, _lib.FLAG_CHECKS if checks else 0, gate, tau)
     o = torch.empty(B, H, L, Dv, dtype=dt, device=dev)
     hkT = torch.empty(B, H, m, Dk, dtype=torch.float32, device=dev) if want_state else None
     hvT = torch.empty(B, H, m, Dv, dtype=torch.float32, device=dev) if want_state else None
@@ -80,10 +81,11 @@ def gsa_fwd(q, k, v, log_a, hk0=None, hv0=None, *, chunk=0, subchunk=0, state_mo
 
 
 def gsa_bwd(q, k, v, log_a, dO, hk0=None, hv0=None, dhkT=None, dhvT=None, *, chunk=0, subchunk=0,
-            state_mode="auto", impl="auto", want_dh0=False, workspace=None, ws_from_fwd=False, checks=False):
-    """Backward of <dO, o> + <dhkT, hkT> + <dhvT, hvT>. Returns a dict with dq, dk, dv, dlog_a and (with
-    want_dh0) dhk0, dhv0. With ws_from_fwd=True `workspace` must be the matching gsa_fwd's, sized for
-    the backward (gsa_bwd_workspace_size)."""
+            state_mode="auto", impl="auto", want_dh0=False, workspace=None, ws_from_fwd=False, checks=False,
+            gate="channel", tau=0.0):
+    """Backward of <dO, o> + <dhkT, hkT> + <dhvT, hvT>. Returns a dict with dq, dk, dv, dlog_a (dL/dz for
+    gate="preact") and (with want_dh0) dhk0, dhv0. With ws_from_fwd=True `workspace` must be the matching
+    gsa_fwd's, sized for the backward (gsa_bwd_workspace_size)."""
     load()
     dev, dt, B, H, L, Dk, Dv, m = _check_inputs(q, k, v, log_a)
     _need(dO, "dO", (B, H, L, Dv), dt, dev)
@@ -94,7 +96,7 @@ def gsa_bwd(q, k, v, log_a, dO, hk0=None, hv0=None, dhkT=None, dhvT=None, *, chu
     if ws_from_fwd and workspace is None:
         raise ValueError("ws_from_fwd needs the forward's workspace")
     flags = (_lib.FLAG_WS_FROM_FWD if ws_from_fwd else 0) | (_lib.FLAG_CHECKS if checks else 0)
-    desc = _desc(q, v, chunk, subchunk, state_mode, impl, flags)
+    desc = _desc(q, v, chunk, subchunk, state_mode, impl, flags, gate, tau)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     dla = torch.empty_like(log_a)
     dhk0 = torch.empty(B, H, m, Dk, dtype=torch.float32, device=dev) if want_dh0 else None
@@ -110,9 +112,9 @@ def gsa_bwd(q, k, v, log_a, dO, hk0=None, hv0=None, dhkT=None, dhvT=None, *, chu
     return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dhk0": dhk0, "dhv0": dhv0}
 
 
-def gsa_step(q, k, v, log_a, hk, hv, o=None, checks=False):
-    """One decode step: q, k [B,H,Dk], v [B,H,Dv], log_a [B,H,m] fp32; the memories hk [B,H,m,Dk] and
-    hv [B,H,m,Dv] (fp32) are updated in place. Returns o [B,H,Dv]."""
+def gsa_step(q, k, v, log_a, hk, hv, o=None, checks=False, gate="channel", tau=0.0):
+    """One decode step: q, k [B,H,Dk], v [B,H,Dv], log_a [B,H,m] fp32 (z for gate="preact"); the memories
+    hk [B,H,m,Dk] and hv [B,H,m,Dv] (fp32) are updated in place. Returns o [B,H,Dv]."""
     load()
     dev, dt = q.device, q.dtype
     B, H, Dk = q.shape
@@ -130,7 +132,7 @@ def gsa_step(q, k, v, log_a, hk, hv, o=None, checks=False):
     if o is None:
         o = torch.empty(B, H, Dv, dtype=dt, device=dev)
     _need(o, "o", (B, H, Dv), dt, dev)
-    desc = make_desc(B, H, 1, Dk, Dv, _dt(q), flags=_lib.FLAG_CHECKS if checks else 0)
+    desc = make_desc(B, H, 1, Dk, Dv, _dt(q), flags=_lib.FLAG_CHECKS if checks else 0, gate=gate, tau=tau)
     with torch.cuda.device(dev):
         st = load().gla_gsa_step(ctypes.byref(desc), m, _ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(hk), _ptr(hv),
                                  _ptr(o), _stream(dev))

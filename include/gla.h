@@ -248,8 +248,10 @@ gla_status gla_state_combine(int64_t G, int64_t BH, int64_t Dk, int64_t Dv, cons
  *
  * Descriptor: B, H, L, Dk (width of q and k), Dv (width of v and o), dtype,
  * chunk, subchunk, impl and state_mode apply to the GLA passes (GLA key width
- * m); `gate` must be GLA_GATE_CHANNEL (log_a is the per-slot gate,
- * GLA_ERR_UNSUPPORTED otherwise); flags: GLA_FLAG_WS_FROM_FWD (backward only:
+ * m); `gate` is GLA_GATE_CHANNEL (log_a is the per-slot log gate) or
+ * GLA_GATE_PREACT (log_a holds the gate's argument z and log a = logsigmoid(z) / gate_tau; the
+ * backward then returns dL/dz in dlog_a), other kinds GLA_ERR_UNSUPPORTED; flags:
+ * GLA_FLAG_WS_FROM_FWD (backward only:
  * `workspace` holds the matching gla_gsa_fwd's workspace, same inputs and
  * options) and GLA_FLAG_CHECKS (gate domain and finite outputs, reported by
  * gla_check_device_error). bf16 with m = 128 and Dk, Dv multiples of 64 takes
@@ -276,9 +278,9 @@ gla_status gla_gsa_fwd(const gla_desc* d, int32_t slots, const void* q, const vo
                        const float* log_a, const float* hk0, const float* hv0, void* o, float* hkT,
                        float* hvT, void* workspace, size_t workspace_bytes, void* stream);
 /* One decode step of gated slot attention for a batch of single tokens: q, k [B,H,Dk], v [B,H,Dv]
- * (d->dtype), log_a [B,H,slots] (fp32), the memories Kmem [B,H,slots,Dk] and Vmem [B,H,slots,Dv] (fp32,
- * updated in place: the step's hkT / hvT), o [B,H,Dv] (d->dtype). d->L is ignored; d->gate must be
- * GLA_GATE_CHANNEL; Dk and Dv multiples of 4. Applied L times from hk0 / hv0 it gives what gla_gsa_fwd
+ * (d->dtype), log_a [B,H,slots] (fp32, or z with GLA_GATE_PREACT), the memories Kmem [B,H,slots,Dk]
+ * and Vmem [B,H,slots,Dv] (fp32, updated in place: the step's hkT / hvT), o [B,H,Dv] (d->dtype). d->L is
+ * ignored; Dk and Dv multiples of 4. Applied L times from hk0 / hv0 it gives what gla_gsa_fwd
  * gives for those L tokens. GLA_FLAG_CHECKS checks the gate domain and that o and both memories are
  * finite. */
 gla_status gla_gsa_step(const gla_desc* d, int32_t slots, const void* q, const void* k, const void* v,

@@ -135,6 +135,8 @@ def test_gsa_rejects_bad_arguments(lib):
     assert gsa_route(lib, 0, dtype=1)[0] == _lib.GLA_ERR_INVALID_ARG
     assert gsa_route(lib, 128, dtype=1, gate=1)[0] == _lib.GLA_ERR_UNSUPPORTED  # slot gates are per slot
     assert gsa_route(lib, 128, dtype=1, gate=9)[0] == _lib.GLA_ERR_INVALID_ARG
+    assert gsa_route(lib, 128, dtype=1, gate=3)[0] == _lib.GLA_ERR_INVALID_ARG  # pre-activation needs tau > 0
+    assert gsa_route(lib, 128, dtype=1, gate=3, gate_tau=8.0, Dk=128, Dv=128) == (0, _lib.IMPL["tc"])
     assert gsa_route(lib, 128, dtype=1, flags=0x40)[0] == _lib.GLA_ERR_INVALID_ARG
     d = desc(dtype=1, L=64, Dk=128, Dv=128)
     ptr = ctypes.c_void_p(256)

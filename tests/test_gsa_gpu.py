@@ -164,3 +164,35 @@ def test_gsa_step_continues_the_forward():
     compare("o (steps)", torch.stack(outs, dim=2), ref["o"][:, :, L:], "bf16")
     compare("hkT", hk, ref["hkT"], "bf16")
     compare("hvT", hv, ref["hvT"], "bf16")
+
+
+# ---------------------------------------------------------------- pre-activation gate
+@pytest.mark.parametrize("dtype,Dk,Dv,m", [("bf16", 128, 128, 128), ("f32", 64, 32, 16)])
+def test_gsa_preact_gate(dtype, Dk, Dv, m):
+    """gate="preact": the caller passes z, log a = logsigmoid(z) / tau; the backward returns
+    dL/dz = dL/dlog a * sigmoid(-z) / tau. Against the oracle run on log a, on both routes: forward,
+    backward and a decode step continuing the forward's memories."""
+    tau = 8.0
+    inp = make_gsa_inputs(1, 2, 333, Dk, Dv, m, dtype, seed=11, q_scale=4.0, h0=True, dhT=True)
+    z = torch.randn(inp["log_a"].shape, generator=torch.Generator().manual_seed(12)) * 2.0
+    inp["log_a"] = (torch.nn.functional.logsigmoid(z) / tau).float()  # what the oracle reads
+    zz = z.numpy().astype(np.float64)
+    ref = run_oracle(inp)
+    d = to_dev(inp)
+    zd = z.float().contiguous().to("cuda")
+    kw = dict(gate="preact", tau=tau)
+    o, hkT, hvT = gsa.gsa_fwd(d["q"], d["k"], d["v"], zd, d["hk0"], d["hv0"], want_state=True, **kw)
+    g = gsa.gsa_bwd(d["q"], d["k"], d["v"], zd, d["dO"], d["hk0"], d["hv0"], d["dhkT"], d["dhvT"], want_dh0=True,
+                    **kw)
+    torch.cuda.synchronize()
+    for n, got in (("o", o), ("hkT", hkT), ("hvT", hvT), ("dq", g["dq"]), ("dk", g["dk"]), ("dv", g["dv"])):
+        compare(n, got, ref[n], dtype)
+    compare("dz", g["dlog_a"], ref["dlog_a"] / (1.0 + np.exp(zz)) / tau, dtype)
+    # one decode step from the final memories continues it
+    hk, hv = hkT.clone(), hvT.clone()
+    step = {n: d[n][:, :, -1].contiguous() for n in ("q", "k", "v")}
+    o1 = gsa.gsa_step(step["q"], step["k"], step["v"], zd[:, :, -1].contiguous(), hk, hv, **kw)
+    torch.cuda.synchronize()
+    f = {n: to_f64_numpy(inp[n][:, :, -1:]) for n in ("q", "k", "v", "log_a")}
+    ref1 = oracle.gsa_fwd(f["q"], f["k"], f["v"], f["log_a"], ref["hkT"], ref["hvT"])
+    compare("o (step)", o1, ref1[0][:, :, 0], dtype)
