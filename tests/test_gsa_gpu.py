@@ -72,7 +72,7 @@ def test_gsa_f32_one_step():
 
 
 # ---------------------------------------------------------------- tensor-core path (bf16, m = 128 or 256)
-@pytest.mark.parametrize("L,Dk,Dv", [(600, 128, 128), (389, 256, 512), (256, 64, 192)])
+@pytest.mark.parametrize("L,Dk,Dv", [(600, 128, 128), (389, 256, 512), (256, 64, 192), (1, 128, 128), (129, 128, 64)])
 def test_gsa_bf16_tensor_core(L, Dk, Dv):
     inp = make_gsa_inputs(1, 2, L, Dk, Dv, 128, "bf16", seed=3, q_scale=4.0, h0=True, dhT=True)
     assert route_of(inp) == "tc"
