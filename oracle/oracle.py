@@ -40,26 +40,43 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
-def _load():
+def _declare(lib):
+    lib.gla_oracle_fwd.argtypes = [_i64] * 5 + [_dp] * 7
+    lib.gla_oracle_fwd.restype = None
+    lib.gla_oracle_step.argtypes = [_i64] * 4 + [_dp] * 6
+    lib.gla_oracle_step.restype = None
+    lib.gla_oracle_bwd.argtypes = [_i64] * 5 + [_dp] * 13 + [_i64]
+    lib.gla_oracle_bwd.restype = None
+    lib.gsa_oracle_fwd.argtypes = [_i64] * 6 + [_dp] * 10
+    lib.gsa_oracle_fwd.restype = None
+    lib.gsa_oracle_bwd.argtypes = [_i64] * 6 + [_dp] * 15 + [_i64]
+    lib.gsa_oracle_bwd.restype = None
+    lib.gla_oracle_num_threads.restype = ctypes.c_int
+    lib.gla_oracle_set_threads.argtypes = [ctypes.c_int]
+    return lib
+
+
+def _load(lib=None):
     global _lib
+    if lib is not None:
+        return lib
     with _lock:
         if _lib is None:
             build()
-            lib = ctypes.CDLL(_LIB)
-            lib.gla_oracle_fwd.argtypes = [_i64] * 5 + [_dp] * 7
-            lib.gla_oracle_fwd.restype = None
-            lib.gla_oracle_step.argtypes = [_i64] * 4 + [_dp] * 6
-            lib.gla_oracle_step.restype = None
-            lib.gla_oracle_bwd.argtypes = [_i64] * 5 + [_dp] * 13 + [_i64]
-            lib.gla_oracle_bwd.restype = None
-            lib.gsa_oracle_fwd.argtypes = [_i64] * 6 + [_dp] * 10
-            lib.gsa_oracle_fwd.restype = None
-            lib.gsa_oracle_bwd.argtypes = [_i64] * 6 + [_dp] * 15 + [_i64]
-            lib.gsa_oracle_bwd.restype = None
-            lib.gla_oracle_num_threads.restype = ctypes.c_int
-            lib.gla_oracle_set_threads.argtypes = [ctypes.c_int]
-            _lib = lib
+            _lib = _declare(ctypes.CDLL(_LIB))
     return _lib
+
+
+def with_library(path: str):
+    """The oracle's functions bound to another build of its C sources (the mutation tests load copies with
+    a planted mistake to show that the pins catch it). Returns a namespace with fwd, bwd, step, gsa_fwd
+    and gsa_bwd."""
+    import functools
+    import types
+
+    lib = _declare(ctypes.CDLL(path))
+    return types.SimpleNamespace(**{f.__name__: functools.partial(f, lib=lib)
+                                    for f in (fwd, bwd, step, gsa_fwd, gsa_bwd)})
 
 
 def _c(a):
@@ -80,9 +97,9 @@ def set_threads(n: int) -> None:
     _load().gla_oracle_set_threads(int(n))
 
 
-def fwd(q, k, v, log_a, h0=None):
+def fwd(q, k, v, log_a, h0=None, lib=None):
     """Step recurrence forward. Returns (o [B,H,L,V], hT [B,H,K,V]) in fp64."""
-    lib = _load()
+    lib = _load(lib)
     q, k, v, log_a = _c(q), _c(k), _c(v), _c(log_a)
     B, H, L, K = q.shape
     V = v.shape[-1]
@@ -96,13 +113,13 @@ def fwd(q, k, v, log_a, h0=None):
     return o, hT
 
 
-def bwd(q, k, v, log_a, dO, h0=None, dhT=None, seg: int = 64):
+def bwd(q, k, v, log_a, dO, h0=None, dhT=None, seg: int = 64, lib=None):
     """Reverse-mode gradients of <dO, o> + <dhT, hT>.
 
     Returns a dict with dq, dk, dv, dlog_a (direct chain rule), dlog_a_cf
     (closed form: reverse cumsum of q*dq - k*dk plus the dhT*hT term) and dh0.
     """
-    lib = _load()
+    lib = _load(lib)
     q, k, v, log_a, dO = _c(q), _c(k), _c(v), _c(log_a), _c(dO)
     B, H, L, K = q.shape
     V = v.shape[-1]
@@ -119,12 +136,12 @@ def bwd(q, k, v, log_a, dO, h0=None, dhT=None, seg: int = 64):
     return {"dq": dq, "dk": dk, "dv": dv, "dlog_a": dla, "dlog_a_cf": dla_cf, "dh0": dh0}
 
 
-def step(q, k, v, log_a, S):
+def step(q, k, v, log_a, S, lib=None):
     """One decode step. q,k,log_a [B,H,K]; v [B,H,V]; S [B,H,K,V].
 
     Returns (o [B,H,V], S_new); the input S is not modified.
     """
-    lib = _load()
+    lib = _load(lib)
     q, k, v, log_a = _c(q), _c(k), _c(v), _c(log_a)
     S = np.array(S, dtype=np.float64, copy=True, order="C")
     B, H, K = q.shape
@@ -135,13 +152,13 @@ def step(q, k, v, log_a, S):
 
 
 # ---- gated slot attention (gsa_oracle.c) ------------------------------------------------------------
-def gsa_fwd(q, k, v, log_a, hk0=None, hv0=None):
+def gsa_fwd(q, k, v, log_a, hk0=None, hv0=None, lib=None):
     """Gated slot attention forward, step by step in fp64.
 
     q, k [B,H,L,K]; v [B,H,L,V]; log_a [B,H,L,m]; hk0 [B,H,m,K], hv0 [B,H,m,V] (None = zero).
     Returns (o [B,H,L,V], s [B,H,L,m] read weights, hkT [B,H,m,K], hvT [B,H,m,V]).
     """
-    lib = _load()
+    lib = _load(lib)
     q, k, v, log_a = _c(q), _c(k), _c(v), _c(log_a)
     B, H, L, K = q.shape
     V, m = v.shape[-1], log_a.shape[-1]
@@ -157,12 +174,12 @@ def gsa_fwd(q, k, v, log_a, hk0=None, hv0=None):
     return o, s, hkT, hvT
 
 
-def gsa_bwd(q, k, v, log_a, dO, hk0=None, hv0=None, dhkT=None, dhvT=None, seg: int = 64):
+def gsa_bwd(q, k, v, log_a, dO, hk0=None, hv0=None, dhkT=None, dhvT=None, seg: int = 64, lib=None):
     """Reverse-mode gradients of <dO, o> + <dhkT, hkT> + <dhvT, hvT> for gated slot attention.
 
     Returns a dict with dq, dk, dv, dlog_a, dhk0, dhv0.
     """
-    lib = _load()
+    lib = _load(lib)
     q, k, v, log_a, dO = _c(q), _c(k), _c(v), _c(log_a), _c(dO)
     B, H, L, K = q.shape
     V, m = v.shape[-1], log_a.shape[-1]
