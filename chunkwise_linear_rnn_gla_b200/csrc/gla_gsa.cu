@@ -424,15 +424,18 @@ __global__ void __launch_bounds__(kStepThreads) k_gsa_step(const T* __restrict__
                                                            float* __restrict__ Vm, T* __restrict__ o, int m, int Dk,
                                                            int Dv) {
     extern __shared__ float sh[];
-    float* qs = sh;
-    float* ks = qs + Dk;
-    float* vs = ks + Dk;
+    // the arrays read as float4 first (Dk and Dv are multiples of 4, so every one starts on 16 bytes),
+    // then the per-slot scalars
+    const int nw = blockDim.x >> 5;
+    float* op = sh;            // [warps][Dv]
+    float* qs = op + nw * Dv;  // [Dk]
+    float* ks = qs + Dk;       // [Dk]
+    float* vs = ks + Dk;       // [Dv]
     float* as = vs + Dv;
     float* ws = as + m;
     float* zs = ws + m;
-    float* op = zs + m;  // [warps][Dv]
     const int64_t bh = blockIdx.x;
-    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5, nw = blockDim.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
     for (int i = tid; i < Dk; i += blockDim.x) {
         qs[i] = ldf(q + bh * Dk + i);
         ks[i] = ldf(k + bh * Dk + i);

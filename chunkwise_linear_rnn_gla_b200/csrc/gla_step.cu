@@ -6,12 +6,13 @@
 // Hardware-Efficient Training", atlas.scime.ai summary, "Approach").
 //
 // The step is a pure stream over the fp32 state (read + write 8*Dk*Dv bytes
-// per head), so the kernel is laid out for HBM: each thread owns four
-// adjacent state columns (16-byte loads/stores, a warp covers 512 contiguous
-// bytes of one state row), a block covers up to 128 columns of one head, and
-// the Dk rows are split over KS row-slices whose partial q.S sums are reduced
-// in shared memory. Each thread loads a batch of rows before storing any, so
-// that the stream has enough loads in flight when the state comes from HBM.
+// per head), so the kernels are laid out for HBM. The default kernel gives
+// each head one block of 16 warps; a warp streams whole state rows, four at a
+// time with their 16-byte loads in flight together, and o is reduced over the
+// warps in shared memory. The fallback (unaligned or very wide states) gives
+// each thread four adjacent state columns of a batch of rows: a block covers
+// up to 128 columns of one head, and the Dk rows are split over KS row-slices
+// whose partial q.S sums are reduced in shared memory.
 
 #include <cstdint>
 
@@ -119,6 +120,73 @@ __global__ void __launch_bounds__(kStepThreads) k_step(const T* __restrict__ q, 
     }
 }
 
+// Row-major kernel (the default): one block of 512 threads per head; a warp takes four state rows at a
+// time, their 16-byte loads issued together with the lanes spread over the columns, so that every warp
+// streams whole 1 KB rows; o sums the warps' partial rows through shared memory in a fixed order.
+constexpr int kRowThreads = 512;
+constexpr int kRowBatch = 4;
+
+template <typename T>
+__global__ void __launch_bounds__(kRowThreads) k_step_rows(const T* __restrict__ q, const T* __restrict__ k,
+                                                           const T* __restrict__ v, GateArgs la,
+                                                           float* __restrict__ S, T* __restrict__ o, int K, int V) {
+    extern __shared__ float sm[];
+    // the arrays read as float4 first (V is a multiple of 4, so every one starts on 16 bytes), then the
+    // per-row scalars
+    const int nw = blockDim.x >> 5;
+    float* op = sm;            // [warps][V]
+    float* vs = op + nw * V;   // [V]
+    float* sq = vs + V;
+    float* sk = sq + K;
+    float* sa = sk + K;
+    const int64_t bh = blockIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, wp = tid >> 5;
+    for (int c = tid; c < K; c += blockDim.x) {
+        sq[c] = ldf(q + bh * K + c);
+        sk[c] = ldf(k + bh * K + c);
+        sa[c] = expf(gate_log_alpha(la, bh, 0, c, 1, K));
+    }
+    for (int x = tid; x < V; x += blockDim.x) vs[x] = ldf(v + bh * V + x);
+    for (int i = tid; i < nw * V; i += blockDim.x) op[i] = 0.f;
+    __syncthreads();
+    const int v4n = V / 4;
+    float4* S4 = reinterpret_cast<float4*>(S + bh * int64_t(K) * V);
+    const float4* v4 = reinterpret_cast<const float4*>(vs);
+    float4* o4 = reinterpret_cast<float4*>(op + wp * V);
+    for (int c0 = wp * kRowBatch; c0 < K; c0 += nw * kRowBatch) {
+        for (int x4 = lane; x4 < v4n; x4 += 32) {
+            float4 r[kRowBatch];
+#pragma unroll
+            for (int u = 0; u < kRowBatch; ++u)
+                if (c0 + u < K) r[u] = S4[int64_t(c0 + u) * v4n + x4];
+            const float4 vv = v4[x4];
+            float4 acc = o4[x4];
+#pragma unroll
+            for (int u = 0; u < kRowBatch; ++u) {
+                if (c0 + u >= K) continue;
+                const float a = sa[c0 + u], kc = sk[c0 + u], qc = sq[c0 + u];
+                float4 y = r[u];
+                y.x = fmaf(a, y.x, kc * vv.x);
+                y.y = fmaf(a, y.y, kc * vv.y);
+                y.z = fmaf(a, y.z, kc * vv.z);
+                y.w = fmaf(a, y.w, kc * vv.w);
+                S4[int64_t(c0 + u) * v4n + x4] = y;
+                acc.x = fmaf(qc, y.x, acc.x);
+                acc.y = fmaf(qc, y.y, acc.y);
+                acc.z = fmaf(qc, y.z, acc.z);
+                acc.w = fmaf(qc, y.w, acc.w);
+            }
+            o4[x4] = acc;
+        }
+    }
+    __syncthreads();
+    for (int x = tid; x < V; x += blockDim.x) {
+        float acc = 0.f;
+        for (int w2 = 0; w2 < nw; ++w2) acc += op[w2 * V + x];
+        stf(o + bh * V + x, acc);
+    }
+}
+
 template <typename T>
 gla_status step_typed(const Problem& p, const T* q, const T* k, const T* v, const float* g, float* S, T* o,
                       cudaStream_t s) {
@@ -126,6 +194,15 @@ gla_status step_typed(const Problem& p, const T* q, const T* k, const T* v, cons
     const int K = int(p.K), V = int(p.V);
     // 16-byte state accesses need a 16-byte aligned state and rows of a multiple of 4 floats
     const bool vec = (V % 4) == 0 && (reinterpret_cast<uintptr_t>(S) & 15) == 0;
+    {
+        // the row-major kernel, while its per-warp partial rows fit the default shared memory
+        const size_t smem = sizeof(float) * (3 * size_t(K) + size_t(V) + size_t(kRowThreads / 32) * V);
+        if (vec && smem <= 48 * 1024) {
+            GLA_LAUNCH("step", k_step_rows<T>, unsigned(p.BH), kRowThreads, smem, s, q, k, v, la, S, o, K, V);
+            return GLA_OK;
+        }
+    }
+    // otherwise (unaligned or very wide states) the column-sliced kernel below
     const int VEC = vec ? 4 : 1;
     const int ncols = V / VEC;
     // 32 column groups (512 bytes of a state row per warp) and 8 row-slices per block: several

@@ -131,7 +131,7 @@ def test_gsa_workload_full_size():
 
 # ---------------------------------------------------------------- decode step
 @pytest.mark.parametrize("dtype,Dk,Dv,m", [("f32", 64, 32, 16), ("f32", 96, 40, 24), ("bf16", 128, 256, 128),
-                                           ("bf16", 256, 512, 128)])
+                                           ("bf16", 256, 512, 128), ("f32", 32, 20, 5), ("bf16", 4, 4, 3)])
 def test_gsa_step_matches_oracle(dtype, Dk, Dv, m):
     """T single-token steps from given memories equal the oracle over those T tokens (o at every step, the
     final memories)."""
