@@ -414,11 +414,11 @@ gla_status simt_route_bwd(const GsaProblem& g, const void* q, const void* k, con
 // A warp takes four slot rows at a time (their loads issued together, 16 bytes per lane); the row dot
 // products reduce by shuffles, the softmax runs in one warp, and o sums the warps' partial rows through
 // shared memory in a fixed order.
-constexpr int kStepThreads = 512;
+constexpr int kStepThreads = 512;  // two blocks per SM (at most 64 registers a thread): 256 heads stay one wave
 constexpr int kStepRows = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(kStepThreads) k_gsa_step(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(kStepThreads, 2) k_gsa_step(const T* __restrict__ q, const T* __restrict__ k,
                                                            const T* __restrict__ v, const float* __restrict__ la,
                                                            float inv_tau, float* __restrict__ Km,
                                                            float* __restrict__ Vm, T* __restrict__ o, int m, int Dk,

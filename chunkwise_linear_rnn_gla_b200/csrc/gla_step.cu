@@ -123,11 +123,11 @@ __global__ void __launch_bounds__(kStepThreads) k_step(const T* __restrict__ q, 
 // Row-major kernel (the default): one block of 512 threads per head; a warp takes four state rows at a
 // time, their 16-byte loads issued together with the lanes spread over the columns, so that every warp
 // streams whole 1 KB rows; o sums the warps' partial rows through shared memory in a fixed order.
-constexpr int kRowThreads = 512;
+constexpr int kRowThreads = 512;  // two blocks per SM (at most 64 registers a thread)
 constexpr int kRowBatch = 4;
 
 template <typename T>
-__global__ void __launch_bounds__(kRowThreads) k_step_rows(const T* __restrict__ q, const T* __restrict__ k,
+__global__ void __launch_bounds__(kRowThreads, 2) k_step_rows(const T* __restrict__ q, const T* __restrict__ k,
                                                            const T* __restrict__ v, GateArgs la,
                                                            float* __restrict__ S, T* __restrict__ o, int K, int V) {
     extern __shared__ float sm[];
