@@ -29,8 +29,8 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-# ~1 ms of device spin (at ~1.9 GHz) between an L2 flush and the start event of a single-call timing:
-# longer than the host needs to marshal and launch any one timed call
+# ~1 ms of device spin (at ~1.9 GHz) between an L2 flush and the start event of a timed call or step:
+# longer than the host needs to marshal and launch it, so the window holds device time only
 HOLD_CYCLES = 2_000_000
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -326,7 +326,7 @@ def gsa_model(B, H, L, K, V, m, C=128):
             "per_token_head": {"bytes": fwd_b + bwd_b, "flops": f_fwd + f_bwd}}
 
 
-def run_gsa(dev, peaks, med_ms, with_cpu=True):
+def run_gsa(dev, peaks, med_ms, flush, with_cpu=True):
     """Gated slot attention, 1.3B-layer shape with 128 slots: device time of fwd+bwd (the backward
     reusing the forward's workspace), the layer roofline of the method's own bytes and FLOPs, the
     per-kernel breakdown from the library's event hooks, and the fp64 oracle on a bounded sample."""
@@ -350,12 +350,15 @@ def run_gsa(dev, peaks, med_ms, with_cpu=True):
     ms = med_ms(fn)
     alg = gsa_model(B, H, L, K, V, m)
     lr = layer_roofline(alg["bytes"], alg["flops"], ms, peaks)
-    # per-kernel device time (an event pair around every launch; shares, not the headline)
+    # per-kernel device time (an event pair around every launch; shares, not the headline), L2 flushed
+    # and the stream held until the step is queued, as for the GLA step
     fn()
     torch.cuda.synchronize(dev)
     gla.gla_profile_reset()
     gla.gla_profile_enable(True)
     for _ in range(3):
+        flush.fill_(1.0)
+        torch.cuda._sleep(HOLD_CYCLES)
         fn()
     torch.cuda.synchronize(dev)
     gla.gla_profile_enable(False)
@@ -478,7 +481,7 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
         del inp, d, o, hT, outs
         torch.cuda.empty_cache()
 
-    out["gsa1p3b_fwdbwd"] = run_gsa(dev, peaks, med_ms, with_cpu)
+    out["gsa1p3b_fwdbwd"] = run_gsa(dev, peaks, med_ms, flush, with_cpu)
 
     # decode: B=64, H=4, d_k=128, d_v=256, one token per call, fp32 state carried
     B, H, K, V = (DECODE[n] for n in ("B", "H", "K", "V"))
@@ -681,6 +684,9 @@ def main():
         gla.gla_profile_enable(kernel_events)
         for i in range(args.steps):
             flush.fill_(float(i))  # evict L2 (126 MB) between timed steps
+            # hold the stream until the host has queued the whole step, so that no launch waits on the
+            # host inside the window (the eager passes issue every kernel from Python)
+            torch.cuda._sleep(HOLD_CYCLES)
             ev[i][0].record(stream)
             if use_graph:
                 graph.replay()

@@ -71,6 +71,7 @@ def time_layer(w, flush):
             gla_profile_reset()
             for _ in range(3):
                 flush.zero_()
+                torch.cuda._sleep(HOLD_CYCLES)
                 fn()
             torch.cuda.synchronize()
             gla_profile_enable(False)
@@ -105,6 +106,7 @@ def time_gsa(flush, reps=10):
             gla_profile_reset()
             for _ in range(3):
                 flush.zero_()
+                torch.cuda._sleep(HOLD_CYCLES)
                 fn()
             torch.cuda.synchronize()
             gla_profile_enable(False)
