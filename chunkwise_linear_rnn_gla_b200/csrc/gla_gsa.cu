@@ -22,11 +22,14 @@
 //     (its dk, dv and dlog_a; its closed-form gate gradient holds as is);
 //   the gate: dlog_a = dla_1 + dla_2 - a * (dw_1 + dw_2).
 // Every step runs in the library's kernels. Two routes:
-//  - tensor cores (bf16, m = 128): the GLA walks, preparation, output and
-//    backward kernels, each memory walked once (the backward reuses the
-//    forward's chunk states), plus the slot-read kernel (gla_gsa_read.cu) that
-//    evaluates the logits and the read gradient in fp32 with the softmax and
-//    its backward fused;
+//  - tensor cores (bf16, m = 128): the GLA walk, output and backward kernels,
+//    each memory walked once (the backward reuses the forward's chunk states),
+//    plus two kernels of this method (gla_gsa_read.cu): the slot gate's
+//    preparation (w and the walks' operands, for both layers) and the slot
+//    read, which evaluates the logits and the read gradient in fp32 with the
+//    softmax and its backward fused, and whose epilogue also forms the next
+//    layer's query operands (Q~ and the masked scores), so no separate GLA
+//    preparation runs;
 //  - CUDA cores (every other shape): the GLA passes in fp32 (bf16 tensors are
 //    converted at the boundary), the logits as the query gradient of layer
 //    one, and the elementwise kernels below.
@@ -193,20 +196,21 @@ TcRoute carve_tc(const GsaProblem& g, Arena& a, bool bwd) {
 }
 
 // w, both memories' chunk states (walks with GLA key w over k and over v), the read weights s, and layer
-// two's preparation (query s, key w). hkT / hvT (nullable) receive the final memories.
+// two's preparation (query s, key w): its K~ and e^Gamma from the gate preparation, its Q~ and scores P
+// from the slot read's epilogue. hkT / hvT (nullable) receive the final memories.
 gla_status tc_forward_state(const GsaProblem& g, const void* q, const void* k, const void* v, const float* la,
                             const float* hk0, const float* hv0, float* hkT, float* hvT, const TcRoute& r,
                             TcBuffers& A, TcBuffers& B, cudaStream_t s) {
     // w, and the walks' operands K~ = w e^{Gamma - B} and e^Gamma
-    gla_status st = tc_gsa_gate_prep_launch(g.A, la, r.w, A.Kt, A.gam, s);
+    gla_status st = tc_gsa_gate_prep_launch(g.A, la, r.w, A.Kt, A.gam, B.Kt, B.gam, s);
     if (st == GLA_OK)
         st = tc_states_walk_launch(g.A, A.Kt, static_cast<const __nv_bfloat16*>(k), A.gam, hk0, hkT, A.hT, A.states,
                                    A.segbuf, false, s, "tc_walk_states");
     if (st == GLA_OK)
         st = tc_states_walk_launch(g.B, A.Kt, static_cast<const __nv_bfloat16*>(v), A.gam, hv0, hvT, B.hT, B.states,
                                    B.segbuf, false, s, "tc_walk_states");
-    if (st == GLA_OK) st = tc_gsa_slot_read_launch(g.A, q, k, A.states, la, nullptr, r.s_b, r.s_f, 0, s);
-    if (st == GLA_OK) st = tc_prep_launch(g.B, r.s_b, r.w, la, B.Qt, B.Kt, B.P, B.gam, GLA_GATE_CHANNEL, s);
+    if (st == GLA_OK)
+        st = tc_gsa_slot_read_launch(g.A, q, k, A.states, la, nullptr, r.s_b, r.s_f, B.Qt, B.P, 0, s);
     return st;
 }
 
@@ -237,14 +241,14 @@ gla_status tc_route_bwd(const GsaProblem& g, const void* q, const void* k, const
     Arena bB = make_arena(g.B, r.wsB, r.capB);
     st = tc_bwd(pB, r.s_b, r.w, v, la, hv0, dO, dhvT, r.junk, r.dw2, dv, dla, dhv0, bB, s);
     // G = dL/dlogits: the read of the value memory with dO, through the softmax backward
-    if (st == GLA_OK) st = tc_gsa_slot_read_launch(g.B, dO, v, B.states, la, r.s_f, r.G, nullptr, 1, s);
+    // with layer one's chunk-local operands (query G; K~ and e^Gamma are the gate preparation's)
+    if (st == GLA_OK)
+        st = tc_gsa_slot_read_launch(g.B, dO, v, B.states, la, r.s_f, r.G, nullptr, A.Qt, A.P, 1, s);
     if (st != GLA_OK) return st;
     // layer one (query G, key w, value k) from the stored key memory: dq is its output, then its backward
     // with dO = q gives dk (its dv), the gradient of w (its dk) and its gate gradient
-    st = tc_prep_launch(g.A, r.G, r.w, la, A.Qt, A.Kt, A.P, A.gam, GLA_GATE_CHANNEL, s);
-    if (st == GLA_OK)
-        st = tc_chunk_out_launch(g.A, A.Qt, A.states, A.P, static_cast<const __nv_bfloat16*>(k), false,
-                                 static_cast<__nv_bfloat16*>(dq), false, s, "tc_output");
+    st = tc_chunk_out_launch(g.A, A.Qt, A.states, A.P, static_cast<const __nv_bfloat16*>(k), false,
+                             static_cast<__nv_bfloat16*>(dq), false, s, "tc_output");
     if (st != GLA_OK) return st;
     Problem pA = g.A;
     pA.flags = GLA_FLAG_WS_FROM_FWD;

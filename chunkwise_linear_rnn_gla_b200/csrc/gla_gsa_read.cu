@@ -25,6 +25,15 @@
 // MMA issuer, 16 compute warps: the gate cumsum (4 threads per slot, 32 rows
 // each), then the epilogue (4 threads per token row, 32 slot columns each; the
 // softmax and <s, r> combine the four partial results through shared memory).
+//
+// The kernel's result x (the read weights s, or the logit gradient G) is the
+// query of the next GLA layer, whose key is w under the same gate. So the
+// epilogue also forms that layer's chunk-local operands, as the GLA preparation
+// would: Q~ = x e^{B} (bf16, stored and staged as a K-major operand in the
+// free part of the ring) and the masked score block P = Q~ Phi^T (s <= j), one
+// more tcgen05.mma into TMEM cols [0,128) with Phi = w e^{-B} as the K-major B
+// operand, plus exact log-space terms x_jc w_sc e^{B_jc - B_sc} for the slots
+// beyond the range bound (their Phi columns are zero).
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -55,9 +64,10 @@ constexpr float kBound2 = 64.f * kLog2e;  // range bound in base-2 units
 
 struct SRBars {
     uint64_t full[2], empty[2];
-    uint64_t a_full, p_ready, phi_ready, l_full, s_full, drain;
+    uint64_t a_full, p_ready, phi_ready, l_full, s_full, qt_ready, q_full, drain;
     uint32_t tmem_slot;
     int abort_flag;
+    int any_beyond;            // some slot of the chunk is beyond the range bound
     uint32_t flag[kSlots];     // 1: the slot's chunk decay passes the range bound
     float tot[kQ][kSlots];     // cumsum: each thread's partial sum over its rows
     float red[2][kQ][C];       // epilogue: per-row partial reductions of the column groups
@@ -65,15 +75,21 @@ struct SRBars {
 
 constexpr size_t kRing = size_t(2) * 3 * PIECE;          // x, y, M pieces, two stages
 constexpr size_t kPhi = size_t(2) * PIECE;               // Phi [128 tokens x 128 slots] bf16
-constexpr size_t kBs = size_t(C) * kSlots * sizeof(float);  // B (base 2) [128 x 128] fp32
+constexpr size_t kBs = size_t(C) * kSlots * sizeof(float);  // e^B, or B (base 2) beyond the bound [128 x 128] fp32
 constexpr size_t kSmem = 1024 + kRing + kPhi + kBs + sizeof(SRBars);
 
 // The read gradient's s tile (fp32 [128 rows x 128 slots], four TMA boxes of 32 columns with the 128-byte
 // swizzle) goes to the ring once the D loop is done, into the four 16 KB pieces that P1 does not use.
 __device__ __forceinline__ uint32_t s_piece(int p) { return uint32_t(2 + p) * PIECE; }
 
-// B2[t][c] lives at t * 128 + (c ^ (t & 31)): a warp reading one column over 32 rows (epilogue) or one
-// row over 32 columns (cumsum) touches 32 different banks.
+// The next layer's query operand Q~ (two K-major pieces): the ring's last two pieces in the forward read
+// (the staged s rows take the first four), the first two (P1's, free after the second GEMM and the exact
+// terms) in the read gradient (the s tile takes the other four).
+template <int MODE>
+__device__ __forceinline__ uint32_t qt_piece() { return MODE == 0 ? 4u * PIECE : 0u; }
+
+// The table entry of (t, c) lives at t * 128 + (c ^ (t & 31)): a warp reading one column over 32 rows
+// (epilogue) or one row over 32 columns (cumsum) touches 32 different banks.
 __device__ __forceinline__ int bs_idx(int t, int c) { return t * kSlots + (c ^ (t & 31)); }
 
 // bf16 write weight, exactly as the elementwise kernel that feeds the GLA passes rounds it
@@ -92,6 +108,37 @@ __device__ __noinline__ float exact_intra(const uint8_t* p1, const float* Bs, co
     return acc;
 }
 
+// e^{min(B, 0)} of row r, slot c: the table holds e^B, or B itself for a slot beyond the range bound
+__device__ __forceinline__ float e_b(const float* Bs, int r, int c, bool beyond) {
+    const float b = Bs[bs_idx(r, c)];
+    // exponents are <= 0 in exact arithmetic; the clamp absorbs cumsum rounding
+    return beyond ? exp2_ftz(fminf(b, 0.f)) : fminf(b, 1.f);
+}
+
+// The next layer's query operand from this thread's 32 columns of row r: Q~ = x e^{B} (one rounding to bf16)
+// into the K-major operand in shared memory (16-byte chunks) and, for a valid row, into global memory
+// (qg: the row's first column of the thread). fmask: the columns' slots beyond the range bound.
+__device__ __forceinline__ void put_qt(uint8_t* qop, const float* Bs, int r, int c0, uint32_t fmask, const float* x,
+                                       __nv_bfloat16* qg) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        uint32_t qpk[8];
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+            const int e = 16 * h + 2 * e2, c = c0 + e;
+            qpk[e2] = pack_bf16x2(x[e] * e_b(Bs, r, c, (fmask >> e) & 1u),
+                                  x[e + 1] * e_b(Bs, r, c + 1, (fmask >> (e + 1)) & 1u));
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int c = c0 + 16 * h + 8 * j;
+            *reinterpret_cast<uint4*>(qop + (c >> 6) * PIECE + sw128_offset(uint32_t(r), uint32_t(c & 63))) =
+                make_uint4(qpk[4 * j], qpk[4 * j + 1], qpk[4 * j + 2], qpk[4 * j + 3]);
+        }
+        if (qg) st_global_v8(qg + 16 * h, qpk);
+    }
+}
+
 // one TMEM column of the warp's 32 lanes
 __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
     uint32_t r;
@@ -108,7 +155,8 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
                     const __grid_constant__ CUtensorMap tmM, const __grid_constant__ CUtensorMap tmS,
                     const float* __restrict__ la,
                     const float* __restrict__ s_in, __nv_bfloat16* __restrict__ s_b, float* __restrict__ s_f,
-                    int64_t L, int64_t N, int64_t D, int* err) {
+                    __nv_bfloat16* __restrict__ Qt, __nv_bfloat16* __restrict__ Pq, int64_t L, int64_t N, int64_t D,
+                    int* err) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* phi = ring + kRing;
@@ -131,8 +179,11 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
         mbar_init(&bar.phi_ready, kNT);
         mbar_init(&bar.l_full, 1);
         mbar_init(&bar.s_full, 1);
+        mbar_init(&bar.qt_ready, kNT);
+        mbar_init(&bar.q_full, 1);
         mbar_init(&bar.drain, 1);
         bar.abort_flag = 0;
+        bar.any_beyond = 0;
         fence_barrier_init();
     }
     if (warp == 1) {
@@ -200,6 +251,18 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
                              sdesc_sw128(ph + kk * 2048, PIECE, 1024), id3, 1u);
                 mma_commit(&bar.l_full);
             }
+            // the next layer's score block P = Q~ Phi^T over the slots (both operands K-major), into cols [0,128)
+            ok = ok && mbar_wait(&bar.qt_ready, 0, err, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                const uint32_t qa = smem_u32(ring + qt_piece<MODE>()), ph = smem_u32(phi);
+                const uint32_t id4 = idesc_bf16_f32(128, 128, false, false);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_bf16(tmem, sdesc_sw128(qa + (kk / 4) * PIECE + (kk % 4) * 32, 16, 1024),
+                             sdesc_sw128(ph + (kk / 4) * PIECE + (kk % 4) * 32, 16, 1024), id4, kk > 0 ? 1u : 0u);
+                mma_commit(&bar.q_full);
+            }
             mma_commit(&bar.drain);
             mbar_drain(&bar.drain, 0);
         }
@@ -230,14 +293,19 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
                 gamma += x;
             }
             const bool beyond = gamma < -kBound2;  // the same for the kQ threads of the slot
-            if (part == 0) bar.flag[c] = beyond ? 1u : 0u;
+            if (part == 0) {
+                bar.flag[c] = beyond ? 1u : 0u;
+                if (beyond) atomicOr(&bar.any_beyond, 1);
+            }
             uint8_t* pp = phi + (c >> 6) * PIECE;
             run = off;
 #pragma unroll
             for (int e = 0; e < kPart; ++e) {
                 const int t = r0 + e;
                 run = fmaf(la_floor(v[e]), kLog2e, run);
-                Bs[bs_idx(t, c)] = run;
+                // e^B for a slot within the bound (the epilogue's factor, formed here under the loads); the
+                // exponent itself (base 2) for a slot beyond it, whose exact terms take differences
+                Bs[bs_idx(t, c)] = beyond ? run : exp2_ftz(run);
                 const float f = (!beyond && t < nvalid) ? write_weight(v[e]) * exp2_ftz(-run) : 0.f;
                 *reinterpret_cast<__nv_bfloat16*>(pp + sw128_offset(uint32_t(t), uint32_t(c & 63))) =
                     __float2bfloat16_rn(f);
@@ -311,7 +379,7 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             }
 #pragma unroll
             for (int e = 0; e < kPart; ++e)
-                if (!((fmask >> e) & 1u)) rr[e] *= exp2_ftz(Bs[bs_idx(r, c0 + e)]);
+                if (!((fmask >> e) & 1u)) rr[e] *= Bs[bs_idx(r, c0 + e)];
         }
         if (MODE == 0) {
             // softmax over the row's 128 slots, spread over kQ threads
@@ -333,28 +401,37 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             sum = 0.f;
 #pragma unroll
             for (int g2 = 0; g2 < kQ; ++g2) sum += bar.red[1][g2][r];
-            // s staged in the ring (free: the second GEMM has read P1; the exact terms above are done, every
-            // thread having passed the first exchange) with a row stride of 129 floats, so that a warp writing
-            // one column over 32 rows, and one reading a row, touch 32 banks; then whole rows are stored
-            float* stg = reinterpret_cast<float*>(ring);
-            constexpr int kStride = kSlots + 1;
             const float inv = 1.f / sum;
+#pragma unroll
+            for (int e = 0; e < kPart; ++e) rr[e] = (ok && valid) ? rr[e] * inv : 0.f;
+            // the next layer's query operand first, so that its MMA runs under the stores below
+            put_qt(ring + qt_piece<MODE>(), Bs, r, c0, fmask, rr,
+                   (ok && valid) ? Qt + (bh * L + t) * kSlots + c0 : nullptr);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar.qt_ready);
+            // s staged in the ring's first four pieces (free: the second GEMM has read P1; the exact terms above
+            // are done, every thread having passed the first exchange), column c of row t at t * 128 + (c ^ (t %
+            // 32)), so that a warp writing one column over 32 rows, and one reading a row, touch 32 banks; then
+            // whole rows are stored
+            float* stg = reinterpret_cast<float*>(ring);
             if (ok) {
 #pragma unroll
-                for (int e = 0; e < kPart; ++e) stg[r * kStride + c0 + e] = rr[e] * inv;
+                for (int e = 0; e < kPart; ++e) stg[r * kSlots + ((c0 + e) ^ (r & 31))] = rr[e];
             }
             named_sync(1, kNT);
             if (ok) {
                 for (int rho = warp - 2; rho < nvalid; rho += kCW) {
-                    const float* srow = stg + rho * kStride;
+                    const float* srow = stg + rho * kSlots;
+                    const int sw = rho & 31;
                     float* df = s_f + (bh * L + t0 + rho) * kSlots;
                     __nv_bfloat16* db = s_b + (bh * L + t0 + rho) * kSlots;
 #pragma unroll
-                    for (int k4 = 0; k4 < kSlots / 32; ++k4) df[32 * k4 + lane] = srow[32 * k4 + lane];
+                    for (int k4 = 0; k4 < kSlots / 32; ++k4) df[32 * k4 + lane] = srow[(32 * k4 + lane) ^ sw];
 #pragma unroll
                     for (int k2 = 0; k2 < kSlots / 64; ++k2) {
                         const int c = 64 * k2 + 2 * lane;
-                        *reinterpret_cast<uint32_t*>(db + c) = pack_bf16x2(srow[c], srow[c + 1]);
+                        *reinterpret_cast<uint32_t*>(db + c) = pack_bf16x2(srow[c ^ sw], srow[(c + 1) ^ sw]);
                     }
                 }
             }
@@ -380,20 +457,72 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             dot = 0.f;
 #pragma unroll
             for (int g2 = 0; g2 < kQ; ++g2) dot += bar.red[0][g2][r];
+#pragma unroll
+            for (int e4 = 0; e4 < kPart / 4; ++e4) {
+                const float4 x = sv[e4];
+                float* y = rr + 4 * e4;
+                const bool on = ok_s && valid;
+                y[0] = on ? x.x * (y[0] - dot) : 0.f;
+                y[1] = on ? x.y * (y[1] - dot) : 0.f;
+                y[2] = on ? x.z * (y[2] - dot) : 0.f;
+                y[3] = on ? x.w * (y[3] - dot) : 0.f;
+            }
+            // the next layer's query operand goes where P1 was: every thread has passed the exact terms
+            // (which read P1) before the exchange above
+            put_qt(ring + qt_piece<MODE>(), Bs, r, c0, fmask, rr,
+                   (ok && valid) ? Qt + (bh * L + t) * kSlots + c0 : nullptr);
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar.qt_ready);
             if (ok_s && valid) {
                 __nv_bfloat16* db = s_b + (bh * L + t) * kSlots + c0;
 #pragma unroll
                 for (int c16 = 0; c16 < kPart / 16; ++c16) {
                     uint32_t wb[8];
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const float4 x = sv[4 * c16 + e4];
-                        const float* y = rr + 16 * c16 + 4 * e4;
-                        wb[2 * e4] = pack_bf16x2(x.x * (y[0] - dot), x.y * (y[1] - dot));
-                        wb[2 * e4 + 1] = pack_bf16x2(x.z * (y[2] - dot), x.w * (y[3] - dot));
-                    }
+                    for (int e2 = 0; e2 < 8; ++e2)
+                        wb[e2] = pack_bf16x2(rr[16 * c16 + 2 * e2], rr[16 * c16 + 2 * e2 + 1]);
                     st_global_v8(db + 16 * c16, wb);
                 }
+            }
+        }
+        // ---- the next layer's score block P: thread = row r, P columns c0 .. c0 + 31 ----
+        // every row of x is stored: the exact terms below read other threads' columns back
+        __threadfence_block();
+        named_sync(1, kNT);
+        if (__all_sync(0xffffffffu, ok && mbar_wait(&bar.q_full, 0, err, abort_flag))) {
+            tc_fence_after();
+            float pv[kPart];
+#pragma unroll
+            for (int cb = 0; cb < kPart / 16; ++cb) tmem_ld16(tmem + lane_off + uint32_t(c0 + 16 * cb), pv + 16 * cb);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < kPart; ++e) pv[e] = (c0 + e <= r) ? pv[e] : 0.f;
+            if (bar.any_beyond && valid) {
+                // slots beyond the range bound: x_rc w_sc e^{B_rc - B_sc} for s <= r, in log space
+                const float* lab = la + (bh * L + t0) * kSlots;
+                const __nv_bfloat16* xrow = s_b + (bh * L + t) * kSlots;
+#pragma unroll 1
+                for (int c = 0; c < kSlots; ++c) {
+                    if (!bar.flag[c]) continue;
+                    const float xr = __bfloat162float(xrow[c]);
+                    const float b2r = Bs[bs_idx(r, c)];
+#pragma unroll
+                    for (int e = 0; e < kPart; ++e) {
+                        const int sj = c0 + e;
+                        if (sj <= r)
+                            pv[e] = fmaf(xr * write_weight(lab[int64_t(sj) * kSlots + c]),
+                                         exp2_ftz(fminf(b2r - Bs[bs_idx(sj, c)], 0.f)), pv[e]);
+                    }
+                }
+            }
+            __nv_bfloat16* dp = Pq + ((bh * N + i) * C + r) * C + c0;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int e2 = 0; e2 < 8; ++e2) pk[e2] = pack_bf16x2(pv[16 * h + 2 * e2], pv[16 * h + 2 * e2 + 1]);
+                st_global_v8(dp + 16 * h, pk);
             }
         }
     }
@@ -407,14 +536,18 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
 
 // Gate preparation of the slot memories' walks, per (chunk, head): the write weight
 // w = bf16(1 - e^{log a}), the walk operand K~ = w e^{Gamma - B} (B the per-chunk cumsum of log a, Gamma
-// its last row) and e^Gamma, as the GLA preparation kernel forms them for a GLA key w. kQ threads per slot
-// (32 rows each): partial sums, a prefix over them through shared memory, then every row's values.
+// its last row) and e^Gamma, as the GLA preparation kernel forms them for a GLA key w. Both GLA layers of
+// the method have key w under this gate, so K~ and e^Gamma also go to the second layer's buffers when
+// given (Kt2, gam2). kQ threads per slot (32 rows each): partial sums, a prefix over them through shared
+// memory, then every row's values.
 constexpr int kGateThreads = kSlots * kQ;
 
 __global__ void __launch_bounds__(kGateThreads, 2) k_gsa_gate_prep(const float* __restrict__ la,
                                                                 __nv_bfloat16* __restrict__ w,
                                                                 __nv_bfloat16* __restrict__ Kt,
-                                                                float* __restrict__ gam, int64_t L, int64_t N) {
+                                                                float* __restrict__ gam,
+                                                                __nv_bfloat16* __restrict__ Kt2,
+                                                                float* __restrict__ gam2, int64_t L, int64_t N) {
     __shared__ float tot[kQ][kSlots];
     const int c = threadIdx.x % kSlots, part = threadIdx.x / kSlots, i = blockIdx.x;
     const int r0 = part * kPart;
@@ -437,7 +570,11 @@ __global__ void __launch_bounds__(kGateThreads, 2) k_gsa_gate_prep(const float* 
         gamma += x;
     }
     // exponents are <= 0 in exact arithmetic; the clamps absorb cumsum rounding
-    if (part == 0) gam[(bh * N + i) * kSlots + c] = __expf(fminf(gamma, 0.f));
+    if (part == 0) {
+        const float eg = __expf(fminf(gamma, 0.f));
+        gam[(bh * N + i) * kSlots + c] = eg;
+        if (gam2) gam2[(bh * N + i) * kSlots + c] = eg;
+    }
     run = off;
 #pragma unroll
     for (int e = 0; e < kPart; ++e) {
@@ -445,8 +582,10 @@ __global__ void __launch_bounds__(kGateThreads, 2) k_gsa_gate_prep(const float* 
         run += la_floor(v[e]);
         if (t < nvalid) {
             const __nv_bfloat16 wb = __float2bfloat16_rn(1.f - __expf(v[e]));
+            const __nv_bfloat16 kt = __float2bfloat16_rn(__bfloat162float(wb) * __expf(fminf(gamma - run, 0.f)));
             w[base + int64_t(t) * kSlots] = wb;
-            Kt[base + int64_t(t) * kSlots] = __float2bfloat16_rn(__bfloat162float(wb) * __expf(fminf(gamma - run, 0.f)));
+            Kt[base + int64_t(t) * kSlots] = kt;
+            if (Kt2) Kt2[base + int64_t(t) * kSlots] = kt;
         }
     }
 }
@@ -465,16 +604,16 @@ bool tc_gsa_slot_read_supported(const Problem& p) {
 }
 
 gla_status tc_gsa_gate_prep_launch(const Problem& p, const float* la, __nv_bfloat16* w, __nv_bfloat16* Kt,
-                                   float* gam, cudaStream_t s) {
+                                   float* gam, __nv_bfloat16* Kt2, float* gam2, cudaStream_t s) {
     if (p.K != kSlots || p.N > 65535 || p.BH > 65535) return GLA_ERR_UNSUPPORTED;
     GLA_LAUNCH("gsa_gate_prep", k_gsa_gate_prep, dim3(unsigned(p.N), unsigned(p.BH)), kGateThreads, 0, s, la, w, Kt,
-               gam, p.L, p.N);
+               gam, Kt2, gam2, p.L, p.N);
     return GLA_OK;
 }
 
 gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* y, const __nv_bfloat16* M,
-                                   const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f, int mode,
-                                   cudaStream_t s) {
+                                   const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f,
+                                   __nv_bfloat16* Qt, __nv_bfloat16* P, int mode, cudaStream_t s) {
     if (!tc_gsa_slot_read_supported(p)) return GLA_ERR_UNSUPPORTED;
     CUtensorMap m[4];
     memset(m, 0, sizeof(m));
@@ -495,7 +634,7 @@ gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* 
         return GLA_ERR_CUDA;
     const dim3 grid(unsigned(p.N), unsigned(p.BH));
     GLA_LAUNCH(mode == 0 ? "gsa_slot_read" : "gsa_slot_read_bwd", fn, grid, kThreadsSR, kSmem, s, m[0], m[1], m[2],
-               m[3], la, s_in, s_b, s_f, p.L, p.N, p.V, device_error_word());
+               m[3], la, s_in, s_b, s_f, Qt, P, p.L, p.N, p.V, device_error_word());
     return GLA_OK;
 }
 

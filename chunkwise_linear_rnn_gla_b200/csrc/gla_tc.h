@@ -35,14 +35,18 @@ TcBuffers tc_carve(const Problem& p, Arena& a, bool bwd);
 // with B the per-chunk cumsum of log a over the slots (exact log-space terms for a slot whose chunk
 // decay passes the range bound). mode 0 (x = q, y = k): s = softmax(r) into s_b (bf16) and s_f
 // (fp32). mode 1 (x = dO, y = v): G = s * (r - <s, r>) into s_b (bf16), s read from s_in (fp32).
+// Either result x (as stored in bf16) is the query of a GLA layer with key w under the same gate; its
+// chunk-local operands come out too, as tc_prep_launch would write them: Qt = x e^{B} [BH][L][m] and
+// the masked scores P [BH][N][128][128].
 gla_status tc_gsa_slot_read_launch(const Problem& p, const void* x, const void* y, const __nv_bfloat16* M,
-                                   const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f, int mode,
-                                   cudaStream_t s);
+                                   const float* la, const float* s_in, __nv_bfloat16* s_b, float* s_f,
+                                   __nv_bfloat16* Qt, __nv_bfloat16* P, int mode, cudaStream_t s);
 bool tc_gsa_slot_read_supported(const Problem& p);
 // The slot gate's preparation for the memories' walks (p: key width m = 128): w = bf16(1 - e^{log a})
-// [BH][L][m], the walk operand K~ = w e^{Gamma - B} [BH][L][m] and e^Gamma [BH][N][m].
+// [BH][L][m], the walk operand K~ = w e^{Gamma - B} [BH][L][m] and e^Gamma [BH][N][m], the last two also
+// into Kt2 / gam2 when given (the second GLA layer's buffers: the same key and gate).
 gla_status tc_gsa_gate_prep_launch(const Problem& p, const float* la, __nv_bfloat16* w, __nv_bfloat16* Kt,
-                                   float* gam, cudaStream_t s);
+                                   float* gam, __nv_bfloat16* Kt2, float* gam2, cudaStream_t s);
 
 // Chunk-parallel gate preparation (gla_tc_prep.cu): Q~, K~, e^Gamma and the
 // masked intra-chunk scores P.
