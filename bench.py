@@ -29,9 +29,6 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-# ~1 ms of device spin (at ~1.9 GHz) between an L2 flush and the start event of a timed call or step:
-# longer than the host needs to marshal and launch it, so the window holds device time only
-HOLD_CYCLES = 2_000_000
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -351,14 +348,13 @@ def run_gsa(dev, peaks, med_ms, flush, with_cpu=True):
     alg = gsa_model(B, H, L, K, V, m)
     lr = layer_roofline(alg["bytes"], alg["flops"], ms, peaks)
     # per-kernel device time (an event pair around every launch; shares, not the headline), L2 flushed
-    # and the stream held until the step is queued, as for the GLA step
+    # before each step as for the GLA step
     fn()
     torch.cuda.synchronize(dev)
     gla.gla_profile_reset()
     gla.gla_profile_enable(True)
     for _ in range(3):
         flush.fill_(1.0)
-        torch.cuda._sleep(HOLD_CYCLES)
         fn()
     torch.cuda.synchronize(dev)
     gla.gla_profile_enable(False)
@@ -384,7 +380,7 @@ def run_gsa(dev, peaks, med_ms, flush, with_cpu=True):
     entry["decode"] = {"B": Bd, "us_per_step": round(step_ms * 1e3, 2), "tokens_per_s": round(Bd / step_ms * 1e3, 1),
                        "memory_GBps": round(mem_bytes / step_ms / 1e6, 1),
                        "hbm_frac": round(mem_bytes / step_ms / 1e6 / peaks["hbm_gbs"], 4),
-                       "how": "median of single calls, L2 flushed and the stream held by a device spin before each; %.1f MB of memories read and "
+                       "how": "median of single calls, L2 flushed before each; %.1f MB of memories read and "
                               "written per step" % (mem_bytes / 1e6)}
     del hk, hv, sd
     if with_cpu:
@@ -427,9 +423,6 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
         ts = []
         for _ in range(reps):
             flush.fill_(1.0)
-            # a spin on the device keeps the stream busy while the host marshals the call, so the start
-            # event fires with the call already queued and the window holds device time only
-            torch.cuda._sleep(HOLD_CYCLES)
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             a.record(stream)
             fn()
@@ -496,7 +489,6 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
     flushed = []
     for t in range(T):
         flush.fill_(1.0)
-        torch.cuda._sleep(HOLD_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         gla.gla_step(q[t], k[t], v[t], la[t], S, o=ob[t])
@@ -534,7 +526,7 @@ def run_workloads(dev, peaks, flush, with_cpu=True, reps=10):
            "l2_flushed": {"us_per_step": round(ms_flushed * 1e3, 3), "tokens_per_s": round(B / ms_flushed * 1e3, 1),
                           "state_GBps": round(state_bytes / ms_flushed / 1e6, 1),
                           "hbm_frac": round(state_bytes / ms_flushed / 1e6 / peaks["hbm_gbs"], 4),
-                          "how": "median of 64 single calls, each after a 512 MB write and a device spin that queues the call before its start event"}}
+                          "how": "median of 64 single calls, each after a 512 MB write"}}
     if with_cpu:
         import oracle
         from chunkwise_linear_rnn_gla_b200.inputs import to_f64_numpy
@@ -684,9 +676,6 @@ def main():
         gla.gla_profile_enable(kernel_events)
         for i in range(args.steps):
             flush.fill_(float(i))  # evict L2 (126 MB) between timed steps
-            # hold the stream until the host has queued the whole step, so that no launch waits on the
-            # host inside the window (the eager passes issue every kernel from Python)
-            torch.cuda._sleep(HOLD_CYCLES)
             ev[i][0].record(stream)
             if use_graph:
                 graph.replay()

@@ -4,8 +4,7 @@
 
 For every bf16 workload of `inputs.WORKLOADS`: the forward and the forward + backward (the backward
 reusing the forward's workspace), with materialised and with non-materialised chunk states. Each
-case is called eagerly with L2 flushed before every call (a 512 MB write, then a short device spin
-so that the call is queued before its start event); the figure is the median
+case is called eagerly with L2 flushed before every call (a 512 MB write); the figure is the median
 of 10 CUDA-event timings around the call, after 3 warm-up calls, followed by the per-kernel split
 from the library's own launch timing over 3 more calls.
 
@@ -28,16 +27,12 @@ from . import gla_step, make_desc
 from .inputs import DECODE, GSA_WORKLOAD, WORKLOADS, make_gsa_inputs, make_inputs, make_step_inputs
 
 FLUSH_BYTES = 512 * 1024 * 1024
-# ~1 ms of device spin (at ~1.9 GHz) after the flush: the host marshals and queues the timed call
-# meanwhile, so the start event fires with the call queued and the window holds device time only
-HOLD_CYCLES = 2_000_000
 
 
 def _median_ms(fn, flush, reps):
     ts = []
     for _ in range(reps):
         flush.zero_()
-        torch.cuda._sleep(HOLD_CYCLES)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
         fn()
@@ -71,7 +66,6 @@ def time_layer(w, flush):
             gla_profile_reset()
             for _ in range(3):
                 flush.zero_()
-                torch.cuda._sleep(HOLD_CYCLES)
                 fn()
             torch.cuda.synchronize()
             gla_profile_enable(False)
@@ -106,7 +100,6 @@ def time_gsa(flush, reps=10):
             gla_profile_reset()
             for _ in range(3):
                 flush.zero_()
-                torch.cuda._sleep(HOLD_CYCLES)
                 fn()
             torch.cuda.synchronize()
             gla_profile_enable(False)
