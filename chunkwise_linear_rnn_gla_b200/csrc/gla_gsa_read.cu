@@ -14,7 +14,7 @@
 // in fp32 up to the softmax (forward) or its backward (the kernel's epilogue).
 //
 // One CTA per (chunk, head); m = 128 slots. Over D in 64-wide pieces:
-//   TMEM cols [0,128)   A1 = x y^T          (M=128 tokens, N=128 tokens)
+//   TMEM cols [0,128)   A1 = x y^T          (M=128 tokens, N=128 tokens; later the next layer's P)
 //   TMEM cols [128,256) L  = x M_[i]^T      (N=128 slots)
 // as ONE N=256 tcgen05.mma per 16-wide k step (the y piece and the M piece sit
 // side by side in shared memory). The epilogue masks A1 (s <= j) into bf16 P1,
@@ -411,28 +411,24 @@ __global__ void __launch_bounds__(kThreadsSR, 1)
             tc_fence_before();
             mbar_arrive(&bar.qt_ready);
             // s staged in the ring's first four pieces (free: the second GEMM has read P1; the exact terms above
-            // are done, every thread having passed the first exchange), column c of row t at t * 128 + (c ^ (t %
-            // 32)), so that a warp writing one column over 32 rows, and one reading a row, touch 32 banks; then
-            // whole rows are stored
+            // are done, every thread having passed the first exchange) in 16-byte chunks, chunk j of row t at
+            // t * 128 + 4 (j ^ (t % 8)) floats, so that a warp writing one chunk over 32 rows, and one reading a
+            // row, touch every bank once per 8 lanes; then whole rows are stored, one 16-byte (fp32) and one
+            // 8-byte (bf16) store per lane and row
             float* stg = reinterpret_cast<float*>(ring);
             if (ok) {
 #pragma unroll
-                for (int e = 0; e < kPart; ++e) stg[r * kSlots + ((c0 + e) ^ (r & 31))] = rr[e];
+                for (int j = 0; j < kPart / 4; ++j)
+                    *reinterpret_cast<float4*>(stg + r * kSlots + 4 * (((c0 >> 2) + j) ^ (r & 7))) =
+                        make_float4(rr[4 * j], rr[4 * j + 1], rr[4 * j + 2], rr[4 * j + 3]);
             }
             named_sync(1, kNT);
             if (ok) {
                 for (int rho = warp - 2; rho < nvalid; rho += kCW) {
-                    const float* srow = stg + rho * kSlots;
-                    const int sw = rho & 31;
-                    float* df = s_f + (bh * L + t0 + rho) * kSlots;
-                    __nv_bfloat16* db = s_b + (bh * L + t0 + rho) * kSlots;
-#pragma unroll
-                    for (int k4 = 0; k4 < kSlots / 32; ++k4) df[32 * k4 + lane] = srow[(32 * k4 + lane) ^ sw];
-#pragma unroll
-                    for (int k2 = 0; k2 < kSlots / 64; ++k2) {
-                        const int c = 64 * k2 + 2 * lane;
-                        *reinterpret_cast<uint32_t*>(db + c) = pack_bf16x2(srow[c ^ sw], srow[(c + 1) ^ sw]);
-                    }
+                    const float4 x = *reinterpret_cast<const float4*>(stg + rho * kSlots + 4 * (lane ^ (rho & 7)));
+                    *reinterpret_cast<float4*>(s_f + (bh * L + t0 + rho) * kSlots + 4 * lane) = x;
+                    *reinterpret_cast<uint2*>(s_b + (bh * L + t0 + rho) * kSlots + 4 * lane) =
+                        make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
                 }
             }
         } else {
