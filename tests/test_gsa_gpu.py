@@ -87,6 +87,19 @@ def test_gsa_bf16_peaked_softmax_and_extreme_gates():
     check_all(inp, "bf16", names=("o", "hkT", "hvT", "dq", "dk", "dv", "dlog_a"))
 
 
+def test_gsa_bf16_gates_straddling_the_range_bound():
+    """Gates whose chunk decays straddle the tensor-core route's range bound: about half of the slots of
+    every full chunk pass it, so the masked scores of the next layer, formed in the slot reads, add their
+    exact log-space terms to the tensor-core product within the same chunk (L = 389: a ragged last chunk)."""
+    inp = make_gsa_inputs(1, 2, 389, 128, 128, 128, "bf16", seed=9, q_scale=4.0, gate_scale=0.62, h0=True,
+                          dhT=True)
+    la = inp["log_a"][0]
+    frac = [(la[:, i:i + 128].sum(1) < -64).float().mean().item() for i in range(0, 384, 128)]
+    assert all(0.3 < f < 0.7 for f in frac), frac
+    assert route_of(inp) == "tc"
+    check_all(inp, "bf16")
+
+
 @pytest.mark.parametrize("L,Dk,Dv,m", [(333, 128, 64, 64), (256, 64, 192, 256)])
 def test_gsa_bf16_cuda_core_slots(L, Dk, Dv, m):
     """Slot counts other than 128: bf16 tensors on the CUDA-core route (fp32 GLA passes)."""
