@@ -77,6 +77,9 @@ constexpr size_t kRing = size_t(2) * 3 * PIECE;          // x, y, M pieces, two 
 constexpr size_t kPhi = size_t(2) * PIECE;               // Phi [128 tokens x 128 slots] bf16
 constexpr size_t kBs = size_t(C) * kSlots * sizeof(float);  // e^B, or B (base 2) beyond the bound [128 x 128] fp32
 constexpr size_t kSmem = 1024 + kRing + kPhi + kBs + sizeof(SRBars);
+static_assert(kSmem <= 232448, "shared memory of one block");
+// the forward read's staged s rows fill the ring's first four pieces, its Q~ operand the last two
+static_assert(size_t(C) * kSlots * sizeof(float) == 4 * PIECE && kRing == 6 * PIECE, "ring areas");
 
 // The read gradient's s tile (fp32 [128 rows x 128 slots], four TMA boxes of 32 columns with the 128-byte
 // swizzle) goes to the ring once the D loop is done, into the four 16 KB pieces that P1 does not use.
