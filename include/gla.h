@@ -268,7 +268,8 @@ gla_status gla_state_combine(int64_t G, int64_t BH, int64_t Dk, int64_t Dv, cons
  * per-slot intermediates (w, s and, in the backward, their gradients). */
 /* The route gla_gsa_fwd / gla_gsa_bwd take for (d, slots): *impl = GLA_IMPL_TC (tensor cores:
  * bf16, slots = 128, both GLA passes on the tensor-core path with materialised states, the logits and
- * the read gradient by a fused fp32 slot-read kernel) or GLA_IMPL_SIMT (both GLA passes on the CUDA
+ * the read gradient by a fused fp32 slot-read kernel that also prepares the next GLA pass's query
+ * operands) or GLA_IMPL_SIMT (both GLA passes on the CUDA
  * cores in fp32; bf16 tensors are converted at the boundary). Returns GLA_ERR_INVALID_ARG /
  * GLA_ERR_UNSUPPORTED like the compute calls. */
 gla_status gla_gsa_resolve(const gla_desc* d, int32_t slots, int32_t* impl);
