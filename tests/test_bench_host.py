@@ -105,3 +105,52 @@ def test_workload_timer_lists_and_validates_without_a_gpu(capsys):
     assert "gla1p3b_fwdbwd" in listed and "decode" in listed and "tiny_f32" not in listed
     with pytest.raises(SystemExit):
         time_workloads.main(["--only", "no_such_workload"])
+
+
+def _gsa_io_bytes(B, H, L, K, V, m):
+    """Gated slot attention: every tensor the method reads or writes once (bf16 q, k, v, o, dO, dq, dk, dv;
+    fp32 gate and its gradient over the m slots), no memories."""
+    th = B * H * L
+    fwd = [("q", th * K, 2), ("k", th * K, 2), ("v", th * V, 2), ("log_a", th * m, 4), ("o", th * V, 2)]
+    bwd = [("q", th * K, 2), ("k", th * K, 2), ("v", th * V, 2), ("dO", th * V, 2), ("log_a", th * m, 4),
+           ("dq", th * K, 2), ("dk", th * K, 2), ("dv", th * V, 2), ("dlog_a", th * m, 4)]
+    return sum(n * e for _, n, e in fwd) + sum(n * e for _, n, e in bwd)
+
+
+def _gsa_flops(B, H, L, K, V, m, C):
+    """The method's contractions per chunk of C tokens (2 flops per multiply-add, causal halves for the
+    intra-chunk products), as two GLA layers over the slots joined by the softmax."""
+    n_chunks = B * H * (L // C)
+
+    def gla_fwd_out(Kg, Vg):  # the output of a GLA with key width Kg and value width Vg, states given
+        return [2 * C * Kg * Vg, C * C * Kg, C * C * Vg]
+
+    def gla_bwd(Kg, Vg):  # a GLA backward with key width Kg, value width Vg
+        return [2 * C * Kg * Vg] * 4 + [C * C * Vg, C * C * Vg, C * C * Kg, C * C * Kg, C * C * Kg]
+
+    def slot_read(Dx):  # the value-side read of a slot memory with a Dx-wide query: inter, q k^T, P1 Phi
+        return [2 * C * Dx * m, C * C * Dx, C * C * m]
+
+    fwd = [2 * C * m * K, 2 * C * m * V]        # both memories' state updates
+    fwd += slot_read(K)                          # layer one: the logits
+    fwd += gla_fwd_out(m, V)                     # layer two: o
+    bwd = gla_bwd(m, V)                          # layer two's backward
+    bwd += slot_read(V)                          # the read of the value memory with dO: ds
+    bwd += gla_fwd_out(m, K)                     # layer one's forward with query G: dq
+    bwd += gla_bwd(m, K)                         # layer one's backward with dO = q
+    return n_chunks * (sum(fwd) + sum(bwd))
+
+
+def test_gsa_model_matches_the_tensor_and_contraction_lists():
+    for (B, H, L, K, V, m) in [(4, 4, 2048, 256, 512, 128), (2, 3, 1024, 128, 64, 64)]:
+        g = bench.gsa_model(B, H, L, K, V, m, C=128)
+        assert g["bytes"] == _gsa_io_bytes(B, H, L, K, V, m)
+        assert g["flops"] == _gsa_flops(B, H, L, K, V, m, 128)
+
+
+def test_gsa_roofline_of_the_1p3b_shape():
+    g = bench.gsa_model(4, 4, 2048, 256, 512, 128)
+    assert g["per_token_head"] == {"bytes": 9728, "flops": 1933312}
+    t_hbm = g["bytes"] / 6551e9
+    assert t_hbm > g["flops"] / 1655.1e12  # bound by HBM
+    assert abs(t_hbm * 1e6 - 48.66) < 0.01
